@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE + multi-LoRA layer on B200: tokens/s of the whole hot path.
+
+One step = one pass of the whole path over one batch resident in HBM:
+  moe_lora_route   router logits x W_r^T, softmax top-k + renormalised weights,
+                   stable (expert, adapter) sort into segments
+  moe_lora_forward gather + gate_up LoRA shrink, tcgen05 gate_up GEMM with the LoRA
+                   expand and SiLU-and-mul fused in its epilogue, down LoRA shrink,
+                   tcgen05 down GEMM with expand and routing weight, fixed-order combine
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--M M]
+    python bench.py --impl reference ...      (the fp64 CPU oracle, same metric)
+
+Default workload: MoE decode, bf16 experts, E=64, top-8, H=2048, I=1408, 8 adapters
+of rank 16 on gate_up and down, M=64 tokens per step.  For N > 1 (torchrun) every
+rank runs an independent replica (weak scaling, no collective on the data path);
+timing is the max over ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import synth  # noqa: E402
+
+METRIC = "MoE+multi-LoRA layer tokens/s; achieved HBM GB/s or TC util vs B200 peak"
+DEFAULT_WORKLOAD = synth.MOE_DECODE_BF16.name
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+# ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM on the
+# default workload, with the hash of the kernel source it was taken on; reported as
+# null when the source has changed since.  Filled from profiles/.
+NCU_TRAFFIC = {"gemm_tc.cu": None, "bytes_per_launch": None}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--M", type=int, default=64)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batches", type=int, default=4, help="distinct token batches cycled over the steps")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [[c.strip() for c in ln.split(",")] for ln in out.strip().splitlines() if ln.count(",") >= 8]
+        if self.uuid:
+            mine = [r for r in rows if self.uuid.replace("GPU-", "") in r[0]]
+            rows = mine or rows
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sm)}
+
+
+def src_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "moe_lora_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def routing_stats(rt: dict, shape: synth.MoEShape):
+    """Touched experts and (adapter, expert) pairs of one routed batch (host side)."""
+    so = rt["seg_offsets"].cpu().numpy().astype(np.int64)
+    cnt = np.diff(so).reshape(shape.E, shape.L + 1)
+    experts = int(np.count_nonzero(cnt.sum(1)))
+    pairs = int(np.count_nonzero(cnt[:, : shape.L]))
+    return experts, pairs
+
+
+def gateup_alg_bytes(shape, M, experts, pairs):
+    """Bytes the gate_up GEMM must move once: touched expert gate_up weights, touched
+    B_gu slices, the gathered x rows, z_gu, and the act it writes."""
+    wb = 1 if shape.wdtype == "e4m3" else 2
+    mk = M * shape.k
+    return (experts * 2 * shape.I * shape.H * wb + pairs * shape.r * 2 * shape.I * 2
+            + mk * shape.H * 2 + mk * shape.r * 4 + mk * shape.I * 2)
+
+
+def layer_alg_bytes(shape, M, experts, pairs):
+    """Bytes the whole layer must move once (intermediates excluded): touched expert
+    weights, touched adapter slices, router weight, x, adapter ids and y."""
+    wb = 1 if shape.wdtype == "e4m3" else 2
+    per_expert = (2 * shape.I * shape.H + shape.H * shape.I) * wb
+    per_pair = shape.r * (shape.H + 2 * shape.I + shape.I + shape.H) * 2
+    return (experts * per_expert + pairs * per_pair + shape.E * shape.H * 2
+            + M * shape.H * 2 * 2 + M * 4)
+
+
+def layer_flops(shape, M):
+    mk = M * shape.k
+    return (2 * mk * (shape.H * 2 * shape.I + shape.I * shape.H)
+            + 2 * mk * shape.r * (2 * shape.H + 3 * shape.I) + 2 * M * shape.H * shape.E)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_tokens_per_s(shape, M, cpu_weights, seconds: float, max_calls: int | None = None,
+                        tokens_per_call: int | None = None):
+    """The fp64 oracle (route from x, sort, forward) on batch 0, repeated until `seconds`
+    of CPU time have passed (or `max_calls`); returns (tokens/s, calls, tokens/call)."""
+    from oracle import formats
+    from oracle import moe_lora_ref as ref
+    from tests.gpu_cases import CpuWeightsOracle
+    OW = CpuWeightsOracle(shape, cpu_weights)
+    x, ad = synth.moe_tokens(shape, M)
+    x64 = formats.to_f64(synth.bits(x), "bf16")
+    ad64 = ad.numpy().astype(np.int64)
+    wr, bias = OW.router()
+    n = M if tokens_per_call is None else max(1, min(M, tokens_per_call))
+    sel = np.arange(n)
+    # weights of the experts this batch touches are decoded once, like a model load
+    lg = ref.router_logits(x64, wr, bias)
+    ids, _ = ref.route_topk(lg, shape.k)
+    for e in np.unique(ids[sel]):
+        OW.expert(int(e))
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        lg = ref.router_logits(x64[sel], wr, bias)
+        ids, w = ref.route_topk(lg, shape.k)
+        ref.sort_pairs(ids, ad64[sel], shape.E, shape.L)
+        ref.moe_lora_forward(x64[sel], ids, w, ad64[sel], shape.I, OW.expert, OW.adapter)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_calls is not None and calls >= max_calls):
+            break
+    return n * calls / el, calls, n, el
+
+
+def reference_arm(args, world, rank):
+    """--impl reference: the oracle on the host cores, same metric/unit/config."""
+    if rank != 0:
+        return
+    shape = synth.WORKLOADS[args.workload]
+    if not isinstance(shape, synth.MoEShape):
+        print(json.dumps({"impl": "reference", "unavailable": "reference arm covers the MoE workloads only"}))
+        return
+    M = args.M
+    cpu = synth.moe_weights(shape, device="cpu")
+    # size one step so that warmup + steps take about two minutes of CPU time
+    tps, _, _, _ = oracle_tokens_per_s(shape, M, cpu, seconds=2.0, max_calls=1, tokens_per_call=1)
+    per_tok = 1.0 / tps
+    budget = 120.0
+    tok = int(max(1, min(M, budget / max(1, args.steps + args.warmup) / per_tok)))
+    oracle_tokens_per_s(shape, M, cpu, seconds=0.0, max_calls=max(1, args.warmup), tokens_per_call=tok)
+    tps, calls, n, el = oracle_tokens_per_s(shape, M, cpu, seconds=1e9, max_calls=args.steps, tokens_per_call=tok)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / calls, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": shape.name, "M": M, "E": shape.E, "k": shape.k, "H": shape.H, "I": shape.I,
+                   "L": shape.L, "r": shape.r, "wdtype": shape.wdtype},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} token(s) of batch 0 per step, {calls} steps, {el:.1f} s"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    import moe_lora_b200 as ml
+
+    shape = synth.WORKLOADS[args.workload]
+    if not isinstance(shape, synth.MoEShape):
+        raise SystemExit("bench.py times the MoE layer workloads; dense SGMV is covered by the tests")
+    dev = torch.device("cuda", local)
+    M, k, L = args.M, shape.k, shape.L
+    cpu = synth.moe_weights(shape, device="cpu")
+    W = {kk: (v.to(dev) if isinstance(v, torch.Tensor) else v) for kk, v in cpu.items()}
+    batches = []
+    for b in range(args.batches):
+        x, ad = synth.moe_tokens(shape, M, batch=b)
+        batches.append((x.to(dev), ad.to(dev)))
+    rws = ml.new_workspace(ml.workspace_size(ml.OP_ROUTE, M, shape.H, 0, shape.E, k, L, 0), dev)
+    fws = ml.new_workspace(ml.workspace_size(ml.OP_FORWARD, M, shape.H, shape.I, shape.E, k, L, shape.r), dev)
+    rbufs = {"topk_ids": torch.empty((M, k), dtype=torch.int32, device=dev),
+             "topk_w": torch.empty((M, k), dtype=torch.float32, device=dev),
+             "sorted_pairs": torch.empty((M * k,), dtype=torch.int32, device=dev),
+             "seg_offsets": torch.empty((shape.E * (L + 1) + 1,), dtype=torch.int32, device=dev)}
+    y = torch.empty((M, shape.H), dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        xb, ab = batches[i % len(batches)]
+        rt = ml.route(ab, k, L, x=xb, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
+        ml.forward(xb, rt, W, k=k, L=L, y=y, workspace=fws)
+        return rt
+
+    # routing statistics of each batch (outside any timed region)
+    stats = []
+    for b in range(len(batches)):
+        rt = step(b)
+        torch.cuda.synchronize()
+        stats.append(routing_stats(rt, shape))
+    ml.check_status(fws)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps on device-resident inputs
+    launches_per_step = 8
+    ml.profile_enable(args.steps * launches_per_step + 64)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.25)
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = ml.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for i in range(args.steps):
+        step(i)
+    ev1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = ml.launch_count() - n0
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    gu_ms, gu_n = ml.profile_read("gemm_gateup")
+    per_kernel = {kname: ml.profile_read(kname) for kname in ("router_logits", "topk", "sort", "shrink",
+                                                            "gemm_gateup", "gemm_down", "combine")}
+    ml.profile_enable(0)
+    ms_max = max_over_ranks(ms, world)
+    value = world * M * args.steps / (ms_max / 1e3)
+
+    # ---- e2e: pinned host inputs -> device, route + forward, y -> pinned host, every step
+    e2e_steps = args.e2e_steps or args.steps
+    hx = [b[0].cpu().pin_memory() for b in batches]
+    ha = [b[1].cpu().pin_memory() for b in batches]
+    hy = torch.empty((M, shape.H), dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(batches[0][0])
+    da = torch.empty_like(batches[0][1])
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        j = i % len(batches)
+        dx.copy_(hx[j], non_blocking=True)
+        da.copy_(ha[j], non_blocking=True)
+        rt = ml.route(da, k, L, x=dx, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
+        ml.forward(dx, rt, W, k=k, L=L, y=y, workspace=fws)
+        hy.copy_(y, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * M * e2e_steps / (e2e_ms / 1e3)
+    ml.check_status(fws)
+    ml.check_status(rws)
+
+    # ---- roofline of the dominant kernel (gate_up GEMM) and of the whole layer
+    peaks, peak_src = load_peaks()
+    n_b = len(batches)
+    mean = lambda f: float(np.mean([f(*stats[i % n_b]) for i in range(args.steps)]))  # noqa: E731
+    gu_bytes = mean(lambda e, p: gateup_alg_bytes(shape, M, e, p))
+    lay_bytes = mean(lambda e, p: layer_alg_bytes(shape, M, e, p))
+    gu_avg_s = (gu_ms / max(gu_n, 1)) / 1e3
+    achieved = gu_bytes / gu_avg_s / 1e9
+    peak = float(peaks["hbm_gbs"])
+    traffic = NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["gemm_tc.cu"] == src_hash("gemm_tc.cu") else None
+    step_s = ms_max / 1e3 / args.steps
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if shape.wdtype == "bf16" else "e4m3/bf16",
+        "data": "synthetic",
+        "config": {"workload": shape.name, "M": M, "tokens_per_step_per_gpu": M, "E": shape.E, "k": k,
+                   "H": shape.H, "I": shape.I, "L": L, "r": shape.r, "wdtype": shape.wdtype,
+                   "adapters": shape.adapter_dist, "parallelism": f"replicas x{world}",
+                   "l2": f"no flush: {lay_bytes / 1e9:.2f} GB of weights per step > 126 MB L2; "
+                         f"{n_b} rotating token batches"},
+        "roofline": {"bound": "hbm", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": traffic, "alg_bytes_per_launch": gu_bytes,
+                     "avg_launch_us": gu_avg_s * 1e6},
+        "layer": {"alg_bytes_per_step": lay_bytes, "achieved_GBps": lay_bytes / step_s / 1e9,
+                  "frac_of_hbm_peak": lay_bytes / step_s / 1e9 / peak,
+                  "TFLOPs": layer_flops(shape, M) / step_s / 1e12,
+                  "kernel_ms_per_step": {kk: v[0] / args.steps for kk, v in per_kernel.items()}},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": M * shape.H * 2 + M * 4,
+                "d2h_bytes_per_step": M * shape.H * 2},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, calls, n, el = oracle_tokens_per_s(shape, M, cpu, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"fp64 oracle on batch 0 ({n} tokens), {calls} calls in {el:.1f} s; "
+                                          "touched expert weights decoded to fp64 once before timing"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

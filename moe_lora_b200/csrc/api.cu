@@ -1,0 +1,662 @@
+// C ABI of libmoe_lora.so: argument validation, workspace layout and the launch
+// sequence of each call.  No allocation, no synchronisation, no host read-back
+// (moe_lora_check_status excepted).
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "prof.h"
+
+#include <atomic>
+#include <vector>
+
+using namespace mlb;
+
+namespace mlb {
+
+namespace {
+struct ProfState {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;
+  size_t next = 0;
+  std::vector<std::pair<int, int>> pairs[K_COUNT];
+  int open[K_COUNT];
+};
+ProfState g_prof;
+std::atomic<long long> g_launches{0};
+}  // namespace
+
+void prof_begin(int id, cudaStream_t st) {
+  if (!g_prof.on || id < 0 || id >= K_COUNT) return;
+  if (g_prof.next >= g_prof.ev.size()) return;
+  g_prof.open[id] = static_cast<int>(g_prof.next);
+  cudaEventRecord(g_prof.ev[g_prof.next++], st);
+}
+
+void prof_end(int id, cudaStream_t st) {
+  if (!g_prof.on || id < 0 || id >= K_COUNT || g_prof.open[id] < 0) return;
+  if (g_prof.next >= g_prof.ev.size()) {
+    g_prof.open[id] = -1;
+    return;
+  }
+  cudaEventRecord(g_prof.ev[g_prof.next], st);
+  g_prof.pairs[id].push_back({g_prof.open[id], static_cast<int>(g_prof.next)});
+  ++g_prof.next;
+  g_prof.open[id] = -1;
+}
+
+void count_launch(int n) { g_launches += n; }
+
+}  // namespace mlb
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+moe_lora_status fail(moe_lora_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+moe_lora_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_LORA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
+
+int num_sms() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  });
+  return n;
+}
+
+moe_lora_status check_device() {
+  static int ok = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      ok = 0;
+      return;
+    }
+    ok = (major == 10 && minor == 0) ? 1 : 2;
+  });
+  if (ok == 0) return fail(MOE_LORA_ERR_CUDA, "no CUDA device available");
+  if (ok == 2) return fail(MOE_LORA_ERR_UNSUPPORTED, "libmoe_lora is built for sm_100a (B200) only");
+  return MOE_LORA_OK;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* v = std::getenv(name);
+  return v ? std::atoi(v) : dflt;
+}
+
+// N tile for the grouped GEMM from the mean number of rows per group.
+int choose_bn(long long rows, int groups) {
+  const int forced = env_int("MOE_LORA_FORCE_BN", 0);
+  if (forced == 16 || forced == 32 || forced == 64 || forced == 128 || forced == 256) return forced;
+  const double avg = groups > 0 ? static_cast<double>(rows) / groups : rows;
+  if (avg <= 12) return 16;
+  if (avg <= 24) return 32;
+  if (avg <= 48) return 64;
+  if (avg <= 96) return 128;
+  return 256;
+}
+
+int shrink_rows_per_cta(long long rows) {
+  long long rb = rows / (2LL * num_sms());
+  if (rb < 1) rb = 1;
+  if (rb > 8) rb = 8;
+  return static_cast<int>(rb);
+}
+
+struct ForwardWs {
+  int* status;
+  __nv_bfloat16* x_sorted;
+  __nv_bfloat16* act;
+  float* z_gu;
+  float* z_d;
+  int32_t* row_adapter;
+  float* o;
+  size_t bytes;
+};
+
+ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r) {
+  const size_t mk = static_cast<size_t>(M) * k;
+  size_t off = kStatusBytes;
+  ForwardWs w{};
+  uint8_t* b = static_cast<uint8_t*>(base);
+  auto take = [&](size_t bytes) {
+    uint8_t* p = b ? b + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  w.status = reinterpret_cast<int*>(b);
+  w.x_sorted = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
+  w.act = reinterpret_cast<__nv_bfloat16*>(take(mk * I * 2));
+  w.z_gu = reinterpret_cast<float*>(take(mk * r * 4));
+  w.z_d = reinterpret_cast<float*>(take(mk * r * 4));
+  w.row_adapter = reinterpret_cast<int32_t*>(take(mk * 4));
+  w.o = reinterpret_cast<float*>(take(mk * H * 4));
+  w.bytes = off;
+  return w;
+}
+
+struct RouteWs {
+  int* status;
+  int32_t* key_count;
+  int32_t* a_key;
+  float* logits;
+  size_t bytes;
+};
+
+RouteWs route_layout(void* base, int M, int E, int L) {
+  size_t off = kStatusBytes;
+  RouteWs w{};
+  uint8_t* b = static_cast<uint8_t*>(base);
+  auto take = [&](size_t bytes) {
+    uint8_t* p = b ? b + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  w.status = reinterpret_cast<int*>(b);
+  w.key_count = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * (L + 1) * 4));
+  w.a_key = reinterpret_cast<int32_t*>(take(static_cast<size_t>(M) * 4));
+  w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(M) * E * 4));
+  w.bytes = off;
+  return w;
+}
+
+struct DenseWs {
+  int* status;
+  float* z;
+  int32_t* row_adapter;
+  size_t bytes;
+};
+
+DenseWs dense_layout(void* base, int T, int r) {
+  size_t off = kStatusBytes;
+  DenseWs w{};
+  uint8_t* b = static_cast<uint8_t*>(base);
+  auto take = [&](size_t bytes) {
+    uint8_t* p = b ? b + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  w.status = reinterpret_cast<int*>(b);
+  w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
+  w.row_adapter = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
+  w.bytes = off;
+  return w;
+}
+
+moe_lora_status check_ws(void* ws, size_t have, size_t need) {
+  if (ws == nullptr) return fail(MOE_LORA_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned16(ws)) return fail(MOE_LORA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  if (have < need)
+    return fail(MOE_LORA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", have, need);
+  return MOE_LORA_OK;
+}
+
+#define ML_REQUIRE(cond, code, ...)              \
+  do {                                           \
+    if (!(cond)) return fail(code, __VA_ARGS__); \
+  } while (0)
+
+#define ML_PTR(p) ML_REQUIRE((p) != nullptr && aligned16(p), MOE_LORA_ERR_INVALID_ARG, \
+                             "%s must be a non-NULL 16-byte aligned device pointer", #p)
+
+#define ML_CUDA(expr, where)                     \
+  do {                                           \
+    cudaError_t _e = (expr);                     \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_lora_last_error(void) { return g_err; }
+
+long long moe_lora_launch_count(void) { return g_launches.load(); }
+
+moe_lora_status moe_lora_profile_enable(int max_launches) {
+  ML_REQUIRE(max_launches >= 0 && max_launches <= (1 << 20), MOE_LORA_ERR_INVALID_ARG,
+             "max_launches must be in [0, 2^20]");
+  for (cudaEvent_t e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.clear();
+  g_prof.next = 0;
+  for (int i = 0; i < K_COUNT; ++i) {
+    g_prof.pairs[i].clear();
+    g_prof.open[i] = -1;
+  }
+  g_prof.on = false;
+  if (max_launches == 0) return MOE_LORA_OK;
+  g_prof.ev.resize(2 * static_cast<size_t>(max_launches));
+  for (auto& e : g_prof.ev) ML_CUDA(cudaEventCreate(&e), "cudaEventCreate");
+  g_prof.on = true;
+  return MOE_LORA_OK;
+}
+
+moe_lora_status moe_lora_profile_read(int kernel_id, double* total_ms, int* launches) {
+  ML_REQUIRE(kernel_id >= 0 && kernel_id < K_COUNT && total_ms && launches, MOE_LORA_ERR_INVALID_ARG,
+             "bad kernel id or output pointer");
+  *total_ms = 0.0;
+  *launches = 0;
+  const auto& v = g_prof.pairs[kernel_id];
+  if (v.empty()) return MOE_LORA_OK;
+  ML_CUDA(cudaEventSynchronize(g_prof.ev[v.back().second]), "cudaEventSynchronize");
+  double tot = 0.0;
+  for (const auto& pr : v) {
+    float ms = 0.f;
+    ML_CUDA(cudaEventElapsedTime(&ms, g_prof.ev[pr.first], g_prof.ev[pr.second]), "cudaEventElapsedTime");
+    tot += ms;
+  }
+  *total_ms = tot;
+  *launches = static_cast<int>(v.size());
+  return MOE_LORA_OK;
+}
+
+const char* moe_lora_version(void) { return "moe_lora_b200 0.1 sm_100a"; }
+
+size_t moe_lora_workspace_size(int op, int M, int H, int I, int E, int k, int L, int r) {
+  if (M < 0 || H < 0 || I < 0 || E < 0 || k < 0 || L < 0 || r < 0) return 0;
+  switch (op) {
+    case MOE_LORA_OP_ROUTE: return route_layout(nullptr, M, E, L).bytes;
+    case MOE_LORA_OP_FORWARD: return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0).bytes;
+    case MOE_LORA_OP_SGMV_SHRINK:
+    case MOE_LORA_OP_SGMV_EXPAND: return kStatusBytes;
+    case MOE_LORA_OP_DENSE: return dense_layout(nullptr, M, L > 0 ? r : 0).bytes;
+    default: return 0;
+  }
+}
+
+moe_lora_status moe_lora_check_status(void* workspace, moe_lora_stream stream) {
+  if (workspace == nullptr) return fail(MOE_LORA_ERR_INVALID_ARG, "workspace is NULL");
+  int h[2] = {0, 0};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  ML_CUDA(cudaStreamSynchronize(st), "cudaStreamSynchronize");
+  ML_CUDA(cudaMemcpy(h, workspace, sizeof(h), cudaMemcpyDeviceToHost), "status read");
+  ML_CUDA(cudaMemset(workspace, 0, sizeof(h)), "status clear");
+  if (h[0] == MOE_LORA_OK) return MOE_LORA_OK;
+  return fail(static_cast<moe_lora_status>(h[0]), "device-side check failed (code %d, detail %d)", h[0], h[1]);
+}
+
+moe_lora_status moe_lora_route(const void* x, const void* w_router, const float* bias,
+                               const float* logits_in, const int32_t* adapter_ids, int M, int H, int E,
+                               int k, int L, float* logits_out, int32_t* topk_ids, float* topk_w,
+                               int32_t* sorted_pairs, int32_t* seg_offsets, void* workspace,
+                               size_t workspace_bytes, moe_lora_stream stream) {
+  ML_REQUIRE(M >= 0 && E >= 1 && k >= 1 && L >= 0, MOE_LORA_ERR_INVALID_ARG,
+             "need M >= 0, E >= 1, k >= 1, L >= 0 (got M=%d E=%d k=%d L=%d)", M, E, k, L);
+  ML_REQUIRE(k <= E && E <= 256 && L <= 64, MOE_LORA_ERR_UNSUPPORTED,
+             "supported: k <= E <= 256, L <= 64 (got k=%d E=%d L=%d)", k, E, L);
+  ML_REQUIRE(static_cast<long long>(M) * k <= (1 << 20), MOE_LORA_ERR_UNSUPPORTED, "M*k > 2^20");
+  ML_PTR(seg_offsets);
+  const RouteWs need = route_layout(nullptr, M, E, L);
+  moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
+  if (st != MOE_LORA_OK) return st;
+  if (M > 0) {
+    ML_PTR(adapter_ids);
+    ML_PTR(topk_ids);
+    ML_PTR(topk_w);
+    ML_PTR(sorted_pairs);
+    if (logits_in == nullptr) {
+      ML_PTR(x);
+      ML_PTR(w_router);
+      ML_REQUIRE(H > 0 && H % 8 == 0, MOE_LORA_ERR_UNSUPPORTED, "H must be a positive multiple of 8");
+      if (bias) ML_PTR(bias);
+    } else {
+      ML_PTR(logits_in);
+    }
+    if (logits_out) ML_PTR(logits_out);
+  }
+  st = check_device();
+  if (st != MOE_LORA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const RouteWs w = route_layout(workspace, M, E, L);
+  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+  RouteArgs a{};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.w_router = static_cast<const __nv_bfloat16*>(w_router);
+  a.bias = bias;
+  a.logits_in = logits_in;
+  a.adapter_ids = adapter_ids;
+  a.M = M;
+  a.H = H;
+  a.E = E;
+  a.k = k;
+  a.L = L;
+  a.logits = logits_out ? logits_out : w.logits;
+  a.logits_out = logits_out;
+  a.topk_ids = topk_ids;
+  a.topk_w = topk_w;
+  a.sorted_pairs = sorted_pairs;
+  a.seg_offsets = seg_offsets;
+  a.key_count = w.key_count;
+  a.a_key = w.a_key;
+  a.status = w.status;
+  ML_CUDA(launch_route(a, cs), "moe_lora_route launch");
+  return MOE_LORA_OK;
+}
+
+moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int k, int L, int r,
+                                 const float* topk_w, const int32_t* sorted_pairs,
+                                 const int32_t* seg_offsets, const void* w_gateup, const void* w_down,
+                                 ml_dtype w_dtype, const float* w_scales, const void* lora_a_gu,
+                                 const void* lora_b_gu, const void* lora_a_d, const void* lora_b_d,
+                                 void* y, void* workspace, size_t workspace_bytes,
+                                 moe_lora_stream stream) {
+  ML_REQUIRE(M >= 0 && H > 0 && I > 0 && E >= 1 && k >= 1 && L >= 0, MOE_LORA_ERR_INVALID_ARG,
+             "need M >= 0, H > 0, I > 0, E >= 1, k >= 1, L >= 0");
+  ML_REQUIRE(w_dtype == ML_BF16 || w_dtype == ML_E4M3, MOE_LORA_ERR_INVALID_ARG,
+             "w_dtype must be ML_BF16 or ML_E4M3");
+  ML_REQUIRE(k <= E && E <= 256 && L <= 64, MOE_LORA_ERR_UNSUPPORTED, "supported: k <= E <= 256, L <= 64");
+  ML_REQUIRE(H % 8 == 0 && I % 8 == 0, MOE_LORA_ERR_UNSUPPORTED, "H and I must be multiples of 8");
+  ML_REQUIRE(static_cast<long long>(M) * k <= (1 << 20), MOE_LORA_ERR_UNSUPPORTED, "M*k > 2^20");
+  if (L > 0) ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
+  const int rr = L > 0 ? r : 0;
+  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr);
+  moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
+  if (st != MOE_LORA_OK) return st;
+  if (w_dtype == ML_E4M3) return fail(MOE_LORA_ERR_UNSUPPORTED, "ML_E4M3 expert weights: not built yet");
+  if (M == 0) return MOE_LORA_OK;
+  ML_PTR(x);
+  ML_PTR(topk_w);
+  ML_PTR(sorted_pairs);
+  ML_PTR(seg_offsets);
+  ML_PTR(w_gateup);
+  ML_PTR(w_down);
+  ML_PTR(y);
+  if (L > 0) {
+    ML_PTR(lora_a_gu);
+    ML_PTR(lora_b_gu);
+    ML_PTR(lora_a_d);
+    ML_PTR(lora_b_d);
+  }
+  st = check_device();
+  if (st != MOE_LORA_OK) return st;
+  if (!tensor_map_encode_available())
+    return fail(MOE_LORA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr);
+  const int mk = M * k;
+  const int nkeys = E * (L + 1);
+  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+
+  // 1. gather x rows into (expert, adapter) order + gate_up shrink z = x A_gu
+  ShrinkArgs s1{};
+  s1.src = x;
+  s1.src_f32 = false;
+  s1.gather = sorted_pairs;
+  s1.gather_div = k;
+  s1.gather_dst = w.x_sorted;
+  s1.nrows = mk;
+  s1.K = H;
+  s1.r = rr;
+  s1.seg_offsets = seg_offsets;
+  s1.nseg = nkeys;
+  s1.seg_adapter = nullptr;
+  s1.L = L;
+  s1.E = E;
+  s1.lora_a = lora_a_gu;
+  s1.z = w.z_gu;
+  s1.row_adapter = w.row_adapter;
+  s1.rows_per_cta = shrink_rows_per_cta(mk);
+  s1.status = w.status;
+  ML_CUDA(launch_shrink(s1, cs), "gate_up shrink launch");
+
+  // 2. gate_up grouped GEMM, LoRA expand + SiLU-and-mul in the epilogue -> act
+  GemmArgs g{};
+  g.epi = EPI_GATEUP;
+  g.w_fp8 = false;
+  g.K = H;
+  g.E = E;
+  g.group_offsets = seg_offsets;
+  g.group_stride = L + 1;
+  g.rows_per_group = 2 * I;
+  g.n_out = I;
+  g.I = I;
+  g.total_rows = mk;
+  g.z = rr ? w.z_gu : nullptr;
+  g.row_adapter = w.row_adapter;
+  g.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
+  g.r = rr;
+  g.L = L;
+  g.out_bf16 = w.act;
+  g.w_scales = w_scales;
+  g.scale_idx = 0;
+  g.status = w.status;
+  g.w = w_gateup;
+  g.b = w.x_sorted;
+  g.bn = choose_bn(mk, E);
+  g.num_sms = num_sms();
+  ML_CUDA(launch_gemm_tc(g, cs), "gate_up GEMM launch");
+
+  // 3. down shrink z_d = act A_d
+  if (rr) {
+    ShrinkArgs s2 = s1;
+    s2.src = w.act;
+    s2.gather = nullptr;
+    s2.gather_dst = nullptr;
+    s2.K = I;
+    s2.lora_a = lora_a_d;
+    s2.z = w.z_d;
+    s2.row_adapter = nullptr;
+    ML_CUDA(launch_shrink(s2, cs), "down shrink launch");
+  }
+
+  // 4. down grouped GEMM, LoRA expand, x routing weight -> o (one row per pair)
+  GemmArgs d = g;
+  d.epi = EPI_DOWN;
+  d.K = I;
+  d.rows_per_group = H;
+  d.n_out = H;
+  d.z = rr ? w.z_d : nullptr;
+  d.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
+  d.out_bf16 = nullptr;
+  d.out_f32 = w.o;
+  d.sorted_pairs = sorted_pairs;
+  d.topk_w = topk_w;
+  d.scale_idx = 1;
+  d.w = w_down;
+  d.b = w.act;
+  ML_CUDA(launch_gemm_tc(d, cs), "down GEMM launch");
+
+  // 5. fixed-order combine over the k slots
+  ML_CUDA(launch_combine(w.o, M, k, H, static_cast<__nv_bfloat16*>(y), cs), "combine launch");
+  return MOE_LORA_OK;
+}
+
+moe_lora_status sgmv_shrink(const void* x, const void* lora_a, const int32_t* seg_offsets,
+                            const int32_t* seg_adapter, int S, int T, int h_in, int r, int L, ml_dtype dt,
+                            float* z, void* workspace, size_t workspace_bytes, moe_lora_stream stream) {
+  ML_REQUIRE(S >= 0 && T >= 0 && L >= 0 && h_in > 0, MOE_LORA_ERR_INVALID_ARG, "need S, T, L >= 0, h_in > 0");
+  ML_REQUIRE(dt == ML_F32 || dt == ML_BF16, MOE_LORA_ERR_INVALID_ARG, "dt must be ML_F32 or ML_BF16");
+  ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
+  ML_REQUIRE(h_in % 8 == 0 && L <= 64, MOE_LORA_ERR_UNSUPPORTED, "h_in must be a multiple of 8, L <= 64");
+  ML_REQUIRE(S >= 1 || T == 0, MOE_LORA_ERR_INVALID_ARG, "segments must cover the T tokens");
+  moe_lora_status st = check_ws(workspace, workspace_bytes, kStatusBytes);
+  if (st != MOE_LORA_OK) return st;
+  if (T == 0) return MOE_LORA_OK;
+  ML_PTR(x);
+  ML_PTR(seg_offsets);
+  ML_PTR(seg_adapter);
+  ML_PTR(z);
+  if (L > 0) ML_PTR(lora_a);
+  st = check_device();
+  if (st != MOE_LORA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+  ShrinkArgs a{};
+  a.src = x;
+  a.src_f32 = dt == ML_F32;
+  a.gather = nullptr;
+  a.gather_div = 1;
+  a.gather_dst = nullptr;
+  a.nrows = T;
+  a.K = h_in;
+  a.r = r;
+  a.seg_offsets = seg_offsets;
+  a.nseg = S;
+  a.seg_adapter = seg_adapter;
+  a.L = L;
+  a.E = 1;
+  a.lora_a = lora_a;
+  a.z = z;
+  a.row_adapter = nullptr;
+  a.rows_per_cta = shrink_rows_per_cta(T);
+  a.status = static_cast<int*>(workspace);
+  ML_CUDA(launch_shrink(a, cs), "sgmv_shrink launch");
+  return MOE_LORA_OK;
+}
+
+moe_lora_status sgmv_expand(const float* z, const void* lora_b, const int32_t* seg_offsets,
+                            const int32_t* seg_adapter, int S, int T, int h_out, int r, int L, ml_dtype dt,
+                            void* y, void* workspace, size_t workspace_bytes, moe_lora_stream stream) {
+  ML_REQUIRE(S >= 0 && T >= 0 && L >= 0 && h_out > 0, MOE_LORA_ERR_INVALID_ARG, "need S, T, L >= 0, h_out > 0");
+  ML_REQUIRE(dt == ML_F32 || dt == ML_BF16, MOE_LORA_ERR_INVALID_ARG, "dt must be ML_F32 or ML_BF16");
+  ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
+  ML_REQUIRE(h_out % 8 == 0 && L <= 64, MOE_LORA_ERR_UNSUPPORTED, "h_out must be a multiple of 8, L <= 64");
+  ML_REQUIRE(S >= 1 || T == 0, MOE_LORA_ERR_INVALID_ARG, "segments must cover the T tokens");
+  moe_lora_status st = check_ws(workspace, workspace_bytes, kStatusBytes);
+  if (st != MOE_LORA_OK) return st;
+  if (T == 0) return MOE_LORA_OK;
+  ML_PTR(z);
+  ML_PTR(seg_offsets);
+  ML_PTR(seg_adapter);
+  ML_PTR(y);
+  if (L > 0) ML_PTR(lora_b);
+  st = check_device();
+  if (st != MOE_LORA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+  ExpandArgs a{};
+  a.z = z;
+  a.lora_b = lora_b;
+  a.f32 = dt == ML_F32;
+  a.seg_offsets = seg_offsets;
+  a.nseg = S;
+  a.seg_adapter = seg_adapter;
+  a.L = L;
+  a.T = T;
+  a.h_out = h_out;
+  a.r = r;
+  a.y = y;
+  a.status = static_cast<int*>(workspace);
+  ML_CUDA(launch_expand(a, cs), "sgmv_expand launch");
+  return MOE_LORA_OK;
+}
+
+moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lora_a, const void* lora_b,
+                                   const int32_t* seg_offsets, const int32_t* seg_adapter, int S, int T,
+                                   int h_in, int h_out, int r, int L, ml_dtype dt, void* y, void* workspace,
+                                   size_t workspace_bytes, moe_lora_stream stream) {
+  ML_REQUIRE(S >= 0 && T >= 0 && L >= 0 && h_in > 0 && h_out > 0, MOE_LORA_ERR_INVALID_ARG,
+             "need S, T, L >= 0 and h_in, h_out > 0");
+  ML_REQUIRE(dt == ML_F32 || dt == ML_BF16, MOE_LORA_ERR_INVALID_ARG, "dt must be ML_F32 or ML_BF16");
+  ML_REQUIRE(h_in % 8 == 0 && h_out % 8 == 0 && L <= 64, MOE_LORA_ERR_UNSUPPORTED,
+             "h_in, h_out must be multiples of 8, L <= 64");
+  if (L > 0) ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
+  ML_REQUIRE(S >= 1 || T == 0, MOE_LORA_ERR_INVALID_ARG, "segments must cover the T tokens");
+  const int rr = L > 0 ? r : 0;
+  const DenseWs need = dense_layout(nullptr, T, rr);
+  moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
+  if (st != MOE_LORA_OK) return st;
+  if (T == 0) return MOE_LORA_OK;
+  ML_PTR(x);
+  ML_PTR(w);
+  ML_PTR(seg_offsets);
+  ML_PTR(seg_adapter);
+  ML_PTR(y);
+  if (L > 0) {
+    ML_PTR(lora_a);
+    ML_PTR(lora_b);
+  }
+  st = check_device();
+  if (st != MOE_LORA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const DenseWs ws = dense_layout(workspace, T, rr);
+  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+
+  ShrinkArgs a{};
+  a.src = x;
+  a.src_f32 = dt == ML_F32;
+  a.gather_div = 1;
+  a.nrows = T;
+  a.K = h_in;
+  a.r = rr;
+  a.seg_offsets = seg_offsets;
+  a.nseg = S;
+  a.seg_adapter = seg_adapter;
+  a.L = L;
+  a.E = 1;
+  a.lora_a = lora_a;
+  a.z = ws.z;
+  a.row_adapter = ws.row_adapter;
+  a.rows_per_cta = shrink_rows_per_cta(T);
+  a.status = ws.status;
+  ML_CUDA(launch_shrink(a, cs), "dense shrink launch");
+
+  if (dt == ML_F32) {
+    DenseF32Args d{};
+    d.x = static_cast<const float*>(x);
+    d.w = static_cast<const float*>(w);
+    d.lora_b = static_cast<const float*>(lora_b);
+    d.z = rr ? ws.z : nullptr;
+    d.row_adapter = ws.row_adapter;
+    d.T = T;
+    d.h_in = h_in;
+    d.h_out = h_out;
+    d.r = rr;
+    d.L = L;
+    d.y = static_cast<float*>(y);
+    ML_CUDA(launch_dense_f32(d, cs), "dense fp32 GEMM launch");
+    return MOE_LORA_OK;
+  }
+  if (!tensor_map_encode_available())
+    return fail(MOE_LORA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  GemmArgs g{};
+  g.epi = EPI_DENSE;
+  g.K = h_in;
+  g.E = 1;
+  g.group_offsets = seg_offsets;  // [0] = 0 and [S] = T bound the single group
+  g.group_stride = S;
+  g.rows_per_group = h_out;
+  g.n_out = h_out;
+  g.I = 0;
+  g.total_rows = T;
+  g.z = rr ? ws.z : nullptr;
+  g.row_adapter = ws.row_adapter;
+  g.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
+  g.r = rr;
+  g.L = L;
+  g.out_bf16 = static_cast<__nv_bfloat16*>(y);
+  g.status = ws.status;
+  g.w = w;
+  g.b = static_cast<const __nv_bfloat16*>(x);
+  g.bn = choose_bn(T, 1);
+  g.num_sms = num_sms();
+  ML_CUDA(launch_gemm_tc(g, cs), "dense GEMM launch");
+  return MOE_LORA_OK;
+}
+
+}  // extern "C"

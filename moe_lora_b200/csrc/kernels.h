@@ -1,0 +1,124 @@
+// Host-side launch interfaces between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mlb {
+
+struct RouteArgs {
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* w_router;
+  const float* bias;
+  const float* logits_in;
+  const int32_t* adapter_ids;
+  int M, H, E, k, L;
+  float* logits;          // where computed logits go (logits_out or workspace)
+  float* logits_out;      // may be null
+  int32_t* topk_ids;
+  float* topk_w;
+  int32_t* sorted_pairs;
+  int32_t* seg_offsets;
+  int32_t* key_count;     // workspace [E*(L+1)]
+  int32_t* a_key;         // workspace [M]
+  int* status;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+
+// Segmented shrink z[s] = src_row(s) . A_seg(s)^T (SIMT: 128-bit loads, warp-shuffle
+// split-K reduction).  Segments come either from a dense (offsets, adapter) table or
+// from MoE keys q = e*(L+1) + a' (seg_adapter == null).
+struct ShrinkArgs {
+  const void* src;            // rows [*, K], f32 or bf16
+  bool src_f32;
+  const int32_t* gather;      // if set: source row of output row s = gather[s] / gather_div
+  int gather_div;
+  __nv_bfloat16* gather_dst;  // if set: copy of the gathered source row (bf16 rows [nrows, K])
+  int nrows, K, r;
+  const int32_t* seg_offsets; // [nseg+1]
+  int nseg;
+  const int32_t* seg_adapter; // dense: [nseg]; null: MoE key decode
+  int L, E;
+  const void* lora_a;         // dense [L][r][K]; MoE [L][E][r][K] (same dtype as src)
+  float* z;                   // [nrows][r]
+  int32_t* row_adapter;       // out: adapter per row (-1 none), may be null
+  int rows_per_cta;
+  int* status;
+};
+cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st);
+
+// y[t] += z[t] . B_a(t) for dense segments (f32 or bf16 y and B).
+struct ExpandArgs {
+  const float* z;
+  const void* lora_b;         // [L][r][h_out]
+  bool f32;
+  const int32_t* seg_offsets;
+  int nseg;
+  const int32_t* seg_adapter;
+  int L, T, h_out, r;
+  void* y;
+  int* status;
+};
+cudaError_t launch_expand(const ExpandArgs& a, cudaStream_t st);
+
+// fp32 SIMT base GEMM with the LoRA expand fused in its epilogue:
+// y[t][f] = sum_k x[t][k] W[f][k] + sum_i z[t][i] B[a(t)][i][f].
+struct DenseF32Args {
+  const float* x;
+  const float* w;
+  const float* lora_b;        // [L][r][h_out]
+  const float* z;             // [T][r]
+  const int32_t* row_adapter; // [T]
+  int T, h_in, h_out, r, L;
+  float* y;
+};
+cudaError_t launch_dense_f32(const DenseF32Args& a, cudaStream_t st);
+
+// Tensor-core grouped GEMM with operand swap: the weight rows fill the 128-row MMA
+// M slot, the tokens of one expert (or of the dense batch) the N slot.
+enum EpiKind : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DENSE = 2 };
+
+struct GemmArgs {
+  int epi;
+  bool w_fp8;
+  int K;                       // reduction length
+  int E;                       // groups (experts); 1 for dense
+  const int32_t* group_offsets;  // row offsets of group g at group_offsets[g * group_stride]
+  int group_stride;
+  int rows_per_group;          // weight rows per expert (2I for gate_up, H for down, h_out)
+  int n_out;                   // output features per group (I for gate_up, H, h_out)
+  int I;                       // gate_up: gate/up split
+  int total_rows;              // rows of the B operand tensor
+  // LoRA expand in the epilogue
+  const float* z;              // [total_rows][r]
+  const int32_t* row_adapter;  // [total_rows]
+  const __nv_bfloat16* lora_b; // MoE [L][E][r][rows_per_group]; dense [L][r][h_out]
+  int r, L;
+  // epilogue outputs
+  __nv_bfloat16* out_bf16;     // gate_up: act [rows][I]; dense: y [T][h_out]
+  float* out_f32;              // down: o [pairs][H] (weighted)
+  const int32_t* sorted_pairs; // down: pair index of each sorted row
+  const float* topk_w;         // down: routing weight per pair
+  const float* w_scales;       // fp8: [E][2]
+  int scale_idx;               // 0 gate_up, 1 down
+  int* status;
+  // operands
+  const void* w;               // weights [E*rows_per_group][K]
+  const __nv_bfloat16* b;      // B operand rows [total_rows][K]
+  int bn;                      // N tile (16..256)
+  int num_sms;
+};
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
+
+// y[t] = sum_j o[t*k + j]  (o already weighted), fixed j order, bf16 out.
+cudaError_t launch_combine(const float* o, int M, int k, int H, __nv_bfloat16* y, cudaStream_t st);
+
+// driver entry point for tensor map encoding (resolved once)
+bool tensor_map_encode_available();
+CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                        uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
+                        uint32_t box_rows, CUtensorMapSwizzle swz);
+
+}  // namespace mlb

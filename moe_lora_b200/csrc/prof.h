@@ -1,0 +1,35 @@
+// Optional per-kernel timing (CUDA events recorded around each launch on its own
+// stream) and a launch counter.  Off by default; enabled through the C ABI
+// (moe_lora_profile_enable) by measurement code.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace mlb {
+
+enum KernelId : int {
+  K_ROUTE_LOGITS = 0,
+  K_TOPK = 1,
+  K_SORT = 2,
+  K_SHRINK = 3,
+  K_GEMM_GATEUP = 4,
+  K_GEMM_DOWN = 5,
+  K_COMBINE = 6,
+  K_EXPAND = 7,
+  K_DENSE_F32 = 8,
+  K_GEMM_DENSE = 9,
+  K_COUNT = 10
+};
+
+void prof_begin(int id, cudaStream_t st);
+void prof_end(int id, cudaStream_t st);
+void count_launch(int n = 1);
+
+struct ProfScope {
+  int id;
+  cudaStream_t st;
+  ProfScope(int i, cudaStream_t s) : id(i), st(s) { prof_begin(id, st); }
+  ~ProfScope() { prof_end(id, st); }
+};
+
+}  // namespace mlb

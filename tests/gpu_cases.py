@@ -1,0 +1,77 @@
+"""Builders shared by the GPU parity tests, the smoke entry point and the bench.
+
+Inputs come from the seeded generator only; expected values come from the oracle
+only.  Nothing computed by the CUDA path is ever fed to the oracle.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import formats
+from oracle import moe_lora_ref as ref
+from tests.oracle_inputs import MoEOracleWeights
+from workloads import synth
+
+TOL_BF16 = 2e-2   # max|err| <= TOL * max|ref| for bf16 expert weights
+TOL_FP8 = 6e-2    # ... for e4m3 expert weights
+
+
+class CpuWeightsOracle(MoEOracleWeights):
+    """Oracle view backed by the generator's CPU tensors (no regeneration)."""
+
+    def __init__(self, shape: synth.MoEShape, cpu: dict):
+        super().__init__(shape, cache=True)
+        self.cpu = cpu
+
+    def _expert(self, e):
+        wdt = self.s.wdtype
+        sc = self.cpu["scales"][e]
+        return (formats.to_f64(synth.bits(self.cpu["w_gu"][e]), wdt),
+                formats.to_f64(synth.bits(self.cpu["w_d"][e]), wdt), float(sc[0]), float(sc[1]))
+
+    def _adapter(self, a, e):
+        return tuple(formats.to_f64(synth.bits(self.cpu[n][a, e]), "bf16") for n in ("a_gu", "b_gu", "a_d", "b_d"))
+
+
+def moe_weights_both(shape: synth.MoEShape, device="cuda"):
+    cpu = synth.moe_weights(shape, device="cpu")
+    dev = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in cpu.items()}
+    return cpu, dev, CpuWeightsOracle(shape, cpu)
+
+
+def oracle_routing_from_logits(logits_cpu: torch.Tensor, adapter_ids: np.ndarray, E: int, k: int, L: int):
+    lg = logits_cpu.numpy().astype(np.float64)
+    ids, w = ref.route_topk(lg, k)
+    sp, so = ref.sort_pairs(ids, adapter_ids, E, L)
+    return ids, w, sp, so
+
+
+def rel_err(y_gpu: torch.Tensor, y_ref: np.ndarray) -> float:
+    yg = y_gpu.detach().float().cpu().numpy().astype(np.float64)
+    denom = float(np.max(np.abs(y_ref))) if y_ref.size else 1.0
+    return float(np.max(np.abs(yg - y_ref))) / max(denom, 1e-30) if y_ref.size else 0.0
+
+
+def run_moe_case(shape: synth.MoEShape, M: int, weights=None, tokens=None):
+    """Route (from the given fp32 logits, so ids are comparable bit for bit) and
+    forward on the GPU; the oracle on the same seeded inputs.
+
+    Returns the GPU outputs, the oracle outputs and the relative error of y over
+    `tokens` (all tokens when None)."""
+    import moe_lora_b200 as ml
+    cpu, dev, OW = weights if weights is not None else moe_weights_both(shape)
+    x, ad = synth.moe_tokens(shape, M)
+    xd, add = x.cuda(), ad.cuda()
+    ad_np = ad.numpy().astype(np.int64)
+    lin = synth.moe_logits_in(shape, M)
+    rt = ml.route(add, shape.k, shape.L, logits_in=lin.cuda())
+    ids, w, sp, so = oracle_routing_from_logits(lin, ad_np, shape.E, shape.k, shape.L)
+    y = ml.forward(xd, rt, dev, k=shape.k, L=shape.L)
+    torch.cuda.synchronize()
+    x64 = formats.to_f64(synth.bits(x), "bf16")
+    sel = np.arange(M) if tokens is None else np.asarray(tokens)
+    y_ref = ref.moe_lora_forward(x64, ids, w, ad_np, shape.I, OW.expert, OW.adapter, tokens=sel)
+    return dict(rt=rt, y=y, ids=ids, w=w, sp=sp, so=so, y_ref=y_ref, tokens=sel,
+                err=rel_err(y[torch.as_tensor(sel, dtype=torch.long, device=y.device)], y_ref),
+                x=x, ad=ad, dev=dev)

@@ -1,0 +1,94 @@
+"""GPU parity of moe_lora_forward (tcgen05 grouped GEMMs + SGMV LoRA) against the oracle."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import moe_lora_b200 as ml
+from tests.gpu_cases import TOL_BF16, TOL_FP8, moe_weights_both, run_moe_case
+from workloads import synth
+
+pytestmark = pytest.mark.gpu
+
+# Small shapes that still span several K blocks (64), several weight tiles (64 gate
+# rows / 128 down rows), several token chunks, and ragged tails in every dimension.
+SMALL = [
+    synth.MoEShape("s_a", 200, E=8, k=2, H=384, I=192, L=3, r=16, no_adapter_frac=0.2),
+    synth.MoEShape("s_ragged", 201, E=6, k=3, H=520, I=136, L=2, r=8, no_adapter_frac=0.25),
+    synth.MoEShape("s_r64", 202, E=4, k=2, H=256, I=128, L=4, r=64, adapter_dist="zipf"),
+    synth.MoEShape("s_r128", 203, E=5, k=2, H=264, I=200, L=2, r=128),
+    synth.MoEShape("s_noadapter", 204, E=8, k=4, H=256, I=256, L=2, r=32, no_adapter_frac=1.0),
+    synth.MoEShape("s_L0", 205, E=8, k=2, H=192, I=128, L=0, r=16),
+    synth.MoEShape("s_kE", 206, E=4, k=4, H=128, I=64, L=1, r=16),
+    synth.MoEShape("s_E1", 207, E=1, k=1, H=256, I=384, L=3, r=16),
+    synth.MoEShape("s_bias_zipf", 208, E=16, k=8, H=512, I=320, L=8, r=32, bias=True, adapter_dist="zipf"),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: s.name)
+@pytest.mark.parametrize("M", [1, 3, 37, 300])
+def test_forward_small_shapes(shape, M):
+    res = run_moe_case(shape, M)
+    assert res["err"] <= TOL_BF16, res["err"]
+
+
+@pytest.mark.parametrize("bn", [16, 32, 64, 128, 256])
+def test_forward_every_n_tile(bn, monkeypatch):
+    monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
+    res = run_moe_case(SMALL[0], 300)
+    assert res["err"] <= TOL_BF16, res["err"]
+    res = run_moe_case(SMALL[1], 37)
+    assert res["err"] <= TOL_BF16, res["err"]
+
+
+@pytest.fixture(scope="module")
+def decode_weights():
+    return moe_weights_both(synth.MOE_DECODE_BF16)
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 64])
+def test_forward_moe_decode_bf16_full(decode_weights, M):
+    res = run_moe_case(synth.MOE_DECODE_BF16, M, weights=decode_weights)
+    assert res["err"] <= TOL_BF16, res["err"]
+    ml.check_status(res["rt"]["workspace"])
+
+
+def test_forward_deterministic(decode_weights):
+    s = synth.MOE_DECODE_BF16
+    a = run_moe_case(s, 64, weights=decode_weights)
+    y2 = ml.forward(a["x"].cuda(), a["rt"], a["dev"], k=s.k, L=s.L)
+    torch.cuda.synchronize()
+    assert torch.equal(a["y"], y2)
+
+
+def test_all_adapters_none_equals_zero_b(decode_weights):
+    """Early exit of adapter -1 and a zero expand B give the same bits."""
+    s = synth.MOE_DECODE_BF16
+    cpu, dev, _ = decode_weights
+    x, ad = synth.moe_tokens(s, 32)
+    lin = synth.moe_logits_in(s, 32).cuda()
+    none = torch.full_like(ad, -1).cuda()
+    rt0 = ml.route(none, s.k, s.L, logits_in=lin)
+    y0 = ml.forward(x.cuda(), rt0, dev, k=s.k, L=s.L)
+    devz = dict(dev)
+    devz["b_gu"] = torch.zeros_like(dev["b_gu"])
+    devz["b_d"] = torch.zeros_like(dev["b_d"])
+    rt1 = ml.route(ad.cuda(), s.k, s.L, logits_in=lin)
+    y1 = ml.forward(x.cuda(), rt1, devz, k=s.k, L=s.L)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+
+
+@pytest.fixture(scope="module")
+def prefill_weights():
+    return moe_weights_both(synth.MOE_PREFILL_BF16)
+
+
+def test_forward_moe_prefill_bf16_full_sampled(prefill_weights):
+    M = 4096
+    toks = np.unique(np.concatenate([np.arange(8), np.arange(M - 8, M),
+                                     np.random.default_rng(1).choice(M, 48, replace=False)]))
+    res = run_moe_case(synth.MOE_PREFILL_BF16, M, weights=prefill_weights, tokens=toks)
+    assert res["err"] <= TOL_BF16, res["err"]
+    ml.check_status(res["rt"]["workspace"])

@@ -130,6 +130,8 @@ def adapter_probs(L: int, dist: str) -> np.ndarray:
 
 def draw_adapter_ids(g: np.random.Generator, n: int, L: int, dist: str,
                      no_adapter_frac: float) -> np.ndarray:
+    if L == 0:
+        return np.full(n, -1, dtype=np.int32)
     ids = g.choice(L, size=n, p=adapter_probs(L, dist)).astype(np.int32)
     if no_adapter_frac > 0:
         ids[g.random(n) < no_adapter_frac] = -1
@@ -138,10 +140,13 @@ def draw_adapter_ids(g: np.random.Generator, n: int, L: int, dist: str,
 
 # ----------------------------------------------------------------------------- MoE slices
 
-def moe_tokens(s: MoEShape, M: int) -> tuple[torch.Tensor, torch.Tensor]:
-    """x bf16 [M, H] and per-token adapter id int32 [M] (-1 = base only)."""
-    x = to_bf16(normal_f32(rng(s.wid, T_X, M), (M, s.H), 1.0))
-    ids = draw_adapter_ids(rng(s.wid, T_ADAPTER, M), M, s.L, s.adapter_dist, s.no_adapter_frac)
+def moe_tokens(s: MoEShape, M: int, batch: int = 0) -> tuple[torch.Tensor, torch.Tensor]:
+    """x bf16 [M, H] and per-token adapter id int32 [M] (-1 = base only).
+
+    `batch` selects one of several independent batches of the same size."""
+    key = (M,) if batch == 0 else (M, batch)
+    x = to_bf16(normal_f32(rng(s.wid, T_X, *key), (M, s.H), 1.0))
+    ids = draw_adapter_ids(rng(s.wid, T_ADAPTER, *key), M, s.L, s.adapter_dist, s.no_adapter_frac)
     return x, torch.from_numpy(ids)
 
 
