@@ -195,6 +195,37 @@ MOE_LORA_API moe_lora_status dense_lora_forward(
     int h_in, int h_out, int r, int L, ml_dtype dt, void* y,
     void* workspace, size_t workspace_bytes, moe_lora_stream stream);
 
+/* ---------------------------------------------------------------------------------
+ * moe_lora_route_noalloc -- moe_lora_route for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this entry point; it exists for callers
+ * that receive only their input and output buffers from a host framework (a plugin
+ * or custom-op interface with no workspace) and may not call cudaMalloc themselves,
+ * because an allocation can synchronise the device, is not allowed during stream
+ * capture, or would break a memory budget planned in advance.
+ *
+ * Arguments, outputs and results are those of moe_lora_route, without the workspace.
+ * The scratch (status word, per-key counts, per-token keys, and the logits when
+ * logits_out is NULL) lives in one fixed array of about 1.07 MiB that the library
+ * defines; every GPU that loads the library holds it until the process exits.
+ *   - Limits: M <= 1024, k <= E <= 256, L <= 64; larger sizes return
+ *     MOE_LORA_ERR_UNSUPPORTED with nothing enqueued.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call uses the same array and leaves its contents behind; each call clears
+ *     what must start at zero.  Calls that overlap on the GPU (concurrent streams, or
+ *     several host threads on one device) race on the array and must be serialised by
+ *     the caller.
+ *   - Nothing is allocated or freed.  Device-side data checks (an adapter id outside
+ *     [-1, L)) are applied as in moe_lora_route, but their status word is not readable
+ *     through this entry point.
+ * ------------------------------------------------------------------------------- */
+MOE_LORA_API moe_lora_status moe_lora_route_noalloc(
+    const void* x, const void* w_router, const float* bias, const float* logits_in,
+    const int32_t* adapter_ids, int M, int H, int E, int k, int L,
+    float* logits_out, int32_t* topk_ids, float* topk_w,
+    int32_t* sorted_pairs, int32_t* seg_offsets, moe_lora_stream stream);
+
 /* Workspace bytes for one call of `op` (arguments not used by the op are ignored;
  * for the SGMV/dense ops pass T as M, h_in as H and h_out as I).  Returns 0 for an
  * unknown op. */

@@ -21,7 +21,8 @@ OP_ROUTE, OP_FORWARD, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_DENSE = range(5)
 
 EXPORTS = ("moe_lora_route", "moe_lora_forward", "sgmv_shrink", "sgmv_expand", "dense_lora_forward",
            "moe_lora_workspace_size", "moe_lora_check_status", "moe_lora_last_error", "moe_lora_version",
-           "moe_lora_profile_enable", "moe_lora_profile_read", "moe_lora_launch_count")
+           "moe_lora_profile_enable", "moe_lora_profile_read", "moe_lora_launch_count",
+           "moe_lora_route_noalloc")
 KERNEL_IDS = {"router_logits": 0, "topk": 1, "sort": 2, "shrink": 3, "gemm_gateup": 4, "gemm_down": 5,
               "combine": 6, "expand": 7, "dense_f32": 8, "gemm_dense": 9}
 

@@ -65,6 +65,15 @@ moe_lora_status fail(moe_lora_status st, const char* fmt, ...) {
   return st;
 }
 
+}  // namespace
+
+namespace mlb {
+// Lets other entry points of the library report through moe_lora_last_error().
+void set_error_message(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace mlb
+
+namespace {
+
 moe_lora_status cuda_fail(cudaError_t e, const char* where) {
   return fail(MOE_LORA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
