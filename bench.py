@@ -44,7 +44,8 @@ L2_BYTES = 126 * 1024 * 1024
 # ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM on the
 # default workload, with the hash of the kernel source it was taken on; reported as
 # null when the source has changed since.  Filled from profiles/.
-NCU_TRAFFIC = {"gemm_tc.cu": None, "bytes_per_launch": None}
+NCU_TRAFFIC = {"gemm_tc.cu": "2c17de826e7599dc", "bytes_per_launch": 746.700032e6 + 5.458432e6,
+               "workload": synth.MOE_DECODE_BF16.name, "M": 64}
 
 
 def parse():
@@ -59,6 +60,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time plain API calls instead of replaying a CUDA graph of them")
     return ap.parse_args()
 
 
@@ -160,12 +163,12 @@ def routing_stats(rt: dict, shape: synth.MoEShape):
 
 
 def gateup_alg_bytes(shape, M, experts, pairs):
-    """Bytes the gate_up GEMM must move once: touched expert gate_up weights, touched
-    B_gu slices, the gathered x rows, z_gu, and the act it writes."""
+    """Bytes the gate_up GEMM must move once: touched expert gate_up weights, the
+    gathered x rows, the LoRA delta it adds (fp32, 2I per row) and the act it writes."""
     wb = 1 if shape.wdtype == "e4m3" else 2
     mk = M * shape.k
-    return (experts * 2 * shape.I * shape.H * wb + pairs * shape.r * 2 * shape.I * 2
-            + mk * shape.H * 2 + mk * shape.r * 4 + mk * shape.I * 2)
+    return (experts * 2 * shape.I * shape.H * wb + mk * shape.H * 2 + mk * 2 * shape.I * 4
+            + mk * shape.I * 2)
 
 
 def layer_alg_bytes(shape, M, experts, pairs):
@@ -307,29 +310,64 @@ def main():
         step(i)
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps on device-resident inputs
-    launches_per_step = 8
+    # ---- per-kernel device times: plain API calls, CUDA events around every launch
+    launches_per_step = 16  # upper bound of library launches per step
     ml.profile_enable(args.steps * launches_per_step + 64)
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = ml.launch_count()
+    p0.record()
+    for i in range(args.steps):
+        step(i)
+    p1.record()
+    torch.cuda.synchronize()
+    launches = ml.launch_count() - n0
+    plain_ms = p0.elapsed_time(p1)
+    gu_ms, gu_n = ml.profile_read("gemm_gateup")
+    per_kernel = {kname: ml.profile_read(kname) for kname in ("router_logits", "topk", "sort", "shrink",
+                                                            "expand", "gemm_gateup", "gemm_down", "combine")}
+    ml.profile_enable(0)
+
+    # ---- the step as a CUDA graph of the same API calls (one graph per token batch)
+    graphs = []
+    if not args.no_graph:
+        gs = torch.cuda.Stream()
+        gs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(gs):
+            for b in range(len(batches)):
+                step(b)  # warm the stream before capture
+        torch.cuda.current_stream().wait_stream(gs)
+        torch.cuda.synchronize()
+        for b in range(len(batches)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(b)
+            graphs.append(g)
+        for i in range(args.warmup):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+
+    def run_step(i):
+        if graphs:
+            graphs[i % len(graphs)].replay()
+        else:
+            step(i)
+
+    # ---- timed region: K steps on device-resident inputs
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.25)
     barrier(world)
     torch.cuda.synchronize()
-    n0 = ml.launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
     for i in range(args.steps):
-        step(i)
+        run_step(i)
     ev1.record()
     torch.cuda.synchronize()
     barrier(world)
-    launches = ml.launch_count() - n0
     ms = ev0.elapsed_time(ev1)
     clk = clocks.stop()
-    gu_ms, gu_n = ml.profile_read("gemm_gateup")
-    per_kernel = {kname: ml.profile_read(kname) for kname in ("router_logits", "topk", "sort", "shrink",
-                                                            "gemm_gateup", "gemm_down", "combine")}
-    ml.profile_enable(0)
     ms_max = max_over_ranks(ms, world)
     value = world * M * args.steps / (ms_max / 1e3)
 
@@ -340,22 +378,37 @@ def main():
     hy = torch.empty((M, shape.H), dtype=torch.bfloat16).pin_memory()
     dx = torch.empty_like(batches[0][0])
     da = torch.empty_like(batches[0][1])
+
+    def e2e_step(j):
+        dx.copy_(hx[j], non_blocking=True)
+        da.copy_(ha[j], non_blocking=True)
+        rt = ml.route(da, k, L, x=dx, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
+        ml.forward(dx, rt, W, k=k, L=L, y=y, workspace=fws)
+        hy.copy_(y, non_blocking=True)
+
+    e2e_graphs = []
+    if not args.no_graph:
+        for j in range(len(batches)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                e2e_step(j)
+            e2e_graphs.append(g)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(e2e_steps):
         j = i % len(batches)
-        dx.copy_(hx[j], non_blocking=True)
-        da.copy_(ha[j], non_blocking=True)
-        rt = ml.route(da, k, L, x=dx, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
-        ml.forward(dx, rt, W, k=k, L=L, y=y, workspace=fws)
-        hy.copy_(y, non_blocking=True)
+        if e2e_graphs:
+            e2e_graphs[j].replay()
+        else:
+            e2e_step(j)
     e1.record()
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = world * M * e2e_steps / (e2e_ms / 1e3)
+    del graphs, e2e_graphs
     ml.check_status(fws)
     ml.check_status(rws)
 
@@ -368,7 +421,8 @@ def main():
     gu_avg_s = (gu_ms / max(gu_n, 1)) / 1e3
     achieved = gu_bytes / gu_avg_s / 1e9
     peak = float(peaks["hbm_gbs"])
-    traffic = NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["gemm_tc.cu"] == src_hash("gemm_tc.cu") else None
+    traffic = (NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["gemm_tc.cu"] == src_hash("gemm_tc.cu")
+               and NCU_TRAFFIC["workload"] == shape.name and NCU_TRAFFIC["M"] == M else None)
     step_s = ms_max / 1e3 / args.steps
 
     line = {
@@ -390,7 +444,10 @@ def main():
                   "TFLOPs": layer_flops(shape, M) / step_s / 1e12,
                   "kernel_ms_per_step": {kk: v[0] / args.steps for kk, v in per_kernel.items()}},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": M * shape.H * 2 + M * 4,
-                "d2h_bytes_per_step": M * shape.H * 2},
+                "d2h_bytes_per_step": M * shape.H * 2,
+                "how": "graph replay of H2D copy, route, forward, D2H copy" if not args.no_graph else "plain API calls"},
+        "timing": {"mode": "CUDA graph replay of the route + forward API calls" if not args.no_graph
+                   else "plain API calls", "plain_api_ms_per_step": plain_ms / args.steps},
         "gpu_launches": launches,
         "clocks": clk,
     }

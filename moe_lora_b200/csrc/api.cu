@@ -141,9 +141,9 @@ struct ForwardWs {
   int* status;
   __nv_bfloat16* x_sorted;
   __nv_bfloat16* act;
-  float* z_gu;
-  float* z_d;
-  int32_t* row_adapter;
+  float* delta_gu;
+  float* delta_d;
+  float* z;
   float* o;
   size_t bytes;
 };
@@ -161,9 +161,9 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r) {
   w.status = reinterpret_cast<int*>(b);
   w.x_sorted = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
   w.act = reinterpret_cast<__nv_bfloat16*>(take(mk * I * 2));
-  w.z_gu = reinterpret_cast<float*>(take(mk * r * 4));
-  w.z_d = reinterpret_cast<float*>(take(mk * r * 4));
-  w.row_adapter = reinterpret_cast<int32_t*>(take(mk * 4));
+  w.delta_gu = reinterpret_cast<float*>(take(r ? mk * 2 * I * 4 : 0));
+  w.delta_d = reinterpret_cast<float*>(take(r ? mk * H * 4 : 0));
+  w.z = reinterpret_cast<float*>(take(mk * r * 4));
   w.o = reinterpret_cast<float*>(take(mk * H * 4));
   w.bytes = off;
   return w;
@@ -196,12 +196,13 @@ RouteWs route_layout(void* base, int M, int E, int L) {
 
 struct DenseWs {
   int* status;
-  float* z;
-  int32_t* row_adapter;
+  float* z;             // fp32 path: shrink output
+  int32_t* row_adapter; // fp32 path
+  float* delta;         // bf16 path: LoRA delta added by the GEMM epilogue
   size_t bytes;
 };
 
-DenseWs dense_layout(void* base, int T, int r) {
+DenseWs dense_layout(void* base, int T, int h_out, int r, bool f32) {
   size_t off = kStatusBytes;
   DenseWs w{};
   uint8_t* b = static_cast<uint8_t*>(base);
@@ -211,8 +212,13 @@ DenseWs dense_layout(void* base, int T, int r) {
     return p;
   };
   w.status = reinterpret_cast<int*>(b);
-  w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
-  w.row_adapter = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
+  if (f32) {
+    w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
+    w.row_adapter = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
+  } else {
+    w.delta = reinterpret_cast<float*>(take(r ? static_cast<size_t>(T) * h_out * 4 : 0));
+    w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
+  }
   w.bytes = off;
   return w;
 }
@@ -293,7 +299,11 @@ size_t moe_lora_workspace_size(int op, int M, int H, int I, int E, int k, int L,
     case MOE_LORA_OP_FORWARD: return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0).bytes;
     case MOE_LORA_OP_SGMV_SHRINK:
     case MOE_LORA_OP_SGMV_EXPAND: return kStatusBytes;
-    case MOE_LORA_OP_DENSE: return dense_layout(nullptr, M, L > 0 ? r : 0).bytes;
+    case MOE_LORA_OP_DENSE: {
+      const size_t a = dense_layout(nullptr, M, I, L > 0 ? r : 0, true).bytes;
+      const size_t b = dense_layout(nullptr, M, I, L > 0 ? r : 0, false).bytes;
+      return a > b ? a : b;
+    }
     default: return 0;
   }
 }
@@ -386,7 +396,10 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr);
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
-  if (w_dtype == ML_E4M3) return fail(MOE_LORA_ERR_UNSUPPORTED, "ML_E4M3 expert weights: not built yet");
+  if (w_dtype == ML_E4M3) {
+    ML_REQUIRE(H % 16 == 0 && I % 16 == 0, MOE_LORA_ERR_UNSUPPORTED,
+               "ML_E4M3 expert weights need H and I multiples of 16 (16-byte rows)");
+  }
   if (M == 0) return MOE_LORA_OK;
   ML_PTR(x);
   ML_PTR(topk_w);
@@ -395,6 +408,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   ML_PTR(w_gateup);
   ML_PTR(w_down);
   ML_PTR(y);
+  if (w_dtype == ML_E4M3) ML_PTR(w_scales);
   if (L > 0) {
     ML_PTR(lora_a_gu);
     ML_PTR(lora_b_gu);
@@ -411,32 +425,33 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   const int nkeys = E * (L + 1);
   ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
 
-  // 1. gather x rows into (expert, adapter) order + gate_up shrink z = x A_gu
-  ShrinkArgs s1{};
-  s1.src = x;
-  s1.src_f32 = false;
-  s1.gather = sorted_pairs;
-  s1.gather_div = k;
-  s1.gather_dst = w.x_sorted;
-  s1.nrows = mk;
-  s1.K = H;
-  s1.r = rr;
-  s1.seg_offsets = seg_offsets;
-  s1.nseg = nkeys;
-  s1.seg_adapter = nullptr;
-  s1.L = L;
-  s1.E = E;
-  s1.lora_a = lora_a_gu;
-  s1.z = w.z_gu;
-  s1.row_adapter = w.row_adapter;
-  s1.rows_per_cta = shrink_rows_per_cta(mk);
-  s1.status = w.status;
-  ML_CUDA(launch_shrink(s1, cs), "gate_up shrink launch");
+  // 1. gather x rows into (expert, adapter) order; gate_up LoRA shrink + expand:
+  //    delta_gu = (x A_gu) B_gu per (adapter, expert) segment, z kept on chip
+  LoraDeltaArgs l1{};
+  l1.src = static_cast<const __nv_bfloat16*>(x);
+  l1.gather = sorted_pairs;
+  l1.gather_div = k;
+  l1.gather_dst = w.x_sorted;
+  l1.nrows = mk;
+  l1.K = H;
+  l1.r = rr;
+  l1.NB = 2 * I;
+  l1.seg_offsets = seg_offsets;
+  l1.nseg = nkeys;
+  l1.seg_adapter = nullptr;
+  l1.L = L;
+  l1.E = E;
+  l1.lora_a = static_cast<const __nv_bfloat16*>(lora_a_gu);
+  l1.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
+  l1.delta = rr ? w.delta_gu : nullptr;
+  l1.z = rr ? w.z : nullptr;
+  l1.status = w.status;
+  ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
 
-  // 2. gate_up grouped GEMM, LoRA expand + SiLU-and-mul in the epilogue -> act
+  // 2. gate_up grouped GEMM; epilogue adds delta_gu and applies SiLU-and-mul -> act
   GemmArgs g{};
   g.epi = EPI_GATEUP;
-  g.w_fp8 = false;
+  g.w_fp8 = w_dtype == ML_E4M3;
   g.K = H;
   g.E = E;
   g.group_offsets = seg_offsets;
@@ -445,42 +460,41 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.n_out = I;
   g.I = I;
   g.total_rows = mk;
-  g.z = rr ? w.z_gu : nullptr;
-  g.row_adapter = w.row_adapter;
-  g.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
-  g.r = rr;
-  g.L = L;
+  g.delta = rr ? w.delta_gu : nullptr;
+  g.delta_cols = 2 * I;
   g.out_bf16 = w.act;
-  g.w_scales = w_scales;
+  g.w_scales = w_dtype == ML_E4M3 ? w_scales : nullptr;
   g.scale_idx = 0;
   g.status = w.status;
   g.w = w_gateup;
   g.b = w.x_sorted;
   g.bn = choose_bn(mk, E);
+  if (g.w_fp8 && g.bn > 64) g.bn = 64;  // the fp8 ring leaves room for N tiles up to 64
   g.num_sms = num_sms();
   ML_CUDA(launch_gemm_tc(g, cs), "gate_up GEMM launch");
 
-  // 3. down shrink z_d = act A_d
+  // 3. down LoRA shrink + expand on act: delta_d = (act A_d) B_d
   if (rr) {
-    ShrinkArgs s2 = s1;
-    s2.src = w.act;
-    s2.gather = nullptr;
-    s2.gather_dst = nullptr;
-    s2.K = I;
-    s2.lora_a = lora_a_d;
-    s2.z = w.z_d;
-    s2.row_adapter = nullptr;
-    ML_CUDA(launch_shrink(s2, cs), "down shrink launch");
+    LoraDeltaArgs l2 = l1;
+    l2.src = w.act;
+    l2.gather = nullptr;
+    l2.gather_dst = nullptr;
+    l2.K = I;
+    l2.NB = H;
+    l2.lora_a = static_cast<const __nv_bfloat16*>(lora_a_d);
+    l2.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
+    l2.delta = w.delta_d;
+    ML_CUDA(launch_lora_delta(l2, cs), "down LoRA launch");
   }
 
-  // 4. down grouped GEMM, LoRA expand, x routing weight -> o (one row per pair)
+  // 4. down grouped GEMM; epilogue adds delta_d and the routing weight -> o (per pair)
   GemmArgs d = g;
   d.epi = EPI_DOWN;
   d.K = I;
   d.rows_per_group = H;
   d.n_out = H;
-  d.z = rr ? w.z_d : nullptr;
-  d.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
+  d.delta = rr ? w.delta_d : nullptr;
+  d.delta_cols = H;
   d.out_bf16 = nullptr;
   d.out_f32 = w.o;
   d.sorted_pairs = sorted_pairs;
@@ -587,7 +601,8 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   if (L > 0) ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
   ML_REQUIRE(S >= 1 || T == 0, MOE_LORA_ERR_INVALID_ARG, "segments must cover the T tokens");
   const int rr = L > 0 ? r : 0;
-  const DenseWs need = dense_layout(nullptr, T, rr);
+  const bool f32 = dt == ML_F32;
+  const DenseWs need = dense_layout(nullptr, T, h_out, rr, f32);
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (T == 0) return MOE_LORA_OK;
@@ -603,29 +618,28 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   st = check_device();
   if (st != MOE_LORA_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const DenseWs ws = dense_layout(workspace, T, rr);
+  const DenseWs ws = dense_layout(workspace, T, h_out, rr, f32);
   ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
 
-  ShrinkArgs a{};
-  a.src = x;
-  a.src_f32 = dt == ML_F32;
-  a.gather_div = 1;
-  a.nrows = T;
-  a.K = h_in;
-  a.r = rr;
-  a.seg_offsets = seg_offsets;
-  a.nseg = S;
-  a.seg_adapter = seg_adapter;
-  a.L = L;
-  a.E = 1;
-  a.lora_a = lora_a;
-  a.z = ws.z;
-  a.row_adapter = ws.row_adapter;
-  a.rows_per_cta = shrink_rows_per_cta(T);
-  a.status = ws.status;
-  ML_CUDA(launch_shrink(a, cs), "dense shrink launch");
-
-  if (dt == ML_F32) {
+  if (f32) {
+    ShrinkArgs a{};
+    a.src = x;
+    a.src_f32 = true;
+    a.gather_div = 1;
+    a.nrows = T;
+    a.K = h_in;
+    a.r = rr;
+    a.seg_offsets = seg_offsets;
+    a.nseg = S;
+    a.seg_adapter = seg_adapter;
+    a.L = L;
+    a.E = 1;
+    a.lora_a = lora_a;
+    a.z = ws.z;
+    a.row_adapter = ws.row_adapter;
+    a.rows_per_cta = shrink_rows_per_cta(T);
+    a.status = ws.status;
+    ML_CUDA(launch_shrink(a, cs), "dense shrink launch");
     DenseF32Args d{};
     d.x = static_cast<const float*>(x);
     d.w = static_cast<const float*>(w);
@@ -643,6 +657,26 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   }
   if (!tensor_map_encode_available())
     return fail(MOE_LORA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (rr) {
+    LoraDeltaArgs l{};
+    l.src = static_cast<const __nv_bfloat16*>(x);
+    l.gather_div = 1;
+    l.nrows = T;
+    l.K = h_in;
+    l.r = rr;
+    l.NB = h_out;
+    l.seg_offsets = seg_offsets;
+    l.nseg = S;
+    l.seg_adapter = seg_adapter;
+    l.L = L;
+    l.E = 1;
+    l.lora_a = static_cast<const __nv_bfloat16*>(lora_a);
+    l.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
+    l.delta = ws.delta;
+    l.z = ws.z;
+    l.status = ws.status;
+    ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
+  }
   GemmArgs g{};
   g.epi = EPI_DENSE;
   g.K = h_in;
@@ -653,11 +687,8 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   g.n_out = h_out;
   g.I = 0;
   g.total_rows = T;
-  g.z = rr ? ws.z : nullptr;
-  g.row_adapter = ws.row_adapter;
-  g.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
-  g.r = rr;
-  g.L = L;
+  g.delta = rr ? ws.delta : nullptr;
+  g.delta_cols = h_out;
   g.out_bf16 = static_cast<__nv_bfloat16*>(y);
   g.status = ws.status;
   g.w = w;

@@ -4,22 +4,29 @@
 // and its N slot the tokens of one expert, so that a decode batch of a few tokens
 // per expert still fills the tensor core's M dimension ([SageMaker MoE kernels
 // page], first item: transpose so the large expert dimension is the first operand).
-// The LoRA expand z B and the base output are added in the epilogue, in registers,
-// before anything is stored ([vLLM MoE-LoRA page], "Otimizações em Nível de
-// Kernel": the LoRA add fused into the expand; "Implementação Técnica no vLLM":
-// fused_moe_lora).  gate_up tiles pair 64 gate rows with the matching 64 up rows so
-// the SiLU-and-mul gate is applied before act leaves the SM; down tiles multiply by
-// the routing weight and store one fp32 row per routing pair for the fixed-order
-// combine (expert aggregation, [SageMaker MoE kernels page], second item).
+// The epilogue adds the LoRA delta (z B, produced by the segmented shrink/expand
+// kernel) to the accumulator before anything is stored ([vLLM MoE-LoRA page],
+// "Otimizações em Nível de Kernel": the LoRA add fused into the base output;
+// "Implementação Técnica no vLLM": fused_moe_lora).  gate_up tiles pair 64 gate rows
+// with the matching 64 up rows so SiLU-and-mul is applied before act leaves the SM;
+// down tiles multiply by the routing weight and store one fp32 row per routing pair
+// for the fixed-order combine (expert aggregation, [SageMaker MoE kernels page],
+// second item).  FP8 (e4m3) expert weights stay one byte per weight in HBM and in the
+// TMA ring; converter warps widen them exactly to bf16 for the kind::f16 MMA and the
+// per-tensor scale is applied in the epilogue (same page, second item).
 //
 // Structure (one CTA per SM, persistent over a device-side tile list):
-//   warp 0      TMA producer: weight tile 128 x 64 (two 64-row boxes) and token
-//               tile BN x 64 per stage, 128-byte swizzle, mbarrier transaction count
+//   warp 0      TMA producer: weight tile 128 x 64 per stage (two 64-row boxes; e4m3:
+//               128 x 128 bytes) and the token tile of the same K range
 //   warp 1      MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM),
-//               M = 128, N = BN, K = 16 x 4 per stage; commits free the smem stage
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, LoRA expand, activation,
-//               stores; two TMEM accumulators so the epilogue of tile i overlaps
-//               the MMAs of tile i+1
+//               M = 128, N = BN, K = 16 per instruction; commits free the smem stage
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, + LoRA delta, activation,
+//               stores; two TMEM accumulators so the epilogue of tile i overlaps the
+//               MMAs of tile i+1
+//   warp 6      epilogue loader (N tiles <= 64): one tile ahead of the epilogue, TMA
+//               of the tile's LoRA delta and, for down, the pair ids and routing
+//               weights, into a two-slot shared-memory ring
+//   warps 7..10 (e4m3 weights) converters: fp8 weight tile -> bf16 stage
 // Every mbarrier wait is bounded; on expiry the CTA records MOE_LORA_ERR_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include "common.cuh"
@@ -34,11 +41,9 @@ namespace mlb {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMaxGroups = 256;
-constexpr int kMaxR = 128;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 struct TcParams {
@@ -50,10 +55,8 @@ struct TcParams {
   int rows_per_group;
   int n_out;
   int I;
-  const float* z;
-  const int32_t* row_adapter;
-  const __nv_bfloat16* lora_b;
-  int r;
+  const float* delta;
+  int delta_cols;
   __nv_bfloat16* out_bf16;
   float* out_f32;
   const int32_t* sorted_pairs;
@@ -63,39 +66,58 @@ struct TcParams {
   int* status;
   int m_tiles;
   int stages;
+  int stages8;
 };
 
-// Non-pipeline shared memory, placed after the stage ring.
-struct SmemMisc {
+// Non-pipeline shared memory, placed after the stage rings.
+struct SmemCore {
   uint64_t full[16];
   uint64_t empty[16];
+  uint64_t full8[16];
+  uint64_t empty8[16];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t sfull[2];
+  uint64_t sempty[2];
   uint64_t tdone;
   uint32_t tmem_base;
   int abort_flag;
   int chunk_pref[kMaxGroups + 1];
   int grp_off[kMaxGroups + 1];
   float ebuf[kBM][33];
-  float zs[32 * kMaxR];
-  int col_ad[32];
   int col_pair[32];
   float col_w[32];
 };
 
+// Epilogue prefetch slot (N tiles <= 64): LoRA delta [2 halves][BN][64] and pair data.
 template <int BN>
+struct EpiSlot {
+  float delta[2 * BN * 64];
+  int col_pair[BN];
+  float col_w[BN];
+};
+
+template <int BN, bool W8>
 struct TileCfg {
-  static constexpr int kBTileBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kATileBytes + kBTileBytes;
-  static constexpr int kAccStride = BN < 32 ? 32 : BN;  // TMEM columns per accumulator
-  static constexpr int kTmemCols = 2 * kAccStride;      // power of two >= 32
+  static constexpr int kBTileBytes = BN * kBK * 2;           // one 64-K token sub-tile
+  // bf16 stage (K = 64): the A tile (+ the token tile for bf16 weights); fp8 stage
+  // (K = 128): the e4m3 weight tile and the two token sub-tiles of the same K range,
+  // converted into two consecutive bf16 stages
+  static constexpr int kStageBytes = W8 ? kATileBytes : kATileBytes + kBTileBytes;
+  static constexpr int kW8StageBytes = kBM * 128 + 2 * kBTileBytes;
+  static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
+  static constexpr int kTmemCols = 2 * kAccStride;           // power of two >= 32
+  static constexpr bool kPrefetch = BN <= 64;                // epilogue loader warp + slots
+  static constexpr int kSlotBytes = kPrefetch ? static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024) : 0;
+  static constexpr int kConvWarp0 = 7;
+  static constexpr int kThreads = W8 ? 352 : 224;
 };
 
 struct TileInfo {
   int g, mt, row0, nvalid;
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const SmemMisc& sm, int t, int m_tiles, int E, int BN) {
+__device__ __forceinline__ TileInfo decode_tile(const SmemCore& sm, int t, int m_tiles, int E, int BN) {
   TileInfo ti;
   const int c = t / m_tiles;
   ti.mt = t - c * m_tiles;
@@ -111,16 +133,44 @@ __device__ __forceinline__ TileInfo decode_tile(const SmemMisc& sm, int t, int m
   return ti;
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+// 16 e4m3 values -> 16 bf16 values, exactly (every e4m3 value is an f16 normal or zero).
+__device__ __forceinline__ void e4m3x16_to_bf16(uint4 q, uint4& lo, uint4& hi) {
+  const uint32_t in[4] = {q.x, q.y, q.z, q.w};
+  uint32_t out[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((in[i] >> (16 * h)) & 0xFFFFu);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      out[2 * i + h] = pack2_bf16(f.x, f.y);
+    }
+  }
+  lo = make_uint4(out[0], out[1], out[2], out[3]);
+  hi = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+// delta column (weight row within the group) of accumulator row m in tile column block f0
+__device__ __forceinline__ int delta_col(int epi, int m, int f0, int I) {
+  if (epi == EPI_GATEUP) return (m < 64) ? f0 + m : I + f0 + (m - 64);
+  return f0 + m;
+}
+
+template <int BN, bool W8>
+__global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
-                   const TcParams p) {
-  using Cfg = TileCfg<BN>;
+                   const __grid_constant__ CUtensorMap tmd, const TcParams p) {
+  using Cfg = TileCfg<BN, W8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SmemMisc& sm = *reinterpret_cast<SmemMisc*>(smem + p.stages * Cfg::kStageBytes);
+  uint8_t* ring8 = smem;                                              // fp8 weight stages
+  uint8_t* ring = smem + (W8 ? p.stages8 * Cfg::kW8StageBytes : 0);  // bf16 stages
+  uint8_t* slots = ring + p.stages * Cfg::kStageBytes;               // epilogue prefetch slots
+  SmemCore& sm = *reinterpret_cast<SmemCore*>(slots + 2 * Cfg::kSlotBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
+  const int S8 = p.stages8;
   volatile int* abort_flag = &sm.abort_flag;
 
   // ---- setup: barriers, TMEM, tile list prefix
@@ -129,9 +179,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
+    for (int s = 0; s < S8; ++s) {
+      mbar_init(&sm.full8[s], 1);
+      mbar_init(&sm.empty8[s], 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
       mbar_init(&sm.tempty[b], kEpiThreads);
+      mbar_init(&sm.sfull[b], 1);
+      mbar_init(&sm.sempty[b], kEpiThreads);
     }
     mbar_init(&sm.tdone, 1);
     sm.abort_flag = 0;
@@ -140,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmw);
     tma_prefetch_desc(&tmb);
+    if (p.delta != nullptr) tma_prefetch_desc(&tmd);
   }
   if (warp == 1) tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
   for (int g = threadIdx.x; g <= p.E; g += blockDim.x)
@@ -180,11 +237,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
   const int total_tiles = sm.chunk_pref[p.E] * p.m_tiles;
-  const int nk = (p.K + kBK - 1) / kBK;
+  const int nk8 = (p.K + 127) / 128;                  // fp8 stages per tile
+  const int nk = W8 ? 2 * nk8 : (p.K + kBK - 1) / kBK;  // bf16 stages per tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      const int SR = W8 ? S8 : S;
+      uint64_t* fullb = W8 ? sm.full8 : sm.full;
+      uint64_t* emptyb = W8 ? sm.empty8 : sm.empty;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t filled_mask = 0, last_parity = 0;
@@ -198,17 +259,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           wrow0 = ti.g * p.rows_per_group + ti.mt * kBM;
           wrow1 = wrow0 + 64;
         }
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort_flag, p.status, kWaitLimitNs, 1)) break;
-          uint8_t* a_s = smem + stage * Cfg::kStageBytes;
-          uint8_t* b_s = a_s + kATileBytes;
-          mbar_arrive_expect_tx(&sm.full[stage], Cfg::kStageBytes);
-          tma_load_2d(a_s, &tmw, &sm.full[stage], kb * kBK, wrow0);
-          tma_load_2d(a_s + kATileBytes / 2, &tmw, &sm.full[stage], kb * kBK, wrow1);
-          tma_load_2d(b_s, &tmb, &sm.full[stage], kb * kBK, ti.row0);
+        for (int kb = 0; kb < (W8 ? nk8 : nk); ++kb) {
+          if (!mbar_wait(&emptyb[stage], phase ^ 1u, abort_flag, p.status, kWaitLimitNs, 1)) break;
+          if constexpr (W8) {
+            uint8_t* a8 = ring8 + stage * Cfg::kW8StageBytes;
+            mbar_arrive_expect_tx(&fullb[stage], Cfg::kW8StageBytes);
+            tma_load_2d(a8, &tmw, &fullb[stage], kb * 128, wrow0);
+            tma_load_2d(a8 + kBM * 64, &tmw, &fullb[stage], kb * 128, wrow1);
+            tma_load_2d(a8 + kBM * 128, &tmb, &fullb[stage], kb * 128, ti.row0);
+            tma_load_2d(a8 + kBM * 128 + Cfg::kBTileBytes, &tmb, &fullb[stage], kb * 128 + 64, ti.row0);
+          } else {
+            uint8_t* a_s = ring + stage * Cfg::kStageBytes;
+            uint8_t* b_s = a_s + kATileBytes;
+            mbar_arrive_expect_tx(&fullb[stage], Cfg::kStageBytes);
+            tma_load_2d(a_s, &tmw, &fullb[stage], kb * kBK, wrow0);
+            tma_load_2d(a_s + kATileBytes / 2, &tmw, &fullb[stage], kb * kBK, wrow1);
+            tma_load_2d(b_s, &tmb, &fullb[stage], kb * kBK, ti.row0);
+          }
           filled_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == S) {
+          if (++stage == SR) {
             stage = 0;
             phase ^= 1u;
           }
@@ -216,10 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag) {
         // let our own copies land before the CTA exits
-        for (int s = 0; s < S; ++s)
+        for (int s = 0; s < SR; ++s)
           if (filled_mask & (1u << s)) {
             volatile int dummy = 0;
-            mbar_wait(&sm.full[s], (last_parity >> s) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
+            mbar_wait(&fullb[s], (last_parity >> s) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
           }
       }
     }
@@ -227,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_bf16(kBM, BN);
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, s8 = 0;
+      uint32_t phase = 0, ph8 = 0;
       int it = 0;
       for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
         const int buf = it & 1;
@@ -238,19 +308,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem_base + buf * Cfg::kAccStride;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 3)) {
+          const int half = kb & 1;  // e4m3: which 64-wide half of the fp8 stage
+          bool got = true;
+          if constexpr (W8)
+            if (half == 0) got = mbar_wait(&sm.full8[s8], ph8, abort_flag, p.status, kWaitLimitNs, 9);
+          if (!got || !mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 3)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * Cfg::kStageBytes);
-          const uint32_t b_addr = a_addr + kATileBytes;
-          const uint64_t adesc = umma_desc_sw128(a_addr);
+          const uint32_t st_addr = smem_u32(ring + stage * Cfg::kStageBytes);
+          const uint32_t b_addr = W8 ? smem_u32(ring8 + s8 * Cfg::kW8StageBytes + kBM * 128 + half * Cfg::kBTileBytes)
+                                     : st_addr + kATileBytes;
+          const uint64_t adesc = umma_desc_sw128(st_addr);
           const uint64_t bdesc = umma_desc_sw128(b_addr);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
             umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit(&sm.empty[stage]);
+          if constexpr (W8) {
+            if (half == 1) {
+              umma_commit(&sm.empty8[s8]);
+              if (++s8 == S8) {
+                s8 = 0;
+                ph8 ^= 1u;
+              }
+            }
+          }
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -264,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int dummy = 0;
       mbar_wait(&sm.tdone, 0, &dummy, nullptr, kWaitLimitNs, 0);
     }
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;   // 0..127
     const int g4 = warp & 3;           // TMEM lane quarter this warp may access
@@ -274,63 +358,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
-      const bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 4);
+      bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 4);
+      if constexpr (Cfg::kPrefetch) got = got && mbar_wait(&sm.sfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 7);
       if (!named_bar_and(2, kEpiThreads, got)) break;  // the four warps leave together
       tc_fence_after();
 
-      // weight row (within the group's rows) held by this thread, and whether it is real
-      int wrow, feat;
+      const int f0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
+      int feat;
       bool row_ok;
       if (p.epi == EPI_GATEUP) {
-        feat = ti.mt * 64 + (m & 63);
-        wrow = (m < 64) ? feat : p.I + feat;
+        feat = f0 + (m & 63);
         row_ok = feat < p.I;
       } else {
-        feat = ti.mt * kBM + m;
-        wrow = feat;
+        feat = f0 + m;
         row_ok = feat < p.n_out;
       }
+      const int dcol = delta_col(p.epi, m, f0, p.I);
       float scale = 1.f;
       if (p.w_scales != nullptr) scale = p.w_scales[ti.g * 2 + p.scale_idx];
+      const EpiSlot<BN>* slot = reinterpret_cast<const EpiSlot<BN>*>(slots + buf * Cfg::kSlotBytes);
 
       for (int c0 = 0; c0 < ti.nvalid; c0 += 32) {
-        named_bar_sync(1, kEpiThreads);
+        named_bar_sync(1, kEpiThreads);  // the previous chunk is done with smem
         const int ncol = min(32, ti.nvalid - c0);
-        if (et < 32) {
-          const int s = ti.row0 + c0 + et;
-          const bool valid = et < ncol;
-          sm.col_ad[et] = (valid && p.row_adapter != nullptr) ? p.row_adapter[s] : -1;
-          if (p.epi == EPI_DOWN) {
-            const int pr = valid ? p.sorted_pairs[s] : 0;
+        if constexpr (!Cfg::kPrefetch) {
+          if (p.epi == EPI_DOWN && et < 32) {
+            const int pr = et < ncol ? p.sorted_pairs[ti.row0 + c0 + et] : 0;
             sm.col_pair[et] = pr;
-            sm.col_w[et] = valid ? p.topk_w[pr] : 0.f;
+            sm.col_w[et] = et < ncol ? p.topk_w[pr] : 0.f;
           }
         }
-        if (p.z != nullptr) {
-          for (int idx = et; idx < 32 * p.r; idx += kEpiThreads) {
-            const int n = idx / p.r;
-            sm.zs[idx] = (n < ncol) ? p.z[static_cast<size_t>(ti.row0 + c0 + n) * p.r + (idx - n * p.r)] : 0.f;
-          }
-        }
-        named_bar_sync(1, kEpiThreads);
-
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) + buf * Cfg::kAccStride + c0, v);
 #pragma unroll
         for (int n = 0; n < 32; ++n) v[n] *= scale;
-
-        if (row_ok && p.z != nullptr) {
+        if (p.delta != nullptr) {
+          if constexpr (Cfg::kPrefetch) {
+            const float* dl = slot->delta + ((m >> 6) * BN + c0) * 64 + (m & 63);
 #pragma unroll
-          for (int n = 0; n < 32; ++n) {
-            const int ad = sm.col_ad[n];
-            if (ad >= 0) {
-              const __nv_bfloat16* bcol = p.lora_b + (static_cast<size_t>(ad) * p.E + ti.g) * p.r * p.rows_per_group + wrow;
-              const float* zr = &sm.zs[n * p.r];
-              float acc = 0.f;
-              for (int i = 0; i < p.r; ++i)
-                acc = fmaf(zr[i], __bfloat162float(bcol[static_cast<size_t>(i) * p.rows_per_group]), acc);
-              v[n] += acc;
-            }
+            for (int n = 0; n < 32; ++n)
+              if (c0 + n < BN) v[n] += dl[n * 64];
+          } else if (dcol < p.delta_cols) {
+            const float* dg = p.delta + static_cast<size_t>(ti.row0 + c0) * p.delta_cols + dcol;
+#pragma unroll
+            for (int n = 0; n < 32; ++n)
+              if (n < ncol) v[n] += dg[static_cast<size_t>(n) * p.delta_cols];
           }
         }
 
@@ -341,8 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = et >> 2;
           const int fq = (et & 3) * 16;
           if (n < ncol) {
-            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(ti.row0 + c0 + n) * p.I + ti.mt * 64 + fq;
-            const int fbase = ti.mt * 64 + fq;
+            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(ti.row0 + c0 + n) * p.I + f0 + fq;
+            const int fbase = f0 + fq;
             uint32_t packed[8];
 #pragma unroll
             for (int f = 0; f < 16; f += 2) {
@@ -363,11 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else if (p.epi == EPI_DOWN) {
+          if constexpr (!Cfg::kPrefetch) named_bar_sync(1, kEpiThreads);  // col_pair / col_w visible
           if (row_ok) {
+            const int* cp = Cfg::kPrefetch ? slot->col_pair + c0 : sm.col_pair;
+            const float* cw = Cfg::kPrefetch ? slot->col_w + c0 : sm.col_w;
 #pragma unroll
             for (int n = 0; n < 32; ++n)
-              if (n < ncol)
-                p.out_f32[static_cast<size_t>(sm.col_pair[n]) * p.n_out + feat] = v[n] * sm.col_w[n];
+              if (n < ncol) p.out_f32[static_cast<size_t>(cp[n]) * p.n_out + feat] = v[n] * cw[n];
           }
         } else {
           if (row_ok) {
@@ -380,6 +454,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&sm.tempty[buf]);
+      if constexpr (Cfg::kPrefetch) mbar_arrive(&sm.sempty[buf]);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ epilogue loader
+    if constexpr (Cfg::kPrefetch) {
+      uint32_t issued_mask = 0, issued_parity = 0;
+      int it = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
+        const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
+        const int buf = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        const bool got = mbar_wait(&sm.sempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 8);
+        if (!__all_sync(0xffffffffu, got)) break;
+        EpiSlot<BN>* slot = reinterpret_cast<EpiSlot<BN>*>(slots + buf * Cfg::kSlotBytes);
+        if (lane == 0 && p.delta != nullptr) {
+          const int f0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
+          const int c1 = (p.epi == EPI_GATEUP) ? p.I + f0 : f0 + 64;
+          mbar_expect_tx(&sm.sfull[buf], 2 * BN * 64 * 4);
+          tma_load_2d(slot->delta, &tmd, &sm.sfull[buf], f0, ti.row0);
+          tma_load_2d(slot->delta + BN * 64, &tmd, &sm.sfull[buf], c1, ti.row0);
+          issued_mask |= 1u << buf;
+          issued_parity = (issued_parity & ~(1u << buf)) | ((use & 1u) << buf);
+        }
+        if (p.epi == EPI_DOWN) {
+          for (int n = lane; n < BN; n += 32) {
+            const int pr = n < ti.nvalid ? p.sorted_pairs[ti.row0 + n] : 0;
+            slot->col_pair[n] = pr;
+            slot->col_w[n] = n < ti.nvalid ? p.topk_w[pr] : 0.f;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sfull[buf]);
+      }
+      if (lane == 0 && *abort_flag) {
+        for (int b = 0; b < 2; ++b)
+          if (issued_mask & (1u << b)) {
+            volatile int dummy = 0;
+            mbar_wait(&sm.sfull[b], (issued_parity >> b) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
+          }
+      }
+    }
+  } else if constexpr (W8) {
+    // ------------------------------------------------------------ fp8 -> bf16 converters
+    // Thread ct owns weight row ct of each stage: it reads the row's 128 e4m3 values from
+    // the fp8 stage (128-byte swizzled rows) and writes them as bf16 into the two 64-wide
+    // 128-byte-swizzled sub-tiles of the bf16 stage the MMA reads.  The token sub-tiles
+    // stay in the fp8 stage, loaded there by the producer.
+    const int ct = threadIdx.x - 32 * Cfg::kConvWarp0;
+    const int sw = ct & 7;
+    int s8 = 0, s16 = 0;
+    uint32_t ph8 = 0, ph16 = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int kb8 = 0; kb8 < nk8 && ok; ++kb8) {
+        const bool got8 = mbar_wait(&sm.full8[s8], ph8, abort_flag, p.status, kWaitLimitNs, 5);
+        const uint8_t* src = ring8 + s8 * Cfg::kW8StageBytes + ct * 128;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const bool got = got8 && mbar_wait(&sm.empty[s16], ph16 ^ 1u, abort_flag, p.status, kWaitLimitNs, 6);
+          if (!named_bar_and(3, 128, got)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = ring + s16 * Cfg::kStageBytes + ct * 128;
+#pragma unroll
+          for (int c = 4 * half; c < 4 * half + 4; ++c) {
+            const uint4 q = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
+            uint4 lo, hi;
+            e4m3x16_to_bf16(q, lo, hi);
+            const int cc = (c & 3) * 2;
+            *reinterpret_cast<uint4*>(dst + ((cc ^ sw) << 4)) = lo;
+            *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ sw) << 4)) = hi;
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(3, 128);
+          if (ct == 0) mbar_arrive(&sm.full[s16]);  // the fp8 stage is released by the MMA
+          if (++s16 == S) {
+            s16 = 0;
+            ph16 ^= 1u;
+          }
+        }
+        if (++s8 == S8) {
+          s8 = 0;
+          ph8 ^= 1u;
+        }
+      }
     }
   }
 
@@ -418,30 +578,56 @@ CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-template <int BN>
+template <int BN, bool W8>
 static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
-  using Cfg = TileCfg<BN>;
-  const int misc = static_cast<int>(sizeof(SmemMisc));
-  const int budget = 232448 - 1024 - misc;
-  int stages = budget / Cfg::kStageBytes;
-  stages = stages > 8 ? 8 : stages;
-  if (stages < 2) return cudaErrorInvalidConfiguration;
-  const size_t smem = 1024 + static_cast<size_t>(stages) * Cfg::kStageBytes + misc;
+  using Cfg = TileCfg<BN, W8>;
+  const int fixed = static_cast<int>(sizeof(SmemCore)) + 2 * Cfg::kSlotBytes;
+  const int budget = 232448 - 1024 - fixed;
+  int stages, stages8 = 0;
+  if (W8) {
+    stages = 4;
+    stages8 = (budget - stages * Cfg::kStageBytes) / Cfg::kW8StageBytes;
+    stages8 = stages8 > 8 ? 8 : stages8;
+    if (stages8 < 2) {
+      stages = 2;
+      stages8 = (budget - stages * Cfg::kStageBytes) / Cfg::kW8StageBytes;
+    }
+    if (stages8 < 2) return cudaErrorInvalidConfiguration;
+  } else {
+    stages = budget / Cfg::kStageBytes;
+    stages = stages > 8 ? 8 : stages;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+  }
+  const size_t smem = 1024 + static_cast<size_t>(stages) * Cfg::kStageBytes +
+                      static_cast<size_t>(stages8) * Cfg::kW8StageBytes + fixed;
+  if (smem > 232448) return cudaErrorInvalidConfiguration;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem > 232448 ? 232448 : smem));
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         232448);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  CUtensorMap tmw, tmb;
+  CUtensorMap tmw, tmb, tmd;
   const uint64_t wrows = static_cast<uint64_t>(a.E) * a.rows_per_group;
-  if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2,
-                     kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  CUresult cr;
+  if (W8)
+    cr = encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, a.K, wrows, static_cast<uint64_t>(a.K), 128, 64,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    cr = encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2,
+                        kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
   if (encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
                      static_cast<uint64_t>(a.K) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  if (a.delta != nullptr && Cfg::kPrefetch) {
+    if (encode_tmap_2d(&tmd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.delta, a.delta_cols, a.total_rows,
+                       static_cast<uint64_t>(a.delta_cols) * 4, 64, BN, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    tmd = tmb;  // unused
+  }
   TcParams p;
   p.epi = a.epi;
   p.K = a.K;
@@ -451,10 +637,8 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.rows_per_group = a.rows_per_group;
   p.n_out = a.n_out;
   p.I = a.I;
-  p.z = a.z;
-  p.row_adapter = a.row_adapter;
-  p.lora_b = a.lora_b;
-  p.r = a.r;
+  p.delta = a.delta;
+  p.delta_cols = a.delta_cols;
   p.out_bf16 = a.out_bf16;
   p.out_f32 = a.out_f32;
   p.sorted_pairs = a.sorted_pairs;
@@ -464,25 +648,34 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.status = a.status;
   p.m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
   p.stages = stages;
+  p.stages8 = stages8;
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
   const long long tiles_ub = chunks_ub * p.m_tiles;
   int grid = a.num_sms;
   if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
   if (grid < 1) grid = 1;
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP : (a.epi == EPI_DOWN ? K_GEMM_DOWN : K_GEMM_DENSE), st);
-  gemm_tc_kernel<BN><<<grid, kThreads, smem, st>>>(tmw, tmb, p);
+  gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tmd, p);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
-  if (a.E > kMaxGroups || a.r > kMaxR || a.w_fp8) return cudaErrorInvalidValue;
+  if (a.E > kMaxGroups) return cudaErrorInvalidValue;
+  if (a.delta != nullptr && a.delta_cols % 8 != 0) return cudaErrorInvalidValue;
+  if (a.w_fp8) {
+    switch (a.bn) {
+      case 16: return launch_bn<16, true>(a, st);
+      case 32: return launch_bn<32, true>(a, st);
+      default: return launch_bn<64, true>(a, st);
+    }
+  }
   switch (a.bn) {
-    case 16: return launch_bn<16>(a, st);
-    case 32: return launch_bn<32>(a, st);
-    case 64: return launch_bn<64>(a, st);
-    case 128: return launch_bn<128>(a, st);
-    case 256: return launch_bn<256>(a, st);
+    case 16: return launch_bn<16, false>(a, st);
+    case 32: return launch_bn<32, false>(a, st);
+    case 64: return launch_bn<64, false>(a, st);
+    case 128: return launch_bn<128, false>(a, st);
+    case 256: return launch_bn<256, false>(a, st);
     default: return cudaErrorInvalidValue;
   }
 }

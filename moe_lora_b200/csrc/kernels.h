@@ -49,6 +49,27 @@ struct ShrinkArgs {
 };
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st);
 
+// Segmented LoRA for the GEMM epilogues: per segment, gather the source rows (optional),
+// shrink z = src . A^T, expand delta = z . B into an fp32 buffer that the GEMM epilogue
+// adds (rows without an adapter get delta = 0).  bf16 only; two kernel launches.
+struct LoraDeltaArgs {
+  const __nv_bfloat16* src;   // rows [*, K]
+  const int32_t* gather;      // if set: source row of output row s = gather[s] / gather_div
+  int gather_div;
+  __nv_bfloat16* gather_dst;  // if set: copy of the gathered source row
+  int nrows, K, r, NB;        // NB = delta features per row
+  const int32_t* seg_offsets; // [nseg+1]
+  int nseg;
+  const int32_t* seg_adapter; // dense: [nseg]; null: MoE key decode
+  int L, E;
+  const __nv_bfloat16* lora_a;  // MoE [L][E][r][K]; dense [L][r][K]
+  const __nv_bfloat16* lora_b;  // MoE [L][E][r][NB]; dense [L][r][NB]
+  float* z;                   // scratch [nrows][r] (shrink -> expand)
+  float* delta;               // [nrows][NB]
+  int* status;
+};
+cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st);
+
 // y[t] += z[t] . B_a(t) for dense segments (f32 or bf16 y and B).
 struct ExpandArgs {
   const float* z;
@@ -91,11 +112,10 @@ struct GemmArgs {
   int n_out;                   // output features per group (I for gate_up, H, h_out)
   int I;                       // gate_up: gate/up split
   int total_rows;              // rows of the B operand tensor
-  // LoRA expand in the epilogue
-  const float* z;              // [total_rows][r]
-  const int32_t* row_adapter;  // [total_rows]
-  const __nv_bfloat16* lora_b; // MoE [L][E][r][rows_per_group]; dense [L][r][h_out]
-  int r, L;
+  // LoRA delta added in the epilogue: [total_rows][delta_cols] fp32, column = weight row
+  // within the group (gate_up: gate rows [0, I), up rows [I, 2I)); null = no LoRA
+  const float* delta;
+  int delta_cols;
   // epilogue outputs
   __nv_bfloat16* out_bf16;     // gate_up: act [rows][I]; dense: y [T][h_out]
   float* out_f32;              // down: o [pairs][H] (weighted)

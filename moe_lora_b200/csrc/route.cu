@@ -51,6 +51,49 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16*
   }
 }
 
+// Small batches: one CTA per (expert, block of RS_TB tokens); the 256 threads split H
+// (128-bit loads, all independent), then a shuffle + shared-memory reduction.  Every
+// CTA reads its W_r row once; the grid has E * ceil(M / RS_TB) CTAs.
+constexpr int RS_TB = 16;
+
+__global__ void __launch_bounds__(256) router_logits_splith_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                   const __nv_bfloat16* __restrict__ wr,
+                                                                   const float* __restrict__ bias, int M,
+                                                                   int H, int E, float* __restrict__ logits) {
+  __shared__ float red[8][RS_TB];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x;
+  const int t0 = blockIdx.y * RS_TB;
+  const int nt = min(RS_TB, M - t0);
+  float acc[RS_TB];
+#pragma unroll
+  for (int i = 0; i < RS_TB; ++i) acc[i] = 0.f;
+  const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * H);
+  const int h8n = H >> 3;
+  for (int h8 = threadIdx.x; h8 < h8n; h8 += blockDim.x) {
+    const uint4 w8 = __ldg(wrow + h8);
+#pragma unroll
+    for (int i = 0; i < RS_TB; ++i) {
+      if (i < nt) {
+        const uint4 x8 = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + i) * H) + h8);
+        acc[i] += dot8_bf16(w8, x8);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RS_TB; ++i) {
+    const float v = warp_sum(acc[i]);
+    if (lane == 0) red[warp][i] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < nt) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w][threadIdx.x];
+    logits[static_cast<size_t>(t0 + threadIdx.x) * E + e] = s + (bias ? bias[e] : 0.f);
+  }
+}
+
 // ---------------------------------------------------------------- top-k + weights
 // One warp per token.  Each lane holds experts lane, lane+32, ... (E <= 256).
 // Selection: k rounds of a warp arg-max on (logit desc, expert asc).
@@ -220,9 +263,14 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   }
   const float* lg = a.logits_in;
   if (lg == nullptr) {
-    dim3 grid((a.M + RT_TB - 1) / RT_TB, (a.E + RT_EB - 1) / RT_EB);
     ProfScope ps(K_ROUTE_LOGITS, st);
-    router_logits_kernel<<<grid, 256, 0, st>>>(a.x, a.w_router, a.bias, a.M, a.H, a.E, a.logits);
+    if (a.M <= 256) {
+      dim3 grid(a.E, (a.M + RS_TB - 1) / RS_TB);
+      router_logits_splith_kernel<<<grid, 256, 0, st>>>(a.x, a.w_router, a.bias, a.M, a.H, a.E, a.logits);
+    } else {
+      dim3 grid((a.M + RT_TB - 1) / RT_TB, (a.E + RT_EB - 1) / RT_EB);
+      router_logits_kernel<<<grid, 256, 0, st>>>(a.x, a.w_router, a.bias, a.M, a.H, a.E, a.logits);
+    }
     count_launch();
     lg = a.logits;
   } else if (a.logits_out != nullptr) {

@@ -29,124 +29,348 @@ __device__ __forceinline__ int find_segment(const int32_t* off, int nseg, int s)
   return lo;
 }
 
+// One CTA per segment q (blockIdx.x < nseg) and row-chunk lane blockIdx.y: the CTA
+// handles chunks y, y + gridDim.y, ... of SH_RB rows of segment q, so the segment's
+// A slice is read from HBM once and then from L1/L2.  blockIdx.x == nseg handles the
+// rows no segment covers (only possible with offsets that do not span [0, nrows)):
+// no adapter, z = 0.
 template <bool F32>
 __global__ void __launch_bounds__(256) shrink_kernel(const ShrinkArgs a) {
-  __shared__ int s_seg[SH_RB];
   __shared__ int s_src[SH_RB];
-  __shared__ int s_ad[SH_RB];
-  __shared__ int s_e[SH_RB];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = blockIdx.x * a.rows_per_cta;
-  const int nr = min(a.rows_per_cta, a.nrows - row0);
-  if (nr <= 0) return;
-
-  // offsets sanity (strided over the grid): monotone, start 0, end nrows
-  for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < a.nseg; q += gridDim.x * blockDim.x)
-    if (a.seg_offsets[q] > a.seg_offsets[q + 1]) set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, q);
-  if (blockIdx.x == 0 && threadIdx.x == 0 &&
-      (a.seg_offsets[0] != 0 || a.seg_offsets[a.nseg] != a.nrows))
-    set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, -1);
-
-  if (threadIdx.x < nr) {
-    const int s = row0 + threadIdx.x;
-    const int q = find_segment(a.seg_offsets, a.nseg, s);
-    int ad = -1, e = 0;
-    if (q >= 0) {
-      if (a.seg_adapter != nullptr) {
-        ad = a.seg_adapter[q];
-      } else {
-        e = q / (a.L + 1);
-        const int ap = q - e * (a.L + 1);
-        ad = (ap == a.L) ? -1 : ap;
-      }
-      if (ad < -1 || ad >= a.L) {
-        set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, s);
-        ad = -1;
-      }
-    }
-    s_seg[threadIdx.x] = (ad >= 0) ? q : -1;
-    s_ad[threadIdx.x] = ad;
-    s_e[threadIdx.x] = e;
-    s_src[threadIdx.x] = a.gather ? a.gather[s] / a.gather_div : s;
-    if (a.row_adapter) a.row_adapter[s] = ad;
-  }
-  __syncthreads();
-
+  const int q = blockIdx.x;
   const size_t K = a.K;
-  if (a.gather_dst != nullptr) {  // bf16 rows, 16 B per thread
-    const int c16 = a.K / 8;
-    for (int idx = threadIdx.x; idx < nr * c16; idx += blockDim.x) {
-      const int i = idx / c16, c = idx - i * c16;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.src) +
-                                                           s_src[i] * K) + c);
-      reinterpret_cast<uint4*>(a.gather_dst + (row0 + i) * K)[c] = v;
-    }
+
+  if (blockIdx.y == 0) {  // offsets sanity, strided over the segments
+    if (threadIdx.x == 0 && q < a.nseg && a.seg_offsets[q] > a.seg_offsets[q + 1])
+      set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, q);
+    if (q == 0 && threadIdx.x == 0 && (a.seg_offsets[0] != 0 || a.seg_offsets[a.nseg] != a.nrows))
+      set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, -1);
   }
 
-  // runs of rows sharing one segment
-  int i0 = 0;
-  while (i0 < nr) {
-    int i1 = i0 + 1;
-    while (i1 < nr && s_seg[i1] == s_seg[i0]) ++i1;
-    const int n = i1 - i0;
-    const int ad = s_ad[i0];
+  int lo, hi, ad = -1, e = 0;
+  if (q < a.nseg) {
+    lo = a.seg_offsets[q];
+    hi = min(a.seg_offsets[q + 1], a.nrows);
+    lo = max(lo, 0);
+    if (a.seg_adapter != nullptr) {
+      ad = a.seg_adapter[q];
+    } else {
+      e = q / (a.L + 1);
+      const int ap = q - e * (a.L + 1);
+      ad = (ap == a.L) ? -1 : ap;
+    }
+    if (ad < -1 || ad >= a.L) {
+      if (threadIdx.x == 0 && blockIdx.y == 0) set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, q);
+      ad = -1;
+    }
+  } else {
+    lo = 0;  // uncovered rows: before the first offset and after the last
+    hi = a.nrows;
+  }
+  const int first = (q < a.nseg) ? lo : 0;
+  const int s_begin = a.seg_offsets[0], s_end = a.seg_offsets[a.nseg];
+  if (q == a.nseg && s_begin <= 0 && s_end >= a.nrows) return;  // every row is covered
+  const size_t abase = (ad >= 0) ? (static_cast<size_t>(ad) * a.E + e) * a.r * K : 0;
+
+  for (int c = blockIdx.y; first + c * SH_RB < hi; c += gridDim.y) {
+    const int r0 = first + c * SH_RB;
+    const int n = min(SH_RB, hi - r0);
+    __syncthreads();  // s_src of the previous chunk is no longer read
+    if (threadIdx.x < SH_RB) {
+      const int s = r0 + threadIdx.x;
+      int src = -1;
+      if (threadIdx.x < n) {
+        const bool mine = (q < a.nseg) || s < s_begin || s >= s_end;
+        if (mine) {
+          src = a.gather ? a.gather[s] / a.gather_div : s;
+          if (a.row_adapter) a.row_adapter[s] = ad;
+        }
+      }
+      s_src[threadIdx.x] = src;
+    }
+    __syncthreads();
+    if (a.gather_dst != nullptr) {  // bf16 rows, 16 B per thread
+      const int c16 = a.K / 8;
+      for (int idx = threadIdx.x; idx < n * c16; idx += blockDim.x) {
+        const int i = idx / c16, cc = idx - i * c16;
+        if (s_src[i] < 0) continue;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.src) +
+                                                             s_src[i] * K) + cc);
+        reinterpret_cast<uint4*>(a.gather_dst + (r0 + i) * K)[cc] = v;
+      }
+    }
     if (ad < 0) {
       for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x)
-        a.z[static_cast<size_t>(row0 + i0) * a.r + idx] = 0.f;
-    } else {
-      const size_t abase = (static_cast<size_t>(ad) * a.E + s_e[i0]) * a.r * K;
-      for (int i = warp; i < a.r; i += 8) {
-        float acc[SH_RB];
+        if (s_src[idx / a.r] >= 0) a.z[static_cast<size_t>(r0) * a.r + idx] = 0.f;
+      continue;
+    }
+    for (int i = warp; i < a.r; i += 8) {
+      float acc[SH_RB];
 #pragma unroll
-        for (int j = 0; j < SH_RB; ++j) acc[j] = 0.f;
-        if constexpr (F32) {
-          const float4* arow = reinterpret_cast<const float4*>(static_cast<const float*>(a.lora_a) + abase + i * K);
-          for (int c = lane; c < a.K / 4; c += 32) {
-            const float4 w4 = __ldg(arow + c);
+      for (int j = 0; j < SH_RB; ++j) acc[j] = 0.f;
+      if constexpr (F32) {
+        const float4* arow = reinterpret_cast<const float4*>(static_cast<const float*>(a.lora_a) + abase + i * K);
+        for (int cc = lane; cc < a.K / 4; cc += 32) {
+          const float4 w4 = __ldg(arow + cc);
 #pragma unroll
-            for (int j = 0; j < SH_RB; ++j) {
-              if (j < n) {
-                const float4 x4 = __ldg(reinterpret_cast<const float4*>(
-                                            static_cast<const float*>(a.src) + s_src[i0 + j] * K) + c);
-                acc[j] += w4.x * x4.x + w4.y * x4.y + w4.z * x4.z + w4.w * x4.w;
-              }
-            }
-          }
-        } else {
-          const uint4* arow = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.lora_a) + abase + i * K);
-          for (int c = lane; c < a.K / 8; c += 32) {
-            const uint4 w8 = __ldg(arow + c);
-#pragma unroll
-            for (int j = 0; j < SH_RB; ++j) {
-              if (j < n) {
-                const uint4 x8 = __ldg(reinterpret_cast<const uint4*>(
-                                           static_cast<const __nv_bfloat16*>(a.src) + s_src[i0 + j] * K) + c);
-                acc[j] += dot8_bf16(w8, x8);
-              }
+          for (int j = 0; j < SH_RB; ++j) {
+            if (j < n) {
+              const float4 x4 = __ldg(reinterpret_cast<const float4*>(
+                                          static_cast<const float*>(a.src) + s_src[j] * K) + cc);
+              acc[j] += w4.x * x4.x + w4.y * x4.y + w4.z * x4.z + w4.w * x4.w;
             }
           }
         }
+      } else {
+        const uint4* arow = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.lora_a) + abase + i * K);
+        for (int cc = lane; cc < a.K / 8; cc += 32) {
+          const uint4 w8 = __ldg(arow + cc);
 #pragma unroll
-        for (int j = 0; j < SH_RB; ++j) {
-          const float v = warp_sum(acc[j]);
-          if (lane == 0 && j < n) a.z[static_cast<size_t>(row0 + i0 + j) * a.r + i] = v;
+          for (int j = 0; j < SH_RB; ++j) {
+            if (j < n) {
+              const uint4 x8 = __ldg(reinterpret_cast<const uint4*>(
+                                         static_cast<const __nv_bfloat16*>(a.src) + s_src[j] * K) + cc);
+              acc[j] += dot8_bf16(w8, x8);
+            }
+          }
         }
       }
+#pragma unroll
+      for (int j = 0; j < SH_RB; ++j) {
+        const float v = warp_sum(acc[j]);
+        if (lane == 0 && j < n) a.z[static_cast<size_t>(r0 + j) * a.r + i] = v;
+      }
     }
-    i0 = i1;
   }
 }
 
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st) {
   if (a.nrows <= 0) return cudaSuccess;
-  const int rb = a.rows_per_cta < 1 ? 1 : (a.rows_per_cta > SH_RB ? SH_RB : a.rows_per_cta);
-  ShrinkArgs b = a;
-  b.rows_per_cta = rb;
-  const int grid = (a.nrows + rb - 1) / rb;
+  // spread long segments over a few CTAs; one CTA per segment at decode sizes
+  long long chunks = (a.nrows + SH_RB - 1) / SH_RB;
+  int ysplit = static_cast<int>(chunks / (a.nseg > 0 ? a.nseg : 1));
+  ysplit = ysplit < 1 ? 1 : (ysplit > 16 ? 16 : ysplit);
+  dim3 grid(a.nseg + 1, ysplit);
   ProfScope ps(K_SHRINK, st);
-  if (a.src_f32) shrink_kernel<true><<<grid, 256, 0, st>>>(b);
-  else shrink_kernel<false><<<grid, 256, 0, st>>>(b);
+  if (a.src_f32) shrink_kernel<true><<<grid, 256, 0, st>>>(a);
+  else shrink_kernel<false><<<grid, 256, 0, st>>>(a);
   count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- segmented LoRA for the GEMMs
+// Two streaming kernels per projection ([Punica review page], "提案手法": SGMV;
+// [vLLM MoE-LoRA page], "O Papel da Multi-LoRA": shrink z = xA then expand zB):
+//   lora_shrink_kernel  grid (segment, rank block of 8, row-chunk lane): warp w computes
+//                       z row i = 8 * block + w for the segment's rows, the whole K range
+//                       in flight (U 16-byte chunks per lane), reduced with shuffles
+//                       (split-K over the lanes, "Otimizações em Nível de Kernel");
+//                       rank block 0 also writes the gathered source rows
+//   lora_expand_kernel  grid (segment, feature block of 2048, row-chunk lane): each thread
+//                       owns 8 features and keeps 8-16 B rows in flight, then writes
+//                       delta = z B (fp32), which the GEMM epilogue adds to its output.
+// Segments without an adapter write delta = 0 (early exit of the LoRA work).
+constexpr int LD_RB = 8;      // rows per chunk
+constexpr int LD_FB = 2048;   // features per expand CTA (256 threads x 8)
+
+struct SegInfo {
+  int lo, hi, ad, e;
+};
+
+__device__ __forceinline__ SegInfo segment_info(const LoraDeltaArgs& a, int q, bool report) {
+  SegInfo si;
+  if (report && threadIdx.x == 0) {
+    if (a.seg_offsets[q] > a.seg_offsets[q + 1]) set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, q);
+    if (q == 0 && (a.seg_offsets[0] != 0 || a.seg_offsets[a.nseg] != a.nrows))
+      set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, -1);
+  }
+  si.lo = max(a.seg_offsets[q], 0);
+  si.hi = min(a.seg_offsets[q + 1], a.nrows);
+  si.e = 0;
+  if (a.seg_adapter != nullptr) {
+    si.ad = a.seg_adapter[q];
+  } else {
+    si.e = q / (a.L + 1);
+    const int ap = q - si.e * (a.L + 1);
+    si.ad = (ap == a.L) ? -1 : ap;
+  }
+  if (si.ad < -1 || si.ad >= a.L) {
+    if (report && threadIdx.x == 0) set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, q);
+    si.ad = -1;
+  }
+  return si;
+}
+
+// z[r0 + j][i] = src_j . arow for j < n; U chunks of every row in flight per lane.
+template <int RB, int U>
+__device__ __forceinline__ void shrink_warp(const LoraDeltaArgs& a, const __nv_bfloat16* arow, const int* s_src,
+                                            int n, int i, int r0, int lane) {
+  const size_t K = a.K;
+  const int k8 = a.K / 8;
+  float acc[RB];
+#pragma unroll
+  for (int j = 0; j < RB; ++j) acc[j] = 0.f;
+  const uint4* ap = reinterpret_cast<const uint4*>(arow);
+  const uint4* xp[RB];
+#pragma unroll
+  for (int j = 0; j < RB; ++j) xp[j] = reinterpret_cast<const uint4*>(a.src + s_src[j < n ? j : 0] * K);
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+  for (int base = 0; base < k8; base += 32 * U) {  // U chunks per lane in flight, tail predicated
+    uint4 w8[U], x8[U][RB];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int cc = base + lane + 32 * u;
+      const bool ok = cc < k8;
+      w8[u] = ok ? __ldg(ap + cc) : zero4;
+#pragma unroll
+      for (int j = 0; j < RB; ++j) x8[u][j] = ok ? __ldg(xp[j] + cc) : zero4;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < RB; ++j) acc[j] += dot8_bf16(w8[u], x8[u][j]);
+  }
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    const float v = warp_sum(acc[j]);
+    if (lane == 0 && j < n) a.z[static_cast<size_t>(r0 + j) * a.r + i] = v;
+  }
+}
+
+__global__ void __launch_bounds__(256) lora_shrink_kernel(const LoraDeltaArgs a) {
+  __shared__ int s_src[LD_RB];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SegInfo si = segment_info(a, blockIdx.x, blockIdx.y == 0 && blockIdx.z == 0);
+  const size_t K = a.K;
+  const int i = blockIdx.y * 8 + warp;
+  const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
+  const bool do_shrink = a.z != nullptr && si.ad >= 0 && i < a.r;
+  if (!do_gather && !(a.z != nullptr && si.ad >= 0)) return;
+  const __nv_bfloat16* arow =
+      a.lora_a + ((static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e) * a.r + (i < a.r ? i : 0)) * K;
+  for (int c = blockIdx.z; si.lo + c * LD_RB < si.hi; c += gridDim.z) {
+    const int r0 = si.lo + c * LD_RB;
+    const int n = min(LD_RB, si.hi - r0);
+    __syncthreads();
+    if (threadIdx.x < LD_RB)
+      s_src[threadIdx.x] = (threadIdx.x < n) ? (a.gather ? a.gather[r0 + threadIdx.x] / a.gather_div : r0 + threadIdx.x) : 0;
+    __syncthreads();
+    if (do_gather) {
+      const int c16 = a.K / 8;
+      for (int idx = threadIdx.x; idx < n * c16; idx += blockDim.x) {
+        const int j = idx / c16, cc = idx - j * c16;
+        reinterpret_cast<uint4*>(a.gather_dst + (r0 + j) * K)[cc] =
+            __ldg(reinterpret_cast<const uint4*>(a.src + s_src[j] * K) + cc);
+      }
+    }
+    if (do_shrink) {
+      if (n <= 1) shrink_warp<1, 8>(a, arow, s_src, n, i, r0, lane);
+      else if (n <= 2) shrink_warp<2, 4>(a, arow, s_src, n, i, r0, lane);
+      else if (n <= 4) shrink_warp<4, 2>(a, arow, s_src, n, i, r0, lane);
+      else shrink_warp<8, 1>(a, arow, s_src, n, i, r0, lane);
+    }
+  }
+}
+
+// delta[r0 + j][f..f+8) = sum_i z[j][i] B_i[f..f+8) for j < n; IB rows of B in flight.
+template <int RB, int IB>
+__device__ __forceinline__ void expand_thread(const LoraDeltaArgs& a, const __nv_bfloat16* bcol, const float* s_z,
+                                              int n, int r0, int f) {
+  float acc[RB][8];
+#pragma unroll
+  for (int j = 0; j < RB; ++j)
+#pragma unroll
+    for (int v = 0; v < 8; ++v) acc[j][v] = 0.f;
+  for (int i0 = 0; i0 < a.r; i0 += IB) {
+    uint4 b8[IB];
+#pragma unroll
+    for (int u = 0; u < IB; ++u) b8[u] = __ldg(reinterpret_cast<const uint4*>(bcol + static_cast<size_t>(i0 + u) * a.NB));
+#pragma unroll
+    for (int u = 0; u < IB; ++u) {
+      float bf[8];
+      unpack8_bf16(b8[u], bf);
+#pragma unroll
+      for (int j = 0; j < RB; ++j) {
+        const float zj = s_z[j * a.r + i0 + u];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[j][v] = fmaf(zj, bf[v], acc[j][v]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    if (j < n) {
+      float4* d = reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f);
+      d[0] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+      d[1] = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256, 2) lora_expand_kernel(const LoraDeltaArgs a) {
+  __shared__ float s_z[LD_RB * 128];
+  const SegInfo si = segment_info(a, blockIdx.x, false);
+  const int f = blockIdx.y * LD_FB + threadIdx.x * 8;
+  const __nv_bfloat16* bcol =
+      a.lora_b + (static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e) * a.r * a.NB + f;
+  for (int c = blockIdx.z; si.lo + c * LD_RB < si.hi; c += gridDim.z) {
+    const int r0 = si.lo + c * LD_RB;
+    const int n = min(LD_RB, si.hi - r0);
+    if (si.ad < 0) {
+      if (f < a.NB) {
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < n; ++j) {
+          float4* d = reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f);
+          d[0] = z4;
+          d[1] = z4;
+        }
+      }
+      continue;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x)
+      s_z[idx] = a.z[static_cast<size_t>(r0) * a.r + idx];
+    __syncthreads();
+    if (f < a.NB) {
+      const bool wide = (a.r % 16) == 0;
+      if (n <= 1) {
+        if (wide) expand_thread<1, 16>(a, bcol, s_z, n, r0, f);
+        else expand_thread<1, 8>(a, bcol, s_z, n, r0, f);
+      } else if (n <= 2) {
+        if (wide) expand_thread<2, 16>(a, bcol, s_z, n, r0, f);
+        else expand_thread<2, 8>(a, bcol, s_z, n, r0, f);
+      } else if (n <= 4) {
+        expand_thread<4, 8>(a, bcol, s_z, n, r0, f);
+      } else {
+        expand_thread<8, 8>(a, bcol, s_z, n, r0, f);
+      }
+    }
+  }
+}
+
+cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
+  if (a.nrows <= 0) return cudaSuccess;
+  if (a.r > 128 || a.r % 8 != 0 || a.NB % 8 != 0) return cudaErrorInvalidValue;
+  const bool lora = a.delta != nullptr && a.z != nullptr && a.r > 0;
+  if (!lora && a.gather_dst == nullptr) return cudaSuccess;  // nothing to do
+  const long long chunks = (a.nrows + LD_RB - 1) / LD_RB;
+  int zsplit = static_cast<int>(chunks / (a.nseg > 0 ? a.nseg : 1));
+  zsplit = zsplit < 1 ? 1 : (zsplit > 16 ? 16 : zsplit);
+  LoraDeltaArgs b = a;
+  if (!lora) b.z = nullptr;
+  {
+    dim3 grid(a.nseg, lora ? a.r / 8 : 1, zsplit);
+    ProfScope ps(K_SHRINK, st);
+    lora_shrink_kernel<<<grid, 256, 0, st>>>(b);
+    count_launch();
+  }
+  if (lora) {
+    dim3 grid(a.nseg, (a.NB + LD_FB - 1) / LD_FB, zsplit);
+    ProfScope ps(K_EXPAND, st);
+    lora_expand_kernel<<<grid, 256, 0, st>>>(a);
+    count_launch();
+  }
   return cudaGetLastError();
 }
 

@@ -92,3 +92,38 @@ def test_forward_moe_prefill_bf16_full_sampled(prefill_weights):
     res = run_moe_case(synth.MOE_PREFILL_BF16, M, weights=prefill_weights, tokens=toks)
     assert res["err"] <= TOL_BF16, res["err"]
     ml.check_status(res["rt"]["workspace"])
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) expert weights
+SMALL_FP8 = [
+    synth.MoEShape("f8_a", 220, E=8, k=2, H=384, I=192, L=3, r=16, wdtype="e4m3", no_adapter_frac=0.2),
+    synth.MoEShape("f8_ragged", 221, E=6, k=3, H=528, I=144, L=2, r=32, wdtype="e4m3", bias=True,
+                   adapter_dist="zipf", no_adapter_frac=0.25),
+    synth.MoEShape("f8_L0", 222, E=4, k=2, H=256, I=128, L=0, r=16, wdtype="e4m3"),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL_FP8, ids=lambda s: s.name)
+@pytest.mark.parametrize("M", [1, 5, 37, 200])
+def test_forward_fp8_small_shapes(shape, M):
+    res = run_moe_case(shape, M)
+    assert res["err"] <= TOL_FP8, res["err"]
+
+
+@pytest.mark.parametrize("bn", [16, 32, 64, 256])
+def test_forward_fp8_every_n_tile(bn, monkeypatch):
+    monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
+    res = run_moe_case(SMALL_FP8[1], 150)
+    assert res["err"] <= TOL_FP8, res["err"]
+
+
+@pytest.fixture(scope="module")
+def fp8_weights():
+    return moe_weights_both(synth.MOE_DECODE_FP8)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16, 64])
+def test_forward_moe_decode_fp8_full(fp8_weights, M):
+    res = run_moe_case(synth.MOE_DECODE_FP8, M, weights=fp8_weights)
+    assert res["err"] <= TOL_FP8, res["err"]
+    ml.check_status(res["rt"]["workspace"])
