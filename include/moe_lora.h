@@ -243,7 +243,8 @@ MOE_LORA_API const char* moe_lora_last_error(void);
  * records one event pair around each kernel launch of the library, on the launch's
  * stream, for up to n launches; n = 0 disables and frees the pool.  Kernel ids:
  *   0 router logits, 1 top-k, 2 sort, 3 SGMV shrink, 4 gate_up GEMM, 5 down GEMM,
- *   6 combine, 7 SGMV expand, 8 fp32 dense GEMM, 9 dense bf16 GEMM.
+ *   6 combine, 7 SGMV expand, 8 fp32 dense GEMM, 9 dense bf16 GEMM,
+ *   10 e4m3 activation planes.
  * moe_lora_profile_read() waits for the recorded events and returns the summed
  * device time (ms) and the number of recorded launches of one kernel id.
  * moe_lora_launch_count() counts every kernel launch of the library since load. */

@@ -24,7 +24,7 @@ EXPORTS = ("moe_lora_route", "moe_lora_forward", "sgmv_shrink", "sgmv_expand", "
            "moe_lora_profile_enable", "moe_lora_profile_read", "moe_lora_launch_count",
            "moe_lora_route_noalloc")
 KERNEL_IDS = {"router_logits": 0, "topk": 1, "sort": 2, "shrink": 3, "gemm_gateup": 4, "gemm_down": 5,
-              "combine": 6, "expand": 7, "dense_f32": 8, "gemm_dense": 9}
+              "combine": 6, "expand": 7, "dense_f32": 8, "gemm_dense": 9, "quant": 10}
 
 
 class MoELoRAError(RuntimeError):

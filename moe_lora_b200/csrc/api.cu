@@ -145,10 +145,13 @@ struct ForwardWs {
   float* delta_d;
   float* z;
   float* o;
+  uint8_t* q_hi;      // e4m3 weights: activation planes [M*k][max(H, I)]
+  uint8_t* q_lo;
+  float* q_scales;    // [M*k][2]
   size_t bytes;
 };
 
-ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r) {
+ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8) {
   const size_t mk = static_cast<size_t>(M) * k;
   size_t off = kStatusBytes;
   ForwardWs w{};
@@ -165,6 +168,10 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r) {
   w.delta_d = reinterpret_cast<float*>(take(r ? mk * H * 4 : 0));
   w.z = reinterpret_cast<float*>(take(mk * r * 4));
   w.o = reinterpret_cast<float*>(take(mk * H * 4));
+  const size_t kmax = H > I ? H : I;
+  w.q_hi = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
+  w.q_lo = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
+  w.q_scales = reinterpret_cast<float*>(take(fp8 ? mk * 2 * 4 : 0));
   w.bytes = off;
   return w;
 }
@@ -296,7 +303,7 @@ size_t moe_lora_workspace_size(int op, int M, int H, int I, int E, int k, int L,
   if (M < 0 || H < 0 || I < 0 || E < 0 || k < 0 || L < 0 || r < 0) return 0;
   switch (op) {
     case MOE_LORA_OP_ROUTE: return route_layout(nullptr, M, E, L).bytes;
-    case MOE_LORA_OP_FORWARD: return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0).bytes;
+    case MOE_LORA_OP_FORWARD: return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, true).bytes;
     case MOE_LORA_OP_SGMV_SHRINK:
     case MOE_LORA_OP_SGMV_EXPAND: return kStatusBytes;
     case MOE_LORA_OP_DENSE: {
@@ -393,7 +400,8 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   ML_REQUIRE(static_cast<long long>(M) * k <= (1 << 20), MOE_LORA_ERR_UNSUPPORTED, "M*k > 2^20");
   if (L > 0) ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
   const int rr = L > 0 ? r : 0;
-  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr);
+  const bool fp8 = w_dtype == ML_E4M3;
+  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr, fp8);
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (w_dtype == ML_E4M3) {
@@ -420,7 +428,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   if (!tensor_map_encode_available())
     return fail(MOE_LORA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr);
+  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8);
   const int mk = M * k;
   const int nkeys = E * (L + 1);
   ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
@@ -469,7 +477,13 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.w = w_gateup;
   g.b = w.x_sorted;
   g.bn = choose_bn(mk, E);
-  if (g.w_fp8 && g.bn > 64) g.bn = 64;  // the fp8 ring leaves room for N tiles up to 64
+  if (fp8) {
+    if (g.bn > 64) g.bn = 64;  // e4m3 tiles use the prefetching epilogue (N <= 64)
+    ML_CUDA(launch_quant_planes(w.x_sorted, mk, H, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
+    g.b_hi = w.q_hi;
+    g.b_lo = w.q_lo;
+    g.b_scales = w.q_scales;
+  }
   g.num_sms = num_sms();
   ML_CUDA(launch_gemm_tc(g, cs), "gate_up GEMM launch");
 
@@ -502,6 +516,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   d.scale_idx = 1;
   d.w = w_down;
   d.b = w.act;
+  if (fp8) ML_CUDA(launch_quant_planes(w.act, mk, I, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
   ML_CUDA(launch_gemm_tc(d, cs), "down GEMM launch");
 
   // 5. fixed-order combine over the k slots

@@ -11,22 +11,24 @@
 // with the matching 64 up rows so SiLU-and-mul is applied before act leaves the SM;
 // down tiles multiply by the routing weight and store one fp32 row per routing pair
 // for the fixed-order combine (expert aggregation, [SageMaker MoE kernels page],
-// second item).  FP8 (e4m3) expert weights stay one byte per weight in HBM and in the
-// TMA ring; converter warps widen them exactly to bf16 for the kind::f16 MMA and the
-// per-tensor scale is applied in the epilogue (same page, second item).
+// second item).  FP8 (e4m3) expert weights stay one byte per weight in HBM, in the TMA
+// ring and in the MMA: the activations are split exactly into two e4m3 planes
+// (hi = RNE(x / s), lo = RNE((x - hi s) / (s / 16)), per-row s), the kind::f8f6f4 MMA
+// runs once per plane into two TMEM accumulators, and the epilogue combines
+// s_w (s acc_hi + s/16 acc_lo) (per-tensor scale, [SageMaker MoE kernels page],
+// second item).
 //
 // Structure (one CTA per SM, persistent over a device-side tile list):
-//   warp 0      TMA producer: weight tile 128 x 64 per stage (two 64-row boxes; e4m3:
-//               128 x 128 bytes) and the token tile of the same K range
-//   warp 1      MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM),
-//               M = 128, N = BN, K = 16 per instruction; commits free the smem stage
+//   warp 0      TMA producer: weight tile 128 x 64 bf16 (or 128 x 128 e4m3) per stage as
+//               two 64-row boxes, and the token tile(s) of the same K range
+//   warp 1      MMA issuer: tcgen05.mma kind::f16 (bf16) or kind::f8f6f4 (e4m3),
+//               M = 128, N = BN; commits free the smem stage
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, + LoRA delta, activation,
 //               stores; two TMEM accumulators so the epilogue of tile i overlaps the
 //               MMAs of tile i+1
 //   warp 6      epilogue loader (N tiles <= 64): one tile ahead of the epilogue, TMA
-//               of the tile's LoRA delta and, for down, the pair ids and routing
-//               weights, into a two-slot shared-memory ring
-//   warps 7..10 (e4m3 weights) converters: fp8 weight tile -> bf16 stage
+//               of the tile's LoRA delta and the per-column data (pair ids, routing
+//               weights, activation plane scales) into a two-slot shared-memory ring
 // Every mbarrier wait is bounded; on expiry the CTA records MOE_LORA_ERR_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include "common.cuh"
@@ -64,17 +66,15 @@ struct TcParams {
   const float* w_scales;
   int scale_idx;
   int* status;
+  const float* b_scales;  // e4m3: [rows][2] = (s, s / 16) of the activation planes
   int m_tiles;
   int stages;
-  int stages8;
 };
 
 // Non-pipeline shared memory, placed after the stage rings.
 struct SmemCore {
   uint64_t full[16];
   uint64_t empty[16];
-  uint64_t full8[16];
-  uint64_t empty8[16];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t sfull[2];
@@ -95,22 +95,22 @@ struct EpiSlot {
   float delta[2 * BN * 64];
   int col_pair[BN];
   float col_w[BN];
+  float col_sh[BN];
+  float col_sl[BN];
 };
 
 template <int BN, bool W8>
 struct TileCfg {
-  static constexpr int kBTileBytes = BN * kBK * 2;           // one 64-K token sub-tile
-  // bf16 stage (K = 64): the A tile (+ the token tile for bf16 weights); fp8 stage
-  // (K = 128): the e4m3 weight tile and the two token sub-tiles of the same K range,
-  // converted into two consecutive bf16 stages
-  static constexpr int kStageBytes = W8 ? kATileBytes : kATileBytes + kBTileBytes;
-  static constexpr int kW8StageBytes = kBM * 128 + 2 * kBTileBytes;
+  static constexpr int kKB = W8 ? 128 : 64;                  // K per stage (128 bytes per row)
+  static constexpr int kBTileBytes = BN * 128;               // one token tile (or plane)
+  static constexpr int kStageBytes = kATileBytes + (W8 ? 2 : 1) * kBTileBytes;
   static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
-  static constexpr int kTmemCols = 2 * kAccStride;           // power of two >= 32
+  static constexpr int kAccPerBuf = W8 ? 2 : 1;              // e4m3: hi and lo accumulators
+  static constexpr int kTmemCols = 2 * kAccPerBuf * kAccStride;  // power of two >= 32
   static constexpr bool kPrefetch = BN <= 64;                // epilogue loader warp + slots
   static constexpr int kSlotBytes = kPrefetch ? static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024) : 0;
-  static constexpr int kConvWarp0 = 7;
-  static constexpr int kThreads = W8 ? 352 : 224;
+  static constexpr int kThreads = 224;
+  static_assert(!W8 || kPrefetch, "e4m3 weights use N tiles <= 64");
 };
 
 struct TileInfo {
@@ -133,24 +133,6 @@ __device__ __forceinline__ TileInfo decode_tile(const SmemCore& sm, int t, int m
   return ti;
 }
 
-// 16 e4m3 values -> 16 bf16 values, exactly (every e4m3 value is an f16 normal or zero).
-__device__ __forceinline__ void e4m3x16_to_bf16(uint4 q, uint4& lo, uint4& hi) {
-  const uint32_t in[4] = {q.x, q.y, q.z, q.w};
-  uint32_t out[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((in[i] >> (16 * h)) & 0xFFFFu);
-      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-      out[2 * i + h] = pack2_bf16(f.x, f.y);
-    }
-  }
-  lo = make_uint4(out[0], out[1], out[2], out[3]);
-  hi = make_uint4(out[4], out[5], out[6], out[7]);
-}
-
 // delta column (weight row within the group) of accumulator row m in tile column block f0
 __device__ __forceinline__ int delta_col(int epi, int m, int f0, int I) {
   if (epi == EPI_GATEUP) return (m < 64) ? f0 + m : I + f0 + (m - 64);
@@ -160,17 +142,16 @@ __device__ __forceinline__ int delta_col(int epi, int m, int f0, int I) {
 template <int BN, bool W8>
 __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
-                   const __grid_constant__ CUtensorMap tmd, const TcParams p) {
+                   const __grid_constant__ CUtensorMap tml, const __grid_constant__ CUtensorMap tmd,
+                   const TcParams p) {
   using Cfg = TileCfg<BN, W8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring8 = smem;                                              // fp8 weight stages
-  uint8_t* ring = smem + (W8 ? p.stages8 * Cfg::kW8StageBytes : 0);  // bf16 stages
-  uint8_t* slots = ring + p.stages * Cfg::kStageBytes;               // epilogue prefetch slots
+  uint8_t* ring = smem;                                 // stages: [A tile][token tile(s)]
+  uint8_t* slots = ring + p.stages * Cfg::kStageBytes;  // epilogue prefetch slots
   SmemCore& sm = *reinterpret_cast<SmemCore*>(slots + 2 * Cfg::kSlotBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
-  const int S8 = p.stages8;
   volatile int* abort_flag = &sm.abort_flag;
 
   // ---- setup: barriers, TMEM, tile list prefix
@@ -178,10 +159,6 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
-    }
-    for (int s = 0; s < S8; ++s) {
-      mbar_init(&sm.full8[s], 1);
-      mbar_init(&sm.empty8[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
@@ -196,6 +173,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmw);
     tma_prefetch_desc(&tmb);
+    if (W8) tma_prefetch_desc(&tml);
     if (p.delta != nullptr) tma_prefetch_desc(&tmd);
   }
   if (warp == 1) tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
@@ -237,15 +215,11 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
   const int total_tiles = sm.chunk_pref[p.E] * p.m_tiles;
-  const int nk8 = (p.K + 127) / 128;                  // fp8 stages per tile
-  const int nk = W8 ? 2 * nk8 : (p.K + kBK - 1) / kBK;  // bf16 stages per tile
+  const int nk = (p.K + Cfg::kKB - 1) / Cfg::kKB;  // stages per tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const int SR = W8 ? S8 : S;
-      uint64_t* fullb = W8 ? sm.full8 : sm.full;
-      uint64_t* emptyb = W8 ? sm.empty8 : sm.empty;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t filled_mask = 0, last_parity = 0;
@@ -259,26 +233,19 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           wrow0 = ti.g * p.rows_per_group + ti.mt * kBM;
           wrow1 = wrow0 + 64;
         }
-        for (int kb = 0; kb < (W8 ? nk8 : nk); ++kb) {
-          if (!mbar_wait(&emptyb[stage], phase ^ 1u, abort_flag, p.status, kWaitLimitNs, 1)) break;
-          if constexpr (W8) {
-            uint8_t* a8 = ring8 + stage * Cfg::kW8StageBytes;
-            mbar_arrive_expect_tx(&fullb[stage], Cfg::kW8StageBytes);
-            tma_load_2d(a8, &tmw, &fullb[stage], kb * 128, wrow0);
-            tma_load_2d(a8 + kBM * 64, &tmw, &fullb[stage], kb * 128, wrow1);
-            tma_load_2d(a8 + kBM * 128, &tmb, &fullb[stage], kb * 128, ti.row0);
-            tma_load_2d(a8 + kBM * 128 + Cfg::kBTileBytes, &tmb, &fullb[stage], kb * 128 + 64, ti.row0);
-          } else {
-            uint8_t* a_s = ring + stage * Cfg::kStageBytes;
-            uint8_t* b_s = a_s + kATileBytes;
-            mbar_arrive_expect_tx(&fullb[stage], Cfg::kStageBytes);
-            tma_load_2d(a_s, &tmw, &fullb[stage], kb * kBK, wrow0);
-            tma_load_2d(a_s + kATileBytes / 2, &tmw, &fullb[stage], kb * kBK, wrow1);
-            tma_load_2d(b_s, &tmb, &fullb[stage], kb * kBK, ti.row0);
-          }
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort_flag, p.status, kWaitLimitNs, 1)) break;
+          uint8_t* a_s = ring + stage * Cfg::kStageBytes;
+          uint8_t* b_s = a_s + kATileBytes;
+          const int kc = kb * Cfg::kKB;  // first K element of the stage
+          mbar_arrive_expect_tx(&sm.full[stage], Cfg::kStageBytes);
+          tma_load_2d(a_s, &tmw, &sm.full[stage], kc, wrow0);
+          tma_load_2d(a_s + kATileBytes / 2, &tmw, &sm.full[stage], kc, wrow1);
+          tma_load_2d(b_s, &tmb, &sm.full[stage], kc, ti.row0);
+          if constexpr (W8) tma_load_2d(b_s + Cfg::kBTileBytes, &tml, &sm.full[stage], kc, ti.row0);
           filled_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == SR) {
+          if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
@@ -286,55 +253,48 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       }
       if (*abort_flag) {
         // let our own copies land before the CTA exits
-        for (int s = 0; s < SR; ++s)
+        for (int s = 0; s < S; ++s)
           if (filled_mask & (1u << s)) {
             volatile int dummy = 0;
-            mbar_wait(&fullb[s], (last_parity >> s) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
+            mbar_wait(&sm.full[s], (last_parity >> s) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
           }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(kBM, BN);
-      int stage = 0, s8 = 0;
-      uint32_t phase = 0, ph8 = 0;
+      const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, BN) : umma_idesc_bf16(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
       int it = 0;
       for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(&sm.tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 2)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + buf * Cfg::kAccStride;
+        const uint32_t d_tmem = tmem_base + buf * Cfg::kAccPerBuf * Cfg::kAccStride;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          const int half = kb & 1;  // e4m3: which 64-wide half of the fp8 stage
-          bool got = true;
-          if constexpr (W8)
-            if (half == 0) got = mbar_wait(&sm.full8[s8], ph8, abort_flag, p.status, kWaitLimitNs, 9);
-          if (!got || !mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 3)) {
+          if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 3)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t st_addr = smem_u32(ring + stage * Cfg::kStageBytes);
-          const uint32_t b_addr = W8 ? smem_u32(ring8 + s8 * Cfg::kW8StageBytes + kBM * 128 + half * Cfg::kBTileBytes)
-                                     : st_addr + kATileBytes;
-          const uint64_t adesc = umma_desc_sw128(st_addr);
-          const uint64_t bdesc = umma_desc_sw128(b_addr);
+          const uint32_t a_addr = smem_u32(ring + stage * Cfg::kStageBytes);
+          const uint64_t adesc = umma_desc_sw128(a_addr);
+          const uint64_t bdesc = umma_desc_sw128(a_addr + kATileBytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
-          umma_commit(&sm.empty[stage]);
-          if constexpr (W8) {
-            if (half == 1) {
-              umma_commit(&sm.empty8[s8]);
-              if (++s8 == S8) {
-                s8 = 0;
-                ph8 ^= 1u;
-              }
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
+            const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
+            if constexpr (W8) {
+              const uint64_t ldesc = umma_desc_sw128(a_addr + kATileBytes + Cfg::kBTileBytes);
+              umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
+              umma_e4m3(d_tmem + Cfg::kAccStride, adesc + 2 * k, ldesc + 2 * k, idesc, acc);
+            } else {
+              umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
             }
           }
+          umma_commit(&sm.empty[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -389,9 +349,19 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           }
         }
         float v[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) + buf * Cfg::kAccStride + c0, v);
+        const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) +
+                               buf * Cfg::kAccPerBuf * Cfg::kAccStride + c0;
+        tmem_ld_32x32b_x32(t_acc, v);
+        if constexpr (W8) {
+          float vl[32];
+          tmem_ld_32x32b_x32(t_acc + Cfg::kAccStride, vl);
 #pragma unroll
-        for (int n = 0; n < 32; ++n) v[n] *= scale;
+          for (int n = 0; n < 32; ++n)
+            if (c0 + n < BN) v[n] = scale * (v[n] * slot->col_sh[c0 + n] + vl[n] * slot->col_sl[c0 + n]);
+        } else {
+#pragma unroll
+          for (int n = 0; n < 32; ++n) v[n] *= scale;
+        }
         if (p.delta != nullptr) {
           if constexpr (Cfg::kPrefetch) {
             const float* dl = slot->delta + ((m >> 6) * BN + c0) * 64 + (m & 63);
@@ -484,6 +454,13 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             slot->col_w[n] = n < ti.nvalid ? p.topk_w[pr] : 0.f;
           }
         }
+        if (W8) {
+          for (int n = lane; n < BN; n += 32) {
+            const bool v = n < ti.nvalid;
+            slot->col_sh[n] = v ? p.b_scales[2 * static_cast<size_t>(ti.row0 + n)] : 0.f;
+            slot->col_sl[n] = v ? p.b_scales[2 * static_cast<size_t>(ti.row0 + n) + 1] : 0.f;
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.sfull[buf]);
       }
@@ -493,52 +470,6 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             volatile int dummy = 0;
             mbar_wait(&sm.sfull[b], (issued_parity >> b) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
           }
-      }
-    }
-  } else if constexpr (W8) {
-    // ------------------------------------------------------------ fp8 -> bf16 converters
-    // Thread ct owns weight row ct of each stage: it reads the row's 128 e4m3 values from
-    // the fp8 stage (128-byte swizzled rows) and writes them as bf16 into the two 64-wide
-    // 128-byte-swizzled sub-tiles of the bf16 stage the MMA reads.  The token sub-tiles
-    // stay in the fp8 stage, loaded there by the producer.
-    const int ct = threadIdx.x - 32 * Cfg::kConvWarp0;
-    const int sw = ct & 7;
-    int s8 = 0, s16 = 0;
-    uint32_t ph8 = 0, ph16 = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-      for (int kb8 = 0; kb8 < nk8 && ok; ++kb8) {
-        const bool got8 = mbar_wait(&sm.full8[s8], ph8, abort_flag, p.status, kWaitLimitNs, 5);
-        const uint8_t* src = ring8 + s8 * Cfg::kW8StageBytes + ct * 128;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const bool got = got8 && mbar_wait(&sm.empty[s16], ph16 ^ 1u, abort_flag, p.status, kWaitLimitNs, 6);
-          if (!named_bar_and(3, 128, got)) {
-            ok = false;
-            break;
-          }
-          uint8_t* dst = ring + s16 * Cfg::kStageBytes + ct * 128;
-#pragma unroll
-          for (int c = 4 * half; c < 4 * half + 4; ++c) {
-            const uint4 q = *reinterpret_cast<const uint4*>(src + ((c ^ sw) << 4));
-            uint4 lo, hi;
-            e4m3x16_to_bf16(q, lo, hi);
-            const int cc = (c & 3) * 2;
-            *reinterpret_cast<uint4*>(dst + ((cc ^ sw) << 4)) = lo;
-            *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ sw) << 4)) = hi;
-          }
-          fence_proxy_async_smem();
-          named_bar_sync(3, 128);
-          if (ct == 0) mbar_arrive(&sm.full[s16]);  // the fp8 stage is released by the MMA
-          if (++s16 == S) {
-            s16 = 0;
-            ph16 ^= 1u;
-          }
-        }
-        if (++s8 == S8) {
-          s8 = 0;
-          ph8 ^= 1u;
-        }
       }
     }
   }
@@ -583,23 +514,10 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   using Cfg = TileCfg<BN, W8>;
   const int fixed = static_cast<int>(sizeof(SmemCore)) + 2 * Cfg::kSlotBytes;
   const int budget = 232448 - 1024 - fixed;
-  int stages, stages8 = 0;
-  if (W8) {
-    stages = 4;
-    stages8 = (budget - stages * Cfg::kStageBytes) / Cfg::kW8StageBytes;
-    stages8 = stages8 > 8 ? 8 : stages8;
-    if (stages8 < 2) {
-      stages = 2;
-      stages8 = (budget - stages * Cfg::kStageBytes) / Cfg::kW8StageBytes;
-    }
-    if (stages8 < 2) return cudaErrorInvalidConfiguration;
-  } else {
-    stages = budget / Cfg::kStageBytes;
-    stages = stages > 8 ? 8 : stages;
-    if (stages < 2) return cudaErrorInvalidConfiguration;
-  }
-  const size_t smem = 1024 + static_cast<size_t>(stages) * Cfg::kStageBytes +
-                      static_cast<size_t>(stages8) * Cfg::kW8StageBytes + fixed;
+  int stages = budget / Cfg::kStageBytes;
+  stages = stages > 8 ? 8 : stages;
+  if (stages < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = 1024 + static_cast<size_t>(stages) * Cfg::kStageBytes + fixed;
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   static bool attr_set = false;
   if (!attr_set) {
@@ -608,19 +526,24 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  CUtensorMap tmw, tmb, tmd;
+  CUtensorMap tmw, tmb, tml, tmd;
   const uint64_t wrows = static_cast<uint64_t>(a.E) * a.rows_per_group;
-  CUresult cr;
-  if (W8)
-    cr = encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, a.K, wrows, static_cast<uint64_t>(a.K), 128, 64,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
-  else
-    cr = encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2,
-                        kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
-                     static_cast<uint64_t>(a.K) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  if (W8) {
+    if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, a.K, wrows, static_cast<uint64_t>(a.K), 128, 64,
+                       CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+        encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_hi, a.K, a.total_rows, static_cast<uint64_t>(a.K),
+                       128, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+        encode_tmap_2d(&tml, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.b_lo, a.K, a.total_rows, static_cast<uint64_t>(a.K),
+                       128, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2, kBK,
+                       64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+        encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
+                       static_cast<uint64_t>(a.K) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    tml = tmb;  // unused
+  }
   if (a.delta != nullptr && Cfg::kPrefetch) {
     if (encode_tmap_2d(&tmd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.delta, a.delta_cols, a.total_rows,
                        static_cast<uint64_t>(a.delta_cols) * 4, 64, BN, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
@@ -646,16 +569,16 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.w_scales = a.w_scales;
   p.scale_idx = a.scale_idx;
   p.status = a.status;
+  p.b_scales = a.b_scales;
   p.m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
   p.stages = stages;
-  p.stages8 = stages8;
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
   const long long tiles_ub = chunks_ub * p.m_tiles;
   int grid = a.num_sms;
   if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
   if (grid < 1) grid = 1;
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP : (a.epi == EPI_DOWN ? K_GEMM_DOWN : K_GEMM_DENSE), st);
-  gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tmd, p);
+  gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, p);
   count_launch();
   return cudaGetLastError();
 }
@@ -664,6 +587,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
   if (a.E > kMaxGroups) return cudaErrorInvalidValue;
   if (a.delta != nullptr && a.delta_cols % 8 != 0) return cudaErrorInvalidValue;
   if (a.w_fp8) {
+    if (a.b_hi == nullptr || a.b_lo == nullptr || a.b_scales == nullptr) return cudaErrorInvalidValue;
     switch (a.bn) {
       case 16: return launch_bn<16, true>(a, st);
       case 32: return launch_bn<32, true>(a, st);

@@ -126,11 +126,19 @@ struct GemmArgs {
   int* status;
   // operands
   const void* w;               // weights [E*rows_per_group][K]
-  const __nv_bfloat16* b;      // B operand rows [total_rows][K]
+  const __nv_bfloat16* b;      // bf16 weights: token rows [total_rows][K]
+  const uint8_t* b_hi;         // e4m3 weights: token rows as two e4m3 planes [total_rows][K]
+  const uint8_t* b_lo;
+  const float* b_scales;       // [total_rows][2] = (s, s / 16)
   int bn;                      // N tile (16..256)
   int num_sms;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
+
+// Rows of bf16 values as two e4m3 planes: hi = RNE(x / s), lo = RNE((x - hi s) / (s / 16)),
+// s = amax(row) / 448; scales[row] = (s, s / 16).
+cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8_t* hi, uint8_t* lo, float* scales,
+                                cudaStream_t st);
 
 // y[t] = sum_j o[t*k + j]  (o already weighted), fixed j order, bf16 out.
 cudaError_t launch_combine(const float* o, int M, int k, int H, __nv_bfloat16* y, cudaStream_t st);

@@ -18,7 +18,8 @@ enum KernelId : int {
   K_EXPAND = 7,
   K_DENSE_F32 = 8,
   K_GEMM_DENSE = 9,
-  K_COUNT = 10
+  K_QUANT = 10,
+  K_COUNT = 11
 };
 
 void prof_begin(int id, cudaStream_t st);

@@ -512,6 +512,73 @@ cudaError_t launch_dense_f32(const DenseF32Args& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- e4m3 activation planes
+// One warp per row: s = amax(|x|) / 448 (1 for an all-zero row); hi = RNE_sat(x / s) and
+// lo = RNE_sat((x - hi s) / (s / 16)) in OCP e4m3, so that x = s hi + (s / 16) lo up to a
+// relative 2^-8; the FP8-weight GEMM multiplies both planes on the kind::f8f6f4 tensor
+// core.  |x / s| <= 448 and |(x - hi s) / (s / 16)| <= 448 by construction.
+__global__ void __launch_bounds__(256) quant_planes_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K,
+                                                          uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
+                                                          float* __restrict__ scales) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k8 = K / 8;
+  for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
+    const uint4* xr = reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * K);
+    float amax = 0.f;
+    for (int c = lane; c < k8; c += 32) {
+      float f[8];
+      unpack8_bf16(__ldg(xr + c), f);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) amax = fmaxf(amax, fabsf(f[v]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = amax > 0.f ? amax / 448.f : 1.f;
+    const float inv = 1.f / s, inv_lo = 16.f / s;
+    for (int c = lane; c < k8; c += 32) {
+      float f[8];
+      unpack8_bf16(__ldg(xr + c), f);
+      uint32_t hq[2], lq[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t hw = 0, lw = 0;
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+          const int v = 4 * h + 2 * pr;
+          const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(make_float2(f[v] * inv, f[v + 1] * inv),
+                                                                  __NV_SATFINITE, __NV_E4M3);
+          const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
+          const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+          const __nv_fp8x2_storage_t ql = __nv_cvt_float2_to_fp8x2(
+              make_float2((f[v] - d.x * s) * inv_lo, (f[v + 1] - d.y * s) * inv_lo), __NV_SATFINITE, __NV_E4M3);
+          hw |= static_cast<uint32_t>(q) << (16 * pr);
+          lw |= static_cast<uint32_t>(ql) << (16 * pr);
+        }
+        hq[h] = hw;
+        lq[h] = lw;
+      }
+      reinterpret_cast<uint2*>(hi + static_cast<size_t>(row) * K)[c] = make_uint2(hq[0], hq[1]);
+      reinterpret_cast<uint2*>(lo + static_cast<size_t>(row) * K)[c] = make_uint2(lq[0], lq[1]);
+    }
+    if (lane == 0) {
+      scales[2 * static_cast<size_t>(row)] = s;
+      scales[2 * static_cast<size_t>(row) + 1] = s / 16.f;
+    }
+  }
+}
+
+cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8_t* hi, uint8_t* lo, float* scales,
+                                cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (K % 16 != 0) return cudaErrorInvalidValue;
+  int grid = (rows + 7) / 8;
+  if (grid > 148 * 8) grid = 148 * 8;
+  ProfScope ps(K_QUANT, st);
+  quant_planes_kernel<<<grid, 256, 0, st>>>(src, rows, K, hi, lo, scales);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- top-k combine
 // y[t, :] = sum_{j=0..k-1} o[t*k + j, :], summed in j order (run-to-run identical).
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o, int M, int k, int H,
