@@ -3,10 +3,11 @@
 
 One step = one pass of the whole path over one batch resident in HBM:
   moe_lora_route   router logits x W_r^T, softmax top-k + renormalised weights,
-                   stable (expert, adapter) sort into segments
-  moe_lora_forward gather + gate_up LoRA shrink, tcgen05 gate_up GEMM with the LoRA
-                   expand and SiLU-and-mul fused in its epilogue, down LoRA shrink,
-                   tcgen05 down GEMM with expand and routing weight, fixed-order combine
+                   stable (expert, adapter) sort into segments (one launch at decode)
+  moe_lora_forward gather + gate_up LoRA shrink, tcgen05 gate_up GEMM running the LoRA
+                   expand as extra MMA K steps and SiLU-and-mul in its epilogue, down
+                   LoRA shrink, tcgen05 down GEMM with the expand and the routing weight,
+                   fixed-order combine
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--M M]
     python bench.py --impl reference ...      (the fp64 CPU oracle, same metric)
@@ -76,7 +77,7 @@ def dist_setup():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    else:
+    elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
 
@@ -164,11 +165,19 @@ def routing_stats(rt: dict, shape: synth.MoEShape):
 
 def gateup_alg_bytes(shape, M, experts, pairs):
     """Bytes the gate_up GEMM must move once: touched expert gate_up weights, the
-    gathered x rows, the LoRA delta it adds (fp32, 2I per row) and the act it writes."""
+    gathered x rows (bf16, or two e4m3 planes and their scales), the z rows and the
+    touched B_gu slices of the LoRA expand it runs, and the act it writes."""
     wb = 1 if shape.wdtype == "e4m3" else 2
     mk = M * shape.k
-    return (experts * 2 * shape.I * shape.H * wb + mk * shape.H * 2 + mk * 2 * shape.I * 4
-            + mk * shape.I * 2)
+    xb = mk * (2 * shape.H + 8) if shape.wdtype == "e4m3" else mk * shape.H * 2
+    return (experts * 2 * shape.I * shape.H * wb + xb + mk * shape.r * 2
+            + pairs * shape.r * 2 * shape.I * 2 + mk * shape.I * 2)
+
+
+def gateup_alg_flops(shape, M):
+    """gate_up base GEMM plus its fused LoRA expand."""
+    mk = M * shape.k
+    return 2 * mk * 2 * shape.I * shape.H + 2 * mk * shape.r * 2 * shape.I
 
 
 def layer_alg_bytes(shape, M, experts, pairs):
@@ -236,7 +245,17 @@ def reference_arm(args, world, rank):
         return
     shape = synth.WORKLOADS[args.workload]
     if not isinstance(shape, synth.MoEShape):
-        print(json.dumps({"impl": "reference", "unavailable": "reference arm covers the MoE workloads only"}))
+        dense_oracle_tokens_per_s(shape, seconds=0.0, max_calls=max(1, args.warmup))
+        tps, calls, n, el = dense_oracle_tokens_per_s(shape, seconds=1e9, max_calls=args.steps)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / calls, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": shape.name, "T": shape.T, "h_in": shape.h_in, "h_out": shape.h_out,
+                       "L": shape.L, "r": shape.r},
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{n} tokens per step, {calls} steps, {el:.1f} s"},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
         return
     M = args.M
     cpu = synth.moe_weights(shape, device="cpu")
@@ -263,53 +282,166 @@ def reference_arm(args, world, rank):
 
 # ----------------------------------------------------------------------------- dense SGMV arm
 
+def dense_oracle_tokens_per_s(shape: synth.DenseShape, seconds: float, max_calls: int | None = None):
+    """The fp64 oracle of one dense multi-LoRA projection on the bench's token batch,
+    repeated until `seconds` of CPU time (or `max_calls`); weights decoded once, like a
+    model load.  Returns (tokens/s, calls, tokens/call, elapsed s)."""
+    from oracle import formats
+    from oracle import moe_lora_ref as ref
+    x, _, offs, segs = synth.dense_tokens(shape)
+    w = synth.dense_weights(shape)
+    f = lambda t: formats.to_f64(synth.bits(t), shape.dtype)  # noqa: E731
+    x64, w64, a64, b64 = f(x), f(w["w"]), f(w["a"]), f(w["b"])
+    so, sa = offs.numpy(), segs.numpy()
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        ref.dense_lora_forward(x64, w64, a64, b64, so, sa)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_calls is not None and calls >= max_calls):
+            break
+    return shape.T * calls / el, calls, shape.T, el
+
+
 def run_dense(args, shape: synth.DenseShape, world, rank, local):
     """One dense projection with segmented multi-LoRA (dense_lora_forward).  Its weight
-    fits in L2, so every timed step is preceded by an L2 flush outside the timed events."""
+    fits in L2, so the steps cycle over enough copies of the weights and adapters that
+    the copy a step reads was evicted by the steps before it (inputs larger than L2)."""
     import moe_lora_b200 as ml
     dev = torch.device("cuda", local)
     T = shape.T
     x, tok_a, offs, segs = synth.dense_tokens(shape)
-    w = synth.dense_weights(shape, device=dev)
+    w0 = synth.dense_weights(shape, device=dev)
     x, offs, segs = x.to(dev), offs.to(dev), segs.to(dev)
+    eb = 2 if shape.dtype == "bf16" else 4
+    copy_bytes = sum(t.numel() for t in w0.values()) * eb
+    n_copies = int(min(512, -(-3 * L2_BYTES // copy_bytes) + 1))
+    copies = [w0] + [{kk: v.clone() for kk, v in w0.items()} for _ in range(n_copies - 1)]
     ws = ml.new_workspace(ml.workspace_size(ml.OP_DENSE, T, shape.h_in, shape.h_out, 1, 1, shape.L, shape.r), dev)
     y = torch.empty((T, shape.h_out), dtype=x.dtype, device=dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    def step():
-        ml.dense_lora_forward(x, w["w"], w["a"], w["b"], offs, segs, y=y, workspace=ws)
+    def step(i, xin=x):
+        w = copies[i % n_copies]
+        ml.dense_lora_forward(xin, w["w"], w["a"], w["b"], offs, segs, y=y, workspace=ws)
 
-    for _ in range(args.warmup):
-        step()
+    for i in range(max(args.warmup, n_copies)):
+        step(i)
     torch.cuda.synchronize()
-    ml.profile_enable(args.steps * 4 + 16)
+    ml.check_status(ws)
+
+    n0 = ml.launch_count()
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
+    launches = ml.launch_count() - n0
+
+    # ---- per-kernel device times: one step per weight copy captured as a CUDA graph
+    #      with event nodes around every launch, replayed; the last replay is read
+    if not args.no_graph:
+        gs = torch.cuda.Stream()
+        gs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(gs):
+            step(0)
+        torch.cuda.current_stream().wait_stream(gs)
+        torch.cuda.synchronize()
+        ml.profile_enable(n_copies * 4 + 16)
+        pgraphs = []
+        for c in range(n_copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(c)
+            pgraphs.append(g)
+        for _ in range(3):
+            for g in pgraphs:
+                g.replay()
+        torch.cuda.synchronize()
+        prof_steps = n_copies
+    else:
+        ml.profile_enable(args.steps * 4 + 16)
+        for i in range(args.steps):
+            step(i)
+        torch.cuda.synchronize()
+        prof_steps = args.steps
+    gemm_ms, gemm_n = ml.profile_read("gemm_dense" if shape.dtype == "bf16" else "dense_f32")
+    per_kernel = {k: ml.profile_read(k)[0] / prof_steps for k in ("lora", "shrink", "gemm_dense", "dense_f32")}
+    ml.profile_enable(0)
+    if not args.no_graph:
+        del pgraphs
+
+    # ---- one CUDA graph per weight copy
+    graphs = []
+    if not args.no_graph:
+        for c in range(n_copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(c)
+            graphs.append(g)
+        for i in range(max(args.warmup, n_copies)):
+            graphs[i % n_copies].replay()
+        torch.cuda.synchronize()
+
+    def run_step(i):
+        if graphs:
+            graphs[i % n_copies].replay()
+        else:
+            step(i)
+
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.25)
     barrier(world)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    n0 = ml.launch_count()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
     for i in range(args.steps):
-        flush.fill_(float(i))  # evict the weight from L2 (outside the timed events)
-        evs[i][0].record()
-        step()
-        evs[i][1].record()
+        run_step(i)
+    ev1.record()
     torch.cuda.synchronize()
     barrier(world)
-    launches = ml.launch_count() - n0
     clk = clocks.stop()
-    ms = sum(a.elapsed_time(b) for a, b in evs)
-    gemm_ms, gemm_n = ml.profile_read("gemm_dense" if shape.dtype == "bf16" else "dense_f32")
-    per_kernel = {k: ml.profile_read(k)[0] / args.steps for k in ("shrink", "expand", "gemm_dense", "dense_f32")}
-    ml.profile_enable(0)
-    ml.check_status(ws)
-    ms_max = max_over_ranks(ms, world)
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world)
     value = world * T * args.steps / (ms_max / 1e3)
-    eb = 2 if shape.dtype == "bf16" else 4
+
+    # ---- e2e: pinned host x -> device, dense_lora_forward, y -> pinned host, every step
+    e2e_steps = args.e2e_steps or args.steps
+    hx = x.cpu().pin_memory()
+    hy = torch.empty((T, shape.h_out), dtype=x.dtype).pin_memory()
+    dx = torch.empty_like(x)
+
+    def e2e_step(i):
+        dx.copy_(hx, non_blocking=True)
+        step(i, dx)
+        hy.copy_(y, non_blocking=True)
+
+    e2e_graphs = []
+    if not args.no_graph:
+        for c in range(n_copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                e2e_step(c)
+            e2e_graphs.append(g)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        if e2e_graphs:
+            e2e_graphs[i % n_copies].replay()
+        else:
+            e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    del graphs, e2e_graphs
+    ml.check_status(ws)
+
     adapters = sorted(set(int(v) for v in tok_a.tolist() if v >= 0))
     lay_bytes = (shape.h_out * shape.h_in + len(adapters) * shape.r * (shape.h_in + shape.h_out)) * eb \
         + T * (shape.h_in + shape.h_out) * eb
-    gemm_bytes = shape.h_out * shape.h_in * eb + T * shape.h_in * eb + T * shape.h_out * (eb + 4)
+    gemm_bytes = shape.h_out * shape.h_in * eb + T * shape.h_in * eb + T * shape.h_out * eb
+    if shape.dtype == "bf16":  # the fused expand: z rows and the touched B slices
+        gemm_bytes += T * shape.r * 2 + len(adapters) * shape.r * shape.h_out * 2
     peaks, peak_src = load_peaks()
     peak = float(peaks["hbm_gbs"])
     g_s = (gemm_ms / max(gemm_n, 1)) / 1e3
@@ -320,16 +452,29 @@ def run_dense(args, shape: synth.DenseShape, world, rank, local):
         "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
         "config": {"workload": shape.name, "T": T, "h_in": shape.h_in, "h_out": shape.h_out, "L": shape.L,
                    "r": shape.r, "adapters": shape.adapter_dist, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every timed step (256 MB write outside the timed events)"},
+                   "l2": f"inputs larger than L2: steps cycle over {n_copies} copies of W, A and B "
+                         f"({n_copies * copy_bytes / 1e6:.0f} MB)"},
         "roofline": {"bound": "hbm", "kernel": "gemm_tc (dense)" if shape.dtype == "bf16" else "dense_f32",
                      "achieved": gemm_bytes / g_s / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": gemm_bytes / g_s / 1e9 / peak, "peak_source": peak_src, "traffic": None,
                      "alg_bytes_per_launch": gemm_bytes, "avg_launch_us": g_s * 1e6},
         "layer": {"alg_bytes_per_step": lay_bytes, "achieved_GBps": lay_bytes / step_s / 1e9,
                   "frac_of_hbm_peak": lay_bytes / step_s / 1e9 / peak,
-                  "kernel_ms_per_step": per_kernel},
+                  "kernel_ms_per_step": per_kernel,
+                  "kernel_times": "CUDA events around each launch inside the replayed step graphs"
+                  if not args.no_graph else "CUDA events around each launch of plain API calls"},
+        "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * shape.h_in * eb, "d2h_bytes_per_step": T * shape.h_out * eb,
+                "how": "graph replay of H2D copy, dense_lora_forward, D2H copy" if not args.no_graph
+                else "plain API calls"},
+        "timing": {"mode": "CUDA graph replay of the API call" if not args.no_graph else "plain API calls"},
         "gpu_launches": launches, "clocks": clk,
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, calls, n, el = dense_oracle_tokens_per_s(shape, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"fp64 oracle, {n} tokens per call, {calls} calls in {el:.1f} s; "
+                                          "weights decoded to fp64 once before timing"}
     if rank == 0:
         print(json.dumps(line))
 
@@ -363,7 +508,8 @@ def main():
         x, ad = synth.moe_tokens(shape, M, batch=b)
         batches.append((x.to(dev), ad.to(dev)))
     rws = ml.new_workspace(ml.workspace_size(ml.OP_ROUTE, M, shape.H, 0, shape.E, k, L, 0), dev)
-    fws = ml.new_workspace(ml.workspace_size(ml.OP_FORWARD, M, shape.H, shape.I, shape.E, k, L, shape.r), dev)
+    fop = ml.OP_FORWARD_E4M3 if shape.wdtype == "e4m3" else ml.OP_FORWARD_BF16
+    fws = ml.new_workspace(ml.workspace_size(fop, M, shape.H, shape.I, shape.E, k, L, shape.r), dev)
     rbufs = {"topk_ids": torch.empty((M, k), dtype=torch.int32, device=dev),
              "topk_w": torch.empty((M, k), dtype=torch.float32, device=dev),
              "sorted_pairs": torch.empty((M * k,), dtype=torch.int32, device=dev),
@@ -387,10 +533,7 @@ def main():
         step(i)
     torch.cuda.synchronize()
 
-    # ---- per-kernel device times: plain API calls, CUDA events around every launch
-    launches_per_step = 16  # upper bound of library launches per step
-    ml.profile_enable(args.steps * launches_per_step + 64)
-    torch.cuda.synchronize()
+    # ---- plain API calls (host enqueue included), for reference
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n0 = ml.launch_count()
     p0.record()
@@ -398,12 +541,45 @@ def main():
         step(i)
     p1.record()
     torch.cuda.synchronize()
-    launches = ml.launch_count() - n0
+    launches_per_step = (ml.launch_count() - n0) / args.steps
     plain_ms = p0.elapsed_time(p1)
-    gu_ms, gu_n = ml.profile_read("gemm_gateup")
-    per_kernel = {kname: ml.profile_read(kname) for kname in ("router_logits", "topk", "sort", "shrink",
-                                                            "expand", "gemm_gateup", "gemm_down", "combine")}
+
+    # ---- per-kernel device times: each batch's step captured as a CUDA graph with an
+    #      event pair around every launch (event nodes), replayed; the last replay of
+    #      every graph is read.  Without graphs: plain calls (host gaps included).
+    names = ("route", "router_logits", "topk", "sort", "lora", "quant", "gemm_gateup", "gemm_down", "combine")
+    if not args.no_graph:
+        gs = torch.cuda.Stream()
+        gs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(gs):
+            for b in range(len(batches)):
+                step(b)  # warm the stream before capture
+        torch.cuda.current_stream().wait_stream(gs)
+        torch.cuda.synchronize()
+        ml.profile_enable(len(batches) * 16 + 64)
+        pgraphs = []
+        for b in range(len(batches)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(b)
+            pgraphs.append(g)
+        for _ in range(5):
+            for g in pgraphs:
+                g.replay()
+        torch.cuda.synchronize()
+        prof_steps = len(batches)
+    else:
+        ml.profile_enable(args.steps * 16 + 64)
+        for i in range(args.steps):
+            step(i)
+        torch.cuda.synchronize()
+        prof_steps = args.steps
+    per_kernel = {kname: ml.profile_read(kname) for kname in names}
     ml.profile_enable(0)
+    if not args.no_graph:
+        del pgraphs
+    gu_ms, gu_n = per_kernel["gemm_gateup"]
+    launches = int(round(launches_per_step * args.steps))
 
     # ---- the step as a CUDA graph of the same API calls (one graph per token batch)
     graphs = []
@@ -496,7 +672,12 @@ def main():
     gu_bytes = mean(lambda e, p: gateup_alg_bytes(shape, M, e, p))
     lay_bytes = mean(lambda e, p: layer_alg_bytes(shape, M, e, p))
     gu_avg_s = (gu_ms / max(gu_n, 1)) / 1e3
-    achieved = gu_bytes / gu_avg_s / 1e9
+    tensor_bound = M * k >= 128 * shape.E  # >= 128 rows per expert: the MMA, not HBM, bounds gate_up
+    if tensor_bound:
+        achieved = gateup_alg_flops(shape, M) / gu_avg_s / 1e12
+        peak_t = float(peaks["bf16_tflops_sustained"]) * (2.0 if shape.wdtype == "e4m3" else 1.0)
+    else:
+        achieved = gu_bytes / gu_avg_s / 1e9
     peak = float(peaks["hbm_gbs"])
     traffic = (NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["gemm_tc.cu"] == src_hash("gemm_tc.cu")
                and NCU_TRAFFIC["workload"] == shape.name and NCU_TRAFFIC["M"] == M else None)
@@ -512,14 +693,23 @@ def main():
                    "adapters": shape.adapter_dist, "parallelism": f"replicas x{world}",
                    "l2": f"no flush: {lay_bytes / 1e9:.2f} GB of weights per step > 126 MB L2; "
                          f"{n_b} rotating token batches"},
-        "roofline": {"bound": "hbm", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src,
-                     "traffic": traffic, "alg_bytes_per_launch": gu_bytes,
-                     "avg_launch_us": gu_avg_s * 1e6},
+        "roofline": ({"bound": "hbm", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved, "peak": peak,
+                      "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src,
+                      "traffic": traffic, "alg_bytes_per_launch": gu_bytes,
+                      "avg_launch_us": gu_avg_s * 1e6} if not tensor_bound else
+                     {"bound": "tensor", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved,
+                      "peak": peak_t, "unit": "TFLOP/s", "frac": achieved / peak_t,
+                      "peak_source": f"{peak_src} bf16 sustained" + (" x2 (fp8 nominal ratio)"
+                                                                    if shape.wdtype == "e4m3" else ""),
+                      "traffic": traffic, "alg_flops_per_launch": gateup_alg_flops(shape, M),
+                      "alg_bytes_per_launch": gu_bytes, "achieved_GBps": gu_bytes / gu_avg_s / 1e9,
+                      "avg_launch_us": gu_avg_s * 1e6}),
         "layer": {"alg_bytes_per_step": lay_bytes, "achieved_GBps": lay_bytes / step_s / 1e9,
                   "frac_of_hbm_peak": lay_bytes / step_s / 1e9 / peak,
                   "TFLOPs": layer_flops(shape, M) / step_s / 1e12,
-                  "kernel_ms_per_step": {kk: v[0] / args.steps for kk, v in per_kernel.items()}},
+                  "kernel_ms_per_step": {kk: v[0] / prof_steps for kk, v in per_kernel.items()},
+                  "kernel_times": "CUDA events around each launch inside the replayed step graphs"
+                  if not args.no_graph else "CUDA events around each launch of plain API calls"},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": M * shape.H * 2 + M * 4,
                 "d2h_bytes_per_step": M * shape.H * 2,
                 "how": "graph replay of H2D copy, route, forward, D2H copy" if not args.no_graph else "plain API calls"},

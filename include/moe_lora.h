@@ -69,7 +69,9 @@ typedef enum {
   MOE_LORA_OP_FORWARD = 1,
   MOE_LORA_OP_SGMV_SHRINK = 2,
   MOE_LORA_OP_SGMV_EXPAND = 3,
-  MOE_LORA_OP_DENSE = 4
+  MOE_LORA_OP_DENSE = 4,
+  MOE_LORA_OP_FORWARD_BF16 = 5,  /* moe_lora_forward with ML_BF16 experts only  */
+  MOE_LORA_OP_FORWARD_E4M3 = 6   /* moe_lora_forward with ML_E4M3 experts only  */
 } moe_lora_op;
 
 /* Supported ranges (outside them: MOE_LORA_ERR_UNSUPPORTED).
@@ -135,7 +137,9 @@ MOE_LORA_API moe_lora_status moe_lora_route(
  *   lora_a_gu    bf16 [L][E][r][H];  lora_b_gu bf16 [L][E][r][2I];
  *   lora_a_d     bf16 [L][E][r][I];  lora_b_d  bf16 [L][E][r][H]  (NULL iff L = 0).
  *   y            bf16 [M, H] output (overwritten).
- *   workspace    >= moe_lora_workspace_size(MOE_LORA_OP_FORWARD, M, H, I, E, k, L, r).
+ *   workspace    >= moe_lora_workspace_size(MOE_LORA_OP_FORWARD, M, H, I, E, k, L, r)
+ *                (either expert type), or the smaller size of MOE_LORA_OP_FORWARD_BF16 /
+ *                MOE_LORA_OP_FORWARD_E4M3 for that expert type.
  * Intermediates (gathered rows, z, act, per-pair outputs) live in the workspace.
  * ------------------------------------------------------------------------------- */
 MOE_LORA_API moe_lora_status moe_lora_forward(
@@ -244,7 +248,10 @@ MOE_LORA_API const char* moe_lora_last_error(void);
  * stream, for up to n launches; n = 0 disables and frees the pool.  Kernel ids:
  *   0 router logits, 1 top-k, 2 sort, 3 SGMV shrink, 4 gate_up GEMM, 5 down GEMM,
  *   6 combine, 7 SGMV expand, 8 fp32 dense GEMM, 9 dense bf16 GEMM,
- *   10 e4m3 activation planes.
+ *   10 e4m3 activation planes, 11 fused segmented LoRA (shrink + expand),
+ *   12 one-launch routing (small batches).
+ * Launches captured into a CUDA graph record their events as graph nodes, so every
+ * replay of the graph re-records them (the last replay's times are read).
  * moe_lora_profile_read() waits for the recorded events and returns the summed
  * device time (ms) and the number of recorded launches of one kernel id.
  * moe_lora_launch_count() counts every kernel launch of the library since load. */

@@ -17,14 +17,15 @@ LIB_PATH = os.path.join(_PKG, "libmoe_lora.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_CHECK, ERR_TIMEOUT = range(6)
 ML_F32, ML_BF16, ML_E4M3 = 0, 1, 2
-OP_ROUTE, OP_FORWARD, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_DENSE = range(5)
+OP_ROUTE, OP_FORWARD, OP_SGMV_SHRINK, OP_SGMV_EXPAND, OP_DENSE, OP_FORWARD_BF16, OP_FORWARD_E4M3 = range(7)
 
 EXPORTS = ("moe_lora_route", "moe_lora_forward", "sgmv_shrink", "sgmv_expand", "dense_lora_forward",
            "moe_lora_workspace_size", "moe_lora_check_status", "moe_lora_last_error", "moe_lora_version",
            "moe_lora_profile_enable", "moe_lora_profile_read", "moe_lora_launch_count",
            "moe_lora_route_noalloc")
 KERNEL_IDS = {"router_logits": 0, "topk": 1, "sort": 2, "shrink": 3, "gemm_gateup": 4, "gemm_down": 5,
-              "combine": 6, "expand": 7, "dense_f32": 8, "gemm_dense": 9, "quant": 10}
+              "combine": 6, "expand": 7, "dense_f32": 8, "gemm_dense": 9, "quant": 10,
+              "lora": 11, "route": 12}
 
 
 class MoELoRAError(RuntimeError):
@@ -171,7 +172,8 @@ def forward(x: torch.Tensor, routing: dict, weights: dict, *, k: int, L: int, y=
     if y is None:
         y = torch.empty((M, H), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = new_workspace(workspace_size(OP_FORWARD, M, H, I, E, k, L, r), x.device)
+        op = OP_FORWARD_E4M3 if wdt == ML_E4M3 else OP_FORWARD_BF16
+        workspace = new_workspace(workspace_size(op, M, H, I, E, k, L, r), x.device)
     scales = weights.get("scales") if wdt == ML_E4M3 else None
     _check(lib().moe_lora_forward(
         _ptr(x), M, H, I, E, k, L, r, _ptr(routing["topk_w"]), _ptr(routing["sorted_pairs"]),

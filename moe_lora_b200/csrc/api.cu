@@ -30,11 +30,21 @@ ProfState g_prof;
 std::atomic<long long> g_launches{0};
 }  // namespace
 
+// Under stream capture an event record becomes a graph node only with the external
+// flag; each replay of the graph then re-records the event.
+static void prof_record(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) == cudaSuccess && cap == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
+}
+
 void prof_begin(int id, cudaStream_t st) {
   if (!g_prof.on || id < 0 || id >= K_COUNT) return;
   if (g_prof.next >= g_prof.ev.size()) return;
   g_prof.open[id] = static_cast<int>(g_prof.next);
-  cudaEventRecord(g_prof.ev[g_prof.next++], st);
+  prof_record(g_prof.ev[g_prof.next++], st);
 }
 
 void prof_end(int id, cudaStream_t st) {
@@ -43,7 +53,7 @@ void prof_end(int id, cudaStream_t st) {
     g_prof.open[id] = -1;
     return;
   }
-  cudaEventRecord(g_prof.ev[g_prof.next], st);
+  prof_record(g_prof.ev[g_prof.next], st);
   g_prof.pairs[id].push_back({g_prof.open[id], static_cast<int>(g_prof.next)});
   ++g_prof.next;
   g_prof.open[id] = -1;
@@ -125,9 +135,21 @@ int choose_bn(long long rows, int groups) {
   const double avg = groups > 0 ? static_cast<double>(rows) / groups : rows;
   if (avg <= 12) return 16;
   if (avg <= 24) return 32;
-  if (avg <= 48) return 64;
+  if (avg <= 64) return 64;
   if (avg <= 96) return 128;
   return 256;
+}
+
+// Where the LoRA expand z B runs.  Long groups (more than 64 rows each: tensor-core
+// tiles of >= 128 tokens) run it inside the grouped GEMM as extra MMA K steps, so no
+// delta round-trips through HBM.  Short groups (decode) run it in the LoRA kernel into
+// an fp32 delta that the GEMM epilogue prefetches and adds: the weight stream of the
+// GEMM stays unbroken.  MOE_LORA_EXPAND=gemm|delta overrides (used by the tests).
+bool expand_in_gemm(long long rows, int groups) {
+  const char* v = std::getenv("MOE_LORA_EXPAND");
+  if (v != nullptr && std::strcmp(v, "gemm") == 0) return true;
+  if (v != nullptr && std::strcmp(v, "delta") == 0) return false;
+  return rows > 64LL * (groups > 0 ? groups : 1);
 }
 
 int shrink_rows_per_cta(long long rows) {
@@ -141,9 +163,9 @@ struct ForwardWs {
   int* status;
   __nv_bfloat16* x_sorted;
   __nv_bfloat16* act;
-  float* delta_gu;
+  float* delta_gu;     // expand in the LoRA kernel: deltas the GEMM epilogues add
   float* delta_d;
-  float* z;
+  __nv_bfloat16* z;    // expand in the GEMMs: the LoRA shrink output [M*k][r]
   float* o;
   uint8_t* q_hi;      // e4m3 weights: activation planes [M*k][max(H, I)]
   uint8_t* q_lo;
@@ -151,7 +173,7 @@ struct ForwardWs {
   size_t bytes;
 };
 
-ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8) {
+ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8, bool fused) {
   const size_t mk = static_cast<size_t>(M) * k;
   size_t off = kStatusBytes;
   ForwardWs w{};
@@ -164,9 +186,9 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
   w.status = reinterpret_cast<int*>(b);
   w.x_sorted = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
   w.act = reinterpret_cast<__nv_bfloat16*>(take(mk * I * 2));
-  w.delta_gu = reinterpret_cast<float*>(take(r ? mk * 2 * I * 4 : 0));
-  w.delta_d = reinterpret_cast<float*>(take(r ? mk * H * 4 : 0));
-  w.z = reinterpret_cast<float*>(take(mk * r * 4));
+  w.delta_gu = reinterpret_cast<float*>(take(r && !fused ? mk * 2 * I * 4 : 0));
+  w.delta_d = reinterpret_cast<float*>(take(r && !fused ? mk * H * 4 : 0));
+  w.z = reinterpret_cast<__nv_bfloat16*>(take(r && fused ? mk * r * 2 : 0));
   w.o = reinterpret_cast<float*>(take(mk * H * 4));
   const size_t kmax = H > I ? H : I;
   w.q_hi = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
@@ -195,7 +217,8 @@ RouteWs route_layout(void* base, int M, int E, int L) {
   };
   w.status = reinterpret_cast<int*>(b);
   w.key_count = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * (L + 1) * 4));
-  w.a_key = reinterpret_cast<int32_t*>(take(static_cast<size_t>(M) * 4));
+  // adapter key per token; tickets of the one-launch routing (ceil(M / 8) + 1)
+  w.a_key = reinterpret_cast<int32_t*>(take(static_cast<size_t>(M > (M + 7) / 8 + 1 ? M : (M + 7) / 8 + 1) * 4));
   w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(M) * E * 4));
   w.bytes = off;
   return w;
@@ -205,11 +228,12 @@ struct DenseWs {
   int* status;
   float* z;             // fp32 path: shrink output
   int32_t* row_adapter; // fp32 path
-  float* delta;         // bf16 path: LoRA delta added by the GEMM epilogue
+  float* delta;         // bf16 path, expand in the LoRA kernel: delta the GEMM adds
+  __nv_bfloat16* zb;    // bf16 path, expand in the GEMM: shrink output
   size_t bytes;
 };
 
-DenseWs dense_layout(void* base, int T, int h_out, int r, bool f32) {
+DenseWs dense_layout(void* base, int T, int h_out, int r, bool f32, bool fused) {
   size_t off = kStatusBytes;
   DenseWs w{};
   uint8_t* b = static_cast<uint8_t*>(base);
@@ -223,8 +247,8 @@ DenseWs dense_layout(void* base, int T, int h_out, int r, bool f32) {
     w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
     w.row_adapter = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
   } else {
-    w.delta = reinterpret_cast<float*>(take(r ? static_cast<size_t>(T) * h_out * 4 : 0));
-    w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
+    w.delta = reinterpret_cast<float*>(take(r && !fused ? static_cast<size_t>(T) * h_out * 4 : 0));
+    w.zb = reinterpret_cast<__nv_bfloat16*>(take(r && fused ? static_cast<size_t>(T) * r * 2 : 0));
   }
   w.bytes = off;
   return w;
@@ -303,12 +327,16 @@ size_t moe_lora_workspace_size(int op, int M, int H, int I, int E, int k, int L,
   if (M < 0 || H < 0 || I < 0 || E < 0 || k < 0 || L < 0 || r < 0) return 0;
   switch (op) {
     case MOE_LORA_OP_ROUTE: return route_layout(nullptr, M, E, L).bytes;
-    case MOE_LORA_OP_FORWARD: return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, true).bytes;
+    case MOE_LORA_OP_FORWARD:
+    case MOE_LORA_OP_FORWARD_E4M3:
+      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, true, expand_in_gemm(1LL * M * k, E)).bytes;
+    case MOE_LORA_OP_FORWARD_BF16:
+      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, false, expand_in_gemm(1LL * M * k, E)).bytes;
     case MOE_LORA_OP_SGMV_SHRINK:
     case MOE_LORA_OP_SGMV_EXPAND: return kStatusBytes;
     case MOE_LORA_OP_DENSE: {
-      const size_t a = dense_layout(nullptr, M, I, L > 0 ? r : 0, true).bytes;
-      const size_t b = dense_layout(nullptr, M, I, L > 0 ? r : 0, false).bytes;
+      const size_t a = dense_layout(nullptr, M, I, L > 0 ? r : 0, true, false).bytes;
+      const size_t b = dense_layout(nullptr, M, I, L > 0 ? r : 0, false, expand_in_gemm(M, 1)).bytes;
       return a > b ? a : b;
     }
     default: return 0;
@@ -401,7 +429,8 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   if (L > 0) ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
   const int rr = L > 0 ? r : 0;
   const bool fp8 = w_dtype == ML_E4M3;
-  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr, fp8);
+  const bool fused = expand_in_gemm(1LL * M * k, E);
+  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr, fp8, fused);
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (w_dtype == ML_E4M3) {
@@ -428,13 +457,14 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   if (!tensor_map_encode_available())
     return fail(MOE_LORA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8);
+  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8, fused);
   const int mk = M * k;
   const int nkeys = E * (L + 1);
   ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
 
-  // 1. gather x rows into (expert, adapter) order; gate_up LoRA shrink + expand:
-  //    delta_gu = (x A_gu) B_gu per (adapter, expert) segment, z kept on chip
+  // 1. gather x rows into (expert, adapter) order; gate_up LoRA shrink z = x A_gu per
+  //    (adapter, expert) segment; the expand z B_gu either runs here (delta_gu, added
+  //    by the GEMM epilogue) or in the GEMM as extra MMA K steps
   LoraDeltaArgs l1{};
   l1.src = static_cast<const __nv_bfloat16*>(x);
   l1.gather = sorted_pairs;
@@ -451,9 +481,10 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   l1.E = E;
   l1.lora_a = static_cast<const __nv_bfloat16*>(lora_a_gu);
   l1.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
-  l1.delta = rr ? w.delta_gu : nullptr;
-  l1.z = rr ? w.z : nullptr;
+  l1.delta = rr && !fused ? w.delta_gu : nullptr;
+  l1.z_out = rr && fused ? w.z : nullptr;
   l1.status = w.status;
+  l1.num_sms = num_sms();
   ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
 
   // 2. gate_up grouped GEMM; epilogue adds delta_gu and applies SiLU-and-mul -> act
@@ -468,8 +499,18 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.n_out = I;
   g.I = I;
   g.total_rows = mk;
-  g.delta = rr ? w.delta_gu : nullptr;
   g.delta_cols = 2 * I;
+  g.delta = rr && !fused ? w.delta_gu : nullptr;
+  if (rr && fused) {
+    g.z = w.z;
+    g.r = rr;
+    g.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
+    g.L = L;
+    g.lseg_off = seg_offsets;
+    g.lseg_stride = L + 1;
+    g.lseg_count = L;
+    g.lseg_adapter = nullptr;
+  }
   g.out_bf16 = w.act;
   g.w_scales = w_dtype == ML_E4M3 ? w_scales : nullptr;
   g.scale_idx = 0;
@@ -497,7 +538,8 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     l2.NB = H;
     l2.lora_a = static_cast<const __nv_bfloat16*>(lora_a_d);
     l2.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
-    l2.delta = w.delta_d;
+    l2.delta = fused ? nullptr : w.delta_d;
+    l2.z_out = fused ? w.z : nullptr;
     ML_CUDA(launch_lora_delta(l2, cs), "down LoRA launch");
   }
 
@@ -507,8 +549,9 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   d.K = I;
   d.rows_per_group = H;
   d.n_out = H;
-  d.delta = rr ? w.delta_d : nullptr;
   d.delta_cols = H;
+  d.delta = rr && !fused ? w.delta_d : nullptr;
+  if (rr && fused) d.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
   d.out_bf16 = nullptr;
   d.out_f32 = w.o;
   d.sorted_pairs = sorted_pairs;
@@ -617,7 +660,8 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   ML_REQUIRE(S >= 1 || T == 0, MOE_LORA_ERR_INVALID_ARG, "segments must cover the T tokens");
   const int rr = L > 0 ? r : 0;
   const bool f32 = dt == ML_F32;
-  const DenseWs need = dense_layout(nullptr, T, h_out, rr, f32);
+  const bool fused = !f32 && expand_in_gemm(T, 1);
+  const DenseWs need = dense_layout(nullptr, T, h_out, rr, f32, fused);
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (T == 0) return MOE_LORA_OK;
@@ -633,7 +677,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   st = check_device();
   if (st != MOE_LORA_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const DenseWs ws = dense_layout(workspace, T, h_out, rr, f32);
+  const DenseWs ws = dense_layout(workspace, T, h_out, rr, f32, fused);
   ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
 
   if (f32) {
@@ -687,9 +731,10 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     l.E = 1;
     l.lora_a = static_cast<const __nv_bfloat16*>(lora_a);
     l.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
-    l.delta = ws.delta;
-    l.z = ws.z;
+    l.delta = fused ? nullptr : ws.delta;
+    l.z_out = fused ? ws.zb : nullptr;
     l.status = ws.status;
+    l.num_sms = num_sms();
     ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
   }
   GemmArgs g{};
@@ -702,8 +747,18 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   g.n_out = h_out;
   g.I = 0;
   g.total_rows = T;
-  g.delta = rr ? ws.delta : nullptr;
   g.delta_cols = h_out;
+  g.delta = rr && !fused ? ws.delta : nullptr;
+  if (rr && fused) {  // expand z B as extra K steps over the dense segments
+    g.z = ws.zb;
+    g.r = rr;
+    g.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
+    g.L = L;
+    g.lseg_off = seg_offsets;
+    g.lseg_stride = 0;
+    g.lseg_count = S;
+    g.lseg_adapter = seg_adapter;
+  }
   g.out_bf16 = static_cast<__nv_bfloat16*>(y);
   g.status = ws.status;
   g.w = w;

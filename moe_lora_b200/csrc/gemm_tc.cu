@@ -4,10 +4,12 @@
 // and its N slot the tokens of one expert, so that a decode batch of a few tokens
 // per expert still fills the tensor core's M dimension ([SageMaker MoE kernels
 // page], first item: transpose so the large expert dimension is the first operand).
-// The epilogue adds the LoRA delta (z B, produced by the segmented shrink/expand
-// kernel) to the accumulator before anything is stored ([vLLM MoE-LoRA page],
-// "Otimizações em Nível de Kernel": the LoRA add fused into the base output;
-// "Implementação Técnica no vLLM": fused_moe_lora).  gate_up tiles pair 64 gate rows
+// The LoRA expand runs inside the tile as extra MMA K steps: for every adapter segment
+// that meets the tile, B_a^T (MN-major TMA boxes of 64 features x r rank rows) times
+// the segment's z rows (written by the shrink kernel, zero outside the segment) is
+// accumulated before anything is stored ([vLLM MoE-LoRA page], "Otimizações em Nível
+// de Kernel": the LoRA add fused into the base output; "Implementação Técnica no
+// vLLM": fused_moe_lora), so no LoRA delta round-trips through HBM.  gate_up tiles pair 64 gate rows
 // with the matching 64 up rows so SiLU-and-mul is applied before act leaves the SM;
 // down tiles multiply by the routing weight and store one fp32 row per routing pair
 // for the fixed-order combine (expert aggregation, [SageMaker MoE kernels page],
@@ -20,9 +22,13 @@
 //
 // Structure (one CTA per SM, persistent over a device-side tile list):
 //   warp 0      TMA producer: weight tile 128 x 64 bf16 (or 128 x 128 e4m3) per stage as
-//               two 64-row boxes, and the token tile(s) of the same K range
+//               two 64-row boxes, and the token tile(s) of the same K range; then one
+//               LoRA stage per (segment, 64 rank rows): B^T boxes by TMA, the z tile
+//               written by the warp in the 128-byte swizzle
 //   warp 1      MMA issuer: tcgen05.mma kind::f16 (bf16) or kind::f8f6f4 (e4m3),
-//               M = 128, N = BN; commits free the smem stage
+//               M = 128, N = BN (rows of a ragged last chunk rounded up to 16); LoRA
+//               stages kind::f16 with A MN-major (into a third accumulator for e4m3,
+//               which the epilogue adds unscaled and re-zeroes); commits free the stage
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, + LoRA delta, activation,
 //               stores; two TMEM accumulators so the epilogue of tile i overlaps the
 //               MMAs of tile i+1
@@ -69,6 +75,16 @@ struct TcParams {
   const float* b_scales;  // e4m3: [rows][2] = (s, s / 16) of the activation planes
   int m_tiles;
   int stages;
+  // LoRA expand as extra K steps of the tile (bf16 weights): for every adapter segment
+  // that meets the tile, acc[f][t] += sum_i B_a[i][f] z[t][i]
+  const __nv_bfloat16* z;       // [total_rows][r] bf16, null = no fused expand
+  int r;
+  int rbox;                     // K rows per LoRA stage: min(64, r rounded up to 16)
+  const int32_t* lseg_off;      // segment CSR; group g's candidates at g * lseg_stride
+  int lseg_stride;
+  int lseg_count;
+  const int32_t* lseg_adapter;  // adapter of candidate c (null: adapter = c)
+  int L;
 };
 
 // Non-pipeline shared memory, placed after the stage rings.
@@ -99,14 +115,20 @@ struct EpiSlot {
   float col_sl[BN];
 };
 
+constexpr int pow2_at_least(int v) {
+  int p = 32;
+  while (p < v) p <<= 1;
+  return p;
+}
+
 template <int BN, bool W8>
 struct TileCfg {
   static constexpr int kKB = W8 ? 128 : 64;                  // K per stage (128 bytes per row)
   static constexpr int kBTileBytes = BN * 128;               // one token tile (or plane)
   static constexpr int kStageBytes = kATileBytes + (W8 ? 2 : 1) * kBTileBytes;
   static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
-  static constexpr int kAccPerBuf = W8 ? 2 : 1;              // e4m3: hi and lo accumulators
-  static constexpr int kTmemCols = 2 * kAccPerBuf * kAccStride;  // power of two >= 32
+  static constexpr int kAccPerBuf = W8 ? 3 : 1;              // e4m3: hi, lo and LoRA accumulators
+  static constexpr int kTmemCols = pow2_at_least(2 * kAccPerBuf * kAccStride);
   static constexpr bool kPrefetch = BN <= 64;                // epilogue loader warp + slots
   static constexpr int kSlotBytes = kPrefetch ? static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024) : 0;
   static constexpr int kThreads = 224;
@@ -139,11 +161,59 @@ __device__ __forceinline__ int delta_col(int epi, int m, int f0, int I) {
   return f0 + m;
 }
 
+// Adapter segments meeting a tile's rows [row0, row0 + nvalid): the segments of group g
+// are candidates c in [0, lseg_count) with ascending row ranges
+// [off[c], off[c + 1]), off = lseg_off + g * lseg_stride.  The producer and the MMA
+// issuer walk the same sequence, so they agree on the stages of every tile.
+struct LoraSeg {
+  int c;        // next candidate
+  int end;      // tile end row
+  int lo, hi;   // rows of the current segment inside the tile
+  int slot;     // (adapter, group) slice of B: row block slot * r
+  int c_start;  // first tile column of the MMA (multiple of 32)
+  int n;        // MMA N (multiple of 16)
+};
+
+__device__ __forceinline__ void lora_seg_begin(const TcParams& p, const TileInfo& ti, LoraSeg& s) {
+  const int32_t* off = p.lseg_off + static_cast<size_t>(ti.g) * p.lseg_stride;
+  int lo = 0, hi = p.lseg_count;  // smallest c with off[c + 1] > row0
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid + 1] > ti.row0) hi = mid;
+    else lo = mid + 1;
+  }
+  s.c = lo;
+  s.end = ti.row0 + ti.nvalid;
+}
+
+// Advances to the next segment with an adapter; false when the tile has no more.
+__device__ __forceinline__ bool lora_seg_next(const TcParams& p, const TileInfo& ti, LoraSeg& s) {
+  const int32_t* off = p.lseg_off + static_cast<size_t>(ti.g) * p.lseg_stride;
+  while (s.c < p.lseg_count) {
+    const int c = s.c++;
+    const int a0 = off[c], a1 = off[c + 1];
+    if (a0 >= s.end) return false;
+    const int lo = max(a0, ti.row0), hi = min(a1, s.end);
+    if (hi <= lo) continue;
+    const int ad = p.lseg_adapter ? p.lseg_adapter[c] : c;
+    if (ad < 0 || ad >= p.L) continue;
+    s.lo = lo;
+    s.hi = hi;
+    s.slot = ad * p.E + ti.g;
+    s.c_start = ((lo - ti.row0) >> 5) << 5;
+    s.n = (hi - ti.row0 - s.c_start + 15) & ~15;
+    return true;
+  }
+  return false;
+}
+
 template <int BN, bool W8>
 __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tml, const __grid_constant__ CUtensorMap tmd,
-                   const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmlb, const TcParams p) {
+  // tml: the lo activation plane (e4m3 weights); tmlb: LoRA B viewed as [L * E * r][NB]
+  // (MN-major boxes of 64 features x rbox rank rows)
   using Cfg = TileCfg<BN, W8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -174,6 +244,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     tma_prefetch_desc(&tmw);
     tma_prefetch_desc(&tmb);
     if (W8) tma_prefetch_desc(&tml);
+    if (p.z != nullptr) tma_prefetch_desc(&tmlb);
     if (p.delta != nullptr) tma_prefetch_desc(&tmd);
   }
   if (warp == 1) tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
@@ -214,27 +285,69 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
+  if constexpr (W8) {
+    // the LoRA accumulators start at zero; the epilogue re-zeroes one after reading it
+    if (p.z != nullptr && warp >= 2 && warp < 6) {
+      for (int b = 0; b < 2; ++b)
+        for (int c = 0; c < Cfg::kAccStride; c += 32)
+          tmem_zero_32x32b_x32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
+                               (b * Cfg::kAccPerBuf + 2) * Cfg::kAccStride + c);
+      tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+  }
   const int total_tiles = sm.chunk_pref[p.E] * p.m_tiles;
   const int nk = (p.K + Cfg::kKB - 1) / Cfg::kKB;  // stages per tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t filled_mask = 0, last_parity = 0;
-      for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
-        const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
-        int wrow0, wrow1;
-        if (p.epi == EPI_GATEUP) {
-          wrow0 = ti.g * p.rows_per_group + ti.mt * 64;
-          wrow1 = ti.g * p.rows_per_group + p.I + ti.mt * 64;
-        } else {
-          wrow0 = ti.g * p.rows_per_group + ti.mt * kBM;
-          wrow1 = wrow0 + 64;
-        }
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort_flag, p.status, kWaitLimitNs, 1)) break;
+    // Lane 0 issues the TMA copies.  The whole warp fills the z tiles of LoRA stages
+    // with cp.async (zero-fill outside the segment); such a stage is completed (copies
+    // waited for, proxy fence, arrive) only when the producer would otherwise block, so
+    // the z loads overlap the following copies instead of stalling them.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t filled_mask = 0, last_parity = 0;
+    uint32_t pend_mask = 0;  // LoRA stages whose z copies are issued but not yet arrived
+    bool ok = true;
+    auto flush_lora = [&]() {
+      if (pend_mask != 0) {
+        cp_async_wait_all();
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the MMA
+        __syncwarp();
+        if (lane == 0)
+          for (int s2 = 0; s2 < S; ++s2)
+            if (pend_mask & (1u << s2)) mbar_arrive(&sm.full[s2]);
+        pend_mask = 0;
+      }
+    };
+    // warp-uniform wait for a free ring slot
+    auto acquire = [&](int where) -> bool {
+      bool got = true;
+      if (lane == 0) got = mbar_try_wait(&sm.empty[stage], phase ^ 1u);
+      if (!__shfl_sync(0xffffffffu, got, 0)) {
+        flush_lora();
+        if (lane == 0) got = mbar_wait(&sm.empty[stage], phase ^ 1u, abort_flag, p.status, kWaitLimitNs, where);
+        got = __shfl_sync(0xffffffffu, got, 0);
+      }
+      return got;
+    };
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      if (__shfl_sync(0xffffffffu, *abort_flag != 0, 0)) break;  // warp-uniform
+      const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
+      int wrow0, wrow1;
+      if (p.epi == EPI_GATEUP) {
+        wrow0 = ti.g * p.rows_per_group + ti.mt * 64;
+        wrow1 = ti.g * p.rows_per_group + p.I + ti.mt * 64;
+      } else {
+        wrow0 = ti.g * p.rows_per_group + ti.mt * kBM;
+        wrow1 = wrow0 + 64;
+      }
+      for (int kb = 0; kb < nk; ++kb) {
+        ok = acquire(1);
+        if (!ok) break;
+        if (lane == 0) {
           uint8_t* a_s = ring + stage * Cfg::kStageBytes;
           uint8_t* b_s = a_s + kATileBytes;
           const int kc = kb * Cfg::kKB;  // first K element of the stage
@@ -245,29 +358,73 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           if constexpr (W8) tma_load_2d(b_s + Cfg::kBTileBytes, &tml, &sm.full[stage], kc, ti.row0);
           filled_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
+        }
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok && p.z != nullptr) {
+        // LoRA stages: A = B_a^T (MN-major: 64 gate/low + 64 up/high features x rbox
+        // rank rows), B = the segment's z rows in tile columns [c_start, c_start + n),
+        // zero outside the segment
+        const int f0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
+        const int col0 = f0, col1 = (p.epi == EPI_GATEUP) ? p.I + f0 : f0 + 64;
+        const int kch = p.rbox / 8;  // 16-byte chunks of a z row per stage
+        LoraSeg ls;
+        lora_seg_begin(p, ti, ls);
+        while (ok && lora_seg_next(p, ti, ls)) {
+          for (int kh = 0; kh * 64 < p.r; ++kh) {
+            ok = acquire(9);
+            if (!ok) break;
+            uint8_t* a_s = ring + stage * Cfg::kStageBytes;
+            uint8_t* b_s = a_s + kATileBytes;
+            if (lane == 0) {
+              const int krow = ls.slot * p.r + kh * 64;
+              mbar_expect_tx(&sm.full[stage], 2 * p.rbox * 128);
+              tma_load_2d(a_s, &tmlb, &sm.full[stage], col0, krow);
+              tma_load_2d(a_s + p.rbox * 128, &tmlb, &sm.full[stage], col1, krow);
+              filled_mask |= 1u << stage;
+              last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+            }
+            for (int idx = lane; idx < ls.n * kch; idx += 32) {
+              const int j = idx / kch, c = idx - j * kch;
+              const int row = ti.row0 + ls.c_start + j;
+              const int el = kh * 64 + c * 8;
+              const bool valid = row >= ls.lo && row < ls.hi && el < p.r;
+              const __nv_bfloat16* src = valid ? p.z + static_cast<size_t>(row) * p.r + el : p.z;
+              cp_async_16_zfill(b_s + j * 128 + ((c ^ (j & 7)) << 4), src, valid);  // 128-byte swizzle
+            }
+            pend_mask |= 1u << stage;
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
       }
-      if (*abort_flag) {
-        // let our own copies land before the CTA exits
-        for (int s = 0; s < S; ++s)
-          if (filled_mask & (1u << s)) {
-            volatile int dummy = 0;
-            mbar_wait(&sm.full[s], (last_parity >> s) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
-          }
-      }
+    }
+    flush_lora();  // every issued stage gets its arrival, also on the abort path
+    if (lane == 0 && *abort_flag) {
+      // let our own copies land before the CTA exits
+      for (int s = 0; s < S; ++s)
+        if (filled_mask & (1u << s)) {
+          volatile int dummy = 0;
+          mbar_wait(&sm.full[s], (last_parity >> s) & 1u, &dummy, nullptr, kWaitLimitNs / 4, 0);
+        }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, BN) : umma_idesc_bf16(kBM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
+        // the last chunk of a group is ragged: N = its rows rounded up to 16, so a
+        // skewed expert load does not pay MMAs on padding rows
+        const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
+        const int n_mma = min(BN, (ti.nvalid + 15) & ~15);
+        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, n_mma) : umma_idesc_bf16(kBM, n_mma);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(&sm.tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 2)) break;
@@ -298,6 +455,34 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
+          }
+        }
+        {
+          if (ok && p.z != nullptr) {
+            // e4m3 weights: LoRA goes to its own accumulator (no weight or plane scale)
+            const uint32_t d_lora = d_tmem + (W8 ? 2 * Cfg::kAccStride : 0);
+            LoraSeg ls;
+            lora_seg_begin(p, ti, ls);
+            while (ok && lora_seg_next(p, ti, ls)) {
+              const uint32_t lidesc = umma_idesc_bf16_amn(kBM, ls.n);
+              for (int kh = 0; kh * 64 < p.r; ++kh) {
+                if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 10)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(ring + stage * Cfg::kStageBytes);
+                const uint64_t adesc = umma_desc_mn_sw128(a_addr, p.rbox * 128);
+                const uint64_t bdesc = umma_desc_sw128(a_addr + kATileBytes);
+                for (int kk = 0; kk < p.rbox / 16; ++kk)  // 16 rank rows (2048 B of A) per instruction
+                  umma_bf16(d_lora + ls.c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
+                umma_commit(&sm.empty[stage]);
+                if (++stage == S) {
+                  stage = 0;
+                  phase ^= 1u;
+                }
+              }
+            }
           }
         }
         if (!ok) break;
@@ -358,6 +543,11 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
 #pragma unroll
           for (int n = 0; n < 32; ++n)
             if (c0 + n < BN) v[n] = scale * (v[n] * slot->col_sh[c0 + n] + vl[n] * slot->col_sl[c0 + n]);
+          if (p.z != nullptr) {
+            tmem_ld_32x32b_x32(t_acc + 2 * Cfg::kAccStride, vl);
+#pragma unroll
+            for (int n = 0; n < 32; ++n) v[n] += vl[n];
+          }
         } else {
 #pragma unroll
           for (int n = 0; n < 32; ++n) v[n] *= scale;
@@ -421,6 +611,12 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
                 p.out_bf16[static_cast<size_t>(ti.row0 + c0 + n) * p.n_out + feat] = __float2bfloat16_rn(v[n]);
           }
         }
+      }
+      if constexpr (W8) {
+        if (p.z != nullptr)
+          for (int c = 0; c < Cfg::kAccStride; c += 32)
+            tmem_zero_32x32b_x32(tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) +
+                                 (buf * Cfg::kAccPerBuf + 2) * Cfg::kAccStride + c);
       }
       tc_fence_before();
       mbar_arrive(&sm.tempty[buf]);
@@ -526,7 +722,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  CUtensorMap tmw, tmb, tml, tmd;
+  CUtensorMap tmw, tmb, tml, tmd, tmlb;
   const uint64_t wrows = static_cast<uint64_t>(a.E) * a.rows_per_group;
   if (W8) {
     if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.w, a.K, wrows, static_cast<uint64_t>(a.K), 128, 64,
@@ -543,6 +739,15 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
                        static_cast<uint64_t>(a.K) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     tml = tmb;  // unused
+  }
+  if (a.z != nullptr) {  // LoRA B as [L * E * r][delta_cols], boxes 64 features x rbox rows
+    const int rbox = a.r >= 64 ? 64 : (a.r + 15) / 16 * 16;
+    if (encode_tmap_2d(&tmlb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.lora_b, a.delta_cols,
+                       static_cast<uint64_t>(a.L) * a.E * a.r, static_cast<uint64_t>(a.delta_cols) * 2, 64, rbox,
+                       CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    tmlb = tmb;  // unused
   }
   if (a.delta != nullptr && Cfg::kPrefetch) {
     if (encode_tmap_2d(&tmd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.delta, a.delta_cols, a.total_rows,
@@ -572,13 +777,21 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.b_scales = a.b_scales;
   p.m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
   p.stages = stages;
+  p.z = a.z;
+  p.r = a.r;
+  p.rbox = a.r >= 64 ? 64 : (a.r + 15) / 16 * 16;
+  p.lseg_off = a.lseg_off;
+  p.lseg_stride = a.lseg_stride;
+  p.lseg_count = a.lseg_count;
+  p.lseg_adapter = a.lseg_adapter;
+  p.L = a.L;
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
   const long long tiles_ub = chunks_ub * p.m_tiles;
   int grid = a.num_sms;
   if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
   if (grid < 1) grid = 1;
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP : (a.epi == EPI_DOWN ? K_GEMM_DOWN : K_GEMM_DENSE), st);
-  gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, p);
+  gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
   count_launch();
   return cudaGetLastError();
 }
@@ -586,6 +799,11 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
   if (a.E > kMaxGroups) return cudaErrorInvalidValue;
   if (a.delta != nullptr && a.delta_cols % 8 != 0) return cudaErrorInvalidValue;
+  if (a.z != nullptr) {
+    if (a.delta != nullptr || a.lora_b == nullptr || a.lseg_off == nullptr || a.r <= 0 ||
+        a.r > 128 || a.r % 8 != 0 || a.delta_cols % 8 != 0 || a.L <= 0)
+      return cudaErrorInvalidValue;
+  }
   if (a.w_fp8) {
     if (a.b_hi == nullptr || a.b_lo == nullptr || a.b_scales == nullptr) return cudaErrorInvalidValue;
     switch (a.bn) {

@@ -22,7 +22,8 @@ struct RouteArgs {
   int32_t* sorted_pairs;
   int32_t* seg_offsets;
   int32_t* key_count;     // workspace [E*(L+1)]
-  int32_t* a_key;         // workspace [M]
+  int32_t* a_key;         // workspace [max(M, ceil(M / 8) + 1)]: adapter keys, or the
+                          // tickets of the one-launch routing
   int* status;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
@@ -49,9 +50,10 @@ struct ShrinkArgs {
 };
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st);
 
-// Segmented LoRA for the GEMM epilogues: per segment, gather the source rows (optional),
-// shrink z = src . A^T, expand delta = z . B into an fp32 buffer that the GEMM epilogue
-// adds (rows without an adapter get delta = 0).  bf16 only; two kernel launches.
+// Segmented LoRA for the GEMMs: per segment, gather the source rows (optional) and
+// shrink z = src . A^T; then either write z (bf16) for a GEMM that runs the expand as
+// extra MMA K steps, or expand delta = z . B into an fp32 buffer that the GEMM epilogue
+// adds (rows without an adapter get delta = 0).  bf16 only; one kernel launch.
 struct LoraDeltaArgs {
   const __nv_bfloat16* src;   // rows [*, K]
   const int32_t* gather;      // if set: source row of output row s = gather[s] / gather_div
@@ -64,9 +66,10 @@ struct LoraDeltaArgs {
   int L, E;
   const __nv_bfloat16* lora_a;  // MoE [L][E][r][K]; dense [L][r][K]
   const __nv_bfloat16* lora_b;  // MoE [L][E][r][NB]; dense [L][r][NB]
-  float* z;                   // scratch [nrows][r] (shrink -> expand)
-  float* delta;               // [nrows][NB]
+  float* delta;               // [nrows][NB] (expand in this kernel) or null
+  __nv_bfloat16* z_out;       // shrink only: z [nrows][r] bf16 for a GEMM that expands
   int* status;
+  int num_sms;
 };
 cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st);
 
@@ -132,6 +135,16 @@ struct GemmArgs {
   const float* b_scales;       // [total_rows][2] = (s, s / 16)
   int bn;                      // N tile (16..256)
   int num_sms;
+  // LoRA expand fused as extra K steps (bf16 weights only; exclusive with delta):
+  // acc[f][t] += sum_i B[slot][i][f] z[t][i] for the rows t of every adapter segment
+  const __nv_bfloat16* z;      // [total_rows][r] bf16 shrink output; null = none
+  int r;
+  const __nv_bfloat16* lora_b; // [L * E * r][delta_cols]: slot (adapter * E + group) rows
+  int L;
+  const int32_t* lseg_off;     // segment CSR, group g's candidates start at g * lseg_stride
+  int lseg_stride;
+  int lseg_count;              // candidates per group
+  const int32_t* lseg_adapter; // adapter of candidate c; null: adapter = c
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
 

@@ -19,7 +19,9 @@ enum KernelId : int {
   K_DENSE_F32 = 8,
   K_GEMM_DENSE = 9,
   K_QUANT = 10,
-  K_COUNT = 11
+  K_LORA = 11,
+  K_ROUTE = 12,
+  K_COUNT = 13
 };
 
 void prof_begin(int id, cudaStream_t st);

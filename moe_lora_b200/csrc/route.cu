@@ -150,6 +150,10 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
       for (int i = 0; i < 8; ++i)
         if (be == lane + 32 * i) used[i] = true;
     }
+    if (be >= E) {  // only NaN logits remain: flag the token, keep the indices in range
+      if (lane == 0) set_status(status, MOE_LORA_ERR_DEVICE_CHECK, t);
+      be = j % E;
+    }
     if (j == 0) top_v0 = bv;
     const float ex = expf(bv - top_v0);
     denom += ex;
@@ -254,13 +258,249 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(const int32_t* __rest
   }
 }
 
+// ---------------------------------------------------------------- one-launch routing
+// Small batches (M k <= RF_MAX_PAIRS): logits, top-k, weights, key counts, CSR offsets
+// and the stable placement in ONE launch, so that a decode step pays one kernel instead
+// of three.  Three phases, handed over by tickets (a_key[0, n_tb) per token block and
+// a_key[n_tb] for all blocks, zeroed on the host before the launch):
+//   1. CTA (expert block of RF_EB, token block of RF_TB) computes its logits, the 8
+//      warps splitting H (128-bit loads, shuffle + fixed-order shared-memory sum);
+//   2. the last CTA of a token block runs the top-k of its RF_TB tokens, one warp per
+//      token as in topk_kernel (given logits: one CTA per token block starts here);
+//   3. the last token block counts the pair keys in shared memory, scans them into
+//      seg_offsets and places the pairs stably: one warp walks the pairs in order and
+//      a warp match on the key ranks each pair among the earlier pairs of its key
+//      (pairs of one token have distinct keys, so pair order is token order).
+constexpr int RF_EB = 4;
+constexpr int RF_TB = 8;
+constexpr int RF_MAX_PAIRS = 1024;
+
+// key counts [E (L+1)], pair keys [M k], unnormalised weights [RF_TB][k]
+size_t route_fused_smem(int E, int L, int M, int k) {
+  return (static_cast<size_t>(E) * (L + 1) + static_cast<size_t>(M) * k + static_cast<size_t>(RF_TB) * k) * 4;
+}
+
+// true in exactly one CTA: the one whose arrival completes `ticket` to `count`
+__device__ __forceinline__ bool arrive_last(int* ticket, int count, int* s_flag) {
+  __syncthreads();  // every write of this CTA is issued
+  if (threadIdx.x == 0) {
+    __threadfence();
+    *s_flag = (atomicAdd(ticket, 1) == count - 1);
+  }
+  __syncthreads();
+  if (!*s_flag) return false;
+  __threadfence();
+  return true;
+}
+
+__global__ void __launch_bounds__(256) route_fused_kernel(const RouteArgs a, const float* lg_in, int n_eb) {
+  extern __shared__ int rf_smem[];
+  __shared__ float s_red[8][RF_EB * RF_TB];
+  __shared__ int s_scan[8];
+  __shared__ int s_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tb = (a.M + RF_TB - 1) / RF_TB;
+  int* tickets = a.a_key;
+  const int LA = a.L + 1;
+  const int nk = a.E * LA;
+  const int mk = a.M * a.k;
+  int* s_cnt = rf_smem;
+  int* s_key = s_cnt + nk;
+  float* s_w = reinterpret_cast<float*>(s_key + mk);
+  const float* lg = lg_in;
+  int tb;
+  if (lg == nullptr) {
+    // ---- phase 1: logits of experts [e0, e0 + 4) x tokens [t0, t0 + 8)
+    const int eb = blockIdx.x % n_eb;
+    tb = blockIdx.x / n_eb;
+    const int e0 = eb * RF_EB, t0 = tb * RF_TB;
+    const int ne = min(RF_EB, a.E - e0), nt = min(RF_TB, a.M - t0);
+    float acc[RF_EB][RF_TB];
+#pragma unroll
+    for (int g = 0; g < RF_EB; ++g)
+#pragma unroll
+      for (int i = 0; i < RF_TB; ++i) acc[g][i] = 0.f;
+    const int h8 = a.H / 8;
+    const int per = (h8 + 7) / 8;
+    const int c0 = warp * per, c1 = min(h8, c0 + per);
+    const uint4* w4 = reinterpret_cast<const uint4*>(a.w_router);
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    for (int cc = c0 + lane; cc < c1; cc += 32) {
+      uint4 wv[RF_EB], xv[RF_TB];
+#pragma unroll
+      for (int g = 0; g < RF_EB; ++g) wv[g] = __ldg(w4 + static_cast<size_t>(e0 + (g < ne ? g : 0)) * h8 + cc);
+#pragma unroll
+      for (int i = 0; i < RF_TB; ++i) xv[i] = __ldg(x4 + static_cast<size_t>(t0 + (i < nt ? i : 0)) * h8 + cc);
+#pragma unroll
+      for (int g = 0; g < RF_EB; ++g)
+#pragma unroll
+        for (int i = 0; i < RF_TB; ++i) acc[g][i] += dot8_bf16(wv[g], xv[i]);
+    }
+#pragma unroll
+    for (int g = 0; g < RF_EB; ++g)
+#pragma unroll
+      for (int i = 0; i < RF_TB; ++i) {
+        const float v = warp_sum(acc[g][i]);
+        if (lane == 0) s_red[warp][g * RF_TB + i] = v;
+      }
+    __syncthreads();
+    if (threadIdx.x < RF_EB * RF_TB) {
+      const int g = threadIdx.x / RF_TB, i = threadIdx.x - g * RF_TB;
+      if (g < ne && i < nt) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) sum += s_red[w][threadIdx.x];
+        a.logits[static_cast<size_t>(t0 + i) * a.E + e0 + g] = sum + (a.bias ? a.bias[e0 + g] : 0.f);
+      }
+    }
+    if (!arrive_last(tickets + tb, n_eb, &s_flag)) return;
+    lg = a.logits;
+  } else {
+    tb = blockIdx.x;
+  }
+
+  // ---- phase 2: top-k of the token block, one warp per token
+  const int t = tb * RF_TB + warp;
+  if (t < a.M) {
+    float v[8];
+    bool used[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = (e < a.E) ? __ldcg(lg + static_cast<size_t>(t) * a.E + e) : -INFINITY;
+      used[i] = (e >= a.E);
+    }
+    int ad = a.adapter_ids[t];
+    if (ad < -1 || ad >= a.L) {
+      if (lane == 0) set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, t);
+      ad = -1;
+    }
+    float top_v0 = 0.f, denom = 0.f;
+    float* wrow = s_w + warp * a.k;
+    for (int j = 0; j < a.k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (!used[i] && (v[i] > bv || (v[i] == bv && e < be))) {
+          bv = v[i];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (be == lane + 32 * i) used[i] = true;
+      }
+      if (be >= a.E) {  // only NaN logits remain: flag the token, keep the indices in range
+        if (lane == 0) set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, t);
+        be = j % a.E;
+      }
+      if (j == 0) top_v0 = bv;
+      const float ex = expf(bv - top_v0);
+      denom += ex;
+      if (lane == 0) {
+        a.topk_ids[t * a.k + j] = be;
+        wrow[j] = ex;
+      }
+    }
+    __syncwarp();
+    const float inv = 1.0f / denom;
+    for (int j = lane; j < a.k; j += 32) a.topk_w[t * a.k + j] = wrow[j] * inv;
+  }
+  if (!arrive_last(tickets + n_tb, n_tb, &s_flag)) return;
+
+  // ---- phase 3: key counts, CSR offsets, stable placement (one CTA)
+  for (int i = threadIdx.x; i < nk; i += blockDim.x) s_cnt[i] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < mk; p += blockDim.x) {
+    const int tt = p / a.k;
+    int ad = a.adapter_ids[tt];
+    if (ad < -1 || ad >= a.L) ad = -1;
+    const int key = __ldcg(a.topk_ids + p) * LA + (ad >= 0 ? ad : a.L);
+    s_key[p] = key;
+    atomicAdd(&s_cnt[key], 1);
+  }
+  __syncthreads();
+  const int per = (nk + blockDim.x - 1) / blockDim.x;
+  const int q0 = threadIdx.x * per, q1 = min(nk, q0 + per);
+  int local = 0;
+  for (int q = q0; q < q1; ++q) local += s_cnt[q];
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_scan[warp] = incl;
+  __syncthreads();
+  int base = incl - local;
+  for (int w = 0; w < warp; ++w) base += s_scan[w];
+  for (int q = q0; q < q1; ++q) {
+    const int c = s_cnt[q];
+    s_cnt[q] = base;
+    a.seg_offsets[q] = base;
+    base += c;
+  }
+  if (threadIdx.x == 0) a.seg_offsets[nk] = mk;
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned lt = (1u << lane) - 1u;
+    for (int p0 = 0; p0 < mk; p0 += 32) {
+      const int p = p0 + lane;
+      const int key = (p < mk) ? s_key[p] : -1 - lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      int pos = 0;
+      if (p < mk) pos = s_cnt[key] + __popc(peers & lt);
+      __syncwarp();
+      if (p < mk) {
+        a.sorted_pairs[pos] = p;
+        if ((peers & lt) == 0) s_cnt[key] += __popc(peers);
+      }
+      __syncwarp();
+    }
+  }
+}
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   const int nk = a.E * (a.L + 1);
+  if (a.M == 0) return cudaMemsetAsync(a.seg_offsets, 0, sizeof(int32_t) * (nk + 1), st);
+  if (static_cast<long long>(a.M) * a.k <= RF_MAX_PAIRS) {
+    // one launch; a_key[0, n_tb] holds the tickets
+    const int n_tb = (a.M + RF_TB - 1) / RF_TB;
+    cudaError_t err = cudaMemsetAsync(a.a_key, 0, sizeof(int32_t) * (n_tb + 1), st);
+    if (err != cudaSuccess) return err;
+    const size_t smem = route_fused_smem(a.E, a.L, a.M, a.k);
+    static bool attr_set = false;
+    if (!attr_set) {
+      const int most = static_cast<int>(route_fused_smem(256, 64, 1, RF_MAX_PAIRS));  // E = 256, L = 64, caps
+      err = cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      if (err != cudaSuccess) return err;
+      attr_set = true;
+    }
+    if (a.logits_in != nullptr && a.logits_out != nullptr) {
+      err = cudaMemcpyAsync(a.logits_out, a.logits_in, sizeof(float) * a.M * a.E, cudaMemcpyDeviceToDevice, st);
+      if (err != cudaSuccess) return err;
+    }
+    const int n_eb = (a.E + RF_EB - 1) / RF_EB;
+    const int grid = a.logits_in ? n_tb : n_eb * n_tb;
+    ProfScope ps(K_ROUTE, st);
+    route_fused_kernel<<<grid, 256, smem, st>>>(a, a.logits_in, n_eb);
+    count_launch();
+    return cudaGetLastError();
+  }
   cudaError_t err = cudaMemsetAsync(a.key_count, 0, sizeof(int32_t) * nk, st);
   if (err != cudaSuccess) return err;
-  if (a.M == 0) {
-    return cudaMemsetAsync(a.seg_offsets, 0, sizeof(int32_t) * (nk + 1), st);
-  }
   const float* lg = a.logits_in;
   if (lg == nullptr) {
     ProfScope ps(K_ROUTE_LOGITS, st);

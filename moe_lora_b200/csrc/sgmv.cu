@@ -9,6 +9,8 @@
 // loads.  The expand adds zB into the output in the same pass (fused add, same
 // section).  These kernels are HBM/L2-bound streams of adapter slices: no tensor
 // cores (r <= 128 outputs per token).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "prof.h"
@@ -160,19 +162,21 @@ cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- segmented LoRA for the GEMMs
-// Two streaming kernels per projection ([Punica review page], "提案手法": SGMV;
-// [vLLM MoE-LoRA page], "O Papel da Multi-LoRA": shrink z = xA then expand zB):
-//   lora_shrink_kernel  grid (segment, rank block of 8, row-chunk lane): warp w computes
-//                       z row i = 8 * block + w for the segment's rows, the whole K range
-//                       in flight (U 16-byte chunks per lane), reduced with shuffles
-//                       (split-K over the lanes, "Otimizações em Nível de Kernel");
-//                       rank block 0 also writes the gathered source rows
-//   lora_expand_kernel  grid (segment, feature block of 2048, row-chunk lane): each thread
-//                       owns 8 features and keeps 8-16 B rows in flight, then writes
-//                       delta = z B (fp32), which the GEMM epilogue adds to its output.
-// Segments without an adapter write delta = 0 (early exit of the LoRA work).
-constexpr int LD_RB = 8;      // rows per chunk
-constexpr int LD_FB = 2048;   // features per expand CTA (256 threads x 8)
+// One fused streaming kernel per projection ([Punica review page], "提案手法": SGMV;
+// [vLLM MoE-LoRA page], "O Papel da Multi-LoRA": shrink z = xA then expand zB, and
+// "Otimizações em Nível de Kernel": split-K for the shrink, fused add of the expand).
+// CTA = (segment, feature slice, row-chunk lane).  For each chunk of up to rb rows of
+// its segment the CTA
+//   1. shrinks: warp w owns K slice (w mod KS) of rank rows (w / KS) + (8 / KS) m;
+//      lanes stream 128-bit chunks of A and of the rows, split-K over lanes (shuffle)
+//      and over the KS warps of a rank row (fixed-order sum in shared memory), so z
+//      stays on chip;
+//   2. expands: each thread owns 8 features of the slice, streams IB rows of B at a
+//      time and writes delta = z B (fp32), which the GEMM epilogue adds to its tile.
+// Segments without an adapter write delta = 0 (early exit of the LoRA work).  The
+// CTAs of feature slice 0 also copy the gathered source rows (gate_up operand).
+constexpr int LF_RB_MAX = 8;   // rows per chunk (4 or 8, chosen on the host)
+constexpr int LF_NI = 4;       // rank rows per warp pass
 
 struct SegInfo {
   int lo, hi, ad, e;
@@ -202,75 +206,52 @@ __device__ __forceinline__ SegInfo segment_info(const LoraDeltaArgs& a, int q, b
   return si;
 }
 
-// z[r0 + j][i] = src_j . arow for j < n; U chunks of every row in flight per lane.
+// Partial shrink of one warp: rank rows i0 + istep g (g < LF_NI) over the 16-byte
+// chunks [c0, c1) of K, for the chunk's rows j < RB (rows j >= n repeat row 0 and
+// are dropped).  out[j * r + i] receives the warp's partial sums.
 template <int RB, int U>
-__device__ __forceinline__ void shrink_warp(const LoraDeltaArgs& a, const __nv_bfloat16* arow, const int* s_src,
-                                            int n, int i, int r0, int lane) {
-  const size_t K = a.K;
-  const int k8 = a.K / 8;
-  float acc[RB];
+__device__ __forceinline__ void shrink_part(const __nv_bfloat16* aseg, const __nv_bfloat16* src, int K,
+                                            const int* s_src, int n, int i0, int istep, int c0, int c1,
+                                            int lane, float* out, int r) {
+  float acc[LF_NI][RB];
 #pragma unroll
-  for (int j = 0; j < RB; ++j) acc[j] = 0.f;
-  const uint4* ap = reinterpret_cast<const uint4*>(arow);
-  const uint4* xp[RB];
+  for (int g = 0; g < LF_NI; ++g)
 #pragma unroll
-  for (int j = 0; j < RB; ++j) xp[j] = reinterpret_cast<const uint4*>(a.src + s_src[j < n ? j : 0] * K);
+    for (int j = 0; j < RB; ++j) acc[g][j] = 0.f;
+  // 16-byte chunk offsets of the rank rows and of the source rows
+  const uint4* a4 = reinterpret_cast<const uint4*>(aseg);
+  const uint4* x4 = reinterpret_cast<const uint4*>(src);
+  const int k8 = K / 8;
+  uint32_t xo[RB];
+#pragma unroll
+  for (int j = 0; j < RB; ++j) xo[j] = static_cast<uint32_t>(s_src[j < n ? j : 0]) * k8;
+  const uint32_t ao = static_cast<uint32_t>(i0) * k8, astep = static_cast<uint32_t>(istep) * k8;
   const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
-  for (int base = 0; base < k8; base += 32 * U) {  // U chunks per lane in flight, tail predicated
-    uint4 w8[U], x8[U][RB];
+  for (int base = c0; base < c1; base += 32 * U) {
+    uint4 w8[U][LF_NI], x8[U][RB];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int cc = base + lane + 32 * u;
-      const bool ok = cc < k8;
-      w8[u] = ok ? __ldg(ap + cc) : zero4;
+      const bool ok = cc < c1;
 #pragma unroll
-      for (int j = 0; j < RB; ++j) x8[u][j] = ok ? __ldg(xp[j] + cc) : zero4;
+      for (int g = 0; g < LF_NI; ++g) w8[u][g] = ok ? __ldg(a4 + (ao + g * astep + cc)) : zero4;
+#pragma unroll
+      for (int j = 0; j < RB; ++j) x8[u][j] = ok ? __ldg(x4 + (static_cast<size_t>(xo[j]) + cc)) : zero4;
     }
 #pragma unroll
     for (int u = 0; u < U; ++u)
 #pragma unroll
-      for (int j = 0; j < RB; ++j) acc[j] += dot8_bf16(w8[u], x8[u][j]);
+      for (int g = 0; g < LF_NI; ++g)
+#pragma unroll
+        for (int j = 0; j < RB; ++j) acc[g][j] += dot8_bf16(w8[u][g], x8[u][j]);
   }
 #pragma unroll
-  for (int j = 0; j < RB; ++j) {
-    const float v = warp_sum(acc[j]);
-    if (lane == 0 && j < n) a.z[static_cast<size_t>(r0 + j) * a.r + i] = v;
-  }
-}
-
-__global__ void __launch_bounds__(256) lora_shrink_kernel(const LoraDeltaArgs a) {
-  __shared__ int s_src[LD_RB];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const SegInfo si = segment_info(a, blockIdx.x, blockIdx.y == 0 && blockIdx.z == 0);
-  const size_t K = a.K;
-  const int i = blockIdx.y * 8 + warp;
-  const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
-  const bool do_shrink = a.z != nullptr && si.ad >= 0 && i < a.r;
-  if (!do_gather && !(a.z != nullptr && si.ad >= 0)) return;
-  const __nv_bfloat16* arow =
-      a.lora_a + ((static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e) * a.r + (i < a.r ? i : 0)) * K;
-  for (int c = blockIdx.z; si.lo + c * LD_RB < si.hi; c += gridDim.z) {
-    const int r0 = si.lo + c * LD_RB;
-    const int n = min(LD_RB, si.hi - r0);
-    __syncthreads();
-    if (threadIdx.x < LD_RB)
-      s_src[threadIdx.x] = (threadIdx.x < n) ? (a.gather ? a.gather[r0 + threadIdx.x] / a.gather_div : r0 + threadIdx.x) : 0;
-    __syncthreads();
-    if (do_gather) {
-      const int c16 = a.K / 8;
-      for (int idx = threadIdx.x; idx < n * c16; idx += blockDim.x) {
-        const int j = idx / c16, cc = idx - j * c16;
-        reinterpret_cast<uint4*>(a.gather_dst + (r0 + j) * K)[cc] =
-            __ldg(reinterpret_cast<const uint4*>(a.src + s_src[j] * K) + cc);
-      }
+  for (int g = 0; g < LF_NI; ++g)
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const float v = warp_sum(acc[g][j]);
+      if (lane == 0 && j < n) out[j * r + i0 + istep * g] = v;
     }
-    if (do_shrink) {
-      if (n <= 1) shrink_warp<1, 8>(a, arow, s_src, n, i, r0, lane);
-      else if (n <= 2) shrink_warp<2, 4>(a, arow, s_src, n, i, r0, lane);
-      else if (n <= 4) shrink_warp<4, 2>(a, arow, s_src, n, i, r0, lane);
-      else shrink_warp<8, 1>(a, arow, s_src, n, i, r0, lane);
-    }
-  }
 }
 
 // delta[r0 + j][f..f+8) = sum_i z[j][i] B_i[f..f+8) for j < n; IB rows of B in flight.
@@ -308,42 +289,89 @@ __device__ __forceinline__ void expand_thread(const LoraDeltaArgs& a, const __nv
   }
 }
 
-__global__ void __launch_bounds__(256, 2) lora_expand_kernel(const LoraDeltaArgs a) {
-  __shared__ float s_z[LD_RB * 128];
-  const SegInfo si = segment_info(a, blockIdx.x, false);
-  const int f = blockIdx.y * LD_FB + threadIdx.x * 8;
-  const __nv_bfloat16* bcol =
-      a.lora_b + (static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e) * a.r * a.NB + f;
-  for (int c = blockIdx.z; si.lo + c * LD_RB < si.hi; c += gridDim.z) {
-    const int r0 = si.lo + c * LD_RB;
-    const int n = min(LD_RB, si.hi - r0);
+template <int RB, int U>
+__device__ __forceinline__ void shrink_chunk(const LoraDeltaArgs& a, const __nv_bfloat16* aseg, const int* s_src,
+                                             int n, int ks, float* s_part, float* s_z) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ig = warp / ks, kp = warp - ig * ks;
+  const int istep = 8 / ks;                 // rank-row groups
+  const int k8 = a.K / 8;
+  const int per = (k8 + ks - 1) / ks;
+  const int c0 = kp * per, c1 = min(k8, c0 + per);
+  float* out = (ks == 1) ? s_z : s_part + kp * (LF_RB_MAX * a.r);
+  for (int m0 = 0; ig + istep * m0 < a.r; m0 += LF_NI)
+    shrink_part<RB, U>(aseg, a.src, a.K, s_src, n, ig + istep * m0, istep, c0, c1, lane, out, a.r);
+  if (ks > 1) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x) {
+      float s = 0.f;
+      for (int p = 0; p < ks; ++p) s += s_part[p * (LF_RB_MAX * a.r) + idx];
+      s_z[idx] = s;
+    }
+  }
+}
+
+// RBMAX = rows per chunk (the host's rb); 4 keeps the decode kernel at three CTAs per SM.
+template <int RBMAX>
+__global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(const LoraDeltaArgs a, int ks, int slice) {
+  constexpr int rb = RBMAX;
+  __shared__ int s_src[LF_RB_MAX];
+  __shared__ float s_z[LF_RB_MAX * 128];
+  __shared__ float s_part[64 * LF_RB_MAX];  // ks * r == 64 whenever ks > 1
+  const SegInfo si = segment_info(a, blockIdx.x, blockIdx.y == 0 && blockIdx.z == 0);
+  const size_t K = a.K;
+  const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
+  const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
+  if (!do_gather && !lora) return;
+  const int f_lo = blockIdx.y * slice, f_hi = min(a.NB, f_lo + slice);
+  const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
+  const __nv_bfloat16* aseg = a.lora_a + slot * a.r * K;
+  const __nv_bfloat16* bseg = a.lora_b + slot * a.r * a.NB;
+  for (int c = blockIdx.z; si.lo + c * rb < si.hi; c += gridDim.z) {
+    const int r0 = si.lo + c * rb;
+    const int n = min(rb, si.hi - r0);
+    __syncthreads();  // s_src / s_z of the previous chunk are no longer read
+    if (threadIdx.x < LF_RB_MAX)
+      s_src[threadIdx.x] = (threadIdx.x < n) ? (a.gather ? a.gather[r0 + threadIdx.x] / a.gather_div : r0 + threadIdx.x) : 0;
+    __syncthreads();
+    if (do_gather) {
+      const int c16 = a.K / 8;
+      for (int idx = threadIdx.x; idx < n * c16; idx += blockDim.x) {
+        const int j = idx / c16, cc = idx - j * c16;
+        reinterpret_cast<uint4*>(a.gather_dst + (r0 + j) * K)[cc] =
+            __ldg(reinterpret_cast<const uint4*>(a.src + s_src[j] * K) + cc);
+      }
+    }
+    if (!lora) continue;
     if (si.ad < 0) {
-      if (f < a.NB) {
-        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < n; ++j) {
-          float4* d = reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f);
-          d[0] = z4;
-          d[1] = z4;
-        }
+      if (a.delta == nullptr) continue;  // shrink only: the GEMM skips rows without an adapter
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int w4 = (f_hi - f_lo) / 4;
+      for (int idx = threadIdx.x; idx < n * w4; idx += blockDim.x) {
+        const int j = idx / w4, cc = idx - j * w4;
+        reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f_lo)[cc] = z4;
       }
       continue;
     }
+    if (n <= 1) shrink_chunk<1, RBMAX == 4 ? 2 : 3>(a, aseg, s_src, n, ks, s_part, s_z);
+    else if (n <= 2) shrink_chunk<2, 2>(a, aseg, s_src, n, ks, s_part, s_z);
+    else if (RBMAX == 4 || n <= 4) shrink_chunk<4, 1>(a, aseg, s_src, n, ks, s_part, s_z);
+    else shrink_chunk<8, 1>(a, aseg, s_src, n, ks, s_part, s_z);
     __syncthreads();
-    for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x)
-      s_z[idx] = a.z[static_cast<size_t>(r0) * a.r + idx];
-    __syncthreads();
-    if (f < a.NB) {
-      const bool wide = (a.r % 16) == 0;
+    if (a.z_out != nullptr) {  // shrink only: z rows (bf16) for the GEMM's expand steps
+      for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x)
+        a.z_out[static_cast<size_t>(r0) * a.r + idx] = __float2bfloat16_rn(s_z[idx]);
+      continue;
+    }
+    for (int f = f_lo + threadIdx.x * 8; f < f_hi; f += blockDim.x * 8) {
       if (n <= 1) {
-        if (wide) expand_thread<1, 16>(a, bcol, s_z, n, r0, f);
-        else expand_thread<1, 8>(a, bcol, s_z, n, r0, f);
+        expand_thread<1, 8>(a, bseg + f, s_z, n, r0, f);
       } else if (n <= 2) {
-        if (wide) expand_thread<2, 16>(a, bcol, s_z, n, r0, f);
-        else expand_thread<2, 8>(a, bcol, s_z, n, r0, f);
-      } else if (n <= 4) {
-        expand_thread<4, 8>(a, bcol, s_z, n, r0, f);
+        expand_thread<2, 8>(a, bseg + f, s_z, n, r0, f);
+      } else if (RBMAX == 4 || n <= 4) {
+        expand_thread<4, 8>(a, bseg + f, s_z, n, r0, f);
       } else {
-        expand_thread<8, 8>(a, bcol, s_z, n, r0, f);
+        expand_thread<8, 8>(a, bseg + f, s_z, n, r0, f);
       }
     }
   }
@@ -352,25 +380,33 @@ __global__ void __launch_bounds__(256, 2) lora_expand_kernel(const LoraDeltaArgs
 cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
   if (a.nrows <= 0) return cudaSuccess;
   if (a.r > 128 || a.r % 8 != 0 || a.NB % 8 != 0) return cudaErrorInvalidValue;
-  const bool lora = a.delta != nullptr && a.z != nullptr && a.r > 0;
+  const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
   if (!lora && a.gather_dst == nullptr) return cudaSuccess;  // nothing to do
-  const long long chunks = (a.nrows + LD_RB - 1) / LD_RB;
-  int zsplit = static_cast<int>(chunks / (a.nseg > 0 ? a.nseg : 1));
-  zsplit = zsplit < 1 ? 1 : (zsplit > 16 ? 16 : zsplit);
-  LoraDeltaArgs b = a;
-  if (!lora) b.z = nullptr;
-  {
-    dim3 grid(a.nseg, lora ? a.r / 8 : 1, zsplit);
-    ProfScope ps(K_SHRINK, st);
-    lora_shrink_kernel<<<grid, 256, 0, st>>>(b);
-    count_launch();
+  const int nseg = a.nseg > 0 ? a.nseg : 1;
+  // rows per chunk: 8 when segments are long (prefill), 4 at decode sizes
+  const int rb = (a.nrows >= 8LL * nseg) ? 8 : 4;
+  const long long chunks = (a.nrows + rb - 1) / rb;
+  // row-chunk lanes: a long segment's chunks run on up to 16 CTAs
+  long long zs = (8 * chunks + nseg - 1) / nseg;
+  const int zsplit = static_cast<int>(zs < 1 ? 1 : (zs > 16 ? 16 : zs));
+  // K split of the shrink over warps: every warp owns 8 rank rows (r <= 64)
+  const int ks = lora ? (a.r >= 64 ? 1 : 64 / a.r) : 1;
+  // feature slices: enough CTAs for two per SM when the chunks are few
+  int nsplit = 1;
+  if (lora && a.delta != nullptr) {
+    const long long busy = std::min<long long>(static_cast<long long>(nseg) * zsplit, chunks + std::min(nseg, a.nrows));
+    const long long want = (2LL * (a.num_sms > 0 ? a.num_sms : 148) + busy - 1) / std::max(1LL, busy);
+    const long long cap = std::max(1, a.NB / 512);
+    nsplit = static_cast<int>(std::max(1LL, std::min(want, cap)));
   }
-  if (lora) {
-    dim3 grid(a.nseg, (a.NB + LD_FB - 1) / LD_FB, zsplit);
-    ProfScope ps(K_EXPAND, st);
-    lora_expand_kernel<<<grid, 256, 0, st>>>(a);
-    count_launch();
-  }
+  int slice = (a.NB + nsplit - 1) / nsplit;
+  slice = (slice + 7) / 8 * 8;
+  nsplit = (a.NB + slice - 1) / slice;
+  dim3 grid(a.nseg, nsplit, zsplit);
+  ProfScope ps(K_LORA, st);
+  if (rb == 8) lora_fused_kernel<8><<<grid, 256, 0, st>>>(a, ks, slice);
+  else lora_fused_kernel<4><<<grid, 256, 0, st>>>(a, ks, slice);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -588,12 +624,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   if (f >= H) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* base = o + static_cast<size_t>(t) * k * H + f;
-  for (int j = 0; j < k; ++j) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(base + static_cast<size_t>(j) * H));
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
+  for (int j0 = 0; j0 < k; j0 += 8) {  // 8 slot rows in flight, summed in slot order
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = (j0 + u < k) ? __ldg(reinterpret_cast<const float4*>(base + static_cast<size_t>(j0 + u) * H))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (j0 + u < k) {
+        acc.x += v[u].x;
+        acc.y += v[u].y;
+        acc.z += v[u].z;
+        acc.w += v[u].w;
+      }
+    }
   }
   uint2 out = make_uint2(pack2_bf16(acc.x, acc.y), pack2_bf16(acc.z, acc.w));
   *reinterpret_cast<uint2*>(y + static_cast<size_t>(t) * H + f) = out;

@@ -39,6 +39,9 @@ def test_workspace_sizes():
     mk = 64 * 8
     assert f >= mk * 2048 * 2 + mk * 1408 * 2 + 2 * mk * 16 * 4 + mk * 4 + mk * 2048 * 4
     assert ml.workspace_size(ml.OP_FORWARD, 0, 2048, 1408, 64, 8, 8, 16) == 256
+    fb = ml.workspace_size(ml.OP_FORWARD_BF16, 64, 2048, 1408, 64, 8, 8, 16)
+    fe = ml.workspace_size(ml.OP_FORWARD_E4M3, 64, 2048, 1408, 64, 8, 8, 16)
+    assert 0 < fb < fe == f   # e4m3 experts add the activation planes
     assert ml.workspace_size(ml.OP_SGMV_SHRINK) == 256
     assert ml.workspace_size(99) == 0
     assert ml.workspace_size(ml.OP_FORWARD, -1) == 0

@@ -33,12 +33,26 @@ def test_forward_small_shapes(shape, M):
     assert res["err"] <= TOL_BF16, res["err"]
 
 
+@pytest.mark.parametrize("where", ["gemm", "delta"])
 @pytest.mark.parametrize("bn", [16, 32, 64, 128, 256])
-def test_forward_every_n_tile(bn, monkeypatch):
+def test_forward_every_n_tile(bn, where, monkeypatch):
+    """Every N tile, with the LoRA expand both as extra MMA K steps of the GEMM and as
+    the fp32 delta of the LoRA kernel added by the GEMM epilogue."""
     monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
+    monkeypatch.setenv("MOE_LORA_EXPAND", where)
     res = run_moe_case(SMALL[0], 300)
     assert res["err"] <= TOL_BF16, res["err"]
     res = run_moe_case(SMALL[1], 37)
+    assert res["err"] <= TOL_BF16, res["err"]
+
+
+@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("shape,M", [(SMALL[1], 37), (SMALL[2], 300), (SMALL[3], 37), (SMALL[7], 37),
+                                     (SMALL[8], 300), (SMALL[8], 1)], ids=lambda v: getattr(v, "name", str(v)))
+def test_forward_expand_placement(shape, M, where, monkeypatch):
+    """Both placements of the LoRA expand on ragged shapes, r = 8 .. 128, E = 1."""
+    monkeypatch.setenv("MOE_LORA_EXPAND", where)
+    res = run_moe_case(shape, M)
     assert res["err"] <= TOL_BF16, res["err"]
 
 
@@ -110,9 +124,11 @@ def test_forward_fp8_small_shapes(shape, M):
     assert res["err"] <= TOL_FP8, res["err"]
 
 
+@pytest.mark.parametrize("where", ["gemm", "delta"])
 @pytest.mark.parametrize("bn", [16, 32, 64, 256])
-def test_forward_fp8_every_n_tile(bn, monkeypatch):
+def test_forward_fp8_every_n_tile(bn, where, monkeypatch):
     monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
+    monkeypatch.setenv("MOE_LORA_EXPAND", where)
     res = run_moe_case(SMALL_FP8[1], 150)
     assert res["err"] <= TOL_FP8, res["err"]
 

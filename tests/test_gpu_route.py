@@ -113,3 +113,37 @@ def test_route_deterministic():
     torch.cuda.synchronize()
     for key in ("topk_ids", "topk_w", "sorted_pairs", "seg_offsets"):
         assert torch.equal(a[key], b[key])
+
+
+@pytest.mark.parametrize("M,E,k,L,H", [(1, 64, 8, 8, 2048), (64, 128, 8, 32, 7168), (128, 64, 8, 8, 512),
+                                       (129, 64, 8, 8, 512), (40, 256, 4, 64, 264), (7, 5, 5, 0, 64)])
+def test_route_from_x_exact_on_gpu_logits(M, E, k, L, H):
+    """Both routing launches (one-launch path for M k <= 1024, three kernels above it):
+    ids, weights, pairs and offsets equal the oracle's routing of the GPU's own fp32
+    logits; the logits themselves agree with the fp64 oracle within fp32 error."""
+    g = np.random.default_rng(M * 31 + E)
+    xb = torch.from_numpy(g.standard_normal((M, H), dtype=np.float32)).to(torch.bfloat16)
+    wr = torch.from_numpy(g.standard_normal((E, H), dtype=np.float32) / np.sqrt(H)).to(torch.bfloat16)
+    bias = torch.from_numpy(g.standard_normal(E).astype(np.float32) * np.float32(0.7))
+    ad = _adapters(M, L, M + E)
+    rt = ml.route(torch.from_numpy(ad).cuda(), k, L, x=xb.cuda(), w_router=wr.cuda(), bias=bias.cuda(),
+                  want_logits=True)
+    torch.cuda.synchronize()
+    lg_gpu = rt["logits"].cpu()
+    ids, w, sp, so = oracle_routing_from_logits(lg_gpu, ad.astype(np.int64), E, k, L)
+    assert np.array_equal(rt["topk_ids"].cpu().numpy(), ids)
+    np.testing.assert_allclose(rt["topk_w"].cpu().numpy(), w, rtol=0, atol=1e-6)
+    assert np.array_equal(rt["sorted_pairs"].cpu().numpy(), sp)
+    assert np.array_equal(rt["seg_offsets"].cpu().numpy(), so)
+    x64 = formats.to_f64(synth.bits(xb), "bf16")
+    w64 = formats.to_f64(synth.bits(wr), "bf16")
+    lg = ref.router_logits(x64, w64, bias.numpy().astype(np.float64))
+    tol = 1e-4 * max(1.0, float(np.max(np.abs(lg))))
+    assert float(np.max(np.abs(lg_gpu.numpy().astype(np.float64) - lg))) <= tol
+    ml.check_status(rt["workspace"])
+    # a second call on the same workspace gives the same bits (phase-1 ticket re-armed)
+    rt2 = ml.route(torch.from_numpy(ad).cuda(), k, L, x=xb.cuda(), w_router=wr.cuda(), bias=bias.cuda(),
+                   want_logits=True, workspace=rt["workspace"])
+    torch.cuda.synchronize()
+    for key in ("logits", "topk_ids", "topk_w", "sorted_pairs", "seg_offsets"):
+        assert torch.equal(rt[key], rt2[key])

@@ -48,8 +48,12 @@ def test_sgmv_shrink_expand(s):
     assert rel_err(y0, d_ref) <= (1e-5 if s.dtype == "f32" else 1e-2)
 
 
+@pytest.mark.parametrize("where", ["gemm", "delta"])
 @pytest.mark.parametrize("s", CASES, ids=lambda s: s.name)
-def test_dense_lora_forward(s):
+def test_dense_lora_forward(s, where, monkeypatch):
+    """bf16: the expand both inside the GEMM (extra MMA K steps) and as the LoRA
+    kernel's delta added by the GEMM epilogue (fp32 cases take the SIMT path)."""
+    monkeypatch.setenv("MOE_LORA_EXPAND", where)
     d = dense_f64(s)
     y = ml.dense_lora_forward(d["x"].cuda(), d["w"]["w"].cuda(), d["w"]["a"].cuda(), d["w"]["b"].cuda(),
                               d["offs"].cuda(), d["segs"].cuda())
