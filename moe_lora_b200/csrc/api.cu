@@ -1,6 +1,7 @@
 // C ABI of libmoe_lora.so: argument validation, workspace layout and the launch
 // sequence of each call.  No allocation, no synchronisation, no host read-back
 // (moe_lora_check_status excepted).
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -166,6 +167,10 @@ struct ForwardWs {
   float* delta_gu;     // expand in the LoRA kernel: deltas the GEMM epilogues add
   float* delta_d;
   __nv_bfloat16* z;    // expand in the GEMMs: the LoRA shrink output [M*k][r]
+  float* z_part;       // split LoRA shrink: fp32 partials [ceil(max(H, I) / 1024)][M*k][r]
+  long long z_part_cap;
+  int2* items;         // LoRA work list and its length
+  int* item_count;
   float* o;
   uint8_t* q_hi;      // e4m3 weights: activation planes [M*k][max(H, I)]
   uint8_t* q_lo;
@@ -173,7 +178,7 @@ struct ForwardWs {
   size_t bytes;
 };
 
-ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8, bool fused) {
+ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8, bool fused, int nkeys) {
   const size_t mk = static_cast<size_t>(M) * k;
   size_t off = kStatusBytes;
   ForwardWs w{};
@@ -189,6 +194,10 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
   w.delta_gu = reinterpret_cast<float*>(take(r && !fused ? mk * 2 * I * 4 : 0));
   w.delta_d = reinterpret_cast<float*>(take(r && !fused ? mk * H * 4 : 0));
   w.z = reinterpret_cast<__nv_bfloat16*>(take(r && fused ? mk * r * 2 : 0));
+  w.z_part_cap = r ? static_cast<long long>((std::max(H, I) + 1023) / 1024) * mk * r : 0;
+  w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
+  w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, 4)) * 8));
+  w.item_count = reinterpret_cast<int*>(take(mk > 0 ? 4 : 0));
   w.o = reinterpret_cast<float*>(take(mk * H * 4));
   const size_t kmax = H > I ? H : I;
   w.q_hi = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
@@ -230,10 +239,14 @@ struct DenseWs {
   int32_t* row_adapter; // fp32 path
   float* delta;         // bf16 path, expand in the LoRA kernel: delta the GEMM adds
   __nv_bfloat16* zb;    // bf16 path, expand in the GEMM: shrink output
+  float* z_part;        // bf16 path, split LoRA shrink partials
+  long long z_part_cap;
+  int2* items;          // bf16 path: LoRA work list and its length
+  int* item_count;
   size_t bytes;
 };
 
-DenseWs dense_layout(void* base, int T, int h_out, int r, bool f32, bool fused) {
+DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, bool fused) {
   size_t off = kStatusBytes;
   DenseWs w{};
   uint8_t* b = static_cast<uint8_t*>(base);
@@ -249,6 +262,10 @@ DenseWs dense_layout(void* base, int T, int h_out, int r, bool f32, bool fused) 
   } else {
     w.delta = reinterpret_cast<float*>(take(r && !fused ? static_cast<size_t>(T) * h_out * 4 : 0));
     w.zb = reinterpret_cast<__nv_bfloat16*>(take(r && fused ? static_cast<size_t>(T) * r * 2 : 0));
+    w.z_part_cap = r ? static_cast<long long>((h_in + 1023) / 1024) * T * r : 0;
+    w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
+    w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(T, T, 4)) * 8));
+    w.item_count = reinterpret_cast<int*>(take(T > 0 ? 4 : 0));
   }
   w.bytes = off;
   return w;
@@ -329,14 +346,16 @@ size_t moe_lora_workspace_size(int op, int M, int H, int I, int E, int k, int L,
     case MOE_LORA_OP_ROUTE: return route_layout(nullptr, M, E, L).bytes;
     case MOE_LORA_OP_FORWARD:
     case MOE_LORA_OP_FORWARD_E4M3:
-      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, true, expand_in_gemm(1LL * M * k, E)).bytes;
+      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, true, expand_in_gemm(1LL * M * k, E), E * (L + 1))
+          .bytes;
     case MOE_LORA_OP_FORWARD_BF16:
-      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, false, expand_in_gemm(1LL * M * k, E)).bytes;
+      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, false, expand_in_gemm(1LL * M * k, E), E * (L + 1))
+          .bytes;
     case MOE_LORA_OP_SGMV_SHRINK:
     case MOE_LORA_OP_SGMV_EXPAND: return kStatusBytes;
     case MOE_LORA_OP_DENSE: {
-      const size_t a = dense_layout(nullptr, M, I, L > 0 ? r : 0, true, false).bytes;
-      const size_t b = dense_layout(nullptr, M, I, L > 0 ? r : 0, false, expand_in_gemm(M, 1)).bytes;
+      const size_t a = dense_layout(nullptr, M, H, I, L > 0 ? r : 0, true, false).bytes;
+      const size_t b = dense_layout(nullptr, M, H, I, L > 0 ? r : 0, false, expand_in_gemm(M, 1)).bytes;
       return a > b ? a : b;
     }
     default: return 0;
@@ -408,6 +427,7 @@ moe_lora_status moe_lora_route(const void* x, const void* w_router, const float*
   a.key_count = w.key_count;
   a.a_key = w.a_key;
   a.status = w.status;
+  a.num_sms = num_sms();
   ML_CUDA(launch_route(a, cs), "moe_lora_route launch");
   return MOE_LORA_OK;
 }
@@ -430,7 +450,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   const int rr = L > 0 ? r : 0;
   const bool fp8 = w_dtype == ML_E4M3;
   const bool fused = expand_in_gemm(1LL * M * k, E);
-  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr, fp8, fused);
+  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr, fp8, fused, E * (L + 1));
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (w_dtype == ML_E4M3) {
@@ -457,7 +477,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   if (!tensor_map_encode_available())
     return fail(MOE_LORA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8, fused);
+  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8, fused, E * (L + 1));
   const int mk = M * k;
   const int nkeys = E * (L + 1);
   ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
@@ -483,8 +503,15 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   l1.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
   l1.delta = rr && !fused ? w.delta_gu : nullptr;
   l1.z_out = rr && fused ? w.z : nullptr;
+  l1.z_part = w.z_part;
+  l1.z_part_cap = w.z_part_cap;
   l1.status = w.status;
   l1.num_sms = num_sms();
+  l1.rb = lora_rows_per_chunk(mk, nkeys);
+  l1.items_bound = lora_items_bound(mk, nkeys, l1.rb);
+  l1.items = w.items;
+  l1.item_count = w.item_count;
+  ML_CUDA(launch_lora_plan(l1, cs), "LoRA plan launch");
   ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
 
   // 2. gate_up grouped GEMM; epilogue adds delta_gu and applies SiLU-and-mul -> act
@@ -661,7 +688,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   const int rr = L > 0 ? r : 0;
   const bool f32 = dt == ML_F32;
   const bool fused = !f32 && expand_in_gemm(T, 1);
-  const DenseWs need = dense_layout(nullptr, T, h_out, rr, f32, fused);
+  const DenseWs need = dense_layout(nullptr, T, h_in, h_out, rr, f32, fused);
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (T == 0) return MOE_LORA_OK;
@@ -677,7 +704,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   st = check_device();
   if (st != MOE_LORA_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const DenseWs ws = dense_layout(workspace, T, h_out, rr, f32, fused);
+  const DenseWs ws = dense_layout(workspace, T, h_in, h_out, rr, f32, fused);
   ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
 
   if (f32) {
@@ -733,8 +760,15 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     l.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
     l.delta = fused ? nullptr : ws.delta;
     l.z_out = fused ? ws.zb : nullptr;
+    l.z_part = ws.z_part;
+    l.z_part_cap = ws.z_part_cap;
     l.status = ws.status;
     l.num_sms = num_sms();
+    l.rb = lora_rows_per_chunk(T, S);
+    l.items_bound = lora_items_bound(T, S, l.rb);
+    l.items = ws.items;
+    l.item_count = ws.item_count;
+    ML_CUDA(launch_lora_plan(l, cs), "LoRA plan launch");
     ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
   }
   GemmArgs g{};

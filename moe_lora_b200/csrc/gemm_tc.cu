@@ -67,6 +67,8 @@ struct TcParams {
   int delta_cols;
   __nv_bfloat16* out_bf16;
   float* out_f32;
+  const float* bias;
+  int total_rows;
   const int32_t* sorted_pairs;
   const float* topk_w;
   const float* w_scales;
@@ -249,7 +251,8 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
   }
   if (warp == 1) tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
   for (int g = threadIdx.x; g <= p.E; g += blockDim.x)
-    sm.grp_off[g] = p.group_offsets[static_cast<size_t>(g) * p.group_stride];
+    sm.grp_off[g] = p.group_offsets ? p.group_offsets[static_cast<size_t>(g) * p.group_stride]
+                                    : (g == 0 ? 0 : p.total_rows);
   __syncthreads();
   if (warp == 0) {
     // exclusive prefix of chunks per group (E <= 256: 8 per lane, then a warp scan)
@@ -603,6 +606,13 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             for (int n = 0; n < 32; ++n)
               if (n < ncol) p.out_f32[static_cast<size_t>(cp[n]) * p.n_out + feat] = v[n] * cw[n];
           }
+        } else if (p.epi == EPI_LOGITS) {
+          if (row_ok) {
+            const float b = p.bias ? p.bias[feat] : 0.f;
+#pragma unroll
+            for (int n = 0; n < 32; ++n)
+              if (n < ncol) p.out_f32[static_cast<size_t>(ti.row0 + c0 + n) * p.n_out + feat] = v[n] + b;
+          }
         } else {
           if (row_ok) {
 #pragma unroll
@@ -769,6 +779,8 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.delta_cols = a.delta_cols;
   p.out_bf16 = a.out_bf16;
   p.out_f32 = a.out_f32;
+  p.bias = a.bias;
+  p.total_rows = a.total_rows;
   p.sorted_pairs = a.sorted_pairs;
   p.topk_w = a.topk_w;
   p.w_scales = a.w_scales;
@@ -790,7 +802,9 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   int grid = a.num_sms;
   if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
   if (grid < 1) grid = 1;
-  ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP : (a.epi == EPI_DOWN ? K_GEMM_DOWN : K_GEMM_DENSE), st);
+  ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP
+               : a.epi == EPI_DOWN ? K_GEMM_DOWN
+               : a.epi == EPI_LOGITS ? K_ROUTE_LOGITS : K_GEMM_DENSE, st);
   gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
   count_launch();
   return cudaGetLastError();

@@ -25,6 +25,7 @@ struct RouteArgs {
   int32_t* a_key;         // workspace [max(M, ceil(M / 8) + 1)]: adapter keys, or the
                           // tickets of the one-launch routing
   int* status;
+  int num_sms;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 
@@ -68,9 +69,19 @@ struct LoraDeltaArgs {
   const __nv_bfloat16* lora_b;  // MoE [L][E][r][NB]; dense [L][r][NB]
   float* delta;               // [nrows][NB] (expand in this kernel) or null
   __nv_bfloat16* z_out;       // shrink only: z [nrows][r] bf16 for a GEMM that expands
+  float* z_part;              // optional scratch for the split form: [ceil(K / 1024)][nrows][r]
+  long long z_part_cap;       // floats available at z_part
+  // work list (launch_lora_plan): one item (segment, first row) per chunk of rb rows
+  int2* items;                // [items_bound]
+  int* item_count;
+  int items_bound;            // lora_items_bound(nrows, nseg, rb)
+  int rb;                     // lora_rows_per_chunk(nrows, nseg)
   int* status;
   int num_sms;
 };
+int lora_rows_per_chunk(int nrows, int nseg);
+int lora_items_bound(int nrows, int nseg, int rb);
+cudaError_t launch_lora_plan(const LoraDeltaArgs& a, cudaStream_t st);
 cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st);
 
 // y[t] += z[t] . B_a(t) for dense segments (f32 or bf16 y and B).
@@ -102,14 +113,15 @@ cudaError_t launch_dense_f32(const DenseF32Args& a, cudaStream_t st);
 
 // Tensor-core grouped GEMM with operand swap: the weight rows fill the 128-row MMA
 // M slot, the tokens of one expert (or of the dense batch) the N slot.
-enum EpiKind : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DENSE = 2 };
+enum EpiKind : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DENSE = 2, EPI_LOGITS = 3 };
 
 struct GemmArgs {
   int epi;
   bool w_fp8;
   int K;                       // reduction length
   int E;                       // groups (experts); 1 for dense
-  const int32_t* group_offsets;  // row offsets of group g at group_offsets[g * group_stride]
+  const int32_t* group_offsets;  // row offsets of group g at group_offsets[g * group_stride];
+                               // null: one group of total_rows rows
   int group_stride;
   int rows_per_group;          // weight rows per expert (2I for gate_up, H for down, h_out)
   int n_out;                   // output features per group (I for gate_up, H, h_out)
@@ -121,7 +133,8 @@ struct GemmArgs {
   int delta_cols;
   // epilogue outputs
   __nv_bfloat16* out_bf16;     // gate_up: act [rows][I]; dense: y [T][h_out]
-  float* out_f32;              // down: o [pairs][H] (weighted)
+  float* out_f32;              // down: o [pairs][H] (weighted); logits: [rows][n_out]
+  const float* bias;           // logits: [n_out] or null
   const int32_t* sorted_pairs; // down: pair index of each sorted row
   const float* topk_w;         // down: routing weight per pair
   const float* w_scales;       // fp8: [E][2]

@@ -502,7 +502,28 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   cudaError_t err = cudaMemsetAsync(a.key_count, 0, sizeof(int32_t) * nk, st);
   if (err != cudaSuccess) return err;
   const float* lg = a.logits_in;
-  if (lg == nullptr) {
+  if (lg == nullptr && a.M >= 256 && tensor_map_encode_available()) {
+    // large batches: logits on the tensor cores (the grouped GEMM with one group, W_r
+    // rows in the MMA M slot, tokens in N, fp32 logits + bias in the epilogue)
+    GemmArgs g{};
+    g.epi = EPI_LOGITS;
+    g.K = a.H;
+    g.E = 1;
+    g.group_offsets = nullptr;
+    g.rows_per_group = a.E;
+    g.n_out = a.E;
+    g.total_rows = a.M;
+    g.out_f32 = a.logits;
+    g.bias = a.bias;
+    g.status = a.status;
+    g.w = a.w_router;
+    g.b = a.x;
+    g.bn = 32;
+    g.num_sms = a.num_sms;
+    err = launch_gemm_tc(g, st);
+    if (err != cudaSuccess) return err;
+    lg = a.logits;
+  } else if (lg == nullptr) {
     ProfScope ps(K_ROUTE_LOGITS, st);
     if (a.M <= 256) {
       dim3 grid(a.E, (a.M + RS_TB - 1) / RS_TB);

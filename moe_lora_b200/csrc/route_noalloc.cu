@@ -111,6 +111,12 @@ extern "C" MOE_LORA_API moe_lora_status moe_lora_route_noalloc(
   a.k = k;
   a.L = L;
   a.status = reinterpret_cast<int*>(base);
+  int nsm = 0;
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, cur) != cudaSuccess || nsm <= 0)
+    nsm = 148;
+  a.num_sms = nsm;
   a.key_count = reinterpret_cast<int32_t*>(base + mlb::kStatusBytes);
   a.a_key = reinterpret_cast<int32_t*>(base + mlb::kStatusBytes + kCountBytes);
   a.logits = logits_out ? logits_out : reinterpret_cast<float*>(base + mlb::kStatusBytes + kCountBytes + kKeyBytes);

@@ -165,8 +165,8 @@ cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st) {
 // One fused streaming kernel per projection ([Punica review page], "提案手法": SGMV;
 // [vLLM MoE-LoRA page], "O Papel da Multi-LoRA": shrink z = xA then expand zB, and
 // "Otimizações em Nível de Kernel": split-K for the shrink, fused add of the expand).
-// CTA = (segment, feature slice, row-chunk lane).  For each chunk of up to rb rows of
-// its segment the CTA
+// CTA = (work item, feature slice); an item is a chunk of up to rb rows of one segment
+// (launch_lora_plan lists the chunks of the non-empty segments).  For its chunk the CTA
 //   1. shrinks: warp w owns K slice (w mod KS) of rank rows (w / KS) + (8 / KS) m;
 //      lanes stream 128-bit chunks of A and of the rows, split-K over lanes (shuffle)
 //      and over the KS warps of a rank row (fixed-order sum in shared memory), so z
@@ -289,15 +289,16 @@ __device__ __forceinline__ void expand_thread(const LoraDeltaArgs& a, const __nv
   }
 }
 
+// z[j][i] (into s_z) over the 16-byte K chunks [kc0, kc1): warps split the chunks ks
+// ways and the rank rows 8 / ks ways; fixed-order sum of the ks partials.
 template <int RB, int U>
 __device__ __forceinline__ void shrink_chunk(const LoraDeltaArgs& a, const __nv_bfloat16* aseg, const int* s_src,
-                                             int n, int ks, float* s_part, float* s_z) {
+                                             int n, int ks, float* s_part, float* s_z, int kc0, int kc1) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ig = warp / ks, kp = warp - ig * ks;
   const int istep = 8 / ks;                 // rank-row groups
-  const int k8 = a.K / 8;
-  const int per = (k8 + ks - 1) / ks;
-  const int c0 = kp * per, c1 = min(k8, c0 + per);
+  const int per = (kc1 - kc0 + ks - 1) / ks;
+  const int c0 = kc0 + kp * per, c1 = min(kc1, c0 + per);
   float* out = (ks == 1) ? s_z : s_part + kp * (LF_RB_MAX * a.r);
   for (int m0 = 0; ig + istep * m0 < a.r; m0 += LF_NI)
     shrink_part<RB, U>(aseg, a.src, a.K, s_src, n, ig + istep * m0, istep, c0, c1, lane, out, a.r);
@@ -318,7 +319,11 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
   __shared__ int s_src[LF_RB_MAX];
   __shared__ float s_z[LF_RB_MAX * 128];
   __shared__ float s_part[64 * LF_RB_MAX];  // ks * r == 64 whenever ks > 1
-  const SegInfo si = segment_info(a, blockIdx.x, blockIdx.y == 0 && blockIdx.z == 0);
+  if (blockIdx.x >= *a.item_count) return;
+  const int2 item = a.items[blockIdx.x];
+  SegInfo si = segment_info(a, item.x, false);
+  si.lo = item.y;  // this CTA's chunk of the segment
+  si.hi = min(si.hi, item.y + rb);
   const size_t K = a.K;
   const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
   const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
@@ -353,10 +358,11 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
       }
       continue;
     }
-    if (n <= 1) shrink_chunk<1, RBMAX == 4 ? 2 : 3>(a, aseg, s_src, n, ks, s_part, s_z);
-    else if (n <= 2) shrink_chunk<2, 2>(a, aseg, s_src, n, ks, s_part, s_z);
-    else if (RBMAX == 4 || n <= 4) shrink_chunk<4, 1>(a, aseg, s_src, n, ks, s_part, s_z);
-    else shrink_chunk<8, 1>(a, aseg, s_src, n, ks, s_part, s_z);
+    const int k8 = a.K / 8;
+    if (n <= 1) shrink_chunk<1, RBMAX == 4 ? 2 : 3>(a, aseg, s_src, n, ks, s_part, s_z, 0, k8);
+    else if (n <= 2) shrink_chunk<2, 2>(a, aseg, s_src, n, ks, s_part, s_z, 0, k8);
+    else if (RBMAX == 4 || n <= 4) shrink_chunk<4, 1>(a, aseg, s_src, n, ks, s_part, s_z, 0, k8);
+    else shrink_chunk<8, 1>(a, aseg, s_src, n, ks, s_part, s_z, 0, k8);
     __syncthreads();
     if (a.z_out != nullptr) {  // shrink only: z rows (bf16) for the GEMM's expand steps
       for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x)
@@ -377,34 +383,192 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
   }
 }
 
+// ---- split form for adapters with long A rows (r K >= 64 Ki elements): the shrink runs
+// on CTAs (segment, K slice of LS_KSLICE, row-chunk lane), each writing fp32 partials
+// z_part[slice][row][r]; then one CTA per (segment, feature slice, row-chunk lane) sums
+// the partials in slice order (deterministic) and expands (delta) or stores z (bf16).
+// Short load chains per CTA, and four to eight times the CTAs of the fused kernel.
+constexpr int LS_KSLICE = 1024;
+
+template <int RBMAX>
+__global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_shrink_part_kernel(const LoraDeltaArgs a, int ks) {
+  constexpr int rb = RBMAX;
+  __shared__ int s_src[LF_RB_MAX];
+  __shared__ float s_z[LF_RB_MAX * 128];
+  __shared__ float s_part[64 * LF_RB_MAX];
+  if (blockIdx.x >= *a.item_count) return;
+  const int2 item = a.items[blockIdx.x];
+  SegInfo si = segment_info(a, item.x, false);
+  si.lo = item.y;
+  si.hi = min(si.hi, item.y + rb);
+  const size_t K = a.K;
+  const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
+  if (!do_gather && si.ad < 0) return;
+  const int k8 = a.K / 8;
+  const int kc0 = blockIdx.y * (LS_KSLICE / 8), kc1 = min(k8, kc0 + LS_KSLICE / 8);
+  const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
+  const __nv_bfloat16* aseg = a.lora_a + slot * a.r * K;
+  float* zp = a.z_part + static_cast<size_t>(blockIdx.y) * a.nrows * a.r;
+  for (int c = blockIdx.z; si.lo + c * rb < si.hi; c += gridDim.z) {
+    const int r0 = si.lo + c * rb;
+    const int n = min(rb, si.hi - r0);
+    __syncthreads();
+    if (threadIdx.x < LF_RB_MAX)
+      s_src[threadIdx.x] = (threadIdx.x < n) ? (a.gather ? a.gather[r0 + threadIdx.x] / a.gather_div : r0 + threadIdx.x) : 0;
+    __syncthreads();
+    if (do_gather) {
+      for (int idx = threadIdx.x; idx < n * k8; idx += blockDim.x) {
+        const int j = idx / k8, cc = idx - j * k8;
+        reinterpret_cast<uint4*>(a.gather_dst + (r0 + j) * K)[cc] =
+            __ldg(reinterpret_cast<const uint4*>(a.src + s_src[j] * K) + cc);
+      }
+    }
+    if (si.ad < 0) continue;
+    if (n <= 1) shrink_chunk<1, RBMAX == 4 ? 2 : 3>(a, aseg, s_src, n, ks, s_part, s_z, kc0, kc1);
+    else if (n <= 2) shrink_chunk<2, 2>(a, aseg, s_src, n, ks, s_part, s_z, kc0, kc1);
+    else if (RBMAX == 4 || n <= 4) shrink_chunk<4, 1>(a, aseg, s_src, n, ks, s_part, s_z, kc0, kc1);
+    else shrink_chunk<8, 1>(a, aseg, s_src, n, ks, s_part, s_z, kc0, kc1);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x) zp[static_cast<size_t>(r0) * a.r + idx] = s_z[idx];
+  }
+}
+
+template <int RBMAX>
+__global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_expand_part_kernel(const LoraDeltaArgs a, int nks,
+                                                                                    int slice) {
+  constexpr int rb = RBMAX;
+  __shared__ float s_z[LF_RB_MAX * 128];
+  if (blockIdx.x >= *a.item_count) return;
+  const int2 item = a.items[blockIdx.x];
+  SegInfo si = segment_info(a, item.x, false);
+  si.lo = item.y;
+  si.hi = min(si.hi, item.y + rb);
+  const int f_lo = blockIdx.y * slice, f_hi = min(a.NB, f_lo + slice);
+  const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
+  const __nv_bfloat16* bseg = a.lora_b + slot * a.r * a.NB;
+  const size_t pstride = static_cast<size_t>(a.nrows) * a.r;
+  for (int c = blockIdx.z; si.lo + c * rb < si.hi; c += gridDim.z) {
+    const int r0 = si.lo + c * rb;
+    const int n = min(rb, si.hi - r0);
+    if (si.ad < 0) {
+      if (a.delta == nullptr) continue;  // z only: the GEMM skips rows without an adapter
+      const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int w4 = (f_hi - f_lo) / 4;
+      for (int idx = threadIdx.x; idx < n * w4; idx += blockDim.x) {
+        const int j = idx / w4, cc = idx - j * w4;
+        reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f_lo)[cc] = z4;
+      }
+      continue;
+    }
+    __syncthreads();  // s_z of the previous chunk is no longer read
+    for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x) {
+      const float* zp = a.z_part + static_cast<size_t>(r0) * a.r + idx;
+      float sum = 0.f;
+      for (int ky = 0; ky < nks; ++ky) sum += __ldcg(zp + ky * pstride);
+      s_z[idx] = sum;
+      if (a.z_out != nullptr && blockIdx.y == 0) a.z_out[static_cast<size_t>(r0) * a.r + idx] = __float2bfloat16_rn(sum);
+    }
+    __syncthreads();
+    if (a.delta == nullptr) continue;
+    for (int f = f_lo + threadIdx.x * 8; f < f_hi; f += blockDim.x * 8) {
+      if (n <= 1) expand_thread<1, 8>(a, bseg + f, s_z, n, r0, f);
+      else if (n <= 2) expand_thread<2, 8>(a, bseg + f, s_z, n, r0, f);
+      else if (RBMAX == 4 || n <= 4) expand_thread<4, 8>(a, bseg + f, s_z, n, r0, f);
+      else expand_thread<8, 8>(a, bseg + f, s_z, n, r0, f);
+    }
+  }
+}
+
+int lora_rows_per_chunk(int nrows, int nseg) { return (nrows >= 8LL * (nseg > 0 ? nseg : 1)) ? 8 : 4; }
+
+int lora_items_bound(int nrows, int nseg, int rb) {
+  return (nrows + rb - 1) / rb + (nseg < nrows ? nseg : nrows);
+}
+
+// Work list of the LoRA kernels: one item (segment q, first row) per chunk of up to rb
+// rows of every non-empty segment, in segment order; also the sanity checks of the
+// offsets and adapter ids (device status).  One CTA: contiguous ranges of segments per
+// thread, block-wide exclusive scan of the item counts.
+__global__ void __launch_bounds__(1024) lora_plan_kernel(const int32_t* __restrict__ off,
+                                                         const int32_t* __restrict__ seg_adapter, int nseg, int L,
+                                                         int nrows, int rb, int2* __restrict__ items,
+                                                         int* __restrict__ count, int cap, int* status) {
+  __shared__ int s_scan[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = (nseg + blockDim.x - 1) / blockDim.x;
+  const int q0 = threadIdx.x * per, q1 = min(nseg, q0 + per);
+  if (threadIdx.x == 0 && (off[0] != 0 || off[nseg] != nrows)) set_status(status, MOE_LORA_ERR_DEVICE_CHECK, -1);
+  int local = 0;
+  for (int q = q0; q < q1; ++q) {
+    const int a0 = off[q], a1 = off[q + 1];
+    if (a0 > a1) set_status(status, MOE_LORA_ERR_DEVICE_CHECK, q);
+    if (seg_adapter != nullptr && (seg_adapter[q] < -1 || seg_adapter[q] >= L))
+      set_status(status, MOE_LORA_ERR_DEVICE_CHECK, q);
+    const int lo = max(a0, 0), hi = min(a1, nrows);
+    if (hi > lo) local += (hi - lo + rb - 1) / rb;
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_scan[warp] = incl;
+  __syncthreads();
+  int base = incl - local;
+  for (int w = 0; w < warp; ++w) base += s_scan[w];
+  for (int q = q0; q < q1; ++q) {
+    const int lo = max(off[q], 0), hi = min(off[q + 1], nrows);
+    for (int r0 = lo; r0 < hi; r0 += rb, ++base)
+      if (base < cap) items[base] = make_int2(q, r0);
+  }
+  if (threadIdx.x == blockDim.x - 1) *count = min(base, cap);
+}
+
+cudaError_t launch_lora_plan(const LoraDeltaArgs& a, cudaStream_t st) {
+  if (a.nrows <= 0) return cudaSuccess;
+  ProfScope ps(K_LORA, st);
+  lora_plan_kernel<<<1, 1024, 0, st>>>(a.seg_offsets, a.seg_adapter, a.nseg, a.L, a.nrows, a.rb, a.items,
+                                       a.item_count, a.items_bound, a.status);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
   if (a.nrows <= 0) return cudaSuccess;
   if (a.r > 128 || a.r % 8 != 0 || a.NB % 8 != 0) return cudaErrorInvalidValue;
+  if (a.items == nullptr || a.item_count == nullptr || (a.rb != 4 && a.rb != 8)) return cudaErrorInvalidValue;
   const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
   if (!lora && a.gather_dst == nullptr) return cudaSuccess;  // nothing to do
-  const int nseg = a.nseg > 0 ? a.nseg : 1;
-  // rows per chunk: 8 when segments are long (prefill), 4 at decode sizes
-  const int rb = (a.nrows >= 8LL * nseg) ? 8 : 4;
-  const long long chunks = (a.nrows + rb - 1) / rb;
-  // row-chunk lanes: a long segment's chunks run on up to 16 CTAs
-  long long zs = (8 * chunks + nseg - 1) / nseg;
-  const int zsplit = static_cast<int>(zs < 1 ? 1 : (zs > 16 ? 16 : zs));
+  const int bound = a.items_bound;
   // K split of the shrink over warps: every warp owns 8 rank rows (r <= 64)
   const int ks = lora ? (a.r >= 64 ? 1 : 64 / a.r) : 1;
-  // feature slices: enough CTAs for two per SM when the chunks are few
+  // feature slices of the expand: enough CTAs for two per SM when the items are few
   int nsplit = 1;
   if (lora && a.delta != nullptr) {
-    const long long busy = std::min<long long>(static_cast<long long>(nseg) * zsplit, chunks + std::min(nseg, a.nrows));
-    const long long want = (2LL * (a.num_sms > 0 ? a.num_sms : 148) + busy - 1) / std::max(1LL, busy);
+    const long long want = (2LL * (a.num_sms > 0 ? a.num_sms : 148) + bound - 1) / std::max(1, bound);
     const long long cap = std::max(1, a.NB / 512);
     nsplit = static_cast<int>(std::max(1LL, std::min(want, cap)));
   }
   int slice = (a.NB + nsplit - 1) / nsplit;
   slice = (slice + 7) / 8 * 8;
   nsplit = (a.NB + slice - 1) / slice;
-  dim3 grid(a.nseg, nsplit, zsplit);
+  const int nks = (a.K + LS_KSLICE - 1) / LS_KSLICE;
+  if (lora && a.z_part != nullptr && static_cast<long long>(a.r) * a.K >= 65536 && nks > 1 &&
+      static_cast<long long>(nks) * a.nrows * a.r <= a.z_part_cap) {
+    ProfScope ps(K_LORA, st);
+    dim3 g1(bound, nks);
+    if (a.rb == 8) lora_shrink_part_kernel<8><<<g1, 256, 0, st>>>(a, ks);
+    else lora_shrink_part_kernel<4><<<g1, 256, 0, st>>>(a, ks);
+    dim3 g2(bound, a.delta != nullptr ? nsplit : 1);
+    if (a.rb == 8) lora_expand_part_kernel<8><<<g2, 256, 0, st>>>(a, nks, slice);
+    else lora_expand_part_kernel<4><<<g2, 256, 0, st>>>(a, nks, slice);
+    count_launch(2);
+    return cudaGetLastError();
+  }
+  dim3 grid(bound, nsplit);
   ProfScope ps(K_LORA, st);
-  if (rb == 8) lora_fused_kernel<8><<<grid, 256, 0, st>>>(a, ks, slice);
+  if (a.rb == 8) lora_fused_kernel<8><<<grid, 256, 0, st>>>(a, ks, slice);
   else lora_fused_kernel<4><<<grid, 256, 0, st>>>(a, ks, slice);
   count_launch();
   return cudaGetLastError();

@@ -23,6 +23,8 @@ SMALL = [
     synth.MoEShape("s_kE", 206, E=4, k=4, H=128, I=64, L=1, r=16),
     synth.MoEShape("s_E1", 207, E=1, k=1, H=256, I=384, L=3, r=16),
     synth.MoEShape("s_bias_zipf", 208, E=16, k=8, H=512, I=320, L=8, r=32, bias=True, adapter_dist="zipf"),
+    # r K >= 65536: the LoRA shrink splits K over CTAs (slices of 1024, ragged last slice)
+    synth.MoEShape("s_split", 209, E=4, k=2, H=1032, I=1096, L=3, r=64, no_adapter_frac=0.2),
 ]
 
 
@@ -48,7 +50,8 @@ def test_forward_every_n_tile(bn, where, monkeypatch):
 
 @pytest.mark.parametrize("where", ["gemm", "delta"])
 @pytest.mark.parametrize("shape,M", [(SMALL[1], 37), (SMALL[2], 300), (SMALL[3], 37), (SMALL[7], 37),
-                                     (SMALL[8], 300), (SMALL[8], 1)], ids=lambda v: getattr(v, "name", str(v)))
+                                     (SMALL[8], 300), (SMALL[8], 1), (SMALL[9], 37), (SMALL[9], 300)],
+                         ids=lambda v: getattr(v, "name", str(v)))
 def test_forward_expand_placement(shape, M, where, monkeypatch):
     """Both placements of the LoRA expand on ragged shapes, r = 8 .. 128, E = 1."""
     monkeypatch.setenv("MOE_LORA_EXPAND", where)

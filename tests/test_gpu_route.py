@@ -116,9 +116,11 @@ def test_route_deterministic():
 
 
 @pytest.mark.parametrize("M,E,k,L,H", [(1, 64, 8, 8, 2048), (64, 128, 8, 32, 7168), (128, 64, 8, 8, 512),
-                                       (129, 64, 8, 8, 512), (40, 256, 4, 64, 264), (7, 5, 5, 0, 64)])
+                                       (129, 64, 8, 8, 512), (40, 256, 4, 64, 264), (7, 5, 5, 0, 64),
+                                       (300, 128, 8, 16, 1024), (260, 256, 4, 4, 264), (1000, 20, 2, 3, 136)])
 def test_route_from_x_exact_on_gpu_logits(M, E, k, L, H):
-    """Both routing launches (one-launch path for M k <= 1024, three kernels above it):
+    """All routing launches (one launch for M k <= 1024; above it SIMT logits for M < 256
+    and tensor-core logits from M = 256, then top-k and sort kernels):
     ids, weights, pairs and offsets equal the oracle's routing of the GPU's own fp32
     logits; the logits themselves agree with the fp64 oracle within fp32 error."""
     g = np.random.default_rng(M * 31 + E)

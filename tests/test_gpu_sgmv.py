@@ -21,6 +21,9 @@ CASES = [
     synth.DENSE_DECODE_BF16.with_(name="bf16_prefillish", wid=302, T=300, h_in=256, h_out=640, L=4,
                                   r=64, adapter_dist="uniform"),
     synth.DENSE_DECODE_BF16.with_(name="bf16_r128", wid=303, T=9, h_in=128, h_out=136, L=2, r=128),
+    # r h_in >= 65536: split LoRA shrink with a ragged last K slice
+    synth.DENSE_DECODE_BF16.with_(name="bf16_split", wid=304, T=45, h_in=2056, h_out=264, L=5, r=32,
+                                  no_adapter_frac=0.2),
 ]
 
 
