@@ -45,7 +45,7 @@ L2_BYTES = 126 * 1024 * 1024
 # ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM on the
 # default workload, with the hash of the kernel source it was taken on; reported as
 # null when the source has changed since.  Filled from profiles/.
-NCU_TRAFFIC = {"gemm_tc.cu": "2c17de826e7599dc", "bytes_per_launch": 746.700032e6 + 5.458432e6,
+NCU_TRAFFIC = {"gemm_tc.cu": "bb8ee476571e2e05", "bytes_per_launch": 746.664192e6 + 6.996224e6,
                "workload": synth.MOE_DECODE_BF16.name, "M": 64}
 
 
@@ -163,15 +163,27 @@ def routing_stats(rt: dict, shape: synth.MoEShape):
     return experts, pairs
 
 
+def expand_in_gemm(shape, M) -> bool:
+    """The library's placement rule for the LoRA expand (inside the GEMM above 64 rows
+    per expert, else the LoRA kernel's fp32 delta)."""
+    return M * shape.k > 64 * shape.E
+
+
 def gateup_alg_bytes(shape, M, experts, pairs):
     """Bytes the gate_up GEMM must move once: touched expert gate_up weights, the
-    gathered x rows (bf16, or two e4m3 planes and their scales), the z rows and the
-    touched B_gu slices of the LoRA expand it runs, and the act it writes."""
+    gathered x rows (bf16, or two e4m3 planes and their scales), its LoRA input (the
+    fp32 delta, or the z rows and touched B_gu slices when it runs the expand), and the
+    act it writes."""
     wb = 1 if shape.wdtype == "e4m3" else 2
     mk = M * shape.k
     xb = mk * (2 * shape.H + 8) if shape.wdtype == "e4m3" else mk * shape.H * 2
-    return (experts * 2 * shape.I * shape.H * wb + xb + mk * shape.r * 2
-            + pairs * shape.r * 2 * shape.I * 2 + mk * shape.I * 2)
+    if shape.L == 0:
+        lora = 0
+    elif expand_in_gemm(shape, M):
+        lora = mk * shape.r * 2 + pairs * shape.r * 2 * shape.I * 2
+    else:
+        lora = mk * 2 * shape.I * 4
+    return experts * 2 * shape.I * shape.H * wb + xb + lora + mk * shape.I * 2
 
 
 def gateup_alg_flops(shape, M):
