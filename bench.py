@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the base-only and same-adapter variants of the MoE step")
     ap.add_argument("--no-graph", action="store_true",
                     help="time plain API calls instead of replaying a CUDA graph of them")
     return ap.parse_args()
@@ -636,6 +638,43 @@ def main():
     ms_max = max_over_ranks(ms, world)
     value = world * M * args.steps / (ms_max / 1e3)
 
+    # ---- secondary measurements: the same step with every adapter id -1 (base only, the
+    #      LoRA work skipped by segment) and with one adapter for every token
+    secondary = None
+    if not args.no_secondary and not args.no_graph:
+        def timed_variant(ids_fn):
+            vb = [(xb, ids_fn(ab)) for xb, ab in batches]
+            vgraphs = []
+            for b, (xb, ab) in enumerate(vb):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    rt = ml.route(ab, k, L, x=xb, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
+                    ml.forward(xb, rt, W, k=k, L=L, y=y, workspace=fws)
+                vgraphs.append(g)
+            n = min(args.steps, 1000)
+            for i in range(min(args.warmup, 20)):
+                vgraphs[i % len(vgraphs)].replay()
+            torch.cuda.synchronize()
+            v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            v0.record()
+            for i in range(n):
+                vgraphs[i % len(vgraphs)].replay()
+            v1.record()
+            torch.cuda.synchronize()
+            del vgraphs
+            return v0.elapsed_time(v1) / n
+
+        t_none = timed_variant(lambda ab: torch.full_like(ab, -1))
+        t_same = timed_variant(lambda ab: torch.zeros_like(ab)) if L > 0 else None
+        t_main = ms_max / args.steps
+        secondary = {
+            "lora_overhead_ms_per_step": t_main - t_none, "base_only_ms_per_step": t_none,
+            "same_adapter_ms_per_step": t_same, "distinct_adapters_ms_per_step": t_main,
+            "adapters": f"{shape.adapter_dist} over L={L}",
+            "swap_ab": "not measured: only the swapped (weights in the 128-row MMA M slot) tile exists; "
+                       "a non-swapped tile would put <= 64 tokens per expert in M = 128",
+        }
+
     # ---- e2e: pinned host inputs -> device, route + forward, y -> pinned host, every step
     e2e_steps = args.e2e_steps or args.steps
     hx = [b[0].cpu().pin_memory() for b in batches]
@@ -730,6 +769,8 @@ def main():
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if secondary is not None:
+        line["secondary"] = secondary
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, calls, n, el = oracle_tokens_per_s(shape, M, cpu, seconds=args.cpu_seconds)
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",

@@ -160,8 +160,16 @@ int shrink_rows_per_cta(long long rows) {
   return static_cast<int>(rb);
 }
 
+// Stream-K scratch of the grouped GEMM (few tiles): flags right after the status word,
+// so the per-call clear of the status also re-arms them, and the partial accumulators.
+constexpr int kSkSlots = 160;                       // >= SMs of the device
+constexpr size_t kSkFlagBytes = kSkSlots * 4;
+constexpr size_t kSkPartFloats = static_cast<size_t>(kSkSlots) * 128 * 64;
+
 struct ForwardWs {
   int* status;
+  int* sk_flag;
+  float* sk_part;
   __nv_bfloat16* x_sorted;
   __nv_bfloat16* act;
   float* delta_gu;     // expand in the LoRA kernel: deltas the GEMM epilogues add
@@ -189,6 +197,7 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
     return p;
   };
   w.status = reinterpret_cast<int*>(b);
+  w.sk_flag = reinterpret_cast<int*>(take(mk > 0 ? kSkFlagBytes : 0));  // must stay first
   w.x_sorted = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
   w.act = reinterpret_cast<__nv_bfloat16*>(take(mk * I * 2));
   w.delta_gu = reinterpret_cast<float*>(take(r && !fused ? mk * 2 * I * 4 : 0));
@@ -198,6 +207,7 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
   w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
   w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, 4)) * 8));
   w.item_count = reinterpret_cast<int*>(take(mk > 0 ? 4 : 0));
+  w.sk_part = reinterpret_cast<float*>(take(mk > 0 ? kSkPartFloats * 4 : 0));
   w.o = reinterpret_cast<float*>(take(mk * H * 4));
   const size_t kmax = H > I ? H : I;
   w.q_hi = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
@@ -235,6 +245,8 @@ RouteWs route_layout(void* base, int M, int E, int L) {
 
 struct DenseWs {
   int* status;
+  int* sk_flag;         // bf16 path: stream-K scratch (see ForwardWs)
+  float* sk_part;
   float* z;             // fp32 path: shrink output
   int32_t* row_adapter; // fp32 path
   float* delta;         // bf16 path, expand in the LoRA kernel: delta the GEMM adds
@@ -256,6 +268,7 @@ DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, bo
     return p;
   };
   w.status = reinterpret_cast<int*>(b);
+  if (!f32) w.sk_flag = reinterpret_cast<int*>(take(T > 0 ? kSkFlagBytes : 0));  // must stay first
   if (f32) {
     w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
     w.row_adapter = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
@@ -266,6 +279,7 @@ DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, bo
     w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
     w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(T, T, 4)) * 8));
     w.item_count = reinterpret_cast<int*>(take(T > 0 ? 4 : 0));
+    w.sk_part = reinterpret_cast<float*>(take(T > 0 ? kSkPartFloats * 4 : 0));
   }
   w.bytes = off;
   return w;
@@ -480,7 +494,8 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8, fused, E * (L + 1));
   const int mk = M * k;
   const int nkeys = E * (L + 1);
-  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+  // status word and the stream-K flags that follow it
+  ML_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes + kSkFlagBytes, cs), "status clear");
 
   // 1. gather x rows into (expert, adapter) order; gate_up LoRA shrink z = x A_gu per
   //    (adapter, expert) segment; the expand z B_gu either runs here (delta_gu, added
@@ -511,6 +526,11 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   l1.items_bound = lora_items_bound(mk, nkeys, l1.rb);
   l1.items = w.items;
   l1.item_count = w.item_count;
+  if (fp8) {  // the same kernel writes the e4m3 planes of the gathered x rows
+    l1.q_hi = w.q_hi;
+    l1.q_lo = w.q_lo;
+    l1.q_scales = w.q_scales;
+  }
   ML_CUDA(launch_lora_plan(l1, cs), "LoRA plan launch");
   ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
 
@@ -547,12 +567,15 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.bn = choose_bn(mk, E);
   if (fp8) {
     if (g.bn > 64) g.bn = 64;  // e4m3 tiles use the prefetching epilogue (N <= 64)
-    ML_CUDA(launch_quant_planes(w.x_sorted, mk, H, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
     g.b_hi = w.q_hi;
     g.b_lo = w.q_lo;
     g.b_scales = w.q_scales;
   }
   g.num_sms = num_sms();
+  g.sk_part = w.sk_part;
+  g.sk_part_cap = static_cast<long long>(kSkPartFloats);
+  g.sk_flag = w.sk_flag;
+  g.sk_slots = kSkSlots;
   ML_CUDA(launch_gemm_tc(g, cs), "gate_up GEMM launch");
 
   // 3. down LoRA shrink + expand on act: delta_d = (act A_d) B_d
@@ -586,7 +609,8 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   d.scale_idx = 1;
   d.w = w_down;
   d.b = w.act;
-  if (fp8) ML_CUDA(launch_quant_planes(w.act, mk, I, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
+  if (fp8 && !rr)  // with adapters the down LoRA kernel wrote the planes of act
+    ML_CUDA(launch_quant_planes(w.act, mk, I, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
   ML_CUDA(launch_gemm_tc(d, cs), "down GEMM launch");
 
   // 5. fixed-order combine over the k slots
@@ -705,7 +729,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   if (st != MOE_LORA_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const DenseWs ws = dense_layout(workspace, T, h_in, h_out, rr, f32, fused);
-  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+  ML_CUDA(cudaMemsetAsync(workspace, 0, f32 ? 8 : kStatusBytes + kSkFlagBytes, cs), "status clear");
 
   if (f32) {
     ShrinkArgs a{};
@@ -799,6 +823,10 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   g.b = static_cast<const __nv_bfloat16*>(x);
   g.bn = choose_bn(T, 1);
   g.num_sms = num_sms();
+  g.sk_part = ws.sk_part;
+  g.sk_part_cap = static_cast<long long>(kSkPartFloats);
+  g.sk_flag = ws.sk_flag;
+  g.sk_slots = kSkSlots;
   ML_CUDA(launch_gemm_tc(g, cs), "dense GEMM launch");
   return MOE_LORA_OK;
 }

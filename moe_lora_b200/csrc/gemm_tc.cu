@@ -43,6 +43,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 namespace mlb {
@@ -87,7 +88,60 @@ struct TcParams {
   int lseg_count;
   const int32_t* lseg_adapter;  // adapter of candidate c (null: adapter = c)
   int L;
+  // stream-K (few tiles): CTA b takes the (tile, K stage) iterations
+  // [b T / G, (b + 1) T / G) of T = tiles * stages; a CTA that starts inside a tile writes
+  // its partial accumulator to sk_part[b] and raises sk_flag[b]; the CTA holding the
+  // tile's first stages adds the partials in CTA order and runs the epilogue
+  int sk;
+  float* sk_part;               // [grid][128][BN] fp32
+  int* sk_flag;                 // [grid], zero on entry, zero again on exit
 };
+
+// A unit of work: tile t, K stages [k0, k1).
+struct Unit {
+  int t, k0, k1;
+};
+struct UnitIter {
+  long long pos, end;
+  int t;
+};
+
+__device__ __forceinline__ long long sk_start(long long b, long long T, long long G) { return b * T / G; }
+// CTA whose stream-K range holds iteration i
+__device__ __forceinline__ int sk_owner(long long i, long long T, long long G) {
+  return static_cast<int>(((i + 1) * G + T - 1) / T - 1);
+}
+
+// CTA bb's stream-K range is non-empty (it holds at least one iteration)
+__device__ __forceinline__ bool sk_busy(long long bb, long long T, long long G) {
+  return sk_start(bb, T, G) < sk_start(bb + 1, T, G);
+}
+
+__device__ __forceinline__ UnitIter unit_begin(const TcParams& p, int total_tiles, int nk) {
+  UnitIter it;
+  it.t = blockIdx.x;
+  const long long T = static_cast<long long>(total_tiles) * nk;
+  it.pos = sk_start(blockIdx.x, T, gridDim.x);
+  it.end = sk_start(blockIdx.x + 1, T, gridDim.x);
+  return it;
+}
+
+__device__ __forceinline__ bool unit_next(const TcParams& p, int total_tiles, int nk, UnitIter& it, Unit& u) {
+  if (!p.sk) {
+    if (it.t >= total_tiles) return false;
+    u.t = it.t;
+    u.k0 = 0;
+    u.k1 = nk;
+    it.t += gridDim.x;
+    return true;
+  }
+  if (it.pos >= it.end) return false;
+  u.t = static_cast<int>(it.pos / nk);
+  u.k0 = static_cast<int>(it.pos - static_cast<long long>(u.t) * nk);
+  u.k1 = static_cast<int>(min(static_cast<long long>(nk), u.k0 + (it.end - it.pos)));
+  it.pos += u.k1 - u.k0;
+  return true;
+}
 
 // Non-pipeline shared memory, placed after the stage rings.
 struct SmemCore {
@@ -336,9 +390,11 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       }
       return got;
     };
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    UnitIter uit = unit_begin(p, total_tiles, nk);
+    Unit u;
+    while (ok && unit_next(p, total_tiles, nk, uit, u)) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0, 0)) break;  // warp-uniform
-      const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
+      const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
       int wrow0, wrow1;
       if (p.epi == EPI_GATEUP) {
         wrow0 = ti.g * p.rows_per_group + ti.mt * 64;
@@ -347,7 +403,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
         wrow0 = ti.g * p.rows_per_group + ti.mt * kBM;
         wrow1 = wrow0 + 64;
       }
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = u.k0; kb < u.k1; ++kb) {
         ok = acquire(1);
         if (!ok) break;
         if (lane == 0) {
@@ -422,10 +478,12 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
+      UnitIter uit = unit_begin(p, total_tiles, nk);
+      Unit u;
+      for (; !*abort_flag && unit_next(p, total_tiles, nk, uit, u); ++it) {
         // the last chunk of a group is ragged: N = its rows rounded up to 16, so a
         // skewed expert load does not pay MMAs on padding rows
-        const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
+        const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
         const int n_mma = min(BN, (ti.nvalid + 15) & ~15);
         const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, n_mma) : umma_idesc_bf16(kBM, n_mma);
         const int buf = it & 1;
@@ -434,7 +492,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * Cfg::kAccPerBuf * Cfg::kAccStride;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = u.k0; kb < u.k1; ++kb) {
           if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 3)) {
             ok = false;
             break;
@@ -445,7 +503,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           const uint64_t bdesc = umma_desc_sw128(a_addr + kATileBytes);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
-            const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
+            const uint32_t acc = (kb != u.k0 || k != 0) ? 1u : 0u;
             if constexpr (W8) {
               const uint64_t ldesc = umma_desc_sw128(a_addr + kATileBytes + Cfg::kBTileBytes);
               umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
@@ -502,12 +560,41 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     const int g4 = warp & 3;           // TMEM lane quarter this warp may access
     const int m = g4 * 32 + lane;      // accumulator row = weight row within the tile
     int it = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
+    UnitIter uit = unit_begin(p, total_tiles, nk);
+    Unit u;
+    const long long skT = static_cast<long long>(total_tiles) * nk;
+    for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
+      const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 4);
       if constexpr (Cfg::kPrefetch) got = got && mbar_wait(&sm.sfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 7);
+      // stream-K roles: a later part stores its partial; the first part of a split tile
+      // waits (bounded) for the later parts' flags, then adds their partials in CTA order
+      const bool sk_store = p.sk && u.k0 != 0;
+      int sk_b1 = 0, sk_b2 = -1;  // CTAs holding the later parts of this tile
+      if (p.sk && u.k0 == 0 && u.k1 != nk) {
+        sk_b1 = static_cast<int>(blockIdx.x) + 1;
+        sk_b2 = sk_owner(static_cast<long long>(u.t) * nk + nk - 1, skT, gridDim.x);
+        if (got && et == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          for (int bb = sk_b1; bb <= sk_b2 && got; ++bb) {
+            if (!sk_busy(bb, skT, gridDim.x)) continue;  // empty range: holds no part
+            while (ld_acquire_gpu(p.sk_flag + bb) == 0) {
+              if (*abort_flag) {
+                got = false;
+                break;
+              }
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                set_status(p.status, MOE_LORA_ERR_TIMEOUT, 11);
+                got = false;
+                break;
+              }
+            }
+          }
+        }
+      }
       if (!named_bar_and(2, kEpiThreads, got)) break;  // the four warps leave together
       tc_fence_after();
 
@@ -554,6 +641,26 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
         } else {
 #pragma unroll
           for (int n = 0; n < 32; ++n) v[n] *= scale;
+        }
+        if (sk_store) {  // later part of a split tile: keep the partial, nothing else
+          float4* dst = reinterpret_cast<float4*>(p.sk_part + (static_cast<size_t>(blockIdx.x) * kBM + m) * BN + c0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (c0 + 4 * q < BN) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          continue;
+        }
+        for (int bb = sk_b1; bb <= sk_b2; ++bb) {  // first part: add the later parts in order
+          if (!sk_busy(bb, skT, gridDim.x)) continue;
+          const float4* src = reinterpret_cast<const float4*>(p.sk_part + (static_cast<size_t>(bb) * kBM + m) * BN + c0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (c0 + 4 * q < BN) {
+              const float4 w4 = __ldcg(src + q);
+              v[4 * q] += w4.x;
+              v[4 * q + 1] += w4.y;
+              v[4 * q + 2] += w4.z;
+              v[4 * q + 3] += w4.w;
+            }
         }
         if (p.delta != nullptr) {
           if constexpr (Cfg::kPrefetch) {
@@ -628,6 +735,18 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             tmem_zero_32x32b_x32(tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) +
                                  (buf * Cfg::kAccPerBuf + 2) * Cfg::kAccStride + c);
       }
+      if (sk_store || sk_b2 >= sk_b1) {
+        __threadfence();                 // this thread's partial row is visible GPU-wide
+        named_bar_sync(1, kEpiThreads);  // every partial row stored / every partial read
+        if (et == 0) {
+          if (sk_store) {
+            __threadfence();
+            st_release_gpu(p.sk_flag + blockIdx.x, 1);
+          } else {
+            for (int bb = sk_b1; bb <= sk_b2; ++bb) p.sk_flag[bb] = 0;  // consumed: re-armed for the next launch
+          }
+        }
+      }
       tc_fence_before();
       mbar_arrive(&sm.tempty[buf]);
       if constexpr (Cfg::kPrefetch) mbar_arrive(&sm.sempty[buf]);
@@ -637,8 +756,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     if constexpr (Cfg::kPrefetch) {
       uint32_t issued_mask = 0, issued_parity = 0;
       int it = 0;
-      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
-        const TileInfo ti = decode_tile(sm, t, p.m_tiles, p.E, BN);
+      UnitIter uit = unit_begin(p, total_tiles, nk);
+      Unit u;
+      for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
+        const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         const bool got = mbar_wait(&sm.sempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 8);
@@ -800,7 +921,21 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
   const long long tiles_ub = chunks_ub * p.m_tiles;
   int grid = a.num_sms;
-  if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
+  // stream-K when the tiles would leave SMs idle or unbalanced (< two waves)
+  p.sk = 0;
+  p.sk_part = a.sk_part;
+  p.sk_flag = a.sk_flag;
+  // Opt-in (MOE_LORA_STREAMK=1), for fewer than two tiles per SM.  Measured on the dense
+  // decode GEMM (86 tiles): all SMs stream but each at half the rate, 40.6 us against
+  // 36.3 us for 86 whole tiles, so whole tiles stay the default.
+  const char* skv = std::getenv("MOE_LORA_STREAMK");
+  const bool sk_want = skv != nullptr && std::atoi(skv) != 0 && tiles_ub < 2LL * grid;
+  if (a.sk_part != nullptr && a.sk_flag != nullptr && a.z == nullptr && BN <= 64 && sk_want &&
+      grid <= a.sk_slots && static_cast<long long>(grid) * kBM * BN <= a.sk_part_cap) {
+    p.sk = 1;
+  } else {
+    if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
+  }
   if (grid < 1) grid = 1;
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP
                : a.epi == EPI_DOWN ? K_GEMM_DOWN

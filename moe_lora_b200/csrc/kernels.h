@@ -69,6 +69,11 @@ struct LoraDeltaArgs {
   const __nv_bfloat16* lora_b;  // MoE [L][E][r][NB]; dense [L][r][NB]
   float* delta;               // [nrows][NB] (expand in this kernel) or null
   __nv_bfloat16* z_out;       // shrink only: z [nrows][r] bf16 for a GEMM that expands
+  // e4m3 experts: the two activation planes of the source rows (in row order), written
+  // by the CTAs of feature slice / K slice 0 (see launch_quant_planes); null otherwise
+  uint8_t* q_hi;
+  uint8_t* q_lo;
+  float* q_scales;            // [nrows][2]
   float* z_part;              // optional scratch for the split form: [ceil(K / 1024)][nrows][r]
   long long z_part_cap;       // floats available at z_part
   // work list (launch_lora_plan): one item (segment, first row) per chunk of rb rows
@@ -158,6 +163,12 @@ struct GemmArgs {
   int lseg_stride;
   int lseg_count;              // candidates per group
   const int32_t* lseg_adapter; // adapter of candidate c; null: adapter = c
+  // optional stream-K scratch (used when the tiles are fewer than two per SM, N <= 64):
+  // partial accumulators [sk_slots][128][BN] fp32 and flags [sk_slots], zero on entry
+  float* sk_part;
+  long long sk_part_cap;       // floats at sk_part
+  int* sk_flag;
+  int sk_slots;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
 

@@ -161,6 +161,58 @@ cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- e4m3 activation planes
+// s = amax(|x|) / 448 per row (1 for an all-zero row); hi = RNE_sat(x / s) and
+// lo = RNE_sat((x - hi s) / (s / 16)) in OCP e4m3, so that x = s hi + (s / 16) lo up to a
+// relative 2^-8; the FP8-weight GEMM multiplies both planes on the kind::f8f6f4 tensor
+// core.  |x / s| <= 448 and |(x - hi s) / (s / 16)| <= 448 by construction.
+// One warp quantises one bf16 row of K elements into the two e4m3 planes (see below).
+__device__ __forceinline__ void quant_row_warp(const __nv_bfloat16* src_row, int K, uint8_t* hi_row, uint8_t* lo_row,
+                                               float* scale2, int lane) {
+  const uint4* xr = reinterpret_cast<const uint4*>(src_row);
+  const int k8 = K / 8;
+  float amax = 0.f;
+  for (int c = lane; c < k8; c += 32) {
+    float f[8];
+    unpack8_bf16(__ldg(xr + c), f);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) amax = fmaxf(amax, fabsf(f[v]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = amax > 0.f ? amax / 448.f : 1.f;
+  const float inv = 1.f / s, inv_lo = 16.f / s;
+  for (int c = lane; c < k8; c += 32) {
+    float f[8];
+    unpack8_bf16(__ldg(xr + c), f);
+    uint32_t hq[2], lq[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t hw = 0, lw = 0;
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const int v = 4 * h + 2 * pr;
+        const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(make_float2(f[v] * inv, f[v + 1] * inv),
+                                                                __NV_SATFINITE, __NV_E4M3);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
+        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        const __nv_fp8x2_storage_t ql = __nv_cvt_float2_to_fp8x2(
+            make_float2((f[v] - d.x * s) * inv_lo, (f[v + 1] - d.y * s) * inv_lo), __NV_SATFINITE, __NV_E4M3);
+        hw |= static_cast<uint32_t>(q) << (16 * pr);
+        lw |= static_cast<uint32_t>(ql) << (16 * pr);
+      }
+      hq[h] = hw;
+      lq[h] = lw;
+    }
+    reinterpret_cast<uint2*>(hi_row)[c] = make_uint2(hq[0], hq[1]);
+    reinterpret_cast<uint2*>(lo_row)[c] = make_uint2(lq[0], lq[1]);
+  }
+  if (lane == 0) {
+    scale2[0] = s;
+    scale2[1] = s / 16.f;
+  }
+}
+
 // ---------------------------------------------------------------- segmented LoRA for the GEMMs
 // One fused streaming kernel per projection ([Punica review page], "提案手法": SGMV;
 // [vLLM MoE-LoRA page], "O Papel da Multi-LoRA": shrink z = xA then expand zB, and
@@ -327,7 +379,8 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
   const size_t K = a.K;
   const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
   const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
-  if (!do_gather && !lora) return;
+  const bool do_quant = a.q_hi != nullptr && blockIdx.y == 0;
+  if (!do_gather && !do_quant && !lora) return;
   const int f_lo = blockIdx.y * slice, f_hi = min(a.NB, f_lo + slice);
   const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
   const __nv_bfloat16* aseg = a.lora_a + slot * a.r * K;
@@ -346,6 +399,12 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
         reinterpret_cast<uint4*>(a.gather_dst + (r0 + j) * K)[cc] =
             __ldg(reinterpret_cast<const uint4*>(a.src + s_src[j] * K) + cc);
       }
+    }
+    if (do_quant) {  // e4m3 experts: the activation planes of the chunk's rows
+      const int w = threadIdx.x >> 5;
+      if (w < n)
+        quant_row_warp(a.src + s_src[w] * K, a.K, a.q_hi + (r0 + w) * K, a.q_lo + (r0 + w) * K,
+                       a.q_scales + 2 * static_cast<size_t>(r0 + w), threadIdx.x & 31);
     }
     if (!lora) continue;
     if (si.ad < 0) {
@@ -403,7 +462,8 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_shrink_part_kern
   si.hi = min(si.hi, item.y + rb);
   const size_t K = a.K;
   const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
-  if (!do_gather && si.ad < 0) return;
+  const bool do_quant = a.q_hi != nullptr && blockIdx.y == 0;
+  if (!do_gather && !do_quant && si.ad < 0) return;
   const int k8 = a.K / 8;
   const int kc0 = blockIdx.y * (LS_KSLICE / 8), kc1 = min(k8, kc0 + LS_KSLICE / 8);
   const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
@@ -422,6 +482,12 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_shrink_part_kern
         reinterpret_cast<uint4*>(a.gather_dst + (r0 + j) * K)[cc] =
             __ldg(reinterpret_cast<const uint4*>(a.src + s_src[j] * K) + cc);
       }
+    }
+    if (do_quant) {  // e4m3 experts: the activation planes of the chunk's rows
+      const int w = threadIdx.x >> 5;
+      if (w < n)
+        quant_row_warp(a.src + s_src[w] * K, a.K, a.q_hi + (r0 + w) * K, a.q_lo + (r0 + w) * K,
+                       a.q_scales + 2 * static_cast<size_t>(r0 + w), threadIdx.x & 31);
     }
     if (si.ad < 0) continue;
     if (n <= 1) shrink_chunk<1, RBMAX == 4 ? 2 : 3>(a, aseg, s_src, n, ks, s_part, s_z, kc0, kc1);
@@ -539,7 +605,8 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
   if (a.r > 128 || a.r % 8 != 0 || a.NB % 8 != 0) return cudaErrorInvalidValue;
   if (a.items == nullptr || a.item_count == nullptr || (a.rb != 4 && a.rb != 8)) return cudaErrorInvalidValue;
   const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
-  if (!lora && a.gather_dst == nullptr) return cudaSuccess;  // nothing to do
+  if (!lora && a.gather_dst == nullptr && a.q_hi == nullptr) return cudaSuccess;  // nothing to do
+  if (a.q_hi != nullptr && a.K % 16 != 0) return cudaErrorInvalidValue;
   const int bound = a.items_bound;
   // K split of the shrink over warps: every warp owns 8 rank rows (r <= 64)
   const int ks = lora ? (a.r >= 64 ? 1 : 64 / a.r) : 1;
@@ -712,59 +779,15 @@ cudaError_t launch_dense_f32(const DenseF32Args& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------- e4m3 activation planes
-// One warp per row: s = amax(|x|) / 448 (1 for an all-zero row); hi = RNE_sat(x / s) and
-// lo = RNE_sat((x - hi s) / (s / 16)) in OCP e4m3, so that x = s hi + (s / 16) lo up to a
-// relative 2^-8; the FP8-weight GEMM multiplies both planes on the kind::f8f6f4 tensor
-// core.  |x / s| <= 448 and |(x - hi s) / (s / 16)| <= 448 by construction.
+// ---------------------------------------------------------------- activation planes (standalone)
+// One warp per row (quant_row_warp); used when no LoRA kernel reads the rows.
 __global__ void __launch_bounds__(256) quant_planes_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K,
                                                           uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
                                                           float* __restrict__ scales) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k8 = K / 8;
-  for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
-    const uint4* xr = reinterpret_cast<const uint4*>(src + static_cast<size_t>(row) * K);
-    float amax = 0.f;
-    for (int c = lane; c < k8; c += 32) {
-      float f[8];
-      unpack8_bf16(__ldg(xr + c), f);
-#pragma unroll
-      for (int v = 0; v < 8; ++v) amax = fmaxf(amax, fabsf(f[v]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = amax > 0.f ? amax / 448.f : 1.f;
-    const float inv = 1.f / s, inv_lo = 16.f / s;
-    for (int c = lane; c < k8; c += 32) {
-      float f[8];
-      unpack8_bf16(__ldg(xr + c), f);
-      uint32_t hq[2], lq[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t hw = 0, lw = 0;
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          const int v = 4 * h + 2 * pr;
-          const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(make_float2(f[v] * inv, f[v + 1] * inv),
-                                                                  __NV_SATFINITE, __NV_E4M3);
-          const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
-          const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-          const __nv_fp8x2_storage_t ql = __nv_cvt_float2_to_fp8x2(
-              make_float2((f[v] - d.x * s) * inv_lo, (f[v + 1] - d.y * s) * inv_lo), __NV_SATFINITE, __NV_E4M3);
-          hw |= static_cast<uint32_t>(q) << (16 * pr);
-          lw |= static_cast<uint32_t>(ql) << (16 * pr);
-        }
-        hq[h] = hw;
-        lq[h] = lw;
-      }
-      reinterpret_cast<uint2*>(hi + static_cast<size_t>(row) * K)[c] = make_uint2(hq[0], hq[1]);
-      reinterpret_cast<uint2*>(lo + static_cast<size_t>(row) * K)[c] = make_uint2(lq[0], lq[1]);
-    }
-    if (lane == 0) {
-      scales[2 * static_cast<size_t>(row)] = s;
-      scales[2 * static_cast<size_t>(row) + 1] = s / 16.f;
-    }
-  }
+  for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8)
+    quant_row_warp(src + static_cast<size_t>(row) * K, K, hi + static_cast<size_t>(row) * K,
+                   lo + static_cast<size_t>(row) * K, scales + 2 * static_cast<size_t>(row), lane);
 }
 
 cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8_t* hi, uint8_t* lo, float* scales,
