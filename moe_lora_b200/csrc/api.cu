@@ -163,6 +163,7 @@ int shrink_rows_per_cta(long long rows) {
 // Stream-K scratch of the grouped GEMM (few tiles): flags right after the status word,
 // so the per-call clear of the status also re-arms them, and the partial accumulators.
 constexpr int kSkSlots = 160;                       // >= SMs of the device
+constexpr int kShrinkBN = 32;                       // N tile of the tensor-core LoRA shrink
 constexpr size_t kSkFlagBytes = kSkSlots * 4;
 constexpr size_t kSkPartFloats = static_cast<size_t>(kSkSlots) * 128 * 64;
 
@@ -179,6 +180,8 @@ struct ForwardWs {
   long long z_part_cap;
   int2* items;         // LoRA work list and its length
   int* item_count;
+  int2* items_tc;      // expand in the GEMMs: tiles of the tensor-core shrink (adapter segments)
+  int* item_count_tc;
   float* o;
   uint8_t* q_hi;      // e4m3 weights: activation planes [M*k][max(H, I)]
   uint8_t* q_lo;
@@ -207,6 +210,9 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
   w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
   w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, 4)) * 8));
   w.item_count = reinterpret_cast<int*>(take(mk > 0 ? 4 : 0));
+  w.items_tc = reinterpret_cast<int2*>(
+      take(r && fused ? static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, kShrinkBN)) * 8 : 0));
+  w.item_count_tc = reinterpret_cast<int*>(take(r && fused ? 4 : 0));
   w.sk_part = reinterpret_cast<float*>(take(mk > 0 ? kSkPartFloats * 4 : 0));
   w.o = reinterpret_cast<float*>(take(mk * H * 4));
   const size_t kmax = H > I ? H : I;
@@ -255,6 +261,8 @@ struct DenseWs {
   long long z_part_cap;
   int2* items;          // bf16 path: LoRA work list and its length
   int* item_count;
+  int2* items_tc;       // bf16 path, expand in the GEMM: tiles of the tensor-core shrink
+  int* item_count_tc;
   size_t bytes;
 };
 
@@ -279,6 +287,8 @@ DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, bo
     w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
     w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(T, T, 4)) * 8));
     w.item_count = reinterpret_cast<int*>(take(T > 0 ? 4 : 0));
+    w.items_tc = reinterpret_cast<int2*>(take(r && fused ? static_cast<size_t>(lora_items_bound(T, T, kShrinkBN)) * 8 : 0));
+    w.item_count_tc = reinterpret_cast<int*>(take(r && fused ? 4 : 0));
     w.sk_part = reinterpret_cast<float*>(take(T > 0 ? kSkPartFloats * 4 : 0));
   }
   w.bytes = off;
@@ -386,6 +396,44 @@ moe_lora_status moe_lora_check_status(void* workspace, moe_lora_stream stream) {
   if (h[0] == MOE_LORA_OK) return MOE_LORA_OK;
   return fail(static_cast<moe_lora_status>(h[0]), "device-side check failed (code %d, detail %d)", h[0], h[1]);
 }
+
+}  // extern "C"
+
+namespace {
+// z = src A_slot^T per adapter segment on the tensor cores: one tile per chunk of up to
+// kShrinkBN rows of a segment with an adapter (work list from the plan kernel), the
+// slot's r rows of LoRA A in the MMA's M slot, bf16 z rows out.
+cudaError_t launch_shrink_tc(const LoraDeltaArgs& l, int2* items, int* count, int E, cudaStream_t cs) {
+  const int bound = lora_items_bound(l.nrows, l.nseg, kShrinkBN);
+  cudaError_t err = launch_lora_plan_adapters(l, kShrinkBN, items, count, bound, cs);
+  if (err != cudaSuccess) return err;
+  GemmArgs s{};
+  s.epi = EPI_ZOUT;
+  s.K = l.K;
+  s.E = 1;
+  s.group_offsets = nullptr;
+  s.rows_per_group = l.L * E * l.r;
+  s.n_out = l.r;
+  s.total_rows = l.nrows;
+  s.w = l.lora_a;
+  s.b = l.gather_dst ? l.gather_dst : l.src;
+  s.out_bf16 = l.z_out;
+  s.status = l.status;
+  s.bn = kShrinkBN;
+  s.num_sms = l.num_sms;
+  s.items = items;
+  s.item_count = count;
+  s.items_bound = bound;
+  s.lseg_off = l.seg_offsets;
+  s.lseg_adapter = l.seg_adapter;
+  s.L = l.L;
+  s.iE = E;
+  s.r = l.r;
+  return launch_gemm_tc(s, cs);
+}
+}  // namespace
+
+extern "C" {
 
 moe_lora_status moe_lora_route(const void* x, const void* w_router, const float* bias,
                                const float* logits_in, const int32_t* adapter_ids, int M, int H, int E,
@@ -516,8 +564,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   l1.E = E;
   l1.lora_a = static_cast<const __nv_bfloat16*>(lora_a_gu);
   l1.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
-  l1.delta = rr && !fused ? w.delta_gu : nullptr;
-  l1.z_out = rr && fused ? w.z : nullptr;
+  l1.delta = rr && !fused ? w.delta_gu : nullptr;  // fused: this launch only gathers (and quantises)
   l1.z_part = w.z_part;
   l1.z_part_cap = w.z_part_cap;
   l1.status = w.status;
@@ -533,6 +580,11 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   }
   ML_CUDA(launch_lora_plan(l1, cs), "LoRA plan launch");
   ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
+  if (rr && fused) {  // the shrink on the tensor cores, z for the GEMM's expand steps
+    LoraDeltaArgs ls = l1;
+    ls.z_out = w.z;
+    ML_CUDA(launch_shrink_tc(ls, w.items_tc, w.item_count_tc, E, cs), "gate_up LoRA shrink launch");
+  }
 
   // 2. gate_up grouped GEMM; epilogue adds delta_gu and applies SiLU-and-mul -> act
   GemmArgs g{};
@@ -588,9 +640,14 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     l2.NB = H;
     l2.lora_a = static_cast<const __nv_bfloat16*>(lora_a_d);
     l2.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
-    l2.delta = fused ? nullptr : w.delta_d;
-    l2.z_out = fused ? w.z : nullptr;
-    ML_CUDA(launch_lora_delta(l2, cs), "down LoRA launch");
+    if (fused) {
+      l2.z_out = w.z;
+      l2.q_hi = nullptr;  // the planes of act come from the plane kernel below
+      ML_CUDA(launch_shrink_tc(l2, w.items_tc, w.item_count_tc, E, cs), "down LoRA shrink launch");
+    } else {
+      l2.delta = w.delta_d;
+      ML_CUDA(launch_lora_delta(l2, cs), "down LoRA launch");
+    }
   }
 
   // 4. down grouped GEMM; epilogue adds delta_d and the routing weight -> o (per pair)
@@ -609,7 +666,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   d.scale_idx = 1;
   d.w = w_down;
   d.b = w.act;
-  if (fp8 && !rr)  // with adapters the down LoRA kernel wrote the planes of act
+  if (fp8 && (!rr || fused))  // otherwise the down LoRA kernel wrote the planes of act
     ML_CUDA(launch_quant_planes(w.act, mk, I, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
   ML_CUDA(launch_gemm_tc(d, cs), "down GEMM launch");
 
@@ -783,7 +840,6 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     l.lora_a = static_cast<const __nv_bfloat16*>(lora_a);
     l.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
     l.delta = fused ? nullptr : ws.delta;
-    l.z_out = fused ? ws.zb : nullptr;
     l.z_part = ws.z_part;
     l.z_part_cap = ws.z_part_cap;
     l.status = ws.status;
@@ -792,8 +848,13 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     l.items_bound = lora_items_bound(T, S, l.rb);
     l.items = ws.items;
     l.item_count = ws.item_count;
-    ML_CUDA(launch_lora_plan(l, cs), "LoRA plan launch");
-    ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
+    if (fused) {  // the shrink on the tensor cores, z for the GEMM's expand steps
+      l.z_out = ws.zb;
+      ML_CUDA(launch_shrink_tc(l, ws.items_tc, ws.item_count_tc, 1, cs), "dense LoRA shrink launch");
+    } else {
+      ML_CUDA(launch_lora_plan(l, cs), "LoRA plan launch");
+      ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
+    }
   }
   GemmArgs g{};
   g.epi = EPI_DENSE;

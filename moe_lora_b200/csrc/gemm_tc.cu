@@ -95,6 +95,11 @@ struct TcParams {
   int sk;
   float* sk_part;               // [grid][128][BN] fp32
   int* sk_flag;                 // [grid], zero on entry, zero again on exit
+  // item tiles (LoRA shrink on the tensor cores): tile t = items[t] = (segment key q,
+  // first row); A rows = slot (a E + e) * r of LoRA A, N = the segment's rows there
+  const int2* items;
+  const int* item_count;
+  int iE;
 };
 
 // A unit of work: tile t, K stages [k0, k1).
@@ -208,6 +213,23 @@ __device__ __forceinline__ TileInfo decode_tile(const SmemCore& sm, int t, int m
   ti.g = lo;
   ti.row0 = sm.grp_off[lo] + (c - sm.chunk_pref[lo]) * BN;
   ti.nvalid = min(BN, sm.grp_off[lo + 1] - ti.row0);
+  return ti;
+}
+
+// Tile of the LoRA shrink: g = the (adapter, expert) slot, rows from the work item.
+__device__ __forceinline__ TileInfo item_tile(const TcParams& p, int t, int BN) {
+  TileInfo ti;
+  const int2 it = p.items[t];
+  if (p.lseg_adapter != nullptr) {  // dense segments: one group, adapter per segment
+    ti.g = p.lseg_adapter[it.x];
+  } else {                          // MoE keys q = e (L + 1) + a
+    const int LA = p.L + 1;
+    const int e = it.x / LA, a = it.x - e * LA;
+    ti.g = a * p.iE + e;
+  }
+  ti.mt = 0;
+  ti.row0 = it.y;
+  ti.nvalid = max(0, min(BN, p.lseg_off[it.x + 1] - it.y));
   return ti;
 }
 
@@ -354,7 +376,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
   }
-  const int total_tiles = sm.chunk_pref[p.E] * p.m_tiles;
+  const int total_tiles = p.items ? *p.item_count : sm.chunk_pref[p.E] * p.m_tiles;
   const int nk = (p.K + Cfg::kKB - 1) / Cfg::kKB;  // stages per tile
 
   if (warp == 0) {
@@ -394,15 +416,21 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     Unit u;
     while (ok && unit_next(p, total_tiles, nk, uit, u)) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0, 0)) break;  // warp-uniform
-      const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
+      const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
       int wrow0, wrow1;
       if (p.epi == EPI_GATEUP) {
         wrow0 = ti.g * p.rows_per_group + ti.mt * 64;
         wrow1 = ti.g * p.rows_per_group + p.I + ti.mt * 64;
+      } else if (p.epi == EPI_ZOUT) {
+        wrow0 = ti.g * p.r;  // the slot's A rows
+        wrow1 = wrow0 + 64;
       } else {
         wrow0 = ti.g * p.rows_per_group + ti.mt * kBM;
         wrow1 = wrow0 + 64;
       }
+      // r <= 64: the second 64-row half of A is not needed (accumulator rows >= r are
+      // never read), so it is not loaded
+      const bool a_half = p.epi == EPI_ZOUT && p.r <= 64;
       for (int kb = u.k0; kb < u.k1; ++kb) {
         ok = acquire(1);
         if (!ok) break;
@@ -410,9 +438,9 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           uint8_t* a_s = ring + stage * Cfg::kStageBytes;
           uint8_t* b_s = a_s + kATileBytes;
           const int kc = kb * Cfg::kKB;  // first K element of the stage
-          mbar_arrive_expect_tx(&sm.full[stage], Cfg::kStageBytes);
+          mbar_arrive_expect_tx(&sm.full[stage], Cfg::kStageBytes - (a_half ? kATileBytes / 2 : 0));
           tma_load_2d(a_s, &tmw, &sm.full[stage], kc, wrow0);
-          tma_load_2d(a_s + kATileBytes / 2, &tmw, &sm.full[stage], kc, wrow1);
+          if (!a_half) tma_load_2d(a_s + kATileBytes / 2, &tmw, &sm.full[stage], kc, wrow1);
           tma_load_2d(b_s, &tmb, &sm.full[stage], kc, ti.row0);
           if constexpr (W8) tma_load_2d(b_s + Cfg::kBTileBytes, &tml, &sm.full[stage], kc, ti.row0);
           filled_mask |= 1u << stage;
@@ -483,7 +511,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       for (; !*abort_flag && unit_next(p, total_tiles, nk, uit, u); ++it) {
         // the last chunk of a group is ragged: N = its rows rounded up to 16, so a
         // skewed expert load does not pay MMAs on padding rows
-        const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
+        const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
         const int n_mma = min(BN, (ti.nvalid + 15) & ~15);
         const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, n_mma) : umma_idesc_bf16(kBM, n_mma);
         const int buf = it & 1;
@@ -564,7 +592,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     Unit u;
     const long long skT = static_cast<long long>(total_tiles) * nk;
     for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
-      const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
+      const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 4);
@@ -713,6 +741,12 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             for (int n = 0; n < 32; ++n)
               if (n < ncol) p.out_f32[static_cast<size_t>(cp[n]) * p.n_out + feat] = v[n] * cw[n];
           }
+        } else if (p.epi == EPI_ZOUT) {
+          if (m < p.r) {
+#pragma unroll
+            for (int n = 0; n < 32; ++n)
+              if (n < ncol) p.out_bf16[static_cast<size_t>(ti.row0 + c0 + n) * p.r + m] = __float2bfloat16_rn(v[n]);
+          }
         } else if (p.epi == EPI_LOGITS) {
           if (row_ok) {
             const float b = p.bias ? p.bias[feat] : 0.f;
@@ -759,7 +793,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       UnitIter uit = unit_begin(p, total_tiles, nk);
       Unit u;
       for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
-        const TileInfo ti = decode_tile(sm, u.t, p.m_tiles, p.E, BN);
+        const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         const bool got = mbar_wait(&sm.sempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 8);
@@ -918,8 +952,11 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.lseg_count = a.lseg_count;
   p.lseg_adapter = a.lseg_adapter;
   p.L = a.L;
+  p.items = a.items;
+  p.item_count = a.item_count;
+  p.iE = a.iE;
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
-  const long long tiles_ub = chunks_ub * p.m_tiles;
+  const long long tiles_ub = a.items ? a.items_bound : chunks_ub * p.m_tiles;
   int grid = a.num_sms;
   // stream-K when the tiles would leave SMs idle or unbalanced (< two waves)
   p.sk = 0;
@@ -939,7 +976,8 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   if (grid < 1) grid = 1;
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP
                : a.epi == EPI_DOWN ? K_GEMM_DOWN
-               : a.epi == EPI_LOGITS ? K_ROUTE_LOGITS : K_GEMM_DENSE, st);
+               : a.epi == EPI_LOGITS ? K_ROUTE_LOGITS
+               : a.epi == EPI_ZOUT ? K_LORA : K_GEMM_DENSE, st);
   gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
   count_launch();
   return cudaGetLastError();
@@ -948,6 +986,9 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
   if (a.E > kMaxGroups) return cudaErrorInvalidValue;
   if (a.delta != nullptr && a.delta_cols % 8 != 0) return cudaErrorInvalidValue;
+  if (a.epi == EPI_ZOUT && (a.items == nullptr || a.item_count == nullptr || a.lseg_off == nullptr || a.w_fp8 ||
+                            a.r <= 0 || a.r > 128 || a.z != nullptr || a.delta != nullptr))
+    return cudaErrorInvalidValue;
   if (a.z != nullptr) {
     if (a.delta != nullptr || a.lora_b == nullptr || a.lseg_off == nullptr || a.r <= 0 ||
         a.r > 128 || a.r % 8 != 0 || a.delta_cols % 8 != 0 || a.L <= 0)

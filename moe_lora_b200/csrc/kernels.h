@@ -87,6 +87,9 @@ struct LoraDeltaArgs {
 int lora_rows_per_chunk(int nrows, int nseg);
 int lora_items_bound(int nrows, int nseg, int rb);
 cudaError_t launch_lora_plan(const LoraDeltaArgs& a, cudaStream_t st);
+// work list of the segments that have an adapter only, chunks of rb rows (tensor-core shrink)
+cudaError_t launch_lora_plan_adapters(const LoraDeltaArgs& a, int rb, int2* items, int* count, int cap,
+                                      cudaStream_t st);
 cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st);
 
 // y[t] += z[t] . B_a(t) for dense segments (f32 or bf16 y and B).
@@ -118,7 +121,7 @@ cudaError_t launch_dense_f32(const DenseF32Args& a, cudaStream_t st);
 
 // Tensor-core grouped GEMM with operand swap: the weight rows fill the 128-row MMA
 // M slot, the tokens of one expert (or of the dense batch) the N slot.
-enum EpiKind : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DENSE = 2, EPI_LOGITS = 3 };
+enum EpiKind : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DENSE = 2, EPI_LOGITS = 3, EPI_ZOUT = 4 };
 
 struct GemmArgs {
   int epi;
@@ -169,6 +172,13 @@ struct GemmArgs {
   long long sk_part_cap;       // floats at sk_part
   int* sk_flag;
   int sk_slots;
+  // EPI_ZOUT (LoRA shrink on the tensor cores): tiles are work items (segment key, first
+  // row) of up to bn rows of one adapter segment; w = LoRA A as [L * E * r][K], b = the
+  // source rows, out_bf16 = z [total_rows][r]; lseg_off = the key CSR, L, r, iE = E
+  const int2* items;
+  const int* item_count;
+  int items_bound;
+  int iE;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
 

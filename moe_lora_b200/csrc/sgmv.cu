@@ -558,12 +558,19 @@ int lora_items_bound(int nrows, int nseg, int rb) {
 __global__ void __launch_bounds__(1024) lora_plan_kernel(const int32_t* __restrict__ off,
                                                          const int32_t* __restrict__ seg_adapter, int nseg, int L,
                                                          int nrows, int rb, int2* __restrict__ items,
-                                                         int* __restrict__ count, int cap, int* status) {
+                                                         int* __restrict__ count, int cap, int* status,
+                                                         int adapters_only) {
   __shared__ int s_scan[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = (nseg + blockDim.x - 1) / blockDim.x;
   const int q0 = threadIdx.x * per, q1 = min(nseg, q0 + per);
   if (threadIdx.x == 0 && (off[0] != 0 || off[nseg] != nrows)) set_status(status, MOE_LORA_ERR_DEVICE_CHECK, -1);
+  // adapters_only: skip segments without an adapter (dense: id -1; MoE keys: a' = L)
+  auto listed = [&](int q) {
+    if (!adapters_only) return true;
+    if (seg_adapter != nullptr) return seg_adapter[q] >= 0 && seg_adapter[q] < L;
+    return q % (L + 1) != L;
+  };
   int local = 0;
   for (int q = q0; q < q1; ++q) {
     const int a0 = off[q], a1 = off[q + 1];
@@ -571,7 +578,7 @@ __global__ void __launch_bounds__(1024) lora_plan_kernel(const int32_t* __restri
     if (seg_adapter != nullptr && (seg_adapter[q] < -1 || seg_adapter[q] >= L))
       set_status(status, MOE_LORA_ERR_DEVICE_CHECK, q);
     const int lo = max(a0, 0), hi = min(a1, nrows);
-    if (hi > lo) local += (hi - lo + rb - 1) / rb;
+    if (hi > lo && listed(q)) local += (hi - lo + rb - 1) / rb;
   }
   int incl = local;
 #pragma unroll
@@ -585,6 +592,7 @@ __global__ void __launch_bounds__(1024) lora_plan_kernel(const int32_t* __restri
   for (int w = 0; w < warp; ++w) base += s_scan[w];
   for (int q = q0; q < q1; ++q) {
     const int lo = max(off[q], 0), hi = min(off[q + 1], nrows);
+    if (!listed(q)) continue;
     for (int r0 = lo; r0 < hi; r0 += rb, ++base)
       if (base < cap) items[base] = make_int2(q, r0);
   }
@@ -595,7 +603,17 @@ cudaError_t launch_lora_plan(const LoraDeltaArgs& a, cudaStream_t st) {
   if (a.nrows <= 0) return cudaSuccess;
   ProfScope ps(K_LORA, st);
   lora_plan_kernel<<<1, 1024, 0, st>>>(a.seg_offsets, a.seg_adapter, a.nseg, a.L, a.nrows, a.rb, a.items,
-                                       a.item_count, a.items_bound, a.status);
+                                       a.item_count, a.items_bound, a.status, 0);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lora_plan_adapters(const LoraDeltaArgs& a, int rb, int2* items, int* count, int cap,
+                                      cudaStream_t st) {
+  if (a.nrows <= 0) return cudaSuccess;
+  ProfScope ps(K_LORA, st);
+  lora_plan_kernel<<<1, 1024, 0, st>>>(a.seg_offsets, a.seg_adapter, a.nseg, a.L, a.nrows, rb, items, count, cap,
+                                       a.status, 1);
   count_launch();
   return cudaGetLastError();
 }
