@@ -100,6 +100,7 @@ struct TcParams {
   const int2* items;
   const int* item_count;
   int iE;
+  int m_tiles2;                 // CTA pairs: pairs of 128-row tiles
 };
 
 // A unit of work: tile t, K stages [k0, k1).
@@ -122,9 +123,13 @@ __device__ __forceinline__ bool sk_busy(long long bb, long long T, long long G) 
   return sk_start(bb, T, G) < sk_start(bb + 1, T, G);
 }
 
+// CTA pairs: unit index space is per cluster (two CTAs walk the same units)
+__device__ __forceinline__ int unit_cta(const TcParams& p) { return p.m_tiles2 ? blockIdx.x >> 1 : blockIdx.x; }
+__device__ __forceinline__ int unit_ctas(const TcParams& p) { return p.m_tiles2 ? gridDim.x >> 1 : gridDim.x; }
+
 __device__ __forceinline__ UnitIter unit_begin(const TcParams& p, int total_tiles, int nk) {
   UnitIter it;
-  it.t = blockIdx.x;
+  it.t = unit_cta(p);
   const long long T = static_cast<long long>(total_tiles) * nk;
   it.pos = sk_start(blockIdx.x, T, gridDim.x);
   it.end = sk_start(blockIdx.x + 1, T, gridDim.x);
@@ -137,7 +142,7 @@ __device__ __forceinline__ bool unit_next(const TcParams& p, int total_tiles, in
     u.t = it.t;
     u.k0 = 0;
     u.k1 = nk;
-    it.t += gridDim.x;
+    it.t += unit_ctas(p);
     return true;
   }
   if (it.pos >= it.end) return false;
@@ -182,10 +187,13 @@ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int BN, bool W8>
+// TWO: the CTA pair (cta_group::2) computes 256 weight rows x BN tokens; each CTA holds
+// its 128 weight rows and half of the BN token rows.
+template <int BN, bool W8, bool TWO = false>
 struct TileCfg {
   static constexpr int kKB = W8 ? 128 : 64;                  // K per stage (128 bytes per row)
-  static constexpr int kBTileBytes = BN * 128;               // one token tile (or plane)
+  static constexpr int kBRows = TWO ? BN / 2 : BN;           // token rows held by this CTA
+  static constexpr int kBTileBytes = kBRows * 128;           // one token tile (or plane)
   static constexpr int kStageBytes = kATileBytes + (W8 ? 2 : 1) * kBTileBytes;
   static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
   static constexpr int kAccPerBuf = W8 ? 3 : 1;              // e4m3: hi, lo and LoRA accumulators
@@ -194,6 +202,7 @@ struct TileCfg {
   static constexpr int kSlotBytes = kPrefetch ? static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024) : 0;
   static constexpr int kThreads = 224;
   static_assert(!W8 || kPrefetch, "e4m3 weights use N tiles <= 64");
+  static_assert(!TWO || (!W8 && BN >= 128), "CTA pairs: bf16 weights, N tiles of 128 or 256");
 };
 
 struct TileInfo {
@@ -279,20 +288,21 @@ __device__ __forceinline__ bool lora_seg_next(const TcParams& p, const TileInfo&
     s.hi = hi;
     s.slot = ad * p.E + ti.g;
     s.c_start = ((lo - ti.row0) >> 5) << 5;
-    s.n = (hi - ti.row0 - s.c_start + 15) & ~15;
+    const int na = p.m_tiles2 ? 31 : 15;  // CTA pairs: N / 2 rows per CTA, a multiple of 16
+    s.n = (hi - ti.row0 - s.c_start + na) & ~na;
     return true;
   }
   return false;
 }
 
-template <int BN, bool W8>
-__global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
+template <int BN, bool W8, bool TWO>
+__global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tml, const __grid_constant__ CUtensorMap tmd,
                    const __grid_constant__ CUtensorMap tmlb, const TcParams p) {
   // tml: the lo activation plane (e4m3 weights); tmlb: LoRA B viewed as [L * E * r][NB]
   // (MN-major boxes of 64 features x rbox rank rows)
-  using Cfg = TileCfg<BN, W8>;
+  using Cfg = TileCfg<BN, W8, TWO>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;                                 // stages: [A tile][token tile(s)]
@@ -301,16 +311,20 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
   volatile int* abort_flag = &sm.abort_flag;
+  // CTA pairs: rank 0 (leader) issues the MMAs for both; the barriers the MMA consumes
+  // live in the leader's shared memory
+  const uint32_t rank = TWO ? cluster_ctarank() : 0;
+  auto leader_bar = [&](uint64_t* bar) -> uint32_t { return TWO ? mapa_shared(smem_u32(bar), 0) : smem_u32(bar); };
 
   // ---- setup: barriers, TMEM, tile list prefix
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.full[s], TWO ? 2 : 1);  // pair: the leader's and the peer's producer
       mbar_init(&sm.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
-      mbar_init(&sm.tempty[b], kEpiThreads);
+      mbar_init(&sm.tempty[b], TWO ? 2 * kEpiThreads : kEpiThreads);
       mbar_init(&sm.sfull[b], 1);
       mbar_init(&sm.sempty[b], kEpiThreads);
     }
@@ -325,7 +339,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     if (p.z != nullptr) tma_prefetch_desc(&tmlb);
     if (p.delta != nullptr) tma_prefetch_desc(&tmd);
   }
-  if (warp == 1) tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
+  if (warp == 1) {
+    if constexpr (TWO) tmem_alloc_pair(&sm.tmem_base, Cfg::kTmemCols);
+    else tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
+  }
   for (int g = threadIdx.x; g <= p.E; g += blockDim.x)
     sm.grp_off[g] = p.group_offsets ? p.group_offsets[static_cast<size_t>(g) * p.group_stride]
                                     : (g == 0 ? 0 : p.total_rows);
@@ -361,7 +378,8 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     if (lane == 31) sm.chunk_pref[p.E] = incl;
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (TWO) cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
   if constexpr (W8) {
@@ -376,7 +394,15 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
   }
-  const int total_tiles = p.items ? *p.item_count : sm.chunk_pref[p.E] * p.m_tiles;
+  const int total_tiles =
+      p.items ? *p.item_count : sm.chunk_pref[p.E] * (TWO ? p.m_tiles2 : p.m_tiles);
+  // this CTA's tile of a unit (pairs: the unit is a pair of 128-row tiles, rank picks one)
+  auto tile_of = [&](int t) -> TileInfo {
+    if (p.items) return item_tile(p, t, BN);
+    TileInfo ti = decode_tile(sm, t, TWO ? p.m_tiles2 : p.m_tiles, p.E, BN);
+    if constexpr (TWO) ti.mt = 2 * ti.mt + static_cast<int>(rank);
+    return ti;
+  };
   const int nk = (p.K + Cfg::kKB - 1) / Cfg::kKB;  // stages per tile
 
   if (warp == 0) {
@@ -397,7 +423,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
         __syncwarp();
         if (lane == 0)
           for (int s2 = 0; s2 < S; ++s2)
-            if (pend_mask & (1u << s2)) mbar_arrive(&sm.full[s2]);
+            if (pend_mask & (1u << s2)) {
+              if constexpr (TWO) mbar_arrive_cluster(leader_bar(&sm.full[s2]));
+              else mbar_arrive(&sm.full[s2]);
+            }
         pend_mask = 0;
       }
     };
@@ -416,7 +445,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     Unit u;
     while (ok && unit_next(p, total_tiles, nk, uit, u)) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0, 0)) break;  // warp-uniform
-      const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
+      const TileInfo ti = tile_of(u.t);
       int wrow0, wrow1;
       if (p.epi == EPI_GATEUP) {
         wrow0 = ti.g * p.rows_per_group + ti.mt * 64;
@@ -438,11 +467,24 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           uint8_t* a_s = ring + stage * Cfg::kStageBytes;
           uint8_t* b_s = a_s + kATileBytes;
           const int kc = kb * Cfg::kKB;  // first K element of the stage
-          mbar_arrive_expect_tx(&sm.full[stage], Cfg::kStageBytes - (a_half ? kATileBytes / 2 : 0));
-          tma_load_2d(a_s, &tmw, &sm.full[stage], kc, wrow0);
-          if (!a_half) tma_load_2d(a_s + kATileBytes / 2, &tmw, &sm.full[stage], kc, wrow1);
-          tma_load_2d(b_s, &tmb, &sm.full[stage], kc, ti.row0);
-          if constexpr (W8) tma_load_2d(b_s + Cfg::kBTileBytes, &tml, &sm.full[stage], kc, ti.row0);
+          if constexpr (TWO) {
+            // both CTAs' copies complete on the leader's barrier: the leader expects the
+            // pair's bytes, the peer adds its arrival
+            const uint32_t fb = leader_bar(&sm.full[stage]);
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2 * Cfg::kStageBytes);
+            tma_load_2d_pair(a_s, &tmw, fb, kc, wrow0);
+            tma_load_2d_pair(a_s + kATileBytes / 2, &tmw, fb, kc, wrow1);
+            // MMA N = the tile's rows rounded to 32; the peer holds columns [N/2, N)
+            const int n_pair = min(BN, (ti.nvalid + 31) & ~31);
+            tma_load_2d_pair(b_s, &tmb, fb, kc, ti.row0 + static_cast<int>(rank) * (n_pair / 2));
+            if (rank != 0) mbar_arrive_cluster(fb);
+          } else {
+            mbar_arrive_expect_tx(&sm.full[stage], Cfg::kStageBytes - (a_half ? kATileBytes / 2 : 0));
+            tma_load_2d(a_s, &tmw, &sm.full[stage], kc, wrow0);
+            if (!a_half) tma_load_2d(a_s + kATileBytes / 2, &tmw, &sm.full[stage], kc, wrow1);
+            tma_load_2d(b_s, &tmb, &sm.full[stage], kc, ti.row0);
+            if constexpr (W8) tma_load_2d(b_s + Cfg::kBTileBytes, &tml, &sm.full[stage], kc, ti.row0);
+          }
           filled_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
         }
@@ -468,15 +510,25 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             uint8_t* b_s = a_s + kATileBytes;
             if (lane == 0) {
               const int krow = ls.slot * p.r + kh * 64;
-              mbar_expect_tx(&sm.full[stage], 2 * p.rbox * 128);
-              tma_load_2d(a_s, &tmlb, &sm.full[stage], col0, krow);
-              tma_load_2d(a_s + p.rbox * 128, &tmlb, &sm.full[stage], col1, krow);
+              if constexpr (TWO) {
+                const uint32_t fb = leader_bar(&sm.full[stage]);
+                if (rank == 0) mbar_expect_tx(&sm.full[stage], 2 * 2 * p.rbox * 128);
+                tma_load_2d_pair(a_s, &tmlb, fb, col0, krow);
+                tma_load_2d_pair(a_s + p.rbox * 128, &tmlb, fb, col1, krow);
+              } else {
+                mbar_expect_tx(&sm.full[stage], 2 * p.rbox * 128);
+                tma_load_2d(a_s, &tmlb, &sm.full[stage], col0, krow);
+                tma_load_2d(a_s + p.rbox * 128, &tmlb, &sm.full[stage], col1, krow);
+              }
               filled_mask |= 1u << stage;
               last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
             }
-            for (int idx = lane; idx < ls.n * kch; idx += 32) {
+            // pairs: this CTA holds rows [rank n / 2, (rank + 1) n / 2) of the unit's n columns
+            const int n_h = TWO ? ls.n / 2 : ls.n;
+            const int col_base = ls.c_start + static_cast<int>(rank) * n_h;
+            for (int idx = lane; idx < n_h * kch; idx += 32) {
               const int j = idx / kch, c = idx - j * kch;
-              const int row = ti.row0 + ls.c_start + j;
+              const int row = ti.row0 + col_base + j;
               const int el = kh * 64 + c * 8;
               const bool valid = row >= ls.lo && row < ls.hi && el < p.r;
               const __nv_bfloat16* src = valid ? p.z + static_cast<size_t>(row) * p.r + el : p.z;
@@ -492,7 +544,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       }
     }
     flush_lora();  // every issued stage gets its arrival, also on the abort path
-    if (lane == 0 && *abort_flag) {
+    if (lane == 0 && *abort_flag && rank == 0) {  // pairs: the leader's barriers count both CTAs' copies
       // let our own copies land before the CTA exits
       for (int s = 0; s < S; ++s)
         if (filled_mask & (1u << s)) {
@@ -502,7 +554,17 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // pairs: the leader issues the MMAs of both CTAs (M = 256: its 128 rows and the
+    // peer's), commits reach both CTAs' barriers; the peer waits for the last commit
+    if (lane == 0 && TWO && rank != 0) {
+      volatile int dummy = 0;
+      mbar_wait(&sm.tdone, 0, &dummy, nullptr, kWaitLimitNs, 0);
+    } else if (lane == 0) {
+      constexpr int kMM = TWO ? 2 * kBM : kBM;  // MMA M
+      auto commit = [&](uint64_t* bar) {
+        if constexpr (TWO) umma_commit_pair(bar, 3);
+        else umma_commit(bar);
+      };
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -511,9 +573,9 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       for (; !*abort_flag && unit_next(p, total_tiles, nk, uit, u); ++it) {
         // the last chunk of a group is ragged: N = its rows rounded up to 16, so a
         // skewed expert load does not pay MMAs on padding rows
-        const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
-        const int n_mma = min(BN, (ti.nvalid + 15) & ~15);
-        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, n_mma) : umma_idesc_bf16(kBM, n_mma);
+        const TileInfo ti = tile_of(u.t);
+        const int n_mma = TWO ? min(BN, (ti.nvalid + 31) & ~31) : min(BN, (ti.nvalid + 15) & ~15);
+        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, n_mma) : umma_idesc_bf16(kMM, n_mma);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(&sm.tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 2)) break;
@@ -536,11 +598,13 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
               const uint64_t ldesc = umma_desc_sw128(a_addr + kATileBytes + Cfg::kBTileBytes);
               umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
               umma_e4m3(d_tmem + Cfg::kAccStride, adesc + 2 * k, ldesc + 2 * k, idesc, acc);
+            } else if constexpr (TWO) {
+              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
             } else {
               umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
             }
           }
-          umma_commit(&sm.empty[stage]);
+          commit(&sm.empty[stage]);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -553,7 +617,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             LoraSeg ls;
             lora_seg_begin(p, ti, ls);
             while (ok && lora_seg_next(p, ti, ls)) {
-              const uint32_t lidesc = umma_idesc_bf16_amn(kBM, ls.n);
+              const uint32_t lidesc = umma_idesc_bf16_amn(kMM, ls.n);
               for (int kh = 0; kh * 64 < p.r; ++kh) {
                 if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 10)) {
                   ok = false;
@@ -563,9 +627,11 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
                 const uint32_t a_addr = smem_u32(ring + stage * Cfg::kStageBytes);
                 const uint64_t adesc = umma_desc_mn_sw128(a_addr, p.rbox * 128);
                 const uint64_t bdesc = umma_desc_sw128(a_addr + kATileBytes);
-                for (int kk = 0; kk < p.rbox / 16; ++kk)  // 16 rank rows (2048 B of A) per instruction
-                  umma_bf16(d_lora + ls.c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
-                umma_commit(&sm.empty[stage]);
+                for (int kk = 0; kk < p.rbox / 16; ++kk) {  // 16 rank rows (2048 B of A) per instruction
+                  if constexpr (TWO) umma_bf16_pair(d_lora + ls.c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
+                  else umma_bf16(d_lora + ls.c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
+                }
+                commit(&sm.empty[stage]);
                 if (++stage == S) {
                   stage = 0;
                   phase ^= 1u;
@@ -575,10 +641,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit(&sm.tfull[buf]);
+        commit(&sm.tfull[buf]);
       }
       // all MMAs issued by this thread complete before TMEM is released
-      umma_commit(&sm.tdone);
+      commit(&sm.tdone);
       volatile int dummy = 0;
       mbar_wait(&sm.tdone, 0, &dummy, nullptr, kWaitLimitNs, 0);
     }
@@ -592,7 +658,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     Unit u;
     const long long skT = static_cast<long long>(total_tiles) * nk;
     for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
-      const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
+      const TileInfo ti = tile_of(u.t);
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 4);
@@ -782,7 +848,8 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&sm.tempty[buf]);
+      if constexpr (TWO) mbar_arrive_cluster(leader_bar(&sm.tempty[buf]));  // the leader's MMA reuses it
+      else mbar_arrive(&sm.tempty[buf]);
       if constexpr (Cfg::kPrefetch) mbar_arrive(&sm.sempty[buf]);
     }
   } else if (warp == 6) {
@@ -793,7 +860,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       UnitIter uit = unit_begin(p, total_tiles, nk);
       Unit u;
       for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
-        const TileInfo ti = p.items ? item_tile(p, u.t, BN) : decode_tile(sm, u.t, p.m_tiles, p.E, BN);
+        const TileInfo ti = tile_of(u.t);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         const bool got = mbar_wait(&sm.sempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 8);
@@ -836,9 +903,13 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (TWO) cluster_sync_all();  // no CTA leaves while its peer may still signal it
+  else __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  if (warp == 1) {
+    if constexpr (TWO) tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+    else tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
 }
 
 // ---------------------------------------------------------------------------- host side
@@ -870,9 +941,9 @@ CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-template <int BN, bool W8>
+template <int BN, bool W8, bool TWO = false>
 static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
-  using Cfg = TileCfg<BN, W8>;
+  using Cfg = TileCfg<BN, W8, TWO>;
   const int fixed = static_cast<int>(sizeof(SmemCore)) + 2 * Cfg::kSlotBytes;
   const int budget = 232448 - 1024 - fixed;
   int stages = budget / Cfg::kStageBytes;
@@ -882,7 +953,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          232448);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -901,7 +972,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2, kBK,
                        64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
-                       static_cast<uint64_t>(a.K) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                       static_cast<uint64_t>(a.K) * 2, kBK, Cfg::kBRows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     tml = tmb;  // unused
   }
@@ -955,8 +1026,9 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.items = a.items;
   p.item_count = a.item_count;
   p.iE = a.iE;
+  p.m_tiles2 = TWO ? (p.m_tiles + 1) / 2 : 0;
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
-  const long long tiles_ub = a.items ? a.items_bound : chunks_ub * p.m_tiles;
+  const long long tiles_ub = a.items ? a.items_bound : chunks_ub * (TWO ? p.m_tiles2 : p.m_tiles);
   int grid = a.num_sms;
   // stream-K when the tiles would leave SMs idle or unbalanced (< two waves)
   p.sk = 0;
@@ -967,20 +1039,50 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   // 36.3 us for 86 whole tiles, so whole tiles stay the default.
   const char* skv = std::getenv("MOE_LORA_STREAMK");
   const bool sk_want = skv != nullptr && std::atoi(skv) != 0 && tiles_ub < 2LL * grid;
-  if (a.sk_part != nullptr && a.sk_flag != nullptr && a.z == nullptr && BN <= 64 && sk_want &&
+  if (!TWO && a.sk_part != nullptr && a.sk_flag != nullptr && a.z == nullptr && BN <= 64 && sk_want &&
       grid <= a.sk_slots && static_cast<long long>(grid) * kBM * BN <= a.sk_part_cap) {
     p.sk = 1;
+  } else if (TWO) {
+    grid = (grid / 2 < tiles_ub ? grid / 2 : static_cast<int>(tiles_ub)) * 2;  // whole pairs
   } else {
     if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
   }
-  if (grid < 1) grid = 1;
+  if (grid < (TWO ? 2 : 1)) grid = TWO ? 2 : 1;
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP
                : a.epi == EPI_DOWN ? K_GEMM_DOWN
                : a.epi == EPI_LOGITS ? K_ROUTE_LOGITS
                : a.epi == EPI_ZOUT ? K_LORA : K_GEMM_DENSE, st);
-  gemm_tc_kernel<BN, W8><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
-  count_launch();
-  return cudaGetLastError();
+  if constexpr (TWO) {  // clusters of two CTAs (the MMA pair)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO>, tmw, tmb, tml, tmd, tmlb, p);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  } else {
+    gemm_tc_kernel<BN, W8, TWO><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
+    count_launch();
+    return cudaGetLastError();
+  }
+}
+
+// N tiles of 128 and 256 on CTA pairs (cta_group::2), opt-in with MOE_LORA_PAIR=1.  On a
+// prefill-shaped case (256 rows per expert, H = 4096) the pair kernel is correct but
+// slower than one CTA per tile (gate_up 283 us against 156 us, tensor pipe active 17.5%),
+// so single-CTA tiles stay the default.
+static bool pairs_on() {
+  const char* v = std::getenv("MOE_LORA_PAIR");
+  return v != nullptr && std::atoi(v) != 0;
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
@@ -1006,8 +1108,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
     case 16: return launch_bn<16, false>(a, st);
     case 32: return launch_bn<32, false>(a, st);
     case 64: return launch_bn<64, false>(a, st);
-    case 128: return launch_bn<128, false>(a, st);
-    case 256: return launch_bn<256, false>(a, st);
+    case 128: return pairs_on() ? launch_bn<128, false, true>(a, st) : launch_bn<128, false>(a, st);
+    case 256: return pairs_on() ? launch_bn<256, false, true>(a, st) : launch_bn<256, false>(a, st);
     default: return cudaErrorInvalidValue;
   }
 }

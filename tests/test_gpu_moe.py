@@ -70,6 +70,19 @@ def test_forward_stream_k(shape, M, monkeypatch):
     assert res["err"] <= TOL_BF16, res["err"]
 
 
+@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("bn", [128, 256])
+def test_forward_cta_pairs(bn, where, monkeypatch):
+    """N tiles of 128 / 256 on CTA pairs (tcgen05 cta_group::2): each CTA holds its 128
+    weight rows and half of the token rows; ragged tiles, odd tile counts, LoRA units."""
+    monkeypatch.setenv("MOE_LORA_PAIR", "1")
+    monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
+    monkeypatch.setenv("MOE_LORA_EXPAND", where)
+    for shape, M in ((SMALL[0], 300), (SMALL[1], 37), (SMALL[3], 37), (SMALL[9], 300)):
+        res = run_moe_case(shape, M)
+        assert res["err"] <= TOL_BF16, (shape.name, res["err"])
+
+
 @pytest.fixture(scope="module")
 def decode_weights():
     return moe_weights_both(synth.MOE_DECODE_BF16)
