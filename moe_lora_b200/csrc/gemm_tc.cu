@@ -15,8 +15,9 @@
 // for the fixed-order combine (expert aggregation, [SageMaker MoE kernels page],
 // second item).  FP8 (e4m3) expert weights stay one byte per weight in HBM, in the TMA
 // ring and in the MMA: the activations are split exactly into two e4m3 planes
-// (hi = RNE(x / s), lo = RNE((x - hi s) / (s / 16)), per-row s), the kind::f8f6f4 MMA
-// runs once per plane into two TMEM accumulators, and the epilogue combines
+// (hi = RNE(x / s), lo = RNE((x - hi s) / (s / 16)), per-row s), one kind::f8f6f4 MMA
+// of N = 2 BN takes both planes (stacked token rows) into adjacent TMEM columns, so
+// the weight tile is read from shared memory once per K step, and the epilogue combines
 // s_w (s acc_hi + s/16 acc_lo) (per-tensor scale, [SageMaker MoE kernels page],
 // second item).
 //
@@ -574,8 +575,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
         // the last chunk of a group is ragged: N = its rows rounded up to 16, so a
         // skewed expert load does not pay MMAs on padding rows
         const TileInfo ti = tile_of(u.t);
+        // e4m3: the hi and lo planes sit back to back in the ring, so one instruction of
+        // N = 2 BN covers both and each weight tile is read from shared memory once
         const int n_mma = TWO ? min(BN, (ti.nvalid + 31) & ~31) : min(BN, (ti.nvalid + 15) & ~15);
-        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, n_mma) : umma_idesc_bf16(kMM, n_mma);
+        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, 2 * BN) : umma_idesc_bf16(kMM, n_mma);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(&sm.tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 2)) break;
@@ -595,9 +598,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
           for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
             const uint32_t acc = (kb != u.k0 || k != 0) ? 1u : 0u;
             if constexpr (W8) {
-              const uint64_t ldesc = umma_desc_sw128(a_addr + kATileBytes + Cfg::kBTileBytes);
-              umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
-              umma_e4m3(d_tmem + Cfg::kAccStride, adesc + 2 * k, ldesc + 2 * k, idesc, acc);
+              umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // columns [0, BN) hi, [BN, 2 BN) lo
             } else if constexpr (TWO) {
               umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
             } else {
@@ -723,7 +724,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
         tmem_ld_32x32b_x32(t_acc, v);
         if constexpr (W8) {
           float vl[32];
-          tmem_ld_32x32b_x32(t_acc + Cfg::kAccStride, vl);
+          tmem_ld_32x32b_x32(t_acc + BN, vl);
 #pragma unroll
           for (int n = 0; n < 32; ++n)
             if (c0 + n < BN) v[n] = scale * (v[n] * slot->col_sh[c0 + n] + vl[n] * slot->col_sl[c0 + n]);
