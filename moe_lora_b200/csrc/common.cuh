@@ -163,6 +163,12 @@ __device__ __forceinline__ void cp_async_16_zfill(void* smem_dst, const void* gs
                : "memory");
 }
 
+// The mbarrier tracks the completion of every cp.async this thread issued so far: its
+// pending count goes up by one now and down by one when those copies have landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

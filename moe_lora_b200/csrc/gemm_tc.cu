@@ -33,9 +33,9 @@
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, + LoRA delta, activation,
 //               stores; two TMEM accumulators so the epilogue of tile i overlaps the
 //               MMAs of tile i+1
-//   warp 6      epilogue loader (N tiles <= 64): one tile ahead of the epilogue, TMA
-//               of the tile's LoRA delta and the per-column data (pair ids, routing
-//               weights, activation plane scales) into a two-slot shared-memory ring
+//   warp 6      epilogue loader: one tile ahead of the epilogue, the per-column data
+//               (pair ids, routing weights, activation plane scales) and, for N tiles
+//               <= 64, a TMA of the tile's LoRA delta into a two-slot shared-memory ring
 // Every mbarrier wait is bounded; on expiry the CTA records MOE_LORA_ERR_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include "common.cuh"
@@ -168,14 +168,18 @@ struct SmemCore {
   int chunk_pref[kMaxGroups + 1];
   int grp_off[kMaxGroups + 1];
   float ebuf[kBM][33];
-  int col_pair[32];
-  float col_w[32];
+  // in-GEMM LoRA expand: LoRA stages of the producer's unit it (mod 16), and per ring
+  // stage holding a LoRA stage its MMA's first tile column and N
+  int tile_nls[16];
+  int lstage_col[16];
+  int lstage_n[16];
 };
 
-// Epilogue prefetch slot (N tiles <= 64): LoRA delta [2 halves][BN][64] and pair data.
+// Epilogue prefetch slot, filled one tile ahead by the loader warp: the tile's pair ids,
+// routing weights and plane scales, and (N tiles <= 64) its LoRA delta [2 halves][BN][64].
 template <int BN>
 struct EpiSlot {
-  float delta[2 * BN * 64];
+  float delta[BN <= 64 ? 2 * BN * 64 : 4];
   int col_pair[BN];
   float col_w[BN];
   float col_sh[BN];
@@ -199,8 +203,8 @@ struct TileCfg {
   static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
   static constexpr int kAccPerBuf = W8 ? 3 : 1;              // e4m3: hi, lo and LoRA accumulators
   static constexpr int kTmemCols = pow2_at_least(2 * kAccPerBuf * kAccStride);
-  static constexpr bool kPrefetch = BN <= 64;                // epilogue loader warp + slots
-  static constexpr int kSlotBytes = kPrefetch ? static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024) : 0;
+  static constexpr bool kPrefetch = BN <= 64;                // LoRA delta prefetched into the slots
+  static constexpr int kSlotBytes = static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024);
   static constexpr int kThreads = 224;
   static_assert(!W8 || kPrefetch, "e4m3 weights use N tiles <= 64");
   static_assert(!TWO || (!W8 && BN >= 128), "CTA pairs: bf16 weights, N tiles of 128 or 256");
@@ -274,6 +278,14 @@ __device__ __forceinline__ void lora_seg_begin(const TcParams& p, const TileInfo
   s.end = ti.row0 + ti.nvalid;
 }
 
+// MMA columns of a segment [lo, hi) inside the tile: from the 32-aligned column at or
+// below lo, N rounded up to 16 (CTA pairs: 32, N / 2 rows per CTA)
+__device__ __forceinline__ void seg_cols(const TcParams& p, const TileInfo& ti, LoraSeg& s) {
+  s.c_start = ((s.lo - ti.row0) >> 5) << 5;
+  const int na = p.m_tiles2 ? 31 : 15;
+  s.n = (s.hi - ti.row0 - s.c_start + na) & ~na;
+}
+
 // Advances to the next segment with an adapter; false when the tile has no more.
 __device__ __forceinline__ bool lora_seg_next(const TcParams& p, const TileInfo& ti, LoraSeg& s) {
   const int32_t* off = p.lseg_off + static_cast<size_t>(ti.g) * p.lseg_stride;
@@ -288,20 +300,111 @@ __device__ __forceinline__ bool lora_seg_next(const TcParams& p, const TileInfo&
     s.lo = lo;
     s.hi = hi;
     s.slot = ad * p.E + ti.g;
-    s.c_start = ((lo - ti.row0) >> 5) << 5;
-    const int na = p.m_tiles2 ? 31 : 15;  // CTA pairs: N / 2 rows per CTA, a multiple of 16
-    s.n = (hi - ti.row0 - s.c_start + na) & ~na;
+    seg_cols(p, ti, s);
     return true;
   }
   return false;
 }
 
-template <int BN, bool W8, bool TWO>
+// Warp-parallel view of the segments that meet a tile: lane l loads candidate
+// base + 32 h + l (h < 2) in one round of independent loads, and a ballot marks the
+// candidates that meet the tile with an adapter.  Candidates past base + 64 (only with
+// very many segments per group) are walked one at a time from global memory.
+struct SegScan {
+  uint32_t mask0, mask1;
+  int lo0, hi0, slot0, lo1, hi1, slot1;  // this lane's candidate of chunk 0 / chunk 1
+  int rest;                             // first candidate after the chunks that may meet the tile, or -1
+};
+
+__device__ __forceinline__ void seg_scan(const TcParams& p, const TileInfo& ti, int lane, SegScan& sc) {
+  const int32_t* off = p.lseg_off + static_cast<size_t>(ti.g) * p.lseg_stride;
+  const int end = ti.row0 + ti.nvalid;
+  int base = 0;
+  if (p.lseg_count > 64) {  // smallest c with off[c + 1] > row0
+    int lo = 0, hi = p.lseg_count;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid + 1] > ti.row0) hi = mid;
+      else lo = mid + 1;
+    }
+    base = lo;
+  }
+  int lo[2], hi[2], slot[2];
+  bool v[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int c = base + 32 * h + lane;
+    v[h] = false;
+    lo[h] = hi[h] = slot[h] = 0;
+    if (c < p.lseg_count) {
+      const int a0 = off[c], a1 = off[c + 1];
+      const int ad = p.lseg_adapter ? p.lseg_adapter[c] : c;
+      lo[h] = max(a0, ti.row0);
+      hi[h] = min(a1, end);
+      v[h] = hi[h] > lo[h] && ad >= 0 && ad < p.L;
+      slot[h] = ad * p.E + ti.g;
+    }
+  }
+  sc.mask0 = __ballot_sync(0xffffffffu, v[0]);
+  sc.mask1 = __ballot_sync(0xffffffffu, v[1]);
+  sc.lo0 = lo[0], sc.hi0 = hi[0], sc.slot0 = slot[0];
+  sc.lo1 = lo[1], sc.hi1 = hi[1], sc.slot1 = slot[1];
+  const int nx = base + 64;
+  sc.rest = (nx < p.lseg_count && off[nx] < end) ? nx : -1;
+}
+
+struct SegIter {
+  int h;
+  uint32_t m;
+  bool in_rest;
+  LoraSeg ls;
+};
+
+__device__ __forceinline__ SegIter seg_iter_begin(const SegScan& sc) {
+  SegIter it;
+  it.h = 0;
+  it.m = sc.mask0;
+  it.in_rest = false;
+  return it;
+}
+
+// Next segment of the tile (warp-uniform: every lane of the warp calls it together).
+__device__ __forceinline__ bool seg_iter_next(const TcParams& p, const TileInfo& ti, const SegScan& sc, SegIter& it,
+                                              LoraSeg& out) {
+  while (it.h < 2) {
+    if (it.m == 0) {
+      if (++it.h == 1) it.m = sc.mask1;
+      continue;
+    }
+    const int b = __ffs(it.m) - 1;
+    it.m &= it.m - 1;
+    const bool h1 = it.h == 1;
+    out.lo = __shfl_sync(0xffffffffu, h1 ? sc.lo1 : sc.lo0, b);
+    out.hi = __shfl_sync(0xffffffffu, h1 ? sc.hi1 : sc.hi0, b);
+    out.slot = __shfl_sync(0xffffffffu, h1 ? sc.slot1 : sc.slot0, b);
+    seg_cols(p, ti, out);
+    return true;
+  }
+  if (sc.rest < 0) return false;
+  if (!it.in_rest) {
+    it.in_rest = true;
+    it.ls.c = sc.rest;
+    it.ls.end = ti.row0 + ti.nvalid;
+  }
+  if (!lora_seg_next(p, ti, it.ls)) return false;
+  out = it.ls;
+  return true;
+}
+
+// LZ: the in-GEMM LoRA expand is compiled in (launches with z); without it the kernel
+// carries none of that code.
+template <int BN, bool W8, bool TWO, bool LZ>
 __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tml, const __grid_constant__ CUtensorMap tmd,
                    const __grid_constant__ CUtensorMap tmlb, const TcParams p) {
   // tml: the lo activation plane (e4m3 weights); tmlb: LoRA B viewed as [L * E * r][NB]
+  const bool lz = LZ && p.z != nullptr;
   // (MN-major boxes of 64 features x rbox rank rows)
   using Cfg = TileCfg<BN, W8, TWO>;
   extern __shared__ uint8_t smem_raw[];
@@ -337,7 +440,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     tma_prefetch_desc(&tmw);
     tma_prefetch_desc(&tmb);
     if (W8) tma_prefetch_desc(&tml);
-    if (p.z != nullptr) tma_prefetch_desc(&tmlb);
+    if (lz) tma_prefetch_desc(&tmlb);
     if (p.delta != nullptr) tma_prefetch_desc(&tmd);
   }
   if (warp == 1) {
@@ -385,7 +488,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
   const uint32_t tmem_base = sm.tmem_base;
   if constexpr (W8) {
     // the LoRA accumulators start at zero; the epilogue re-zeroes one after reading it
-    if (p.z != nullptr && warp >= 2 && warp < 6) {
+    if (lz && warp >= 2 && warp < 6) {
       for (int b = 0; b < 2; ++b)
         for (int c = 0; c < Cfg::kAccStride; c += 32)
           tmem_zero_32x32b_x32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
@@ -409,9 +512,11 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // Lane 0 issues the TMA copies.  The whole warp fills the z tiles of LoRA stages
-    // with cp.async (zero-fill outside the segment); such a stage is completed (copies
-    // waited for, proxy fence, arrive) only when the producer would otherwise block, so
-    // the z loads overlap the following copies instead of stalling them.
+    // with cp.async (zero-fill outside the segment) whose completion is tracked by the
+    // stage's full barrier (cp.async.mbarrier.arrive), so the producer never waits for
+    // them; the MMA thread issues a proxy fence before it reads such a stage.  CTA pairs
+    // signal the leader's barrier, which cp.async cannot: there the stage is completed
+    // (copies waited for, fence, remote arrive) when the producer would otherwise block.
     int stage = 0;
     uint32_t phase = 0;
     uint32_t filled_mask = 0, last_parity = 0;
@@ -444,6 +549,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     };
     UnitIter uit = unit_begin(p, total_tiles, nk);
     Unit u;
+    int itp = 0;  // unit index, the same sequence as the MMA thread's
     while (ok && unit_next(p, total_tiles, nk, uit, u)) {
       if (__shfl_sync(0xffffffffu, *abort_flag != 0, 0)) break;  // warp-uniform
       const TileInfo ti = tile_of(u.t);
@@ -461,7 +567,35 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
       // r <= 64: the second 64-row half of A is not needed (accumulator rows >= r are
       // never read), so it is not loaded
       const bool a_half = p.epi == EPI_ZOUT && p.r <= 64;
-      for (int kb = u.k0; kb < u.k1; ++kb) {
+      const bool lora = lz;
+      const int nb = u.k1 - u.k0;  // base stages of the unit
+      // LoRA stages (in-GEMM expand), after the unit's base stages: A = B_a^T (MN-major:
+      // 64 gate/low + 64 up/high features x rbox rank rows), B = the segment's z rows in
+      // tile columns [c_start, c_start + n), zero outside the segment.  Their count goes
+      // to shared memory before the last base stage's arrival and each one's MMA columns
+      // before its own, for the MMA thread.  (Spreading them between the base stages
+      // measured slower: mixed MMA kinds slowed the tensor pipe more than the earlier
+      // loads saved.)
+      const int lf0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
+      const int lcol1 = (p.epi == EPI_GATEUP) ? p.I + lf0 : lf0 + 64;
+      const int kch = p.rbox / 8;  // 16-byte chunks of a z row per stage
+      const int per = lora ? (p.r + 63) / 64 : 0;
+      SegScan sc;
+      int nls = 0;
+      for (int i = 0; i < nb; ++i) {
+        // the segment scan waits for global loads: midway, while the ring is full
+        if (lora && i == nb / 2) {
+          seg_scan(p, ti, lane, sc);
+          nls = (__popc(sc.mask0) + __popc(sc.mask1)) * per;
+          if (sc.rest >= 0) {  // very many segments: count the rest one by one
+            LoraSeg rs;
+            rs.c = sc.rest;
+            rs.end = ti.row0 + ti.nvalid;
+            while (lora_seg_next(p, ti, rs)) nls += per;
+          }
+          if (lane == 0) sm.tile_nls[itp & 15] = nls;
+        }
+        const int kb = u.k0 + i;
         ok = acquire(1);
         if (!ok) break;
         if (lane == 0) {
@@ -494,32 +628,28 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
           phase ^= 1u;
         }
       }
-      if (ok && p.z != nullptr) {
-        // LoRA stages: A = B_a^T (MN-major: 64 gate/low + 64 up/high features x rbox
-        // rank rows), B = the segment's z rows in tile columns [c_start, c_start + n),
-        // zero outside the segment
-        const int f0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
-        const int col0 = f0, col1 = (p.epi == EPI_GATEUP) ? p.I + f0 : f0 + 64;
-        const int kch = p.rbox / 8;  // 16-byte chunks of a z row per stage
+      if (ok && nls > 0) {
+        SegIter si = seg_iter_begin(sc);
         LoraSeg ls;
-        lora_seg_begin(p, ti, ls);
-        while (ok && lora_seg_next(p, ti, ls)) {
-          for (int kh = 0; kh * 64 < p.r; ++kh) {
+        while (ok && seg_iter_next(p, ti, sc, si, ls)) {  // warp-uniform
+          for (int kh = 0; kh < per; ++kh) {
             ok = acquire(9);
             if (!ok) break;
             uint8_t* a_s = ring + stage * Cfg::kStageBytes;
             uint8_t* b_s = a_s + kATileBytes;
             if (lane == 0) {
+              sm.lstage_col[stage] = ls.c_start;
+              sm.lstage_n[stage] = ls.n;
               const int krow = ls.slot * p.r + kh * 64;
               if constexpr (TWO) {
                 const uint32_t fb = leader_bar(&sm.full[stage]);
                 if (rank == 0) mbar_expect_tx(&sm.full[stage], 2 * 2 * p.rbox * 128);
-                tma_load_2d_pair(a_s, &tmlb, fb, col0, krow);
-                tma_load_2d_pair(a_s + p.rbox * 128, &tmlb, fb, col1, krow);
+                tma_load_2d_pair(a_s, &tmlb, fb, lf0, krow);
+                tma_load_2d_pair(a_s + p.rbox * 128, &tmlb, fb, lcol1, krow);
               } else {
                 mbar_expect_tx(&sm.full[stage], 2 * p.rbox * 128);
-                tma_load_2d(a_s, &tmlb, &sm.full[stage], col0, krow);
-                tma_load_2d(a_s + p.rbox * 128, &tmlb, &sm.full[stage], col1, krow);
+                tma_load_2d(a_s, &tmlb, &sm.full[stage], lf0, krow);
+                tma_load_2d(a_s + p.rbox * 128, &tmlb, &sm.full[stage], lcol1, krow);
               }
               filled_mask |= 1u << stage;
               last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -535,7 +665,13 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
               const __nv_bfloat16* src = valid ? p.z + static_cast<size_t>(row) * p.r + el : p.z;
               cp_async_16_zfill(b_s + j * 128 + ((c ^ (j & 7)) << 4), src, valid);  // 128-byte swizzle
             }
-            pend_mask |= 1u << stage;
+            if constexpr (TWO) {
+              pend_mask |= 1u << stage;
+            } else {
+              cp_async_mbar_arrive(&sm.full[stage]);     // each lane: +1 now, -1 when its copies land
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.full[stage]);  // the stage's counted arrival
+            }
             if (++stage == S) {
               stage = 0;
               phase ^= 1u;
@@ -543,8 +679,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
           }
         }
       }
+      ++itp;
     }
     flush_lora();  // every issued stage gets its arrival, also on the abort path
+    cp_async_wait_all();  // no copy into this CTA's shared memory outlives the producer
     if (lane == 0 && *abort_flag && rank == 0) {  // pairs: the leader's barriers count both CTAs' copies
       // let our own copies land before the CTA exits
       for (int s = 0; s < S; ++s)
@@ -611,33 +749,33 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
             phase ^= 1u;
           }
         }
-        {
-          if (ok && p.z != nullptr) {
-            // e4m3 weights: LoRA goes to its own accumulator (no weight or plane scale)
-            const uint32_t d_lora = d_tmem + (W8 ? 2 * Cfg::kAccStride : 0);
-            LoraSeg ls;
-            lora_seg_begin(p, ti, ls);
-            while (ok && lora_seg_next(p, ti, ls)) {
-              const uint32_t lidesc = umma_idesc_bf16_amn(kMM, ls.n);
-              for (int kh = 0; kh * 64 < p.r; ++kh) {
-                if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 10)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-                const uint32_t a_addr = smem_u32(ring + stage * Cfg::kStageBytes);
-                const uint64_t adesc = umma_desc_mn_sw128(a_addr, p.rbox * 128);
-                const uint64_t bdesc = umma_desc_sw128(a_addr + kATileBytes);
-                for (int kk = 0; kk < p.rbox / 16; ++kk) {  // 16 rank rows (2048 B of A) per instruction
-                  if constexpr (TWO) umma_bf16_pair(d_lora + ls.c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
-                  else umma_bf16(d_lora + ls.c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
-                }
-                commit(&sm.empty[stage]);
-                if (++stage == S) {
-                  stage = 0;
-                  phase ^= 1u;
-                }
-              }
+        if (ok && lz) {
+          // e4m3 weights: LoRA goes to its own accumulator (no weight or plane scale).
+          // The count and each stage's columns come from the producer's shared-memory
+          // records, so no segment table is read on this thread's critical path.
+          const uint32_t d_lora = d_tmem + (W8 ? 2 * Cfg::kAccStride : 0);
+          const int nls = static_cast<volatile int*>(sm.tile_nls)[it & 15];
+          for (int j = 0; j < nls; ++j) {
+            if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kWaitLimitNs, 10)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if constexpr (!TWO) fence_proxy_async_smem();  // z written by cp.async (generic proxy)
+            const int c_start = static_cast<volatile int*>(sm.lstage_col)[stage];
+            const int n_l = static_cast<volatile int*>(sm.lstage_n)[stage];
+            const uint32_t lidesc = umma_idesc_bf16_amn(kMM, n_l);
+            const uint32_t a_addr = smem_u32(ring + stage * Cfg::kStageBytes);
+            const uint64_t adesc = umma_desc_mn_sw128(a_addr, p.rbox * 128);
+            const uint64_t bdesc = umma_desc_sw128(a_addr + kATileBytes);
+            for (int kk = 0; kk < p.rbox / 16; ++kk) {  // 16 rank rows (2048 B of A) per instruction
+              if constexpr (TWO) umma_bf16_pair(d_lora + c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
+              else umma_bf16(d_lora + c_start, adesc + 128 * kk, bdesc + 2 * kk, lidesc, 1u);
+            }
+            commit(&sm.empty[stage]);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
             }
           }
         }
@@ -663,7 +801,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 4);
-      if constexpr (Cfg::kPrefetch) got = got && mbar_wait(&sm.sfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 7);
+      got = got && mbar_wait(&sm.sfull[buf], use & 1u, abort_flag, p.status, kWaitLimitNs, 7);
       // stream-K roles: a later part stores its partial; the first part of a split tile
       // waits (bounded) for the later parts' flags, then adds their partials in CTA order
       const bool sk_store = p.sk && u.k0 != 0;
@@ -711,13 +849,6 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
       for (int c0 = 0; c0 < ti.nvalid; c0 += 32) {
         named_bar_sync(1, kEpiThreads);  // the previous chunk is done with smem
         const int ncol = min(32, ti.nvalid - c0);
-        if constexpr (!Cfg::kPrefetch) {
-          if (p.epi == EPI_DOWN && et < 32) {
-            const int pr = et < ncol ? p.sorted_pairs[ti.row0 + c0 + et] : 0;
-            sm.col_pair[et] = pr;
-            sm.col_w[et] = et < ncol ? p.topk_w[pr] : 0.f;
-          }
-        }
         float v[32];
         const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) +
                                buf * Cfg::kAccPerBuf * Cfg::kAccStride + c0;
@@ -728,7 +859,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
 #pragma unroll
           for (int n = 0; n < 32; ++n)
             if (c0 + n < BN) v[n] = scale * (v[n] * slot->col_sh[c0 + n] + vl[n] * slot->col_sl[c0 + n]);
-          if (p.z != nullptr) {
+          if (lz) {
             tmem_ld_32x32b_x32(t_acc + 2 * Cfg::kAccStride, vl);
 #pragma unroll
             for (int n = 0; n < 32; ++n) v[n] += vl[n];
@@ -800,10 +931,9 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
             }
           }
         } else if (p.epi == EPI_DOWN) {
-          if constexpr (!Cfg::kPrefetch) named_bar_sync(1, kEpiThreads);  // col_pair / col_w visible
           if (row_ok) {
-            const int* cp = Cfg::kPrefetch ? slot->col_pair + c0 : sm.col_pair;
-            const float* cw = Cfg::kPrefetch ? slot->col_w + c0 : sm.col_w;
+            const int* cp = slot->col_pair + c0;
+            const float* cw = slot->col_w + c0;
 #pragma unroll
             for (int n = 0; n < 32; ++n)
               if (n < ncol) p.out_f32[static_cast<size_t>(cp[n]) * p.n_out + feat] = v[n] * cw[n];
@@ -831,7 +961,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
         }
       }
       if constexpr (W8) {
-        if (p.z != nullptr)
+        if (lz)
           for (int c = 0; c < Cfg::kAccStride; c += 32)
             tmem_zero_32x32b_x32(tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) +
                                  (buf * Cfg::kAccPerBuf + 2) * Cfg::kAccStride + c);
@@ -851,11 +981,11 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
       tc_fence_before();
       if constexpr (TWO) mbar_arrive_cluster(leader_bar(&sm.tempty[buf]));  // the leader's MMA reuses it
       else mbar_arrive(&sm.tempty[buf]);
-      if constexpr (Cfg::kPrefetch) mbar_arrive(&sm.sempty[buf]);
+      mbar_arrive(&sm.sempty[buf]);
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------ epilogue loader
-    if constexpr (Cfg::kPrefetch) {
+    {
       uint32_t issued_mask = 0, issued_parity = 0;
       int it = 0;
       UnitIter uit = unit_begin(p, total_tiles, nk);
@@ -867,14 +997,16 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
         const bool got = mbar_wait(&sm.sempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, kWaitLimitNs, 8);
         if (!__all_sync(0xffffffffu, got)) break;
         EpiSlot<BN>* slot = reinterpret_cast<EpiSlot<BN>*>(slots + buf * Cfg::kSlotBytes);
-        if (lane == 0 && p.delta != nullptr) {
-          const int f0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
-          const int c1 = (p.epi == EPI_GATEUP) ? p.I + f0 : f0 + 64;
-          mbar_expect_tx(&sm.sfull[buf], 2 * BN * 64 * 4);
-          tma_load_2d(slot->delta, &tmd, &sm.sfull[buf], f0, ti.row0);
-          tma_load_2d(slot->delta + BN * 64, &tmd, &sm.sfull[buf], c1, ti.row0);
-          issued_mask |= 1u << buf;
-          issued_parity = (issued_parity & ~(1u << buf)) | ((use & 1u) << buf);
+        if constexpr (Cfg::kPrefetch) {
+          if (lane == 0 && p.delta != nullptr) {
+            const int f0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
+            const int c1 = (p.epi == EPI_GATEUP) ? p.I + f0 : f0 + 64;
+            mbar_expect_tx(&sm.sfull[buf], 2 * BN * 64 * 4);
+            tma_load_2d(slot->delta, &tmd, &sm.sfull[buf], f0, ti.row0);
+            tma_load_2d(slot->delta + BN * 64, &tmd, &sm.sfull[buf], c1, ti.row0);
+            issued_mask |= 1u << buf;
+            issued_parity = (issued_parity & ~(1u << buf)) | ((use & 1u) << buf);
+          }
         }
         if (p.epi == EPI_DOWN) {
           for (int n = lane; n < BN; n += 32) {
@@ -954,8 +1086,11 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         232448);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               232448);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -1066,12 +1201,15 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO>, tmw, tmb, tml, tmd, tmlb, p);
+    cudaError_t e = a.z != nullptr
+                        ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO, true>, tmw, tmb, tml, tmd, tmlb, p)
+                        : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO, false>, tmw, tmb, tml, tmd, tmlb, p);
     count_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   } else {
-    gemm_tc_kernel<BN, W8, TWO><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
+    if (a.z != nullptr) gemm_tc_kernel<BN, W8, TWO, true><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
+    else gemm_tc_kernel<BN, W8, TWO, false><<<grid, Cfg::kThreads, smem, st>>>(tmw, tmb, tml, tmd, tmlb, p);
     count_launch();
     return cudaGetLastError();
   }

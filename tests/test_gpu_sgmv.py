@@ -98,3 +98,25 @@ def test_sgmv_bad_adapter_sets_status():
     with pytest.raises(ml.MoELoRAError) as ei:
         ml.check_status(ws)
     assert ei.value.status == ml.ERR_DEVICE_CHECK
+
+
+@pytest.mark.parametrize("where", ["gemm", "delta"])
+def test_dense_many_segments(where, monkeypatch):
+    """Tokens in arrival order (not grouped by adapter): every maximal run of one adapter
+    is a segment, ~200 of them, so a 256-token tile meets more than 64 segments (the
+    GEMM's segment scan then also walks candidates one by one)."""
+    monkeypatch.setenv("MOE_LORA_EXPAND", where)
+    s = synth.DENSE_DECODE_BF16.with_(name="bf16_many_segs", wid=305, T=300, h_in=256, h_out=640, L=4,
+                                      r=64, adapter_dist="uniform")
+    d = dense_f64(s)
+    ids = np.random.default_rng(305).integers(-1, s.L, size=s.T)
+    starts = [0] + [i for i in range(1, s.T) if ids[i] != ids[i - 1]]
+    offs = np.array(starts + [s.T], dtype=np.int32)
+    segs = ids[starts].astype(np.int32)
+    assert len(segs) > 150
+    y = ml.dense_lora_forward(d["x"].cuda(), d["w"]["w"].cuda(), d["w"]["a"].cuda(), d["w"]["b"].cuda(),
+                              torch.from_numpy(offs).cuda(), torch.from_numpy(segs).cuda())
+    torch.cuda.synchronize()
+    y_ref = ref.dense_lora_forward(d["x64"], d["w64"], d["a64"], d["b64"], offs, segs)
+    err = rel_err(y, y_ref)
+    assert err <= TOL_BF16, err
