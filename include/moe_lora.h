@@ -34,6 +34,20 @@
  *     the up projection in rows [I, 2I); expert down w_d [E][H][I]; dense W [h_out][h_in].
  *     LoRA A is stored transposed as [.. ][r][h_in]; LoRA B as [.. ][r][h_out].
  *   - No alpha/r scaling is applied: y = xW + (xA)B exactly; fold any scale into B.
+ *
+ * Environment switches (read at each call; none changes a result beyond rounding order)
+ *   MOE_LORA_EXPAND=gemm|delta  where the LoRA expand z B runs: inside the grouped GEMM
+ *                               as extra tensor-core K steps, or in the LoRA kernel into an
+ *                               fp32 delta the GEMM epilogue adds.  Default: inside the GEMM
+ *                               above 64 rows per expert (prefill), the delta below (decode).
+ *   MOE_LORA_FORCE_BN=16|32|64|128|256  the GEMM's token tile (default: from the mean rows
+ *                               per group: <= 12 -> 16, <= 24 -> 32, <= 64 -> 64, <= 96 -> 128,
+ *                               else 256).
+ *   MOE_LORA_STREAMK=1          stream-K split of the GEMM's (tile, K stage) iterations over
+ *                               all SMs when there are fewer than two tiles per SM (off by
+ *                               default: measured slower on the dense decode GEMM).
+ *   MOE_LORA_PAIR=1             N tiles of 128/256 on CTA pairs (tcgen05 cta_group::2, M = 256;
+ *                               off by default: measured slower at prefill).
  */
 #ifndef MOE_LORA_H
 #define MOE_LORA_H
