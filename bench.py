@@ -106,6 +106,24 @@ def max_over_ranks(v: float, world: int) -> float:
     return float(t.item())
 
 
+def step_percentiles(run_step, n_steps: int) -> dict:
+    """Device time of each of up to 200 further steps, run after the timed region (not part
+    of `value`): median and 10th / 90th percentiles in ms."""
+    try:
+        n = max(1, min(n_steps, 200))
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        evs[0].record()
+        for i in range(n):
+            run_step(i)
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        d = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(n))
+        q = lambda f: d[min(n - 1, int(round(f * (n - 1))))]  # noqa: E731
+        return {"p10_ms": q(0.1), "p50_ms": q(0.5), "p90_ms": q(0.9), "steps": n}
+    except Exception as e:  # a side measurement never costs the line
+        return {"error": f"{type(e).__name__}: {str(e)[:120]}"}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -422,6 +440,7 @@ def run_dense(args, shape: synth.DenseShape, world, rank, local):
     clk = clocks.stop()
     ms_max = max_over_ranks(ev0.elapsed_time(ev1), world)
     value = world * T * args.steps / (ms_max / 1e3)
+    per_step = step_percentiles(run_step, args.steps)
 
     # ---- e2e: pinned host x -> device, dense_lora_forward, y -> pinned host, every step
     e2e_steps = args.e2e_steps or args.steps
@@ -488,7 +507,8 @@ def run_dense(args, shape: synth.DenseShape, world, rank, local):
                 "h2d_bytes_per_step": T * shape.h_in * eb, "d2h_bytes_per_step": T * shape.h_out * eb,
                 "how": "graph replay of H2D copy, dense_lora_forward, D2H copy" if not args.no_graph
                 else "plain API calls"},
-        "timing": {"mode": "CUDA graph replay of the API call" if not args.no_graph else "plain API calls"},
+        "timing": {"mode": "CUDA graph replay of the API call" if not args.no_graph else "plain API calls",
+                   "per_step": per_step},
         "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -644,6 +664,7 @@ def main():
     clk = clocks.stop()
     ms_max = max_over_ranks(ms, world)
     value = world * M * args.steps / (ms_max / 1e3)
+    per_step = step_percentiles(run_step, args.steps)
 
     # ---- secondary measurements: the same step with every adapter id -1 (base only, the
     #      LoRA work skipped by segment) and with one adapter for every token
@@ -772,7 +793,8 @@ def main():
                 "d2h_bytes_per_step": M * shape.H * 2,
                 "how": "graph replay of H2D copy, route, forward, D2H copy" if not args.no_graph else "plain API calls"},
         "timing": {"mode": "CUDA graph replay of the route + forward API calls" if not args.no_graph
-                   else "plain API calls", "plain_api_ms_per_step": plain_ms / args.steps},
+                   else "plain API calls", "plain_api_ms_per_step": plain_ms / args.steps,
+                   "per_step": per_step},
         "gpu_launches": launches,
         "clocks": clk,
     }
