@@ -24,6 +24,8 @@ Modules:
 Pins (tests/test_oracle_*.py, ``-m "not gpu"``): brute force on tiny inputs,
 hand-derived golden cases (tests/golden/), library routines (torch casts, softmax),
 closed forms and invariants (zero adapters, merged weights, linearity, top-k = E,
-permutation invariance of SGMV).  Parity of end-to-end values beyond those pins is
-unpinned: the pages print no worked numeric example.
+permutation invariance of SGMV).  Every public function here is checked by at least one
+of them (helpers through the functions that call them).  The pages print no worked
+numeric example, so no pin is a value printed by the pages; the golden cases are closed
+forms derived by hand from the definitions.
 """
