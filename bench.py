@@ -3,19 +3,22 @@
 
 One step = one pass of the whole path over one batch resident in HBM:
   moe_lora_route   router logits x W_r^T, softmax top-k + renormalised weights,
-                   stable (expert, adapter) sort into segments (one launch at decode)
-  moe_lora_forward gather + gate_up LoRA shrink, tcgen05 gate_up GEMM running the LoRA
-                   expand as extra MMA K steps and SiLU-and-mul in its epilogue, down
-                   LoRA shrink, tcgen05 down GEMM with the expand and the routing weight,
-                   fixed-order combine
+                   stable (expert, adapter) sort into segments
+  moe_lora_forward gather + LoRA shrink, tcgen05 gate_up GEMM (LoRA expand, SiLU-and-mul),
+                   down LoRA, tcgen05 down GEMM (LoRA expand, routing weight), fixed-order
+                   combine
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--M M]
     python bench.py --impl reference ...      (the fp64 CPU oracle, same metric)
 
-Default workload: MoE decode, bf16 experts, E=64, top-8, H=2048, I=1408, 8 adapters
-of rank 16 on gate_up and down, M=64 tokens per step.  For N > 1 (torchrun) every
-rank runs an independent replica (weak scaling, no collective on the data path);
-timing is the max over ranks.  Prints one JSON line on rank 0.
+Default workload: the MoE prefill layer, the largest configuration that fits one GPU:
+4096 tokens, bf16 experts, E=128, top-8, H=4096, I=1536, 16 adapters of rank 64 on
+gate_up and down (Zipf adapter ids, router bias skewing the expert load).  The same line
+carries a `sweep` of the decode layers (bf16 E=64 at M = 1, 8, 32, 64; e4m3 experts
+E=128 at M = 1, 4, 16, 64) and the dense decode projection, measured in the same
+process.  For N > 1 (torchrun) every rank runs an independent replica (weak scaling, no
+collective on the data path); timing is the max over ranks.  Prints one JSON line on
+rank 0.
 """
 from __future__ import annotations
 
@@ -24,6 +27,7 @@ import datetime
 import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -38,24 +42,26 @@ sys.path.insert(0, ROOT)
 from workloads import synth  # noqa: E402
 
 METRIC = "MoE+multi-LoRA layer tokens/s; achieved HBM GB/s or TC util vs B200 peak"
-DEFAULT_WORKLOAD = synth.MOE_DECODE_BF16.name
+DEFAULT_WORKLOAD = synth.MOE_PREFILL_BF16.name
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
+# decode layers measured in the same process as the headline line
+SWEEP = ((synth.MOE_DECODE_BF16.name, (1, 8, 32, 64)), (synth.MOE_DECODE_FP8.name, (1, 4, 16, 64)),
+         (synth.DENSE_DECODE_BF16.name, (64,)))
 
-# ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM on the
-# default workload, with the hash of the kernel source it was taken on; reported as
-# null when the source has changed since.  Filled from profiles/.
-NCU_TRAFFIC = {"gemm_tc.cu": "6ca23e0dc6e3bec3", "bytes_per_launch": 746.644224e6 + 5.415680e6,
-               "workload": synth.MOE_DECODE_BF16.name, "M": 64}
+# ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM, with the
+# hash of the kernel source it was taken on and the case it was taken on; reported as
+# null when the source has changed since or the case differs.  Filled from profiles/.
+NCU_TRAFFIC = {"gemm_tc.cu": "", "bytes_per_launch": 0.0, "workload": "", "M": 0}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--M", type=int, default=64)
+    ap.add_argument("--M", type=int, default=0, help="tokens per step (0: the workload's largest)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batches", type=int, default=4, help="distinct token batches cycled over the steps")
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps")
@@ -63,9 +69,15 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the base-only and same-adapter variants of the MoE step")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the decode sweep")
+    ap.add_argument("--sweep-seconds", type=float, default=0.25, help="timed device seconds per sweep entry")
     ap.add_argument("--no-graph", action="store_true",
                     help="time plain API calls instead of replaying a CUDA graph of them")
-    return ap.parse_args()
+    a = ap.parse_args(argv)
+    if a.M <= 0:
+        shape = synth.WORKLOADS[a.workload]
+        a.M = shape.M_list[-1] if isinstance(shape, synth.MoEShape) else shape.T
+    return a
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -131,6 +143,17 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 class ClockSampler:
@@ -235,6 +258,22 @@ def layer_flops(shape, M):
             + 2 * mk * shape.r * (2 * shape.H + 3 * shape.I) + 2 * M * shape.H * shape.E)
 
 
+def gateup_tensor_bound(shape, M) -> bool:
+    """>= 128 rows per expert on average: the MMA, not the weight stream, bounds gate_up."""
+    return M * shape.k >= 128 * shape.E
+
+
+def scaled_kernel_times(event_ms: dict, instrumented_step_ms: float, step_ms: float) -> dict:
+    """Per-kernel device time per step, reconciled with the uninstrumented step: each
+    kernel's share of the instrumented step (event pairs around every launch inside the
+    replayed graphs) applied to the step time measured without events.  The event nodes
+    serialise the graph and add a few microseconds each, so the raw event sums exceed the
+    plain step; the shares do not depend on that overhead's absolute size."""
+    if instrumented_step_ms <= 0:
+        return {k: 0.0 for k in event_ms}
+    return {k: v / instrumented_step_ms * step_ms for k, v in event_ms.items()}
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -244,82 +283,74 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def cores_desc() -> dict:
+    return {"cores": blas_threads(), "cpu_model": cpu_model(), "host_cpus": os.cpu_count()}
+
+
 # ----------------------------------------------------------------------------- oracle timing
 
-def oracle_tokens_per_s(shape, M, cpu_weights, seconds: float, max_calls: int | None = None,
-                        tokens_per_call: int | None = None):
-    """The fp64 oracle (route from x, sort, forward) on batch 0, repeated until `seconds`
-    of CPU time have passed (or `max_calls`); returns (tokens/s, calls, tokens/call)."""
+class StoredSlices:
+    """Expert and adapter slices of one MoE workload at their stored precision (bf16 or
+    e4m3 bits), drawn once from the seeded generator before timing; every get widens
+    the slice to fp64 anew, so the oracle's timed region runs from the stored weights
+    to y, conversion included (generation excluded)."""
+
+    def __init__(self, shape: synth.MoEShape):
+        self.s = shape
+        self.e, self.a = {}, {}
+
+    def prepare(self, ids: np.ndarray, adapter_ids: np.ndarray):
+        import concurrent.futures as cf
+        need_e = sorted({int(e) for e in ids.reshape(-1)} - set(self.e))
+        need_a = sorted({(int(adapter_ids[t]), int(e)) for t in range(ids.shape[0]) for e in ids[t]
+                         if adapter_ids[t] >= 0} - set(self.a))
+        with cf.ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1))) as ex:
+            for e, v in zip(need_e, ex.map(lambda e: synth.moe_expert(self.s, e), need_e)):
+                self.e[e] = (synth.bits(v[0]), synth.bits(v[1]), float(v[2]), float(v[3]))
+            for ae, v in zip(need_a, ex.map(lambda ae: synth.moe_adapter(self.s, *ae), need_a)):
+                self.a[ae] = tuple(synth.bits(t) for t in v)
+
+    def expert(self, e):
+        from oracle import formats
+        gu, d, sg, sd = self.e[int(e)]
+        return formats.to_f64(gu, self.s.wdtype), formats.to_f64(d, self.s.wdtype), sg, sd
+
+    def adapter(self, a, e):
+        from oracle import formats
+        return tuple(formats.to_f64(t, "bf16") for t in self.a[(int(a), int(e))])
+
+
+def oracle_tokens_per_s(shape, M, seconds: float, max_calls: int | None = None,
+                        tokens_per_call: int | None = None, slices: StoredSlices | None = None):
+    """The fp64 oracle (route from x, sort, forward) on the first tokens of batch 0,
+    repeated until `seconds` of CPU time have passed (or `max_calls`); returns
+    (tokens/s, calls, tokens/call, elapsed s).  The touched expert and adapter slices are
+    drawn at stored precision before timing; their fp64 conversion is timed."""
     from oracle import formats
     from oracle import moe_lora_ref as ref
-    from tests.gpu_cases import CpuWeightsOracle
-    OW = CpuWeightsOracle(shape, cpu_weights)
     x, ad = synth.moe_tokens(shape, M)
     x64 = formats.to_f64(synth.bits(x), "bf16")
     ad64 = ad.numpy().astype(np.int64)
-    wr, bias = OW.router()
+    wr_t, bias_t = synth.moe_router(shape)
+    wr = formats.to_f64(synth.bits(wr_t), "bf16")
+    bias = None if bias_t is None else bias_t.numpy().astype(np.float64)
     n = M if tokens_per_call is None else max(1, min(M, tokens_per_call))
     sel = np.arange(n)
-    # weights of the experts this batch touches are decoded once, like a model load
-    lg = ref.router_logits(x64, wr, bias)
-    ids, _ = ref.route_topk(lg, shape.k)
-    for e in np.unique(ids[sel]):
-        OW.expert(int(e))
+    sl = slices if slices is not None else StoredSlices(shape)
+    ids, _ = ref.route_topk(ref.router_logits(x64[sel], wr, bias), shape.k)
+    sl.prepare(ids, ad64[sel])
     calls, t0 = 0, time.perf_counter()
     while True:
         lg = ref.router_logits(x64[sel], wr, bias)
         ids, w = ref.route_topk(lg, shape.k)
         ref.sort_pairs(ids, ad64[sel], shape.E, shape.L)
-        ref.moe_lora_forward(x64[sel], ids, w, ad64[sel], shape.I, OW.expert, OW.adapter)
+        ref.moe_lora_forward(x64[sel], ids, w, ad64[sel], shape.I, sl.expert, sl.adapter)
         calls += 1
         el = time.perf_counter() - t0
         if el >= seconds or (max_calls is not None and calls >= max_calls):
             break
     return n * calls / el, calls, n, el
 
-
-def reference_arm(args, world, rank):
-    """--impl reference: the oracle on the host cores, same metric/unit/config."""
-    if rank != 0:
-        return
-    shape = synth.WORKLOADS[args.workload]
-    if not isinstance(shape, synth.MoEShape):
-        dense_oracle_tokens_per_s(shape, seconds=0.0, max_calls=max(1, args.warmup))
-        tps, calls, n, el = dense_oracle_tokens_per_s(shape, seconds=1e9, max_calls=args.steps)
-        print(json.dumps({
-            "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / calls, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": shape.name, "T": shape.T, "h_in": shape.h_in, "h_out": shape.h_out,
-                       "L": shape.L, "r": shape.r},
-            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"{n} tokens per step, {calls} steps, {el:.1f} s"},
-            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
-        return
-    M = args.M
-    cpu = synth.moe_weights(shape, device="cpu")
-    # size one step so that warmup + steps take about two minutes of CPU time
-    tps, _, _, _ = oracle_tokens_per_s(shape, M, cpu, seconds=2.0, max_calls=1, tokens_per_call=1)
-    per_tok = 1.0 / tps
-    budget = 120.0
-    tok = int(max(1, min(M, budget / max(1, args.steps + args.warmup) / per_tok)))
-    oracle_tokens_per_s(shape, M, cpu, seconds=0.0, max_calls=max(1, args.warmup), tokens_per_call=tok)
-    tps, calls, n, el = oracle_tokens_per_s(shape, M, cpu, seconds=1e9, max_calls=args.steps, tokens_per_call=tok)
-    cores = blas_threads()
-    line = {
-        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / calls, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": shape.name, "M": M, "E": shape.E, "k": shape.k, "H": shape.H, "I": shape.I,
-                   "L": shape.L, "r": shape.r, "wdtype": shape.wdtype},
-        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{n} token(s) of batch 0 per step, {calls} steps, {el:.1f} s"},
-        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line))
-
-
-# ----------------------------------------------------------------------------- dense SGMV arm
 
 def dense_oracle_tokens_per_s(shape: synth.DenseShape, seconds: float, max_calls: int | None = None):
     """The fp64 oracle of one dense multi-LoRA projection on the bench's token batch,
@@ -342,10 +373,53 @@ def dense_oracle_tokens_per_s(shape: synth.DenseShape, seconds: float, max_calls
     return shape.T * calls / el, calls, shape.T, el
 
 
-def run_dense(args, shape: synth.DenseShape, world, rank, local):
+def reference_arm(args, world, rank):
+    """--impl reference: the oracle on the host cores, same metric/unit/config."""
+    if rank != 0:
+        return
+    shape = synth.WORKLOADS[args.workload]
+    base = {"impl": "reference", "metric": METRIC, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic"}
+    if not isinstance(shape, synth.MoEShape):
+        dense_oracle_tokens_per_s(shape, seconds=0.0, max_calls=max(1, args.warmup))
+        tps, calls, n, el = dense_oracle_tokens_per_s(shape, seconds=1e9, max_calls=args.steps)
+        print(json.dumps({
+            **base, "value": tps, "ms_per_step": 1e3 * el / calls,
+            "config": {"workload": shape.name, "T": shape.T, "h_in": shape.h_in, "h_out": shape.h_out,
+                       "L": shape.L, "r": shape.r},
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", **cores_desc(), "kind": "oracle",
+                             "sample": f"{n} tokens per step, {calls} steps, {el:.1f} s"},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return
+    M = args.M
+    sl = StoredSlices(shape)
+    # size one step so that warmup + steps take about two minutes of CPU time
+    tps, _, _, _ = oracle_tokens_per_s(shape, M, seconds=2.0, max_calls=1, tokens_per_call=1, slices=sl)
+    per_tok = 1.0 / tps
+    budget = 120.0
+    tok = int(max(1, min(M, 64, budget / max(1, args.steps + args.warmup) / per_tok)))
+    oracle_tokens_per_s(shape, M, seconds=0.0, max_calls=max(1, args.warmup), tokens_per_call=tok, slices=sl)
+    tps, calls, n, el = oracle_tokens_per_s(shape, M, seconds=1e9, max_calls=args.steps, tokens_per_call=tok,
+                                            slices=sl)
+    line = {
+        **base, "value": tps, "ms_per_step": 1e3 * el / calls,
+        "config": {"workload": shape.name, "M": M, "E": shape.E, "k": shape.k, "H": shape.H, "I": shape.I,
+                   "L": shape.L, "r": shape.r, "wdtype": shape.wdtype},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", **cores_desc(), "kind": "oracle",
+                         "sample": f"{n} token(s) of batch 0 per step, {calls} steps, {el:.1f} s"},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ----------------------------------------------------------------------------- dense arm
+
+def measure_dense(args, shape: synth.DenseShape, world, local, *, steps, warmup, full):
     """One dense projection with segmented multi-LoRA (dense_lora_forward).  Its weight
     fits in L2, so the steps cycle over enough copies of the weights and adapters that
-    the copy a step reads was evicted by the steps before it (inputs larger than L2)."""
+    the copy a step reads was evicted by the steps before it (inputs larger than L2).
+    Returns the measurement fields of a line (full: also e2e, percentiles and clocks)."""
     import moe_lora_b200 as ml
     dev = torch.device("cuda", local)
     T = shape.T
@@ -363,61 +437,68 @@ def run_dense(args, shape: synth.DenseShape, world, rank, local):
         w = copies[i % n_copies]
         ml.dense_lora_forward(xin, w["w"], w["a"], w["b"], offs, segs, y=y, workspace=ws)
 
-    for i in range(max(args.warmup, n_copies)):
+    for i in range(max(warmup, n_copies)):
         step(i)
     torch.cuda.synchronize()
     ml.check_status(ws)
-
     n0 = ml.launch_count()
-    for i in range(args.steps):
+    for i in range(n_copies):
         step(i)
     torch.cuda.synchronize()
-    launches = ml.launch_count() - n0
+    launches_per_step = (ml.launch_count() - n0) / n_copies
 
-    # ---- per-kernel device times: one step per weight copy captured as a CUDA graph
-    #      with event nodes around every launch, replayed; the last replay is read
-    if not args.no_graph:
+    def capture(fn):
         gs = torch.cuda.Stream()
         gs.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(gs):
-            step(0)
+            fn(0)
         torch.cuda.current_stream().wait_stream(gs)
         torch.cuda.synchronize()
-        ml.profile_enable(n_copies * 4 + 16)
-        pgraphs = []
+        out = []
         for c in range(n_copies):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                step(c)
-            pgraphs.append(g)
+                fn(c)
+            out.append(g)
+        return out
+
+    # ---- per-kernel device times: event pairs around every launch inside the graphs
+    names = ("lora", "shrink", "gemm_dense", "dense_f32")
+    if not args.no_graph:
+        ml.profile_enable(n_copies * 4 + 16)
+        pgraphs = capture(step)
         for _ in range(3):
             for g in pgraphs:
                 g.replay()
         torch.cuda.synchronize()
+        per_kernel = {k: ml.profile_read(k) for k in names}
+        i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        i0.record()
+        for g in pgraphs:
+            g.replay()
+        i1.record()
+        torch.cuda.synchronize()
+        instr_ms = i0.elapsed_time(i1) / n_copies
+        ml.profile_enable(0)
+        del pgraphs
         prof_steps = n_copies
     else:
-        ml.profile_enable(args.steps * 4 + 16)
-        for i in range(args.steps):
+        ml.profile_enable(steps * 4 + 16)
+        for i in range(steps):
             step(i)
         torch.cuda.synchronize()
-        prof_steps = args.steps
-    gemm_ms, gemm_n = ml.profile_read("gemm_dense" if shape.dtype == "bf16" else "dense_f32")
-    per_kernel = {k: ml.profile_read(k)[0] / prof_steps for k in ("lora", "shrink", "gemm_dense", "dense_f32")}
-    ml.profile_enable(0)
-    if not args.no_graph:
-        del pgraphs
+        per_kernel = {k: ml.profile_read(k) for k in names}
+        ml.profile_enable(0)
+        prof_steps, instr_ms = steps, 0.0
+    gemm_ms, gemm_n = per_kernel["gemm_dense" if shape.dtype == "bf16" else "dense_f32"]
+    event_ms = {k: v[0] / prof_steps for k, v in per_kernel.items()}
+    if args.no_graph:
+        instr_ms = sum(event_ms.values())
 
-    # ---- one CUDA graph per weight copy
-    graphs = []
-    if not args.no_graph:
-        for c in range(n_copies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                step(c)
-            graphs.append(g)
-        for i in range(max(args.warmup, n_copies)):
-            graphs[i % n_copies].replay()
-        torch.cuda.synchronize()
+    graphs = capture(step) if not args.no_graph else []
+    for i in range(max(warmup, n_copies)):
+        graphs[i % n_copies].replay() if graphs else step(i)
+    torch.cuda.synchronize()
 
     def run_step(i):
         if graphs:
@@ -425,125 +506,91 @@ def run_dense(args, shape: synth.DenseShape, world, rank, local):
         else:
             step(i)
 
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.25)
+    clocks = ClockSampler(local) if full else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.25)
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
-    for i in range(args.steps):
+    for i in range(steps):
         run_step(i)
     ev1.record()
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks else None
     ms_max = max_over_ranks(ev0.elapsed_time(ev1), world)
-    value = world * T * args.steps / (ms_max / 1e3)
-    per_step = step_percentiles(run_step, args.steps)
-
-    # ---- e2e: pinned host x -> device, dense_lora_forward, y -> pinned host, every step
-    e2e_steps = args.e2e_steps or args.steps
-    hx = x.cpu().pin_memory()
-    hy = torch.empty((T, shape.h_out), dtype=x.dtype).pin_memory()
-    dx = torch.empty_like(x)
-
-    def e2e_step(i):
-        dx.copy_(hx, non_blocking=True)
-        step(i, dx)
-        hy.copy_(y, non_blocking=True)
-
-    e2e_graphs = []
-    if not args.no_graph:
-        for c in range(n_copies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                e2e_step(c)
-            e2e_graphs.append(g)
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(e2e_steps):
-        if e2e_graphs:
-            e2e_graphs[i % n_copies].replay()
-        else:
-            e2e_step(i)
-    e1.record()
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    del graphs, e2e_graphs
-    ml.check_status(ws)
+    step_ms = ms_max / steps
 
     adapters = sorted(set(int(v) for v in tok_a.tolist() if v >= 0))
     lay_bytes = (shape.h_out * shape.h_in + len(adapters) * shape.r * (shape.h_in + shape.h_out)) * eb \
         + T * (shape.h_in + shape.h_out) * eb
     gemm_bytes = shape.h_out * shape.h_in * eb + T * shape.h_in * eb + T * shape.h_out * eb
-    if shape.dtype == "bf16":  # the fused expand: z rows and the touched B slices
+    if shape.dtype == "bf16" and T > 64:  # expand inside the GEMM: z rows and the touched B slices
         gemm_bytes += T * shape.r * 2 + len(adapters) * shape.r * shape.h_out * 2
+    elif shape.dtype == "bf16":  # fp32 delta of the LoRA kernel
+        gemm_bytes += T * shape.h_out * 4
     peaks, peak_src = load_peaks()
     peak = float(peaks["hbm_gbs"])
     g_s = (gemm_ms / max(gemm_n, 1)) / 1e3
-    step_s = ms_max / 1e3 / args.steps
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
-        "config": {"workload": shape.name, "T": T, "h_in": shape.h_in, "h_out": shape.h_out, "L": shape.L,
-                   "r": shape.r, "adapters": shape.adapter_dist, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: steps cycle over {n_copies} copies of W, A and B "
-                         f"({n_copies * copy_bytes / 1e6:.0f} MB)"},
+    out = {
+        "value": world * T / (step_ms / 1e3), "ms_per_step": step_ms, "steps": steps,
         "roofline": {"bound": "hbm", "kernel": "gemm_tc (dense)" if shape.dtype == "bf16" else "dense_f32",
                      "achieved": gemm_bytes / g_s / 1e9, "peak": peak, "unit": "GB/s",
-                     "frac": gemm_bytes / g_s / 1e9 / peak, "peak_source": peak_src, "traffic": None,
-                     "alg_bytes_per_launch": gemm_bytes, "avg_launch_us": g_s * 1e6},
-        "layer": {"alg_bytes_per_step": lay_bytes, "achieved_GBps": lay_bytes / step_s / 1e9,
-                  "frac_of_hbm_peak": lay_bytes / step_s / 1e9 / peak,
-                  "kernel_ms_per_step": per_kernel,
-                  "kernel_times": "CUDA events around each launch inside the replayed step graphs"
-                  if not args.no_graph else "CUDA events around each launch of plain API calls"},
-        "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * shape.h_in * eb, "d2h_bytes_per_step": T * shape.h_out * eb,
-                "how": "graph replay of H2D copy, dense_lora_forward, D2H copy" if not args.no_graph
-                else "plain API calls"},
-        "timing": {"mode": "CUDA graph replay of the API call" if not args.no_graph else "plain API calls",
-                   "per_step": per_step},
-        "gpu_launches": launches, "clocks": clk,
+                     "frac": gemm_bytes / g_s / 1e9 / peak, "peak_source": f"{peak_src} HBM copy",
+                     "traffic": None, "alg_bytes_per_launch": gemm_bytes, "avg_launch_us": g_s * 1e6},
+        "layer": {"alg_bytes_per_step": lay_bytes, "achieved_GBps": lay_bytes / (step_ms / 1e3) / 1e9,
+                  "frac_of_hbm_peak": lay_bytes / (step_ms / 1e3) / 1e9 / peak,
+                  "kernel_ms_per_step": scaled_kernel_times(event_ms, instr_ms, step_ms),
+                  "instrumented_step_ms": instr_ms},
+        "gpu_launches": int(round(launches_per_step * steps)),
+        "l2": f"inputs larger than L2: steps cycle over {n_copies} copies of W, A and B "
+              f"({n_copies * copy_bytes / 1e6:.0f} MB)",
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, calls, n, el = dense_oracle_tokens_per_s(shape, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"fp64 oracle, {n} tokens per call, {calls} calls in {el:.1f} s; "
-                                          "weights decoded to fp64 once before timing"}
-    if rank == 0:
-        print(json.dumps(line))
+    if full:
+        out["clocks"] = clk
+        out["timing_per_step"] = step_percentiles(run_step, steps)
+        e2e_steps = args.e2e_steps or steps
+        hx = x.cpu().pin_memory()
+        hy = torch.empty((T, shape.h_out), dtype=x.dtype).pin_memory()
+        dx = torch.empty_like(x)
+
+        def e2e_step(i):
+            dx.copy_(hx, non_blocking=True)
+            step(i, dx)
+            hy.copy_(y, non_blocking=True)
+
+        e2e_graphs = capture(e2e_step) if not args.no_graph else []
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(e2e_steps):
+            e2e_graphs[i % n_copies].replay() if e2e_graphs else e2e_step(i)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        del e2e_graphs
+        out["e2e"] = {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": T * shape.h_in * eb, "d2h_bytes_per_step": T * shape.h_out * eb,
+                      "how": "graph replay of H2D copy, dense_lora_forward, D2H copy" if not args.no_graph
+                      else "plain API calls"}
+    del graphs
+    ml.check_status(ws)
+    return out
 
 
-# ----------------------------------------------------------------------------- our arm
+# ----------------------------------------------------------------------------- MoE arm
 
-def main():
-    args = parse()
-    world, rank, local = dist_setup()
-    if args.impl == "reference":
-        reference_arm(args, world, rank)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return
+def measure_moe(args, shape: synth.MoEShape, M: int, W: dict, world, local, *, steps, warmup, full):
+    """Route + forward of one MoE layer at M tokens per step, timed as CUDA-graph replays
+    of the two API calls over `args.batches` rotating token batches.  Returns the
+    measurement fields of a line (full: also e2e, percentiles, clocks, secondary)."""
     import moe_lora_b200 as ml
-
-    shape = synth.WORKLOADS[args.workload]
-    if not isinstance(shape, synth.MoEShape):
-        run_dense(args, shape, world, rank, local)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return
     dev = torch.device("cuda", local)
-    M, k, L = args.M, shape.k, shape.L
-    cpu = synth.moe_weights(shape, device="cpu")
-    W = {kk: (v.to(dev) if isinstance(v, torch.Tensor) else v) for kk, v in cpu.items()}
+    k, L = shape.k, shape.L
     batches = []
     for b in range(args.batches):
         x, ad = synth.moe_tokens(shape, M, batch=b)
@@ -557,136 +604,176 @@ def main():
              "seg_offsets": torch.empty((shape.E * (L + 1) + 1,), dtype=torch.int32, device=dev)}
     y = torch.empty((M, shape.H), dtype=torch.bfloat16, device=dev)
 
-    def step(i):
-        xb, ab = batches[i % len(batches)]
+    def call(xb, ab):
         rt = ml.route(ab, k, L, x=xb, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
         ml.forward(xb, rt, W, k=k, L=L, y=y, workspace=fws)
         return rt
 
-    # routing statistics of each batch (outside any timed region)
-    stats = []
+    def step(i):
+        return call(*batches[i % len(batches)])
+
+    stats = []  # routing statistics of each batch (outside any timed region)
     for b in range(len(batches)):
         rt = step(b)
         torch.cuda.synchronize()
         stats.append(routing_stats(rt, shape))
     ml.check_status(fws)
-    for i in range(args.warmup):
+    ml.check_status(rws)
+    for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
 
-    # ---- plain API calls (host enqueue included), for reference
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n0 = ml.launch_count()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_plain = len(batches) if not full else max(len(batches), min(steps, 200))
     p0.record()
-    for i in range(args.steps):
+    for i in range(n_plain):
         step(i)
     p1.record()
     torch.cuda.synchronize()
-    launches_per_step = (ml.launch_count() - n0) / args.steps
-    plain_ms = p0.elapsed_time(p1)
+    launches_per_step = (ml.launch_count() - n0) / n_plain
+    plain_ms = p0.elapsed_time(p1) / n_plain
 
-    # ---- per-kernel device times: each batch's step captured as a CUDA graph with an
-    #      event pair around every launch (event nodes), replayed; the last replay of
-    #      every graph is read.  Without graphs: plain calls (host gaps included).
-    names = ("route", "router_logits", "topk", "sort", "lora", "quant", "gemm_gateup", "gemm_down", "combine")
-    if not args.no_graph:
+    def capture(fn, nb):
         gs = torch.cuda.Stream()
         gs.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(gs):
-            for b in range(len(batches)):
-                step(b)  # warm the stream before capture
+            for b in range(nb):
+                fn(b)  # warm the stream before capture
         torch.cuda.current_stream().wait_stream(gs)
         torch.cuda.synchronize()
-        ml.profile_enable(len(batches) * 16 + 64)
-        pgraphs = []
-        for b in range(len(batches)):
+        out = []
+        for b in range(nb):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                step(b)
-            pgraphs.append(g)
+                fn(b)
+            out.append(g)
+        return out
+
+    # ---- per-kernel device times: each batch's step captured as a CUDA graph with an
+    #      event pair around every launch (event nodes), replayed; the last replay of
+    #      every graph is read, and the instrumented replay itself is timed
+    names = ("route", "router_logits", "topk", "sort", "lora", "quant", "gemm_gateup", "gemm_down", "combine")
+    nb = len(batches)
+    if not args.no_graph:
+        ml.profile_enable(nb * 24 + 64)
+        pgraphs = capture(step, nb)
         for _ in range(5):
             for g in pgraphs:
                 g.replay()
         torch.cuda.synchronize()
-        prof_steps = len(batches)
+        per_kernel = {kname: ml.profile_read(kname) for kname in names}
+        i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        i0.record()
+        for g in pgraphs:
+            g.replay()
+        i1.record()
+        torch.cuda.synchronize()
+        instr_ms = i0.elapsed_time(i1) / nb
+        ml.profile_enable(0)
+        del pgraphs
+        prof_steps = nb
     else:
-        ml.profile_enable(args.steps * 16 + 64)
-        for i in range(args.steps):
+        ml.profile_enable(steps * 24 + 64)
+        for i in range(steps):
             step(i)
         torch.cuda.synchronize()
-        prof_steps = args.steps
-    per_kernel = {kname: ml.profile_read(kname) for kname in names}
-    ml.profile_enable(0)
-    if not args.no_graph:
-        del pgraphs
+        per_kernel = {kname: ml.profile_read(kname) for kname in names}
+        ml.profile_enable(0)
+        prof_steps, instr_ms = steps, 0.0
+    event_ms = {kk: v[0] / prof_steps for kk, v in per_kernel.items()}
+    if args.no_graph:
+        instr_ms = sum(event_ms.values())
     gu_ms, gu_n = per_kernel["gemm_gateup"]
-    launches = int(round(launches_per_step * args.steps))
 
     # ---- the step as a CUDA graph of the same API calls (one graph per token batch)
-    graphs = []
-    if not args.no_graph:
-        gs = torch.cuda.Stream()
-        gs.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(gs):
-            for b in range(len(batches)):
-                step(b)  # warm the stream before capture
-        torch.cuda.current_stream().wait_stream(gs)
-        torch.cuda.synchronize()
-        for b in range(len(batches)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                step(b)
-            graphs.append(g)
-        for i in range(args.warmup):
-            graphs[i % len(graphs)].replay()
-        torch.cuda.synchronize()
+    graphs = capture(step, nb) if not args.no_graph else []
+    for i in range(warmup):
+        graphs[i % nb].replay() if graphs else step(i)
+    torch.cuda.synchronize()
 
     def run_step(i):
         if graphs:
-            graphs[i % len(graphs)].replay()
+            graphs[i % nb].replay()
         else:
             step(i)
 
     # ---- timed region: K steps on device-resident inputs
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.25)
+    clocks = ClockSampler(local) if full else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.25)
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
-    for i in range(args.steps):
+    for i in range(steps):
         run_step(i)
     ev1.record()
     torch.cuda.synchronize()
     barrier(world)
-    ms = ev0.elapsed_time(ev1)
-    clk = clocks.stop()
-    ms_max = max_over_ranks(ms, world)
-    value = world * M * args.steps / (ms_max / 1e3)
-    per_step = step_percentiles(run_step, args.steps)
+    clk = clocks.stop() if clocks else None
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world)
+    step_ms = ms_max / steps
+
+    # ---- roofline of the dominant kernel (gate_up GEMM) and of the whole layer
+    peaks, peak_src = load_peaks()
+    mean = lambda f: float(np.mean([f(*stats[i % nb]) for i in range(steps)]))  # noqa: E731
+    gu_bytes = mean(lambda e, p: gateup_alg_bytes(shape, M, e, p))
+    lay_bytes = mean(lambda e, p: layer_alg_bytes(shape, M, e, p))
+    gu_avg_s = (gu_ms / max(gu_n, 1)) / 1e3
+    peak = float(peaks["hbm_gbs"])
+    traffic = (NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["gemm_tc.cu"] == src_hash("gemm_tc.cu")
+               and NCU_TRAFFIC["workload"] == shape.name and NCU_TRAFFIC["M"] == M else None)
+    if gateup_tensor_bound(shape, M):
+        fp8 = shape.wdtype == "e4m3"
+        peak_t = float(peaks["bf16_tflops_sustained"]) * (2.0 if fp8 else 1.0)
+        achieved = gateup_alg_flops(shape, M) / gu_avg_s / 1e12
+        roof = {"bound": "tensor", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved, "peak": peak_t,
+                "unit": "TFLOP/s", "frac": achieved / peak_t,
+                "peak_source": f"{peak_src} bf16 sustained" + (" x2 (fp8 nominal ratio)" if fp8 else ""),
+                "traffic": traffic, "alg_flops_per_launch": gateup_alg_flops(shape, M),
+                "alg_bytes_per_launch": gu_bytes, "achieved_GBps": gu_bytes / gu_avg_s / 1e9,
+                "avg_launch_us": gu_avg_s * 1e6}
+    else:
+        achieved = gu_bytes / gu_avg_s / 1e9
+        roof = {"bound": "hbm", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_src} HBM copy",
+                "traffic": traffic, "alg_bytes_per_launch": gu_bytes, "avg_launch_us": gu_avg_s * 1e6}
+    out = {
+        "value": world * M / (step_ms / 1e3), "ms_per_step": step_ms, "steps": steps,
+        "roofline": roof,
+        "layer": {"alg_bytes_per_step": lay_bytes, "achieved_GBps": lay_bytes / (step_ms / 1e3) / 1e9,
+                  "frac_of_hbm_peak": lay_bytes / (step_ms / 1e3) / 1e9 / peak,
+                  "TFLOPs": layer_flops(shape, M) / (step_ms / 1e3) / 1e12,
+                  "kernel_ms_per_step": scaled_kernel_times(event_ms, instr_ms, step_ms),
+                  "instrumented_step_ms": instr_ms,
+                  "touched_experts": float(np.mean([s[0] for s in stats])),
+                  "touched_adapter_expert_pairs": float(np.mean([s[1] for s in stats]))},
+        "gpu_launches": int(round(launches_per_step * steps)),
+        "plain_api_ms_per_step": plain_ms,
+        "l2": f"no flush: {lay_bytes / 1e9:.2f} GB of weights per step > 126 MB L2; {nb} rotating token batches",
+    }
+    if not full:
+        del graphs
+        return out
+    out["clocks"] = clk
+    out["timing_per_step"] = step_percentiles(run_step, steps)
 
     # ---- secondary measurements: the same step with every adapter id -1 (base only, the
     #      LoRA work skipped by segment) and with one adapter for every token
-    secondary = None
     if not args.no_secondary and not args.no_graph:
         def timed_variant(ids_fn):
             vb = [(xb, ids_fn(ab)) for xb, ab in batches]
-            vgraphs = []
-            for b, (xb, ab) in enumerate(vb):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    rt = ml.route(ab, k, L, x=xb, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
-                    ml.forward(xb, rt, W, k=k, L=L, y=y, workspace=fws)
-                vgraphs.append(g)
-            n = min(args.steps, 1000)
-            for i in range(min(args.warmup, 20)):
-                vgraphs[i % len(vgraphs)].replay()
+            vgraphs = capture(lambda b: call(*vb[b]), nb)
+            n = max(10, min(steps, 200))
+            for i in range(min(warmup, 20)):
+                vgraphs[i % nb].replay()
             torch.cuda.synchronize()
             v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             v0.record()
             for i in range(n):
-                vgraphs[i % len(vgraphs)].replay()
+                vgraphs[i % nb].replay()
             v1.record()
             torch.cuda.synchronize()
             del vgraphs
@@ -694,17 +781,15 @@ def main():
 
         t_none = timed_variant(lambda ab: torch.full_like(ab, -1))
         t_same = timed_variant(lambda ab: torch.zeros_like(ab)) if L > 0 else None
-        t_main = ms_max / args.steps
-        secondary = {
-            "lora_overhead_ms_per_step": t_main - t_none, "base_only_ms_per_step": t_none,
-            "same_adapter_ms_per_step": t_same, "distinct_adapters_ms_per_step": t_main,
+        out["secondary"] = {
+            "lora_overhead_ms_per_step": step_ms - t_none, "base_only_ms_per_step": t_none,
+            "same_adapter_ms_per_step": t_same, "distinct_adapters_ms_per_step": step_ms,
             "adapters": f"{shape.adapter_dist} over L={L}",
-            "swap_ab": "not measured: only the swapped (weights in the 128-row MMA M slot) tile exists; "
-                       "a non-swapped tile would put <= 64 tokens per expert in M = 128",
+            "swap_ab": "not measured: only the swapped (weights in the 128-row MMA M slot) tile exists",
         }
 
     # ---- e2e: pinned host inputs -> device, route + forward, y -> pinned host, every step
-    e2e_steps = args.e2e_steps or args.steps
+    e2e_steps = args.e2e_steps or steps
     hx = [b[0].cpu().pin_memory() for b in batches]
     ha = [b[1].cpu().pin_memory() for b in batches]
     hy = torch.empty((M, shape.H), dtype=torch.bfloat16).pin_memory()
@@ -714,97 +799,133 @@ def main():
     def e2e_step(j):
         dx.copy_(hx[j], non_blocking=True)
         da.copy_(ha[j], non_blocking=True)
-        rt = ml.route(da, k, L, x=dx, w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
-        ml.forward(dx, rt, W, k=k, L=L, y=y, workspace=fws)
+        call(dx, da)
         hy.copy_(y, non_blocking=True)
 
-    e2e_graphs = []
-    if not args.no_graph:
-        for j in range(len(batches)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                e2e_step(j)
-            e2e_graphs.append(g)
+    e2e_graphs = capture(e2e_step, nb) if not args.no_graph else []
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(e2e_steps):
-        j = i % len(batches)
-        if e2e_graphs:
-            e2e_graphs[j].replay()
-        else:
-            e2e_step(j)
+        e2e_graphs[i % nb].replay() if e2e_graphs else e2e_step(i % nb)
     e1.record()
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * M * e2e_steps / (e2e_ms / 1e3)
     del graphs, e2e_graphs
     ml.check_status(fws)
     ml.check_status(rws)
+    out["e2e"] = {"value": world * M * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                  "h2d_bytes_per_step": M * shape.H * 2 + M * 4, "d2h_bytes_per_step": M * shape.H * 2,
+                  "how": "graph replay of H2D copy, route, forward, D2H copy" if not args.no_graph
+                  else "plain API calls"}
+    return out
 
-    # ---- roofline of the dominant kernel (gate_up GEMM) and of the whole layer
-    peaks, peak_src = load_peaks()
-    n_b = len(batches)
-    mean = lambda f: float(np.mean([f(*stats[i % n_b]) for i in range(args.steps)]))  # noqa: E731
-    gu_bytes = mean(lambda e, p: gateup_alg_bytes(shape, M, e, p))
-    lay_bytes = mean(lambda e, p: layer_alg_bytes(shape, M, e, p))
-    gu_avg_s = (gu_ms / max(gu_n, 1)) / 1e3
-    tensor_bound = M * k >= 128 * shape.E  # >= 128 rows per expert: the MMA, not HBM, bounds gate_up
-    if tensor_bound:
-        achieved = gateup_alg_flops(shape, M) / gu_avg_s / 1e12
-        peak_t = float(peaks["bf16_tflops_sustained"]) * (2.0 if shape.wdtype == "e4m3" else 1.0)
+
+def sweep_steps(est_ms: float, seconds: float) -> int:
+    return int(min(4000, max(20, seconds * 1e3 / max(est_ms, 1e-3))))
+
+
+def run_sweep(args, world, local, skip: str) -> list:
+    """The decode layers (and the dense decode projection) measured in the same process:
+    tokens/s, the layer's fraction of the HBM copy peak and the gate_up GEMM's roofline,
+    per workload and token count.  Weights are drawn on the device (seeded)."""
+    dev = torch.device("cuda", local)
+    res = []
+    for name, Ms in SWEEP:
+        shape = synth.WORKLOADS[name]
+        if isinstance(shape, synth.DenseShape):
+            if name == skip:
+                continue
+            est = measure_dense(args, shape, world, local, steps=20, warmup=3, full=False)
+            n = sweep_steps(est["ms_per_step"], args.sweep_seconds)
+            m = measure_dense(args, shape, world, local, steps=n, warmup=10, full=False)
+            res.append({"workload": name, "M": shape.T, "tokens_per_s": m["value"], "ms_per_step": m["ms_per_step"],
+                        "steps": n, "layer_frac_of_hbm_peak": m["layer"]["frac_of_hbm_peak"],
+                        "gemm": {kk: m["roofline"][kk] for kk in ("bound", "achieved", "unit", "frac")},
+                        "kernel_ms_per_step": m["layer"]["kernel_ms_per_step"], "gpu_launches": m["gpu_launches"]})
+            continue
+        W = synth.moe_weights_device(shape, dev)
+        for M in Ms:
+            if name == skip and M == args.M:
+                continue
+            est = measure_moe(args, shape, M, W, world, local, steps=10, warmup=3, full=False)
+            n = sweep_steps(est["ms_per_step"], args.sweep_seconds)
+            m = measure_moe(args, shape, M, W, world, local, steps=n, warmup=10, full=False)
+            res.append({"workload": name, "M": M, "tokens_per_s": m["value"], "ms_per_step": m["ms_per_step"],
+                        "steps": n, "layer_frac_of_hbm_peak": m["layer"]["frac_of_hbm_peak"],
+                        "gate_up": {kk: m["roofline"][kk] for kk in ("bound", "achieved", "unit", "frac")},
+                        "kernel_ms_per_step": m["layer"]["kernel_ms_per_step"], "gpu_launches": m["gpu_launches"]})
+        del W
+        torch.cuda.empty_cache()
+    return res
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    import moe_lora_b200  # noqa: F401  (fails loudly without the CUDA library)
+
+    shape = synth.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic"}
+    if isinstance(shape, synth.MoEShape):
+        M = args.M
+        W = synth.moe_weights_device(shape, dev)
+        m = measure_moe(args, shape, M, W, world, local, steps=args.steps, warmup=args.warmup, full=True)
+        del W
+        torch.cuda.empty_cache()
+        line["dtype"] = "bf16" if shape.wdtype == "bf16" else "e4m3/bf16"
+        line["config"] = {"workload": shape.name, "M": M, "tokens_per_step_per_gpu": M, "E": shape.E, "k": shape.k,
+                          "H": shape.H, "I": shape.I, "L": shape.L, "r": shape.r, "wdtype": shape.wdtype,
+                          "adapters": shape.adapter_dist, "router_bias": shape.bias,
+                          "parallelism": f"replicas x{world}", "l2": m.pop("l2"),
+                          "weights": "expert and adapter weights drawn on the device (seeded); router, bias, "
+                                     "tokens and adapter ids from the seeded slice generator"}
     else:
-        achieved = gu_bytes / gu_avg_s / 1e9
-    peak = float(peaks["hbm_gbs"])
-    traffic = (NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["gemm_tc.cu"] == src_hash("gemm_tc.cu")
-               and NCU_TRAFFIC["workload"] == shape.name and NCU_TRAFFIC["M"] == M else None)
-    step_s = ms_max / 1e3 / args.steps
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if shape.wdtype == "bf16" else "e4m3/bf16",
-        "data": "synthetic",
-        "config": {"workload": shape.name, "M": M, "tokens_per_step_per_gpu": M, "E": shape.E, "k": k,
-                   "H": shape.H, "I": shape.I, "L": L, "r": shape.r, "wdtype": shape.wdtype,
-                   "adapters": shape.adapter_dist, "parallelism": f"replicas x{world}",
-                   "l2": f"no flush: {lay_bytes / 1e9:.2f} GB of weights per step > 126 MB L2; "
-                         f"{n_b} rotating token batches"},
-        "roofline": ({"bound": "hbm", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved, "peak": peak,
-                      "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_src,
-                      "traffic": traffic, "alg_bytes_per_launch": gu_bytes,
-                      "avg_launch_us": gu_avg_s * 1e6} if not tensor_bound else
-                     {"bound": "tensor", "kernel": "gemm_tc (gate_up, tcgen05)", "achieved": achieved,
-                      "peak": peak_t, "unit": "TFLOP/s", "frac": achieved / peak_t,
-                      "peak_source": f"{peak_src} bf16 sustained" + (" x2 (fp8 nominal ratio)"
-                                                                    if shape.wdtype == "e4m3" else ""),
-                      "traffic": traffic, "alg_flops_per_launch": gateup_alg_flops(shape, M),
-                      "alg_bytes_per_launch": gu_bytes, "achieved_GBps": gu_bytes / gu_avg_s / 1e9,
-                      "avg_launch_us": gu_avg_s * 1e6}),
-        "layer": {"alg_bytes_per_step": lay_bytes, "achieved_GBps": lay_bytes / step_s / 1e9,
-                  "frac_of_hbm_peak": lay_bytes / step_s / 1e9 / peak,
-                  "TFLOPs": layer_flops(shape, M) / step_s / 1e12,
-                  "kernel_ms_per_step": {kk: v[0] / prof_steps for kk, v in per_kernel.items()},
-                  "kernel_times": "CUDA events around each launch inside the replayed step graphs"
-                  if not args.no_graph else "CUDA events around each launch of plain API calls"},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": M * shape.H * 2 + M * 4,
-                "d2h_bytes_per_step": M * shape.H * 2,
-                "how": "graph replay of H2D copy, route, forward, D2H copy" if not args.no_graph else "plain API calls"},
-        "timing": {"mode": "CUDA graph replay of the route + forward API calls" if not args.no_graph
-                   else "plain API calls", "plain_api_ms_per_step": plain_ms / args.steps,
-                   "per_step": per_step},
-        "gpu_launches": launches,
-        "clocks": clk,
-    }
-    if secondary is not None:
-        line["secondary"] = secondary
+        M = shape.T
+        m = measure_dense(args, shape, world, local, steps=args.steps, warmup=args.warmup, full=True)
+        line["dtype"] = shape.dtype
+        line["config"] = {"workload": shape.name, "T": shape.T, "h_in": shape.h_in, "h_out": shape.h_out,
+                          "L": shape.L, "r": shape.r, "adapters": shape.adapter_dist,
+                          "parallelism": f"replicas x{world}", "l2": m.pop("l2")}
+    clk = m.pop("clocks", None)
+    per_step = m.pop("timing_per_step", None)
+    plain = m.pop("plain_api_ms_per_step", None)
+    line.update(m)
+    line["steps"] = args.steps
+    line["timing"] = {"mode": "CUDA graph replay of the API calls" if not args.no_graph else "plain API calls",
+                      "plain_api_ms_per_step": plain, "per_step": per_step}
+    line["clocks"] = clk
+    if not args.no_sweep:
+        line["sweep"] = run_sweep(args, world, local, skip=shape.name)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, calls, n, el = oracle_tokens_per_s(shape, M, cpu, seconds=args.cpu_seconds)
-        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"fp64 oracle on batch 0 ({n} tokens), {calls} calls in {el:.1f} s; "
-                                          "touched expert weights decoded to fp64 once before timing"}
+        if isinstance(shape, synth.MoEShape):
+            # a bounded sample: the first tokens of batch 0, sized to about cpu_seconds
+            sl = StoredSlices(shape)
+            tps1, _, _, _ = oracle_tokens_per_s(shape, M, seconds=0.0, max_calls=1, tokens_per_call=1, slices=sl)
+            tok = int(max(1, min(M, 64, args.cpu_seconds / 4.0 * tps1)))
+            tps, calls, n, el = oracle_tokens_per_s(shape, M, seconds=args.cpu_seconds, tokens_per_call=tok,
+                                                    slices=sl)
+            sample = (f"fp64 oracle (route, sort, forward) on the first {n} tokens of batch 0, {calls} calls in "
+                      f"{el:.1f} s; the fp64 conversion of the touched stored-precision slices is timed, "
+                      "their generation is not")
+        else:
+            tps, calls, n, el = dense_oracle_tokens_per_s(shape, args.cpu_seconds)
+            sample = (f"fp64 oracle, {n} tokens per call, {calls} calls in {el:.1f} s; "
+                      "weights decoded to fp64 once before timing")
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", **cores_desc(), "kind": "oracle",
+                                "sample": sample}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -95,34 +95,50 @@ constexpr size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
 
+}  // namespace
+
+namespace mlb {
+int current_device_index() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+moe_lora_status check_current_device() {
+  // 0 = not looked up yet, 1 = sm_100a, 2 = another architecture
+  static std::atomic<int> state[kMaxDevices];
+  const int dev = current_device_index();
+  if (dev < 0) return fail(MOE_LORA_ERR_CUDA, "no CUDA device available");
+  int s = state[dev].load(std::memory_order_acquire);
+  if (s == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return fail(MOE_LORA_ERR_CUDA, "cannot query device %d", dev);
+    s = (major == 10 && minor == 0) ? 1 : 2;
+    state[dev].store(s, std::memory_order_release);
+  }
+  if (s == 2) return fail(MOE_LORA_ERR_UNSUPPORTED, "libmoe_lora is built for sm_100a (B200) only");
+  return MOE_LORA_OK;
+}
+}  // namespace mlb
+
+namespace {
+
+// SM count of the current device (cached per device; 148 if it cannot be read).
 int num_sms() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    cudaGetDevice(&dev);
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device_index();
+  if (dev < 0) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  });
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
   return n;
 }
 
-moe_lora_status check_device() {
-  static int ok = -1;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0, major = 0, minor = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-      ok = 0;
-      return;
-    }
-    ok = (major == 10 && minor == 0) ? 1 : 2;
-  });
-  if (ok == 0) return fail(MOE_LORA_ERR_CUDA, "no CUDA device available");
-  if (ok == 2) return fail(MOE_LORA_ERR_UNSUPPORTED, "libmoe_lora is built for sm_100a (B200) only");
-  return MOE_LORA_OK;
-}
+moe_lora_status check_device() { return check_current_device(); }
 
 int env_int(const char* name, int dflt) {
   const char* v = std::getenv(name);

@@ -44,6 +44,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -1084,15 +1085,18 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   if (stages < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = 1024 + static_cast<size_t>(stages) * Cfg::kStageBytes + fixed;
   if (smem > 232448) return cudaErrorInvalidConfiguration;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the raised shared-memory limit is a per-device function attribute
+  static std::atomic<bool> attr_set[kMaxDevices];
+  const int dev = current_device_index();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                232448);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   CUtensorMap tmw, tmb, tml, tmd, tmlb;
   const uint64_t wrows = static_cast<uint64_t>(a.E) * a.rows_per_group;

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/moe_lora.h"
+
 namespace mlb {
 
 struct RouteArgs {
@@ -189,6 +191,14 @@ cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8
 
 // y[t] = sum_j o[t*k + j]  (o already weighted), fixed j order, bf16 out.
 cudaError_t launch_combine(const float* o, int M, int k, int H, __nv_bfloat16* y, cudaStream_t st);
+
+// Host state that CUDA keeps per device (function attributes, SM counts, capability)
+// is cached per device index, for processes that drive several GPUs.
+constexpr int kMaxDevices = 64;
+// The current device's index in [0, kMaxDevices), or -1 when there is none.
+int current_device_index();
+// MOE_LORA_OK on an sm_100a device; the library's status code otherwise (message set).
+moe_lora_status check_current_device();
 
 // driver entry point for tensor map encoding (resolved once)
 bool tensor_map_encode_available();

@@ -11,6 +11,8 @@
 #include "kernels.h"
 #include "prof.h"
 
+#include <atomic>
+
 namespace mlb {
 
 // ---------------------------------------------------------------- router logits
@@ -481,12 +483,15 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
     cudaError_t err = cudaMemsetAsync(a.a_key, 0, sizeof(int32_t) * (n_tb + 1), st);
     if (err != cudaSuccess) return err;
     const size_t smem = route_fused_smem(a.E, a.L, a.M, a.k);
-    static bool attr_set = false;
-    if (!attr_set) {
+    // the raised shared-memory limit is a per-device function attribute
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const int dev = current_device_index();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
       const int most = static_cast<int>(route_fused_smem(256, 64, 1, RF_MAX_PAIRS));  // E = 256, L = 64, caps
       err = cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
       if (err != cudaSuccess) return err;
-      attr_set = true;
+      attr_set[dev].store(true, std::memory_order_release);
     }
     if (a.logits_in != nullptr && a.logits_out != nullptr) {
       err = cudaMemcpyAsync(a.logits_out, a.logits_in, sizeof(float) * a.M * a.E, cudaMemcpyDeviceToDevice, st);

@@ -36,7 +36,7 @@ constexpr size_t kScratchBytes = mlb::kStatusBytes + kCountBytes + kKeyBytes + k
 // the symbol: its device address comes from cudaGetSymbolAddress (below).
 __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
+using mlb::kMaxDevices;
 void* g_scratch_ptr[kMaxDevices] = {};
 std::mutex g_scratch_mutex;
 
@@ -93,6 +93,9 @@ extern "C" MOE_LORA_API moe_lora_status moe_lora_route_noalloc(
     }
     if (logits_out != nullptr && !al16(logits_out)) return noalloc_fail(MOE_LORA_ERR_INVALID_ARG, "logits_out misaligned");
   }
+  // the same answer as moe_lora_route on a device that is not sm_100a (or no device)
+  const moe_lora_status dst = mlb::check_current_device();
+  if (dst != MOE_LORA_OK) return dst;
   unsigned char* base = nullptr;
   if (scratch_for_current_device(&base) != cudaSuccess)
     return noalloc_fail(MOE_LORA_ERR_CUDA, "cudaGetSymbolAddress of the scratch array failed");

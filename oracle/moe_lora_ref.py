@@ -158,14 +158,6 @@ def moe_lora_forward(x: np.ndarray, topk_ids: np.ndarray, topk_w: np.ndarray,
 
 # ----------------------------------------------------------------------------- SGMV
 
-def segment_adapter_per_token(seg_offsets: np.ndarray, seg_adapter: np.ndarray, T: int) -> np.ndarray:
-    """Adapter id of every token from contiguous segments [off[s], off[s+1]); -1 if none."""
-    a = np.full(T, -1, dtype=np.int64)
-    for s in range(len(seg_adapter)):
-        a[int(seg_offsets[s]):int(seg_offsets[s + 1])] = int(seg_adapter[s])
-    return a
-
-
 def sgmv_shrink(x: np.ndarray, lora_a: np.ndarray, seg_offsets, seg_adapter) -> np.ndarray:
     """z_t = x_t A_a(t)^T per segment (segmented gather, [Punica review page], "提案手法");
     rows of segments with adapter -1 are zero."""

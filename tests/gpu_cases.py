@@ -15,13 +15,19 @@ from workloads import synth
 
 TOL_BF16 = 2e-2   # max|err| <= TOL * max|ref| for bf16 expert weights
 TOL_FP8 = 6e-2    # ... for e4m3 expert weights
+# The e4m3-weight GEMM splits each bf16 activation row exactly into two e4m3 planes
+# (hi and a residual plane at 1/16 of the scale), which carries every activation to a
+# relative 2^-8.  The forward error of that design is then of the size of the bf16
+# path's (act and y rounded to bf16), well inside this bound; a kernel that dropped the
+# residual plane (activations at e4m3 precision, ~2^-4 relative) lands above it.
+FP8_DESIGN_BOUND = 1e-2
 
 
 class CpuWeightsOracle(MoEOracleWeights):
     """Oracle view backed by the generator's CPU tensors (no regeneration)."""
 
-    def __init__(self, shape: synth.MoEShape, cpu: dict):
-        super().__init__(shape, cache=True)
+    def __init__(self, shape: synth.MoEShape, cpu: dict, cache: bool = True):
+        super().__init__(shape, cache=cache)
         self.cpu = cpu
 
     def _expert(self, e):

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import moe_lora_b200 as ml
-from tests.gpu_cases import TOL_BF16, TOL_FP8, moe_weights_both, run_moe_case
+from tests.gpu_cases import FP8_DESIGN_BOUND, TOL_BF16, TOL_FP8, CpuWeightsOracle, moe_weights_both, run_moe_case
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
@@ -126,16 +126,30 @@ def prefill_weights():
     return moe_weights_both(synth.MOE_PREFILL_BF16)
 
 
-def test_forward_moe_prefill_bf16_full_sampled(prefill_weights):
-    M = 4096
-    toks = np.unique(np.concatenate([np.arange(8), np.arange(M - 8, M),
-                                     np.random.default_rng(1).choice(M, 48, replace=False)]))
-    res = run_moe_case(synth.MOE_PREFILL_BF16, M, weights=prefill_weights, tokens=toks)
+def test_forward_moe_prefill_bf16_full(prefill_weights):
+    """All 4096 tokens of the prefill layer against the oracle: every expert's ragged
+    last 256-row chunk and every (expert, adapter) segment boundary is checked.  The
+    oracle view decodes one expert (and its adapters) at a time, so the fp64 weights
+    are never all resident."""
+    cpu, dev, _ = prefill_weights
+    s = synth.MOE_PREFILL_BF16
+    res = run_moe_case(s, 4096, weights=(cpu, dev, CpuWeightsOracle(s, cpu, cache=False)))
+    print(f"prefill M=4096: max|err|/max|ref| = {res['err']:.3e} over {len(res['tokens'])} tokens")
+    assert len(res["tokens"]) == 4096
     assert res["err"] <= TOL_BF16, res["err"]
     ml.check_status(res["rt"]["workspace"])
 
 
 # ---------------------------------------------------------------- FP8 (e4m3) expert weights
+def check_fp8(res, label, record_property):
+    """The stated FP8 gate and the tighter bound of the two-plane activation design;
+    the achieved error is printed and recorded for every case."""
+    print(f"fp8 {label}: max|err|/max|ref| = {res['err']:.3e}")
+    record_property("fp8_rel_err", res["err"])
+    assert res["err"] <= TOL_FP8, res["err"]
+    assert res["err"] <= FP8_DESIGN_BOUND, res["err"]
+
+
 SMALL_FP8 = [
     synth.MoEShape("f8_a", 220, E=8, k=2, H=384, I=192, L=3, r=16, wdtype="e4m3", no_adapter_frac=0.2),
     synth.MoEShape("f8_ragged", 221, E=6, k=3, H=528, I=144, L=2, r=32, wdtype="e4m3", bias=True,
@@ -146,18 +160,16 @@ SMALL_FP8 = [
 
 @pytest.mark.parametrize("shape", SMALL_FP8, ids=lambda s: s.name)
 @pytest.mark.parametrize("M", [1, 5, 37, 200])
-def test_forward_fp8_small_shapes(shape, M):
-    res = run_moe_case(shape, M)
-    assert res["err"] <= TOL_FP8, res["err"]
+def test_forward_fp8_small_shapes(shape, M, record_property):
+    check_fp8(run_moe_case(shape, M), f"{shape.name} M={M}", record_property)
 
 
 @pytest.mark.parametrize("where", ["gemm", "delta"])
 @pytest.mark.parametrize("bn", [16, 32, 64, 256])
-def test_forward_fp8_every_n_tile(bn, where, monkeypatch):
+def test_forward_fp8_every_n_tile(bn, where, monkeypatch, record_property):
     monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
-    res = run_moe_case(SMALL_FP8[1], 150)
-    assert res["err"] <= TOL_FP8, res["err"]
+    check_fp8(run_moe_case(SMALL_FP8[1], 150), f"{SMALL_FP8[1].name} bn={bn} {where}", record_property)
 
 
 @pytest.fixture(scope="module")
@@ -166,7 +178,7 @@ def fp8_weights():
 
 
 @pytest.mark.parametrize("M", [1, 4, 16, 64])
-def test_forward_moe_decode_fp8_full(fp8_weights, M):
+def test_forward_moe_decode_fp8_full(fp8_weights, M, record_property):
     res = run_moe_case(synth.MOE_DECODE_FP8, M, weights=fp8_weights)
-    assert res["err"] <= TOL_FP8, res["err"]
+    check_fp8(res, f"{synth.MOE_DECODE_FP8.name} M={M}", record_property)
     ml.check_status(res["rt"]["workspace"])

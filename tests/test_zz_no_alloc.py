@@ -79,6 +79,21 @@ def test_noalloc_route_matches_workspace_route_two_calls_in_a_row():
     _same(got3, ref1)
 
 
+def test_noalloc_route_largest_scratch_case():
+    """The limits themselves: M = 1024, E = 256, k = 8, L = 64, logits computed from x on
+    the tensor cores into the scratch (M * E fp32 values, the largest region), twice."""
+    s = synth.MoEShape("noalloc_max", 230, E=256, k=8, H=512, I=64, L=64, r=16, bias=True)
+    x, a = synth.moe_tokens(s, 1024)
+    wr, b = synth.moe_router(s)
+    x, a, wr, b = x.cuda(), a.cuda(), wr.cuda(), b.cuda()
+    a[::5] = -1
+    ref = ml.route(a, s.k, s.L, x=x, w_router=wr, bias=b)
+    for _ in range(2):
+        got = _call_noalloc(a, s.k, s.L, s.E, x=x, w_router=wr, bias=b)
+        torch.cuda.synchronize()
+        _same(got, ref)
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     f = _fn()
     fake = 0x7F0000000000
@@ -86,4 +101,8 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert st == ml.ERR_UNSUPPORTED
     assert b"M <= 1024" in ml.lib().moe_lora_last_error()
     st = f(None, None, None, fake, fake, 16, 0, 257, 8, 8, None, fake, fake, fake, fake, None)
+    assert st == ml.ERR_UNSUPPORTED
+    st = f(None, None, None, fake, fake, 16, 0, 8, 9, 8, None, fake, fake, fake, fake, None)  # k > E
+    assert st == ml.ERR_UNSUPPORTED
+    st = f(None, None, None, fake, fake, 16, 0, 64, 8, 65, None, fake, fake, fake, fake, None)  # L = 65
     assert st == ml.ERR_UNSUPPORTED

@@ -230,6 +230,44 @@ def moe_weights(s: MoEShape, device="cpu") -> dict:
     return out
 
 
+def moe_weights_device(s: MoEShape, device, seed: int = 0) -> dict:
+    """The same layout and distributions as moe_weights, drawn on the device by torch's
+    seeded generator (one stream per workload and seed) instead of the per-slice numpy
+    streams: gigabytes in well under a second, for timing runs whose results are not
+    compared with the oracle.  The router weight and bias come from the numpy streams
+    (moe_router), so routing of a given token batch is the same as with moe_weights."""
+    g = torch.Generator(device=device)
+    g.manual_seed(BASE_SEED * 1000 + s.wid * 10 + seed)
+    wdt = torch.bfloat16 if s.wdtype == "bf16" else torch.float8_e4m3fn
+
+    def draw(shape, var):
+        return torch.randn(shape, generator=g, device=device, dtype=torch.float32).mul_(float(np.sqrt(var)))
+
+    out = {"w_gu": torch.empty((s.E, 2 * s.I, s.H), dtype=wdt, device=device),
+           "w_d": torch.empty((s.E, s.H, s.I), dtype=wdt, device=device),
+           "scales": torch.ones((s.E, 2), dtype=torch.float32, device=device)}
+    for e in range(s.E):
+        for name, shape, var, col in (("w_gu", (2 * s.I, s.H), 1.0 / s.H, 0), ("w_d", (s.H, s.I), 1.0 / s.I, 1)):
+            w = draw(shape, var)
+            if s.wdtype == "bf16":
+                out[name][e].copy_(w)
+            else:  # per-tensor e4m3: scale = amax / 448, code = RNE(w / scale)
+                amax = float(w.abs().max())
+                sc = np.float32(amax / 448.0) if amax > 0 else np.float32(1.0)
+                out[name][e].copy_((w / torch.tensor(sc, dtype=torch.float32, device=device)).to(wdt))
+                out["scales"][e, col] = float(sc)
+    for name, cols, var in (("a_gu", s.H, 1.0 / s.H), ("b_gu", 2 * s.I, 1.0 / s.r),
+                            ("a_d", s.I, 1.0 / s.I), ("b_d", s.H, 1.0 / s.r)):
+        t = torch.empty((s.L, s.E, s.r, cols), dtype=torch.bfloat16, device=device)
+        for a in range(s.L):
+            t[a].copy_(draw((s.E, s.r, cols), var))
+        out[name] = t
+    wr, bias = moe_router(s)
+    out["w_router"] = wr.to(device)
+    out["bias"] = None if bias is None else bias.to(device)
+    return out
+
+
 # ----------------------------------------------------------------------------- dense slices
 
 def dense_tokens(s: DenseShape, T: int | None = None):
