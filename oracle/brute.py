@@ -92,9 +92,12 @@ def silu(g: float) -> float:
     return g / (1.0 + math.exp(-g))
 
 
-def moe_layer(x, ids, ws, adapters, I, experts, lora):
+def moe_layer(x, ids, ws, adapters, I, experts, lora, split=False, scale_gu=1.0, scale_d=1.0):
     """experts[e] = (w_gu rows [2I][H], w_d rows [H][I], s_gu, s_d);
-    lora[(a, e)] = (A_gu [r][H], B_gu [r][2I], A_d [r][I], B_d [r][H]); all floats."""
+    lora[(a, e)] = (A_gu [r][H], B_gu [r][2I], A_d [r][I], B_d [r][H]); all floats.
+    split: A_gu = (A_gate [r][H], A_up [r][H]) and B_gu = (B_gate [r][I], B_up [r][I]),
+    each feature of the gate half taking its delta from the gate adapter, the up half
+    from the up adapter.  scale_gu / scale_d multiply each projection's delta."""
     H = len(x[0])
     y = []
     for t, xt in enumerate(x):
@@ -105,14 +108,17 @@ def moe_layer(x, ids, ws, adapters, I, experts, lora):
             h = [s_gu * v for v in matvec(w_gu, xt)]
             if a >= 0:
                 ag, bg, _, _ = lora[(a, e)]
-                d = vecmat_t(matvec(ag, xt), bg)
-                h = [u + v for u, v in zip(h, d)]
+                if split:
+                    d = vecmat_t(matvec(ag[0], xt), bg[0]) + vecmat_t(matvec(ag[1], xt), bg[1])
+                else:
+                    d = vecmat_t(matvec(ag, xt), bg)
+                h = [u + scale_gu * v for u, v in zip(h, d)]
             act = [silu(h[i]) * h[I + i] for i in range(I)]
             o = [s_d * v for v in matvec(w_d, act)]
             if a >= 0:
                 _, _, ad, bd = lora[(a, e)]
                 d = vecmat_t(matvec(ad, act), bd)
-                o = [u + v for u, v in zip(o, d)]
+                o = [u + scale_d * v for u, v in zip(o, d)]
             for n in range(H):
                 acc[n] += ws[t][j] * o[n]
         y.append(acc)

@@ -108,35 +108,52 @@ def swiglu(h: np.ndarray, I: int) -> np.ndarray:
     return silu(h[:, :I]) * h[:, I:]
 
 
+def gate_up_lora_delta(v: np.ndarray, a_gu: np.ndarray, b_gu: np.ndarray, I: int) -> np.ndarray:
+    """The gate_up adapter delta [n, 2I] in either layout.
+
+    Fused (a_gu [r, H], b_gu [r, 2I]): one adapter on the fused projection.  Split
+    (a_gu [2, r, H], b_gu [2, r, I]): the gate and the up projection each carry their own
+    adapter, as every projection does on the vLLM MoE-LoRA page ("O Papel da
+    Multi-LoRA": one A and one B per projection): gate columns (v A_g) B_g, up columns
+    (v A_u) B_u."""
+    if a_gu.ndim == 2:
+        return lora_delta(v, a_gu, b_gu)
+    return np.concatenate([lora_delta(v, a_gu[0], b_gu[0]), lora_delta(v, a_gu[1], b_gu[1])], axis=1)
+
+
 def expert_ffn(xe: np.ndarray, adapters: np.ndarray, I: int, w_gu: np.ndarray, w_d: np.ndarray,
-               s_gu: float, s_d: float, get_adapter) -> np.ndarray:
+               s_gu: float, s_d: float, get_adapter, scale_gu: float = 1.0, scale_d: float = 1.0) -> np.ndarray:
     """One expert on its gathered rows xe [n, H] with per-row adapter id (-1 = none).
 
     gate_up expands H -> 2I, the gate is applied, down compresses I -> H
     ([vLLM MoE-LoRA page], "Entendendo os Modelos MoE"); each projection adds the
     row's own adapter delta, y = xW + xAB ("O Papel da Multi-LoRA"), with adapters
-    owned per (adapter, expert) ("these operations per expert, per adapter")."""
+    owned per (adapter, expert) ("these operations per expert, per adapter").
+    scale_gu / scale_d multiply each projection's delta (an alpha / r factor; 1 = the
+    page's y = xW + xAB)."""
     h = s_gu * (xe @ w_gu.T)
     present = sorted(set(int(a) for a in adapters if a >= 0))
     lw = {a: get_adapter(a) for a in present}
     for a in present:
         rows = np.nonzero(adapters == a)[0]
-        h[rows] += lora_delta(xe[rows], lw[a][0], lw[a][1])
+        h[rows] += scale_gu * gate_up_lora_delta(xe[rows], lw[a][0], lw[a][1], I)
     act = swiglu(h, I)
     o = s_d * (act @ w_d.T)
     for a in present:
         rows = np.nonzero(adapters == a)[0]
-        o[rows] += lora_delta(act[rows], lw[a][2], lw[a][3])
+        o[rows] += scale_d * lora_delta(act[rows], lw[a][2], lw[a][3])
     return o
 
 
 def moe_lora_forward(x: np.ndarray, topk_ids: np.ndarray, topk_w: np.ndarray,
                      adapter_ids: np.ndarray, I: int, get_expert, get_adapter,
-                     tokens: np.ndarray | None = None) -> np.ndarray:
+                     tokens: np.ndarray | None = None, scale_gu: float = 1.0,
+                     scale_d: float = 1.0) -> np.ndarray:
     """y [M, H] (or only the rows listed in ``tokens``) in fp64.
 
     get_expert(e) -> (W_gu [2I,H], W_d [H,I], s_gu, s_d) widened to fp64;
-    get_adapter(a, e) -> (A_gu [r,H], B_gu [r,2I], A_d [r,I], B_d [r,H]) fp64.
+    get_adapter(a, e) -> (A_gu [r,H], B_gu [r,2I], A_d [r,I], B_d [r,H]) fp64, or with
+    separate gate and up adapters A_gu [2,r,H], B_gu [2,r,I] (gate_up_lora_delta).
     The selected experts' outputs are summed with the routing weights
     ([vLLM MoE-LoRA page], "Entendendo os Modelos MoE": outputs are aggregated)."""
     M, H = x.shape
@@ -151,7 +168,7 @@ def moe_lora_forward(x: np.ndarray, topk_ids: np.ndarray, topk_w: np.ndarray,
         t = t_of[sel]
         w_gu, w_d, s_gu, s_d = get_expert(int(e))
         o = expert_ffn(x[t], adapter_ids[t], I, w_gu, w_d, s_gu, s_d,
-                       lambda a, e=int(e): get_adapter(a, e))
+                       lambda a, e=int(e): get_adapter(a, e), scale_gu, scale_d)
         y[sel // k] += topk_w[t, j_of[sel]][:, None] * o
     return y
 

@@ -119,3 +119,54 @@ def test_weights_sum_to_one_on_workload_router():
     wr, bias = W.router()
     _, w = ref.route_topk(ref.router_logits(x64, wr, bias), s.k)
     np.testing.assert_allclose(w.sum(1), 1.0, atol=1e-15)
+
+
+# ---------------------------------------------------------------- separate gate / up adapters
+SPLIT = TINY.with_(name="tiny_split", wid=130, gu_split=True)
+
+
+def test_split_gate_up_matches_brute_loops_with_scales():
+    """Separate gate and up adapters and per-projection scales against scalar loops."""
+    M = 7
+    W, x64, ad, ids, w = _route(SPLIT, M)
+    ag, bg, _, _ = W.adapter(0, 0)
+    assert ag.shape == (2, SPLIT.r, SPLIT.H) and bg.shape == (2, SPLIT.r, SPLIT.I)
+    y = ref.moe_lora_forward(x64, ids, w, ad, SPLIT.I, W.expert, W.adapter, scale_gu=0.5, scale_d=2.0)
+    experts, lora = _brute_inputs(SPLIT, W)
+    yb = brute.moe_layer(x64.tolist(), ids.tolist(), w.tolist(), ad.tolist(), SPLIT.I, experts, lora,
+                         split=True, scale_gu=0.5, scale_d=2.0)
+    np.testing.assert_allclose(y, np.array(yb), rtol=1e-12, atol=1e-12)
+
+
+def test_split_gate_up_is_fused_rank_2r_with_block_diagonal_b():
+    """Two adapters on the gate and up halves equal one fused adapter of rank 2r whose A
+    stacks A_gate over A_up and whose B is block-diagonal (B_gate on the gate columns, B_up
+    on the up columns) -- a different computation path through the fused layout."""
+    M = 7
+    W, x64, ad, ids, w = _route(SPLIT, M)
+    I, r = SPLIT.I, SPLIT.r
+
+    def fused(a, e):
+        ag, bg, a_d, b_d = W.adapter(a, e)
+        bf = np.zeros((2 * r, 2 * I))
+        bf[:r, :I] = bg[0]
+        bf[r:, I:] = bg[1]
+        return np.concatenate([ag[0], ag[1]], axis=0), bf, a_d, b_d
+
+    ys = ref.moe_lora_forward(x64, ids, w, ad, I, W.expert, W.adapter)
+    yf = ref.moe_lora_forward(x64, ids, w, ad, I, W.expert, fused)
+    np.testing.assert_allclose(ys, yf, rtol=1e-12, atol=1e-13)
+
+
+def test_scale_equals_b_scaled():
+    """A projection's scale multiplies its delta: the same as scaling that projection's B."""
+    M = 7
+    W, x64, ad, ids, w = _route(TINY, M)
+
+    def scaled_b(a, e):
+        ag, bg, a_d, b_d = W.adapter(a, e)
+        return ag, 0.25 * bg, a_d, -3.0 * b_d
+
+    y1 = ref.moe_lora_forward(x64, ids, w, ad, TINY.I, W.expert, W.adapter, scale_gu=0.25, scale_d=-3.0)
+    y2 = ref.moe_lora_forward(x64, ids, w, ad, TINY.I, W.expert, scaled_b)
+    np.testing.assert_allclose(y1, y2, rtol=1e-12, atol=1e-13)

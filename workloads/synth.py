@@ -53,6 +53,7 @@ class MoEShape:
     adapter_dist: str = "uniform"  # "uniform" or "zipf"
     M_list: tuple = (64,)
     no_adapter_frac: float = 0.0  # share of tokens with adapter id -1 (base only)
+    gu_split: bool = False        # separate gate and up adapters (A [2][r][H], B [2][r][I])
 
     def with_(self, **kw) -> "MoEShape":
         return replace(self, **kw)
@@ -182,11 +183,16 @@ def moe_expert(s: MoEShape, e: int):
 
 
 def moe_adapter(s: MoEShape, a: int, e: int):
-    """Adapter a on expert e, bf16: A_gu [r, H], B_gu [r, 2I], A_d [r, I], B_d [r, H].
+    """Adapter a on expert e, bf16: A_gu [r, H], B_gu [r, 2I], A_d [r, I], B_d [r, H]; with
+    separate gate and up adapters (gu_split) A_gu [2, r, H] and B_gu [2, r, I] (gate, up).
 
     A is stored transposed (r rows, each contiguous over h_in); B as r rows over h_out."""
-    ag = to_bf16(normal_f32(rng(s.wid, T_AGU, a, e), (s.r, s.H), 1.0 / s.H))
-    bg = to_bf16(normal_f32(rng(s.wid, T_BGU, a, e), (s.r, 2 * s.I), 1.0 / s.r))
+    if s.gu_split:
+        ag = to_bf16(normal_f32(rng(s.wid, T_AGU, a, e), (2, s.r, s.H), 1.0 / s.H))
+        bg = to_bf16(normal_f32(rng(s.wid, T_BGU, a, e), (2, s.r, s.I), 1.0 / s.r))
+    else:
+        ag = to_bf16(normal_f32(rng(s.wid, T_AGU, a, e), (s.r, s.H), 1.0 / s.H))
+        bg = to_bf16(normal_f32(rng(s.wid, T_BGU, a, e), (s.r, 2 * s.I), 1.0 / s.r))
     ad = to_bf16(normal_f32(rng(s.wid, T_AD, a, e), (s.r, s.I), 1.0 / s.I))
     bd = to_bf16(normal_f32(rng(s.wid, T_BD, a, e), (s.r, s.H), 1.0 / s.r))
     return ag, bg, ad, bd
@@ -206,8 +212,10 @@ def moe_weights(s: MoEShape, device="cpu") -> dict:
         "w_gu": torch.empty((s.E, 2 * s.I, s.H), dtype=wdt, device=device),
         "w_d": torch.empty((s.E, s.H, s.I), dtype=wdt, device=device),
         "scales": torch.ones((s.E, 2), dtype=torch.float32),
-        "a_gu": torch.empty((s.L, s.E, s.r, s.H), dtype=torch.bfloat16, device=device),
-        "b_gu": torch.empty((s.L, s.E, s.r, 2 * s.I), dtype=torch.bfloat16, device=device),
+        "a_gu": torch.empty((s.L, s.E, 2, s.r, s.H) if s.gu_split else (s.L, s.E, s.r, s.H),
+                            dtype=torch.bfloat16, device=device),
+        "b_gu": torch.empty((s.L, s.E, 2, s.r, s.I) if s.gu_split else (s.L, s.E, s.r, 2 * s.I),
+                            dtype=torch.bfloat16, device=device),
         "a_d": torch.empty((s.L, s.E, s.r, s.I), dtype=torch.bfloat16, device=device),
         "b_d": torch.empty((s.L, s.E, s.r, s.H), dtype=torch.bfloat16, device=device),
     }
@@ -256,11 +264,13 @@ def moe_weights_device(s: MoEShape, device, seed: int = 0) -> dict:
                 sc = np.float32(amax / 448.0) if amax > 0 else np.float32(1.0)
                 out[name][e].copy_((w / torch.tensor(sc, dtype=torch.float32, device=device)).to(wdt))
                 out["scales"][e, col] = float(sc)
-    for name, cols, var in (("a_gu", s.H, 1.0 / s.H), ("b_gu", 2 * s.I, 1.0 / s.r),
-                            ("a_d", s.I, 1.0 / s.I), ("b_d", s.H, 1.0 / s.r)):
-        t = torch.empty((s.L, s.E, s.r, cols), dtype=torch.bfloat16, device=device)
+    sp = (2,) if s.gu_split else ()
+    for name, lead, cols, var in (("a_gu", sp, s.H, 1.0 / s.H),
+                                  ("b_gu", sp, s.I if s.gu_split else 2 * s.I, 1.0 / s.r),
+                                  ("a_d", (), s.I, 1.0 / s.I), ("b_d", (), s.H, 1.0 / s.r)):
+        t = torch.empty((s.L, s.E, *lead, s.r, cols), dtype=torch.bfloat16, device=device)
         for a in range(s.L):
-            t[a].copy_(draw((s.E, s.r, cols), var))
+            t[a].copy_(draw((s.E, *lead, s.r, cols), var))
         out[name] = t
     wr, bias = moe_router(s)
     out["w_router"] = wr.to(device)
