@@ -213,33 +213,36 @@ def routing_stats(rt: dict, shape: synth.MoEShape):
     return experts, pairs
 
 
-def expand_in_gemm(shape, M) -> bool:
-    """The library's placement rule for the LoRA expand (inside the GEMM above 64 rows
-    per expert, else the LoRA kernel's fp32 delta)."""
-    return M * shape.k > 64 * shape.E
+def lora_place(shape, M) -> str:
+    """The library's placement of the LoRA work of the grouped GEMMs (MOE_LORA_EXPAND
+    overrides): "tc" above 64 rows per expert (the tensor-core LoRA kernel writes bf16
+    deltas: gate_up's is added by the GEMM epilogue, down's by the combine), else "delta"
+    (the SIMT LoRA kernel's fp32 deltas)."""
+    v = os.environ.get("MOE_LORA_EXPAND")
+    if v in ("delta", "tc"):
+        return v
+    return "tc" if M * shape.k > 64 * shape.E else "delta"
 
 
 def gateup_alg_bytes(shape, M, experts, pairs):
     """Bytes the gate_up GEMM must move once: touched expert gate_up weights, the
     gathered x rows (bf16, or two e4m3 planes and their scales), its LoRA input (the
-    fp32 delta, or the z rows and touched B_gu slices when it runs the expand), and the
-    act it writes."""
+    fp32 or bf16 delta) and the act it writes."""
     wb = 1 if shape.wdtype == "e4m3" else 2
     mk = M * shape.k
     xb = mk * (2 * shape.H + 8) if shape.wdtype == "e4m3" else mk * shape.H * 2
     if shape.L == 0:
         lora = 0
-    elif expand_in_gemm(shape, M):
-        lora = mk * shape.r * 2 + pairs * shape.r * 2 * shape.I * 2
+    elif lora_place(shape, M) == "tc":
+        lora = mk * 2 * shape.I * 2
     else:
         lora = mk * 2 * shape.I * 4
     return experts * 2 * shape.I * shape.H * wb + xb + lora + mk * shape.I * 2
 
 
 def gateup_alg_flops(shape, M):
-    """gate_up base GEMM plus its fused LoRA expand."""
-    mk = M * shape.k
-    return 2 * mk * 2 * shape.I * shape.H + 2 * mk * shape.r * 2 * shape.I
+    """The gate_up base GEMM (its LoRA expand runs in the LoRA kernels)."""
+    return 2 * M * shape.k * 2 * shape.I * shape.H
 
 
 def layer_alg_bytes(shape, M, experts, pairs):
@@ -447,13 +450,15 @@ def measure_dense(args, shape: synth.DenseShape, world, local, *, steps, warmup,
     torch.cuda.synchronize()
     launches_per_step = (ml.launch_count() - n0) / n_copies
 
-    def capture(fn):
+    def capture(fn, profile=0):
         gs = torch.cuda.Stream()
         gs.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(gs):
             fn(0)
         torch.cuda.current_stream().wait_stream(gs)
         torch.cuda.synchronize()
+        if profile:  # event pairs only around the captured launches, not the warm-up
+            ml.profile_enable(profile)
         out = []
         for c in range(n_copies):
             g = torch.cuda.CUDAGraph()
@@ -465,8 +470,7 @@ def measure_dense(args, shape: synth.DenseShape, world, local, *, steps, warmup,
     # ---- per-kernel device times: event pairs around every launch inside the graphs
     names = ("lora", "shrink", "gemm_dense", "dense_f32")
     if not args.no_graph:
-        ml.profile_enable(n_copies * 4 + 16)
-        pgraphs = capture(step)
+        pgraphs = capture(step, profile=n_copies * 4 + 16)
         for _ in range(3):
             for g in pgraphs:
                 g.replay()
@@ -634,7 +638,7 @@ def measure_moe(args, shape: synth.MoEShape, M: int, W: dict, world, local, *, s
     launches_per_step = (ml.launch_count() - n0) / n_plain
     plain_ms = p0.elapsed_time(p1) / n_plain
 
-    def capture(fn, nb):
+    def capture(fn, nb, profile=0):
         gs = torch.cuda.Stream()
         gs.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(gs):
@@ -642,6 +646,8 @@ def measure_moe(args, shape: synth.MoEShape, M: int, W: dict, world, local, *, s
                 fn(b)  # warm the stream before capture
         torch.cuda.current_stream().wait_stream(gs)
         torch.cuda.synchronize()
+        if profile:  # event pairs only around the captured launches, not the warm-up
+            ml.profile_enable(profile)
         out = []
         for b in range(nb):
             g = torch.cuda.CUDAGraph()
@@ -656,8 +662,7 @@ def measure_moe(args, shape: synth.MoEShape, M: int, W: dict, world, local, *, s
     names = ("route", "router_logits", "topk", "sort", "lora", "quant", "gemm_gateup", "gemm_down", "combine")
     nb = len(batches)
     if not args.no_graph:
-        ml.profile_enable(nb * 24 + 64)
-        pgraphs = capture(step, nb)
+        pgraphs = capture(step, nb, profile=nb * 24 + 64)
         for _ in range(5):
             for g in pgraphs:
                 g.replay()

@@ -33,13 +33,16 @@
  *     reduction dim): expert gate_up w_gu [E][2I][H] with the gate in rows [0, I) and
  *     the up projection in rows [I, 2I); expert down w_d [E][H][I]; dense W [h_out][h_in].
  *     LoRA A is stored transposed as [.. ][r][h_in]; LoRA B as [.. ][r][h_out].
- *   - No alpha/r scaling is applied: y = xW + (xA)B exactly; fold any scale into B.
+ *   - Adapter scaling: y = xW + s (xA)B with s = 1 unless moe_lora_forward's format sets
+ *     a per-projection scale (an alpha / r factor).
  *
  * Environment switches (read at each call; none changes a result beyond rounding order)
- *   MOE_LORA_EXPAND=gemm|delta  where the LoRA expand z B runs: inside the grouped GEMM
- *                               as extra tensor-core K steps, or in the LoRA kernel into an
- *                               fp32 delta the GEMM epilogue adds.  Default: inside the GEMM
- *                               above 64 rows per expert (prefill), the delta below (decode).
+ *   MOE_LORA_EXPAND=delta|tc    where the LoRA work of the grouped GEMMs runs: "delta", the
+ *                               segmented CUDA-core LoRA kernel writes fp32 deltas (decode:
+ *                               gate_up's added by the GEMM epilogue, down's by the
+ *                               combine); "tc", the tensor-core LoRA kernel (shrink and
+ *                               expand on tcgen05, z on chip) writes bf16 deltas (prefill).
+ *                               Default: "tc" above 64 rows per expert, "delta" below.
  *   MOE_LORA_FORCE_BN=16|32|64|128|256  the GEMM's token tile (default: from the mean rows
  *                               per group: <= 12 -> 16, <= 24 -> 32, <= 64 -> 64, <= 96 -> 128,
  *                               else 256).
@@ -128,13 +131,30 @@ MOE_LORA_API moe_lora_status moe_lora_route(
     int32_t* sorted_pairs, int32_t* seg_offsets,
     void* workspace, size_t workspace_bytes, moe_lora_stream stream);
 
+/* Layout and scaling of the adapters given to moe_lora_forward (NULL: the defaults,
+ * which are {0, 1.0f, 1.0f}).  Each projection carries its own adapter on the pages
+ * ([vLLM MoE-LoRA page], "O Papel da Multi-LoRA": one A and one B per projection).
+ *   gate_up_split  0: one adapter on the fused gate_up projection,
+ *                     lora_a_gu [L][E][r][H], lora_b_gu [L][E][r][2I];
+ *                  1: separate gate and up adapters, lora_a_gu [L][E][2][r][H] and
+ *                     lora_b_gu [L][E][2][r][I] (index 0 = gate, 1 = up); needs r <= 64.
+ *   scale_gu       multiplies the gate_up delta (both halves), e.g. alpha / r.
+ *   scale_d        multiplies the down delta. */
+typedef struct {
+  int gate_up_split;
+  float scale_gu;
+  float scale_d;
+} moe_lora_adapter_format;
+
 /* ---------------------------------------------------------------------------------
  * moe_lora_forward -- the MoE FFN with per-(adapter, expert) LoRA on gate_up and
  * down, and the top-k weighted combine.  For every routing pair p = (t, j), with
  * e = topk_ids[t, j] and a = a(t):
- *   h   = s_gu[e] * W_gu[e] x_t + [a >= 0] (x_t A_gu[a,e]) B_gu[a,e]        (2I)
+ *   h   = s_gu[e] * W_gu[e] x_t + [a >= 0] c_gu (x_t A_gu[a,e]) B_gu[a,e]   (2I)
  *   act = silu(h[0:I]) * h[I:2I],  silu(g) = g / (1 + exp(-g))             (I)
- *   o   = s_d[e] * W_d[e] act + [a >= 0] (act A_d[a,e]) B_d[a,e]            (H)
+ *   o   = s_d[e] * W_d[e] act + [a >= 0] c_d (act A_d[a,e]) B_d[a,e]        (H)
+ * (c_gu, c_d: the format's scales; with separate gate and up adapters the gate half of
+ * the gate_up delta is (x_t A_gate) B_gate and the up half (x_t A_up) B_up)
  *   y_t = sum_j topk_w[t, j] * o_(t, j)      (fixed j order: deterministic)
  * Defines: expert gate_up/down ([vLLM MoE-LoRA page], "Entendendo os Modelos MoE"),
  * y = xW + xAB per projection, per expert and per adapter ("O Papel da Multi-LoRA"),
@@ -148,8 +168,9 @@ MOE_LORA_API moe_lora_status moe_lora_route(
  *   w_gateup     [E][2I][H], w_down [E][H][I], of type w_dtype (ML_BF16 or ML_E4M3).
  *   w_scales     fp32 [E][2] = (s_gu, s_d) per expert when w_dtype = ML_E4M3; NULL
  *                for ML_BF16 (scales 1).
- *   lora_a_gu    bf16 [L][E][r][H];  lora_b_gu bf16 [L][E][r][2I];
+ *   lora_a_gu    bf16 [L][E][r][H];  lora_b_gu bf16 [L][E][r][2I] (split: see above);
  *   lora_a_d     bf16 [L][E][r][I];  lora_b_d  bf16 [L][E][r][H]  (NULL iff L = 0).
+ *   format       adapter layout and scales, or NULL for the defaults.
  *   y            bf16 [M, H] output (overwritten).
  *   workspace    >= moe_lora_workspace_size(MOE_LORA_OP_FORWARD, M, H, I, E, k, L, r)
  *                (either expert type), or the smaller size of MOE_LORA_OP_FORWARD_BF16 /
@@ -161,7 +182,8 @@ MOE_LORA_API moe_lora_status moe_lora_forward(
     const float* topk_w, const int32_t* sorted_pairs, const int32_t* seg_offsets,
     const void* w_gateup, const void* w_down, ml_dtype w_dtype, const float* w_scales,
     const void* lora_a_gu, const void* lora_b_gu, const void* lora_a_d, const void* lora_b_d,
-    void* y, void* workspace, size_t workspace_bytes, moe_lora_stream stream);
+    const moe_lora_adapter_format* format, void* y, void* workspace, size_t workspace_bytes,
+    moe_lora_stream stream);
 
 /* ---------------------------------------------------------------------------------
  * sgmv_shrink -- segmented gather matrix-vector shrink: z_t = x_t A_{a(s)} for every

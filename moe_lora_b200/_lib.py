@@ -28,6 +28,12 @@ KERNEL_IDS = {"router_logits": 0, "topk": 1, "sort": 2, "shrink": 3, "gemm_gateu
               "lora": 11, "route": 12}
 
 
+class AdapterFormat(ctypes.Structure):
+    """moe_lora_adapter_format: gate_up adapter layout (0 fused, 1 separate gate and up
+    adapters) and the per-projection scales of the LoRA deltas."""
+    _fields_ = [("gate_up_split", ctypes.c_int), ("scale_gu", ctypes.c_float), ("scale_d", ctypes.c_float)]
+
+
 class MoELoRAError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"moe_lora status {status}: {msg}")
@@ -49,7 +55,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         L.moe_lora_route.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.moe_lora_forward.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P,
-                                       _P, _P, _P, _P, _P, _P, _SZ, _P]
+                                       _P, _P, _P, _P, ctypes.POINTER(AdapterFormat), _P, _P, _SZ, _P]
         L.sgmv_shrink.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]
         L.sgmv_expand.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]
         L.dense_lora_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]
@@ -161,13 +167,17 @@ def route(adapter_ids: torch.Tensor, k: int, L: int, *, x=None, w_router=None, b
 
 
 def forward(x: torch.Tensor, routing: dict, weights: dict, *, k: int, L: int, y=None, workspace=None,
-            stream=None) -> torch.Tensor:
+            stream=None, scale_gu: float = 1.0, scale_d: float = 1.0) -> torch.Tensor:
     """moe_lora_forward.  weights: w_gu [E,2I,H], w_d [E,H,I] (bf16 or e4m3), scales [E,2]
-    (e4m3 only), a_gu [L,E,r,H], b_gu [L,E,r,2I], a_d [L,E,r,I], b_d [L,E,r,H] (bf16)."""
+    (e4m3 only), a_gu [L,E,r,H], b_gu [L,E,r,2I] -- or separate gate and up adapters
+    a_gu [L,E,2,r,H], b_gu [L,E,2,r,I] -- a_d [L,E,r,I], b_d [L,E,r,H] (bf16).
+    scale_gu / scale_d multiply each projection's delta."""
     M, H = x.shape
     E, twoI, _ = weights["w_gu"].shape
     I = twoI // 2
-    r = weights["a_gu"].shape[2] if L > 0 else 0
+    split = L > 0 and weights["a_gu"].dim() == 5
+    r = weights["a_gu"].shape[-2] if L > 0 else 0
+    fmt = AdapterFormat(1 if split else 0, float(scale_gu), float(scale_d))
     wdt = _dt(weights["w_gu"])
     if y is None:
         y = torch.empty((M, H), dtype=torch.bfloat16, device=x.device)
@@ -179,7 +189,7 @@ def forward(x: torch.Tensor, routing: dict, weights: dict, *, k: int, L: int, y=
         _ptr(x), M, H, I, E, k, L, r, _ptr(routing["topk_w"]), _ptr(routing["sorted_pairs"]),
         _ptr(routing["seg_offsets"]), _ptr(weights["w_gu"]), _ptr(weights["w_d"]), wdt, _ptr(scales),
         _ptr(weights["a_gu"]) if L else None, _ptr(weights["b_gu"]) if L else None,
-        _ptr(weights["a_d"]) if L else None, _ptr(weights["b_d"]) if L else None,
+        _ptr(weights["a_d"]) if L else None, _ptr(weights["b_d"]) if L else None, ctypes.byref(fmt),
         _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)))
     return y
 

@@ -157,16 +157,20 @@ int choose_bn(long long rows, int groups) {
   return 256;
 }
 
-// Where the LoRA expand z B runs.  Long groups (more than 64 rows each: tensor-core
-// tiles of >= 128 tokens) run it inside the grouped GEMM as extra MMA K steps, so no
-// delta round-trips through HBM.  Short groups (decode) run it in the LoRA kernel into
-// an fp32 delta that the GEMM epilogue prefetches and adds: the weight stream of the
-// GEMM stays unbroken.  MOE_LORA_EXPAND=gemm|delta overrides (used by the tests).
-bool expand_in_gemm(long long rows, int groups) {
+// Where the LoRA work of the grouped GEMMs runs.
+//   LORA_DELTA  short groups (decode, <= 64 rows per group): the SIMT segmented LoRA
+//               kernel writes an fp32 delta that the GEMM epilogue prefetches and adds,
+//               so the GEMM's weight stream stays unbroken.
+//   LORA_TC     long groups (prefill): the tensor-core LoRA kernel (shrink and expand on
+//               tcgen05, z on chip) writes a bf16 delta that the GEMM epilogue adds.
+// MOE_LORA_EXPAND=delta|tc overrides (used by the tests and the measurements).
+enum LoraPlace { LORA_DELTA = 0, LORA_TC = 1 };
+
+LoraPlace lora_place(long long rows, int groups) {
   const char* v = std::getenv("MOE_LORA_EXPAND");
-  if (v != nullptr && std::strcmp(v, "gemm") == 0) return true;
-  if (v != nullptr && std::strcmp(v, "delta") == 0) return false;
-  return rows > 64LL * (groups > 0 ? groups : 1);
+  if (v != nullptr && std::strcmp(v, "delta") == 0) return LORA_DELTA;
+  if (v != nullptr && std::strcmp(v, "tc") == 0) return LORA_TC;
+  return rows > 64LL * (groups > 0 ? groups : 1) ? LORA_TC : LORA_DELTA;
 }
 
 int shrink_rows_per_cta(long long rows) {
@@ -179,7 +183,6 @@ int shrink_rows_per_cta(long long rows) {
 // Stream-K scratch of the grouped GEMM (few tiles): flags right after the status word,
 // so the per-call clear of the status also re-arms them, and the partial accumulators.
 constexpr int kSkSlots = 160;                       // >= SMs of the device
-constexpr int kShrinkBN = 32;                       // N tile of the tensor-core LoRA shrink
 constexpr size_t kSkFlagBytes = kSkSlots * 4;
 constexpr size_t kSkPartFloats = static_cast<size_t>(kSkSlots) * 128 * 64;
 
@@ -191,22 +194,24 @@ struct ForwardWs {
   __nv_bfloat16* act;
   float* delta_gu;     // expand in the LoRA kernel: deltas the GEMM epilogues add
   float* delta_d;
-  __nv_bfloat16* z;    // expand in the GEMMs: the LoRA shrink output [M*k][r]
+  __nv_bfloat16* dgu;  // tensor-core LoRA: bf16 deltas [M*k][2I] and [M*k][H]
+  __nv_bfloat16* dd;
   float* z_part;       // split LoRA shrink: fp32 partials [ceil(max(H, I) / 1024)][M*k][r]
   long long z_part_cap;
   int2* items;         // LoRA work list and its length
   int* item_count;
   int2* items_tc;      // expand in the GEMMs: tiles of the tensor-core shrink (adapter segments)
   int* item_count_tc;
-  float* o;
+  __nv_bfloat16* o;   // per-pair weighted outputs [M*k][H], summed by the combine
   uint8_t* q_hi;      // e4m3 weights: activation planes [M*k][max(H, I)]
   uint8_t* q_lo;
   float* q_scales;    // [M*k][2]
   size_t bytes;
 };
 
-ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8, bool fused, int nkeys) {
+ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8, LoraPlace place, int nkeys) {
   const size_t mk = static_cast<size_t>(M) * k;
+  const bool dl = r && place == LORA_DELTA, tc = r && place == LORA_TC;
   size_t off = kStatusBytes;
   ForwardWs w{};
   uint8_t* b = static_cast<uint8_t*>(base);
@@ -219,18 +224,20 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
   w.sk_flag = reinterpret_cast<int*>(take(mk > 0 ? kSkFlagBytes : 0));  // must stay first
   w.x_sorted = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
   w.act = reinterpret_cast<__nv_bfloat16*>(take(mk * I * 2));
-  w.delta_gu = reinterpret_cast<float*>(take(r && !fused ? mk * 2 * I * 4 : 0));
-  w.delta_d = reinterpret_cast<float*>(take(r && !fused ? mk * H * 4 : 0));
-  w.z = reinterpret_cast<__nv_bfloat16*>(take(r && fused ? mk * r * 2 : 0));
-  w.z_part_cap = r ? static_cast<long long>((std::max(H, I) + 1023) / 1024) * mk * r : 0;
+  w.delta_gu = reinterpret_cast<float*>(take(dl ? mk * 2 * I * 4 : 0));
+  w.delta_d = reinterpret_cast<float*>(take(dl ? mk * H * 4 : 0));
+  w.dgu = reinterpret_cast<__nv_bfloat16*>(take(tc ? mk * 2 * I * 2 : 0));
+  w.dd = reinterpret_cast<__nv_bfloat16*>(take(tc ? mk * H * 2 : 0));
+  // split LoRA shrink partials: rank r, or 2 r for separate gate and up adapters (r <= 64)
+  w.z_part_cap = dl ? static_cast<long long>((std::max(H, I) + 1023) / 1024) * mk * (r <= 64 ? 2 * r : r) : 0;
   w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
   w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, 4)) * 8));
   w.item_count = reinterpret_cast<int*>(take(mk > 0 ? 4 : 0));
   w.items_tc = reinterpret_cast<int2*>(
-      take(r && fused ? static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, kShrinkBN)) * 8 : 0));
-  w.item_count_tc = reinterpret_cast<int*>(take(r && fused ? 4 : 0));
+      take(tc ? static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, kLtN)) * 8 : 0));
+  w.item_count_tc = reinterpret_cast<int*>(take(tc ? 4 : 0));
   w.sk_part = reinterpret_cast<float*>(take(mk > 0 ? kSkPartFloats * 4 : 0));
-  w.o = reinterpret_cast<float*>(take(mk * H * 4));
+  w.o = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
   const size_t kmax = H > I ? H : I;
   w.q_hi = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
   w.q_lo = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
@@ -272,7 +279,7 @@ struct DenseWs {
   float* z;             // fp32 path: shrink output
   int32_t* row_adapter; // fp32 path
   float* delta;         // bf16 path, expand in the LoRA kernel: delta the GEMM adds
-  __nv_bfloat16* zb;    // bf16 path, expand in the GEMM: shrink output
+  __nv_bfloat16* dbf;   // bf16 path, tensor-core LoRA: bf16 delta [T][h_out]
   float* z_part;        // bf16 path, split LoRA shrink partials
   long long z_part_cap;
   int2* items;          // bf16 path: LoRA work list and its length
@@ -282,7 +289,8 @@ struct DenseWs {
   size_t bytes;
 };
 
-DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, bool fused) {
+DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, LoraPlace place) {
+  const bool dl = r && place == LORA_DELTA, tc = r && place == LORA_TC;
   size_t off = kStatusBytes;
   DenseWs w{};
   uint8_t* b = static_cast<uint8_t*>(base);
@@ -297,14 +305,14 @@ DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, bo
     w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
     w.row_adapter = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
   } else {
-    w.delta = reinterpret_cast<float*>(take(r && !fused ? static_cast<size_t>(T) * h_out * 4 : 0));
-    w.zb = reinterpret_cast<__nv_bfloat16*>(take(r && fused ? static_cast<size_t>(T) * r * 2 : 0));
-    w.z_part_cap = r ? static_cast<long long>((h_in + 1023) / 1024) * T * r : 0;
+    w.delta = reinterpret_cast<float*>(take(dl ? static_cast<size_t>(T) * h_out * 4 : 0));
+    w.dbf = reinterpret_cast<__nv_bfloat16*>(take(tc ? static_cast<size_t>(T) * h_out * 2 : 0));
+    w.z_part_cap = dl ? static_cast<long long>((h_in + 1023) / 1024) * T * r : 0;
     w.z_part = reinterpret_cast<float*>(take(static_cast<size_t>(w.z_part_cap) * 4));
     w.items = reinterpret_cast<int2*>(take(static_cast<size_t>(lora_items_bound(T, T, 4)) * 8));
     w.item_count = reinterpret_cast<int*>(take(T > 0 ? 4 : 0));
-    w.items_tc = reinterpret_cast<int2*>(take(r && fused ? static_cast<size_t>(lora_items_bound(T, T, kShrinkBN)) * 8 : 0));
-    w.item_count_tc = reinterpret_cast<int*>(take(r && fused ? 4 : 0));
+    w.items_tc = reinterpret_cast<int2*>(take(tc ? static_cast<size_t>(lora_items_bound(T, T, kLtN)) * 8 : 0));
+    w.item_count_tc = reinterpret_cast<int*>(take(tc ? 4 : 0));
     w.sk_part = reinterpret_cast<float*>(take(T > 0 ? kSkPartFloats * 4 : 0));
   }
   w.bytes = off;
@@ -386,16 +394,16 @@ size_t moe_lora_workspace_size(int op, int M, int H, int I, int E, int k, int L,
     case MOE_LORA_OP_ROUTE: return route_layout(nullptr, M, E, L).bytes;
     case MOE_LORA_OP_FORWARD:
     case MOE_LORA_OP_FORWARD_E4M3:
-      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, true, expand_in_gemm(1LL * M * k, E), E * (L + 1))
+      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, true, lora_place(1LL * M * k, E), E * (L + 1))
           .bytes;
     case MOE_LORA_OP_FORWARD_BF16:
-      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, false, expand_in_gemm(1LL * M * k, E), E * (L + 1))
+      return forward_layout(nullptr, M, H, I, k, L > 0 ? r : 0, false, lora_place(1LL * M * k, E), E * (L + 1))
           .bytes;
     case MOE_LORA_OP_SGMV_SHRINK:
     case MOE_LORA_OP_SGMV_EXPAND: return kStatusBytes;
     case MOE_LORA_OP_DENSE: {
-      const size_t a = dense_layout(nullptr, M, H, I, L > 0 ? r : 0, true, false).bytes;
-      const size_t b = dense_layout(nullptr, M, H, I, L > 0 ? r : 0, false, expand_in_gemm(M, 1)).bytes;
+      const size_t a = dense_layout(nullptr, M, H, I, L > 0 ? r : 0, true, LORA_DELTA).bytes;
+      const size_t b = dense_layout(nullptr, M, H, I, L > 0 ? r : 0, false, lora_place(M, 1)).bytes;
       return a > b ? a : b;
     }
     default: return 0;
@@ -415,39 +423,6 @@ moe_lora_status moe_lora_check_status(void* workspace, moe_lora_stream stream) {
 
 }  // extern "C"
 
-namespace {
-// z = src A_slot^T per adapter segment on the tensor cores: one tile per chunk of up to
-// kShrinkBN rows of a segment with an adapter (work list from the plan kernel), the
-// slot's r rows of LoRA A in the MMA's M slot, bf16 z rows out.
-cudaError_t launch_shrink_tc(const LoraDeltaArgs& l, int2* items, int* count, int E, cudaStream_t cs) {
-  const int bound = lora_items_bound(l.nrows, l.nseg, kShrinkBN);
-  cudaError_t err = launch_lora_plan_adapters(l, kShrinkBN, items, count, bound, cs);
-  if (err != cudaSuccess) return err;
-  GemmArgs s{};
-  s.epi = EPI_ZOUT;
-  s.K = l.K;
-  s.E = 1;
-  s.group_offsets = nullptr;
-  s.rows_per_group = l.L * E * l.r;
-  s.n_out = l.r;
-  s.total_rows = l.nrows;
-  s.w = l.lora_a;
-  s.b = l.gather_dst ? l.gather_dst : l.src;
-  s.out_bf16 = l.z_out;
-  s.status = l.status;
-  s.bn = kShrinkBN;
-  s.num_sms = l.num_sms;
-  s.items = items;
-  s.item_count = count;
-  s.items_bound = bound;
-  s.lseg_off = l.seg_offsets;
-  s.lseg_adapter = l.seg_adapter;
-  s.L = l.L;
-  s.iE = E;
-  s.r = l.r;
-  return launch_gemm_tc(s, cs);
-}
-}  // namespace
 
 extern "C" {
 
@@ -515,8 +490,8 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
                                  const int32_t* seg_offsets, const void* w_gateup, const void* w_down,
                                  ml_dtype w_dtype, const float* w_scales, const void* lora_a_gu,
                                  const void* lora_b_gu, const void* lora_a_d, const void* lora_b_d,
-                                 void* y, void* workspace, size_t workspace_bytes,
-                                 moe_lora_stream stream) {
+                                 const moe_lora_adapter_format* format, void* y, void* workspace,
+                                 size_t workspace_bytes, moe_lora_stream stream) {
   ML_REQUIRE(M >= 0 && H > 0 && I > 0 && E >= 1 && k >= 1 && L >= 0, MOE_LORA_ERR_INVALID_ARG,
              "need M >= 0, H > 0, I > 0, E >= 1, k >= 1, L >= 0");
   ML_REQUIRE(w_dtype == ML_BF16 || w_dtype == ML_E4M3, MOE_LORA_ERR_INVALID_ARG,
@@ -527,8 +502,17 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   if (L > 0) ML_REQUIRE(rank_ok(r), MOE_LORA_ERR_UNSUPPORTED, "r must be one of 8, 16, 32, 64, 128");
   const int rr = L > 0 ? r : 0;
   const bool fp8 = w_dtype == ML_E4M3;
-  const bool fused = expand_in_gemm(1LL * M * k, E);
-  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr, fp8, fused, E * (L + 1));
+  const moe_lora_adapter_format fmt = format ? *format : moe_lora_adapter_format{0, 1.0f, 1.0f};
+  ML_REQUIRE(fmt.gate_up_split == 0 || fmt.gate_up_split == 1, MOE_LORA_ERR_INVALID_ARG,
+             "format->gate_up_split must be 0 or 1");
+  const bool split = fmt.gate_up_split == 1 && rr > 0;
+  if (split) ML_REQUIRE(r <= 64, MOE_LORA_ERR_UNSUPPORTED, "separate gate and up adapters need r <= 64");
+  const LoraPlace place = lora_place(1LL * M * k, E);
+  // the tensor-core LoRA kernel takes separate gate and up adapters at whole 64-feature boxes
+  if (split && place == LORA_TC)
+    ML_REQUIRE(I % 64 == 0, MOE_LORA_ERR_UNSUPPORTED,
+               "separate gate and up adapters with more than 64 rows per expert need I a multiple of 64");
+  const ForwardWs need = forward_layout(nullptr, M, H, I, k, rr, fp8, place, E * (L + 1));
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (w_dtype == ML_E4M3) {
@@ -555,19 +539,22 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   if (!tensor_map_encode_available())
     return fail(MOE_LORA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8, fused, E * (L + 1));
+  const ForwardWs w = forward_layout(workspace, M, H, I, k, rr, fp8, place, E * (L + 1));
+  const bool tcl = rr && place == LORA_TC;  // tensor-core LoRA kernel, bf16 deltas
   const int mk = M * k;
   const int nkeys = E * (L + 1);
   // status word and the stream-K flags that follow it
   ML_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes + kSkFlagBytes, cs), "status clear");
 
-  // 1. gather x rows into (expert, adapter) order; gate_up LoRA shrink z = x A_gu per
-  //    (adapter, expert) segment; the expand z B_gu either runs here (delta_gu, added
-  //    by the GEMM epilogue) or in the GEMM as extra MMA K steps
+  // 1. gather x rows into (expert, adapter) order, and the gate_up LoRA:
+  //    LORA_DELTA: one SIMT kernel gathers, shrinks z = x A_gu per (adapter, expert)
+  //                segment chunk and expands z B_gu into an fp32 delta;
+  //    LORA_TC:    a row gather, then the tensor-core LoRA kernel (bf16 delta);
   LoraDeltaArgs l1{};
   l1.src = static_cast<const __nv_bfloat16*>(x);
   l1.gather = sorted_pairs;
   l1.gather_div = k;
+  l1.nsrc = M;
   l1.gather_dst = w.x_sorted;
   l1.nrows = mk;
   l1.K = H;
@@ -580,7 +567,11 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   l1.E = E;
   l1.lora_a = static_cast<const __nv_bfloat16*>(lora_a_gu);
   l1.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
-  l1.delta = rr && !fused ? w.delta_gu : nullptr;  // fused: this launch only gathers (and quantises)
+  l1.r_exp = rr;
+  l1.split_I = split ? I : 0;
+  l1.scale = fmt.scale_gu;
+  if (split) l1.r = 2 * rr;  // the shrink covers both adapters' rows
+  l1.delta = rr && place == LORA_DELTA ? w.delta_gu : nullptr;  // otherwise this launch only gathers
   l1.z_part = w.z_part;
   l1.z_part_cap = w.z_part_cap;
   l1.status = w.status;
@@ -589,17 +580,57 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   l1.items_bound = lora_items_bound(mk, nkeys, l1.rb);
   l1.items = w.items;
   l1.item_count = w.item_count;
-  if (fp8) {  // the same kernel writes the e4m3 planes of the gathered x rows
-    l1.q_hi = w.q_hi;
-    l1.q_lo = w.q_lo;
-    l1.q_scales = w.q_scales;
-  }
-  ML_CUDA(launch_lora_plan(l1, cs), "LoRA plan launch");
-  ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
-  if (rr && fused) {  // the shrink on the tensor cores, z for the GEMM's expand steps
-    LoraDeltaArgs ls = l1;
-    ls.z_out = w.z;
-    ML_CUDA(launch_shrink_tc(ls, w.items_tc, w.item_count_tc, E, cs), "gate_up LoRA shrink launch");
+  LoraTcArgs t1{};
+  if (tcl) {
+    ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs),
+            "row gather launch");
+    if (fp8)
+      ML_CUDA(launch_quant_planes(w.x_sorted, mk, H, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
+    const int bound = lora_items_bound(mk, nkeys, kLtN);
+    ML_CUDA(launch_lora_plan_all(seg_offsets, nullptr, nkeys, L, mk, kLtN, w.items_tc, w.item_count_tc, bound,
+                                 w.status, cs),
+            "LoRA work list launch");
+    t1.src = w.x_sorted;
+    t1.nrows = mk;
+    t1.K = H;
+    t1.r = rr;
+    t1.F = 2 * I;
+    t1.seg_offsets = seg_offsets;
+    t1.nseg = nkeys;
+    t1.seg_adapter = nullptr;
+    t1.L = L;
+    t1.E = E;
+    t1.lora_a = static_cast<const __nv_bfloat16*>(lora_a_gu);
+    t1.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
+    t1.r = split ? 2 * rr : rr;
+    t1.r_exp = rr;
+    t1.split_I = split ? I : 0;
+    t1.scale = fmt.scale_gu;
+    t1.items = w.items_tc;
+    t1.item_count = w.item_count_tc;
+    t1.items_bound = bound;
+    t1.delta = w.dgu;
+    t1.status = w.status;
+    t1.work_counter = w.status + 2;  // inside the status block: cleared with it by every call
+    t1.num_sms = num_sms();
+    ML_CUDA(launch_lora_tc(t1, cs), "gate_up tensor-core LoRA launch");
+  } else {
+    // the GEMM's operand first (gathered x rows, or their e4m3 planes), then the LoRA
+    // kernel, which lets the GEMM start at once: the GEMM streams its weights while the
+    // LoRA kernel runs, and only its epilogue loader waits for the delta
+    if (fp8)
+      ML_CUDA(launch_gather_quant(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.q_hi, w.q_lo,
+                                  w.q_scales, cs),
+              "activation planes launch");
+    else
+      ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs),
+              "row gather launch");
+    if (rr) {
+      l1.gather_dst = nullptr;
+      l1.pdl_trigger = 1;
+      ML_CUDA(launch_lora_plan(l1, cs), "LoRA plan launch");
+      ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
+    }
   }
 
   // 2. gate_up grouped GEMM; epilogue adds delta_gu and applies SiLU-and-mul -> act
@@ -615,17 +646,9 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.I = I;
   g.total_rows = mk;
   g.delta_cols = 2 * I;
-  g.delta = rr && !fused ? w.delta_gu : nullptr;
-  if (rr && fused) {
-    g.z = w.z;
-    g.r = rr;
-    g.lora_b = static_cast<const __nv_bfloat16*>(lora_b_gu);
-    g.L = L;
-    g.lseg_off = seg_offsets;
-    g.lseg_stride = L + 1;
-    g.lseg_count = L;
-    g.lseg_adapter = nullptr;
-  }
+  g.delta = rr && place == LORA_DELTA ? w.delta_gu : nullptr;
+  g.delta_bf16 = tcl ? w.dgu : nullptr;
+  g.pdl_secondary = rr && place == LORA_DELTA ? 1 : 0;
   g.out_bf16 = w.act;
   g.w_scales = w_dtype == ML_E4M3 ? w_scales : nullptr;
   g.scale_idx = 0;
@@ -644,50 +667,78 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.sk_part_cap = static_cast<long long>(kSkPartFloats);
   g.sk_flag = w.sk_flag;
   g.sk_slots = kSkSlots;
+  // tests only: the gate_up GEMM's first stage in CTA 0 never arrives and every bounded
+  // wait is shortened to MOE_LORA_TEST_STALL milliseconds (exercises the abort path)
+  g.test_stall_ms = env_int("MOE_LORA_TEST_STALL", 0);
   ML_CUDA(launch_gemm_tc(g, cs), "gate_up GEMM launch");
+  g.test_stall_ms = 0;
 
-  // 3. down LoRA shrink + expand on act: delta_d = (act A_d) B_d
-  if (rr) {
-    LoraDeltaArgs l2 = l1;
-    l2.src = w.act;
-    l2.gather = nullptr;
-    l2.gather_dst = nullptr;
-    l2.K = I;
-    l2.NB = H;
-    l2.lora_a = static_cast<const __nv_bfloat16*>(lora_a_d);
-    l2.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
-    if (fused) {
-      l2.z_out = w.z;
-      l2.q_hi = nullptr;  // the planes of act come from the plane kernel below
-      ML_CUDA(launch_shrink_tc(l2, w.items_tc, w.item_count_tc, E, cs), "down LoRA shrink launch");
-    } else {
-      l2.delta = w.delta_d;
-      ML_CUDA(launch_lora_delta(l2, cs), "down LoRA launch");
-    }
+  g.pdl_secondary = 0;
+
+  // 3. down LoRA shrink + expand on act: delta_d = (act A_d) B_d (LORA_DELTA: after the
+  //    down GEMM's launch, overlapped with it, into a pair-order delta the combine adds)
+  if (tcl) {
+    LoraTcArgs t2 = t1;
+    t2.src = w.act;
+    t2.K = I;
+    t2.F = H;
+    t2.lora_a = static_cast<const __nv_bfloat16*>(lora_a_d);
+    t2.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
+    t2.r = rr;
+    t2.r_exp = rr;
+    t2.split_I = 0;
+    t2.scale = fmt.scale_d;
+    t2.delta = w.dd;
+    t2.scatter = sorted_pairs;  // pair order: the combine adds it
+    t2.work_counter = w.status + 3;
+    ML_CUDA(launch_lora_tc(t2, cs), "down tensor-core LoRA launch");
   }
 
-  // 4. down grouped GEMM; epilogue adds delta_d and the routing weight -> o (per pair)
+  // 4. down grouped GEMM; the epilogue applies the routing weight -> o (per pair, bf16);
+  //    the combine adds the weighted down LoRA delta
   GemmArgs d = g;
   d.epi = EPI_DOWN;
   d.K = I;
   d.rows_per_group = H;
   d.n_out = H;
   d.delta_cols = H;
-  d.delta = rr && !fused ? w.delta_d : nullptr;
-  if (rr && fused) d.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
-  d.out_bf16 = nullptr;
-  d.out_f32 = w.o;
+  d.delta = nullptr;
+  d.delta_bf16 = nullptr;  // the down LoRA delta (delta and tc placements) goes to the combine
+  d.pdl_trigger = rr && place == LORA_DELTA ? 1 : 0;
+  d.out_bf16 = w.o;
+  d.out_f32 = nullptr;
   d.sorted_pairs = sorted_pairs;
   d.topk_w = topk_w;
   d.scale_idx = 1;
   d.w = w_down;
   d.b = w.act;
-  if (fp8 && (!rr || fused))  // otherwise the down LoRA kernel wrote the planes of act
-    ML_CUDA(launch_quant_planes(w.act, mk, I, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
+  if (fp8) ML_CUDA(launch_quant_planes(w.act, mk, I, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
   ML_CUDA(launch_gemm_tc(d, cs), "down GEMM launch");
+  if (rr && place == LORA_DELTA) {
+    LoraDeltaArgs l2 = l1;
+    l2.src = w.act;
+    l2.gather = nullptr;
+    l2.gather_dst = nullptr;
+    l2.q_hi = nullptr;
+    l2.K = I;
+    l2.NB = H;
+    l2.lora_a = static_cast<const __nv_bfloat16*>(lora_a_d);
+    l2.lora_b = static_cast<const __nv_bfloat16*>(lora_b_d);
+    l2.r = rr;
+    l2.r_exp = rr;
+    l2.split_I = 0;
+    l2.scale = fmt.scale_d;
+    l2.delta = w.delta_d;
+    l2.scatter = sorted_pairs;  // pair order, for the combine
+    l2.pdl_trigger = 0;
+    l2.pdl_secondary = 1;
+    ML_CUDA(launch_lora_delta(l2, cs), "down LoRA launch");
+  }
 
-  // 5. fixed-order combine over the k slots
-  ML_CUDA(launch_combine(w.o, M, k, H, static_cast<__nv_bfloat16*>(y), cs), "combine launch");
+  // 5. fixed-order combine over the k slots (+ the weighted down LoRA delta)
+  ML_CUDA(launch_combine(w.o, M, k, H, rr && place == LORA_DELTA ? w.delta_d : nullptr, tcl ? w.dd : nullptr,
+                         topk_w, static_cast<__nv_bfloat16*>(y), cs),
+          "combine launch");
   return MOE_LORA_OK;
 }
 
@@ -784,8 +835,8 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   ML_REQUIRE(S >= 1 || T == 0, MOE_LORA_ERR_INVALID_ARG, "segments must cover the T tokens");
   const int rr = L > 0 ? r : 0;
   const bool f32 = dt == ML_F32;
-  const bool fused = !f32 && expand_in_gemm(T, 1);
-  const DenseWs need = dense_layout(nullptr, T, h_in, h_out, rr, f32, fused);
+  const LoraPlace place = f32 ? LORA_DELTA : lora_place(T, 1);
+  const DenseWs need = dense_layout(nullptr, T, h_in, h_out, rr, f32, place);
   moe_lora_status st = check_ws(workspace, workspace_bytes, need.bytes);
   if (st != MOE_LORA_OK) return st;
   if (T == 0) return MOE_LORA_OK;
@@ -801,7 +852,8 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   st = check_device();
   if (st != MOE_LORA_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const DenseWs ws = dense_layout(workspace, T, h_in, h_out, rr, f32, fused);
+  const DenseWs ws = dense_layout(workspace, T, h_in, h_out, rr, f32, place);
+  const bool tcl = rr && place == LORA_TC;  // tensor-core LoRA kernel, bf16 delta
   ML_CUDA(cudaMemsetAsync(workspace, 0, f32 ? 8 : kStatusBytes + kSkFlagBytes, cs), "status clear");
 
   if (f32) {
@@ -855,7 +907,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     l.E = 1;
     l.lora_a = static_cast<const __nv_bfloat16*>(lora_a);
     l.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
-    l.delta = fused ? nullptr : ws.delta;
+    l.delta = place == LORA_DELTA ? ws.delta : nullptr;
     l.z_part = ws.z_part;
     l.z_part_cap = ws.z_part_cap;
     l.status = ws.status;
@@ -864,10 +916,36 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     l.items_bound = lora_items_bound(T, S, l.rb);
     l.items = ws.items;
     l.item_count = ws.item_count;
-    if (fused) {  // the shrink on the tensor cores, z for the GEMM's expand steps
-      l.z_out = ws.zb;
-      ML_CUDA(launch_shrink_tc(l, ws.items_tc, ws.item_count_tc, 1, cs), "dense LoRA shrink launch");
+    if (tcl) {  // shrink and expand on the tensor cores, bf16 delta for the epilogue
+      const int bound = lora_items_bound(T, S, kLtN);
+      ML_CUDA(launch_lora_plan_all(seg_offsets, seg_adapter, S, L, T, kLtN, ws.items_tc, ws.item_count_tc, bound,
+                                   ws.status, cs),
+              "LoRA work list launch");
+      LoraTcArgs t{};
+      t.src = static_cast<const __nv_bfloat16*>(x);
+      t.nrows = T;
+      t.K = h_in;
+      t.r = rr;
+      t.F = h_out;
+      t.seg_offsets = seg_offsets;
+      t.nseg = S;
+      t.seg_adapter = seg_adapter;
+      t.L = L;
+      t.E = 1;
+      t.lora_a = static_cast<const __nv_bfloat16*>(lora_a);
+      t.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
+      t.items = ws.items_tc;
+      t.item_count = ws.item_count_tc;
+      t.items_bound = bound;
+      t.delta = ws.dbf;
+      t.status = ws.status;
+      t.work_counter = ws.status + 2;  // inside the status block: cleared with it by every call
+      t.num_sms = num_sms();
+      ML_CUDA(launch_lora_tc(t, cs), "dense tensor-core LoRA launch");
     } else {
+      // the LoRA kernel lets the GEMM start at once: the GEMM streams W while it runs,
+      // and only the GEMM's epilogue loader waits for the delta
+      l.pdl_trigger = 1;
       ML_CUDA(launch_lora_plan(l, cs), "LoRA plan launch");
       ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
     }
@@ -883,22 +961,15 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   g.I = 0;
   g.total_rows = T;
   g.delta_cols = h_out;
-  g.delta = rr && !fused ? ws.delta : nullptr;
-  if (rr && fused) {  // expand z B as extra K steps over the dense segments
-    g.z = ws.zb;
-    g.r = rr;
-    g.lora_b = static_cast<const __nv_bfloat16*>(lora_b);
-    g.L = L;
-    g.lseg_off = seg_offsets;
-    g.lseg_stride = 0;
-    g.lseg_count = S;
-    g.lseg_adapter = seg_adapter;
-  }
+  g.delta = rr && place == LORA_DELTA ? ws.delta : nullptr;
+  g.delta_bf16 = tcl ? ws.dbf : nullptr;
   g.out_bf16 = static_cast<__nv_bfloat16*>(y);
   g.status = ws.status;
   g.w = w;
   g.b = static_cast<const __nv_bfloat16*>(x);
   g.bn = choose_bn(T, 1);
+  g.pdl_secondary = rr && place == LORA_DELTA ? 1 : 0;
+
   g.num_sms = num_sms();
   g.sk_part = ws.sk_part;
   g.sk_part_cap = static_cast<long long>(kSkPartFloats);

@@ -71,6 +71,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start before the kernel
+// ahead of it in the stream has finished.  pdl_wait() blocks the calling thread until
+// that kernel has completed and its memory is visible (immediately when there is none);
+// pdl_trigger() lets the kernel behind this one start once every CTA of this grid has
+// triggered or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ shared memory / mbarrier
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -155,6 +164,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// The box at {c0, c1} of a tensor map heads for L2 (no shared-memory destination, no
+// barrier): issued some stages ahead of the box's real load, it turns the load's DRAM
+// latency into an L2 hit.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // 16-byte global -> shared copy that does not block the thread; zero-fills when !valid
 // (no bytes read; `gsrc` must still be a mapped address).
 __device__ __forceinline__ void cp_async_16_zfill(void* smem_dst, const void* gsrc, bool valid) {
@@ -167,6 +185,13 @@ __device__ __forceinline__ void cp_async_16_zfill(void* smem_dst, const void* gs
 // pending count goes up by one now and down by one when those copies have landed.
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Asks the memory system to bring [p, p + bytes) into L2 without waiting (bulk, no
+// destination): p 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
 }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }

@@ -61,6 +61,7 @@ struct LoraDeltaArgs {
   const __nv_bfloat16* src;   // rows [*, K]
   const int32_t* gather;      // if set: source row of output row s = gather[s] / gather_div
   int gather_div;
+  int nsrc;                   // source rows (bound of the gathered indices)
   __nv_bfloat16* gather_dst;  // if set: copy of the gathered source row
   int nrows, K, r, NB;        // NB = delta features per row
   const int32_t* seg_offsets; // [nseg+1]
@@ -70,7 +71,6 @@ struct LoraDeltaArgs {
   const __nv_bfloat16* lora_a;  // MoE [L][E][r][K]; dense [L][r][K]
   const __nv_bfloat16* lora_b;  // MoE [L][E][r][NB]; dense [L][r][NB]
   float* delta;               // [nrows][NB] (expand in this kernel) or null
-  __nv_bfloat16* z_out;       // shrink only: z [nrows][r] bf16 for a GEMM that expands
   // e4m3 experts: the two activation planes of the source rows (in row order), written
   // by the CTAs of feature slice / K slice 0 (see launch_quant_planes); null otherwise
   uint8_t* q_hi;
@@ -85,14 +85,64 @@ struct LoraDeltaArgs {
   int rb;                     // lora_rows_per_chunk(nrows, nseg)
   int* status;
   int num_sms;
+  // delta row of gathered row s: scatter[s] (a routing pair, so that the combine reads
+  // delta in pair order) instead of s; null = s
+  const int32_t* scatter;
+  // expand: r_exp rank rows of B per delta feature (r for fused adapters); split_I > 0:
+  // separate gate and up adapters (A = the 2 r_exp rows of both, B = [2][r_exp][split_I]);
+  // every delta value is multiplied by scale
+  int r_exp;
+  int split_I;
+  float scale;
+  // programmatic dependent launch: pdl_trigger lets the next kernel start right away;
+  // pdl_secondary launches this one behind the running kernel ahead of it, and the
+  // kernel then waits for that kernel before it exits.  Either forces the one-kernel form.
+  int pdl_trigger;
+  int pdl_secondary;
 };
 int lora_rows_per_chunk(int nrows, int nseg);
 int lora_items_bound(int nrows, int nseg, int rb);
 cudaError_t launch_lora_plan(const LoraDeltaArgs& a, cudaStream_t st);
-// work list of the segments that have an adapter only, chunks of rb rows (tensor-core shrink)
-cudaError_t launch_lora_plan_adapters(const LoraDeltaArgs& a, int rb, int2* items, int* count, int cap,
-                                      cudaStream_t st);
 cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st);
+
+// Tensor-core segmented LoRA for long segments: per work item (a chunk of up to kLtN
+// rows of one segment) shrink z = src A_a and expand delta = z B_a on tcgen05, z kept on
+// chip; delta rows (bf16, [nrows][F]) for the grouped GEMM's epilogue.  Items of
+// segments without an adapter write delta = 0 rows.  Work list: lora_plan over every
+// segment with chunks of kLtN rows.
+constexpr int kLtN = 128;
+struct LoraTcArgs {
+  const __nv_bfloat16* src;     // rows [nrows][K] (gathered x, or act)
+  int nrows, K, r, F;
+  const int32_t* seg_offsets;   // [nseg + 1]
+  int nseg;
+  const int32_t* seg_adapter;   // dense: [nseg]; null: MoE keys q = e (L + 1) + a'
+  int L, E;
+  const __nv_bfloat16* lora_a;  // MoE [L][E][r][K]; dense [L][r][K]
+  const __nv_bfloat16* lora_b;  // MoE [L][E][r][F]; dense [L][r][F]
+  const int2* items;
+  const int* item_count;
+  int items_bound;
+  __nv_bfloat16* delta;         // [nrows][F]
+  const int32_t* scatter;       // delta row of gathered row s: scatter[s] (pair order); null = s
+  int* status;
+  int* work_counter;            // int in device memory, zero before the launch (work claiming)
+  int num_sms;
+  // separate gate and up adapters: split_I = I (a multiple of 64), r = 2 r_exp (A holds
+  // both adapters' rows), B [L][E][2][r_exp][I]; 0 = one fused adapter (B [..][r][F])
+  int split_I;
+  int r_exp;
+  float scale;                  // multiplies every delta value
+};
+cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st);
+
+// dst[i] = src[gather[i] / div] for i < rows (bf16 rows of K elements; a source index
+// outside [0, nsrc) gives a zero row).
+cudaError_t launch_gather_rows(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
+                               __nv_bfloat16* dst, cudaStream_t st);
+// Work list of every non-empty segment (with or without an adapter), chunks of rb rows.
+cudaError_t launch_lora_plan_all(const int32_t* seg_offsets, const int32_t* seg_adapter, int nseg, int L, int nrows,
+                                 int rb, int2* items, int* count, int cap, int* status, cudaStream_t st);
 
 // y[t] += z[t] . B_a(t) for dense segments (f32 or bf16 y and B).
 struct ExpandArgs {
@@ -123,7 +173,7 @@ cudaError_t launch_dense_f32(const DenseF32Args& a, cudaStream_t st);
 
 // Tensor-core grouped GEMM with operand swap: the weight rows fill the 128-row MMA
 // M slot, the tokens of one expert (or of the dense batch) the N slot.
-enum EpiKind : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DENSE = 2, EPI_LOGITS = 3, EPI_ZOUT = 4 };
+enum EpiKind : int { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DENSE = 2, EPI_LOGITS = 3 };
 
 struct GemmArgs {
   int epi;
@@ -141,9 +191,12 @@ struct GemmArgs {
   // within the group (gate_up: gate rows [0, I), up rows [I, 2I)); null = no LoRA
   const float* delta;
   int delta_cols;
+  // the same as a bf16 delta (from the tensor-core LoRA kernel), read by the epilogue
+  // straight from global memory; exclusive with delta
+  const __nv_bfloat16* delta_bf16;
   // epilogue outputs
-  __nv_bfloat16* out_bf16;     // gate_up: act [rows][I]; dense: y [T][h_out]
-  float* out_f32;              // down: o [pairs][H] (weighted); logits: [rows][n_out]
+  __nv_bfloat16* out_bf16;     // gate_up: act [rows][I]; down: o [pairs][H] (weighted); dense: y [T][h_out]
+  float* out_f32;              // logits: [rows][n_out]
   const float* bias;           // logits: [n_out] or null
   const int32_t* sorted_pairs; // down: pair index of each sorted row
   const float* topk_w;         // down: routing weight per pair
@@ -158,29 +211,21 @@ struct GemmArgs {
   const float* b_scales;       // [total_rows][2] = (s, s / 16)
   int bn;                      // N tile (16..256)
   int num_sms;
-  // LoRA expand fused as extra K steps (bf16 weights only; exclusive with delta):
-  // acc[f][t] += sum_i B[slot][i][f] z[t][i] for the rows t of every adapter segment
-  const __nv_bfloat16* z;      // [total_rows][r] bf16 shrink output; null = none
-  int r;
-  const __nv_bfloat16* lora_b; // [L * E * r][delta_cols]: slot (adapter * E + group) rows
-  int L;
-  const int32_t* lseg_off;     // segment CSR, group g's candidates start at g * lseg_stride
-  int lseg_stride;
-  int lseg_count;              // candidates per group
-  const int32_t* lseg_adapter; // adapter of candidate c; null: adapter = c
   // optional stream-K scratch (used when the tiles are fewer than two per SM, N <= 64):
   // partial accumulators [sk_slots][128][BN] fp32 and flags [sk_slots], zero on entry
   float* sk_part;
   long long sk_part_cap;       // floats at sk_part
   int* sk_flag;
   int sk_slots;
-  // EPI_ZOUT (LoRA shrink on the tensor cores): tiles are work items (segment key, first
-  // row) of up to bn rows of one adapter segment; w = LoRA A as [L * E * r][K], b = the
-  // source rows, out_bf16 = z [total_rows][r]; lseg_off = the key CSR, L, r, iE = E
-  const int2* items;
-  const int* item_count;
-  int items_bound;
-  int iE;
+  // tests only: > 0 makes CTA 0 skip the copies of its first stage and shortens every
+  // bounded wait to this many milliseconds (the MMA's wait runs out: MOE_LORA_ERR_TIMEOUT)
+  int test_stall_ms;
+  // programmatic dependent launch: pdl_trigger lets the next kernel start right away;
+  // pdl_secondary launches the GEMM behind the running kernel ahead of it (the LoRA
+  // kernel that writes the fp32 delta): only the epilogue's loader waits for that kernel,
+  // so the weight stream and the MMAs start at once
+  int pdl_trigger;
+  int pdl_secondary;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
 
@@ -189,8 +234,14 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
 cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8_t* hi, uint8_t* lo, float* scales,
                                 cudaStream_t st);
 
-// y[t] = sum_j o[t*k + j]  (o already weighted), fixed j order, bf16 out.
-cudaError_t launch_combine(const float* o, int M, int k, int H, __nv_bfloat16* y, cudaStream_t st);
+// y[t] = sum_j (o[t*k + j] + w[t*k + j] delta[t*k + j])  (o bf16, already weighted; delta
+// in pair order, fp32 or bf16, optional), fixed j order, fp32 sum, bf16 out.
+cudaError_t launch_combine(const __nv_bfloat16* o, int M, int k, int H, const float* delta,
+                           const __nv_bfloat16* delta_bf16, const float* topk_w, __nv_bfloat16* y, cudaStream_t st);
+// The e4m3 activation planes of gathered rows (see launch_quant_planes): plane row i from
+// src[gather[i] / div].
+cudaError_t launch_gather_quant(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
+                                uint8_t* hi, uint8_t* lo, float* scales, cudaStream_t st);
 
 // Host state that CUDA keeps per device (function attributes, SM counts, capability)
 // is cached per device index, for processes that drive several GPUs.

@@ -258,6 +258,18 @@ __device__ __forceinline__ SegInfo segment_info(const LoraDeltaArgs& a, int q, b
   return si;
 }
 
+// Source row of gathered row s: gather[s] / gather_div, or s without a gather.  An index
+// outside [0, nsrc) (a corrupted pair index) is flagged and replaced by row 0.
+__device__ __forceinline__ int gather_src(const LoraDeltaArgs& a, int s) {
+  if (a.gather == nullptr) return s;
+  const int v = a.gather[s] / a.gather_div;
+  if (v < 0 || v >= a.nsrc) {
+    set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, s);
+    return 0;
+  }
+  return v;
+}
+
 // Partial shrink of one warp: rank rows i0 + istep g (g < LF_NI) over the 16-byte
 // chunks [c0, c1) of K, for the chunk's rows j < RB (rows j >= n repeat row 0 and
 // are dropped).  out[j * r + i] receives the warp's partial sums.
@@ -306,26 +318,66 @@ __device__ __forceinline__ void shrink_part(const __nv_bfloat16* aseg, const __n
     }
 }
 
-// delta[r0 + j][f..f+8) = sum_i z[j][i] B_i[f..f+8) for j < n; IB rows of B in flight.
+// Row of delta that gathered row s writes: s itself, or scatter[s] (the routing pair of
+// sorted row s, for a delta the combine reads in pair order).  An index outside
+// [0, nrows) is flagged and the row is not written (-1).
+__device__ __forceinline__ int delta_row(const LoraDeltaArgs& a, int s) {
+  if (a.scatter == nullptr) return s;
+  const int d = a.scatter[s];
+  if (d < 0 || d >= a.nrows) {
+    set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, s);
+    return -1;
+  }
+  return d;
+}
+
+// Where the expand reads B for delta features [f, f + 8): the column pointer, its row
+// stride, the B rows (rank) and the first z value they pair with.  Fused adapters: the
+// slot's r rows of NB features.  Separate gate and up adapters (split_I = I): the slot holds
+// the gate adapter's r_exp rows of I features, then the up adapter's; gate features pair
+// with z[0, r_exp), up features with z[r_exp, 2 r_exp).
+struct BCol {
+  const __nv_bfloat16* p;
+  int stride, zoff;
+};
+
+__device__ __forceinline__ BCol expand_bcol(const LoraDeltaArgs& a, size_t slot, int f) {
+  BCol c;
+  if (a.split_I == 0) {
+    c.p = a.lora_b + slot * a.r_exp * a.NB + f;
+    c.stride = a.NB;
+    c.zoff = 0;
+  } else {
+    const bool up = f >= a.split_I;
+    c.p = a.lora_b + (slot * 2 + (up ? 1 : 0)) * a.r_exp * a.split_I + (up ? f - a.split_I : f);
+    c.stride = a.split_I;
+    c.zoff = up ? a.r_exp : 0;
+  }
+  return c;
+}
+
+// delta[row(r0 + j)][f..f+8) = scale sum_i z[j][zoff + i] B_i[f..f+8) for j < n; IB rows of
+// B in flight.
 template <int RB, int IB>
-__device__ __forceinline__ void expand_thread(const LoraDeltaArgs& a, const __nv_bfloat16* bcol, const float* s_z,
-                                              int n, int r0, int f) {
+__device__ __forceinline__ void expand_thread(const LoraDeltaArgs& a, const BCol& bc, const float* s_z, int n,
+                                              int r0, int f) {
   float acc[RB][8];
 #pragma unroll
   for (int j = 0; j < RB; ++j)
 #pragma unroll
     for (int v = 0; v < 8; ++v) acc[j][v] = 0.f;
-  for (int i0 = 0; i0 < a.r; i0 += IB) {
+  for (int i0 = 0; i0 < a.r_exp; i0 += IB) {
     uint4 b8[IB];
 #pragma unroll
-    for (int u = 0; u < IB; ++u) b8[u] = __ldg(reinterpret_cast<const uint4*>(bcol + static_cast<size_t>(i0 + u) * a.NB));
+    for (int u = 0; u < IB; ++u)
+      b8[u] = __ldg(reinterpret_cast<const uint4*>(bc.p + static_cast<size_t>(i0 + u) * bc.stride));
 #pragma unroll
     for (int u = 0; u < IB; ++u) {
       float bf[8];
       unpack8_bf16(b8[u], bf);
 #pragma unroll
       for (int j = 0; j < RB; ++j) {
-        const float zj = s_z[j * a.r + i0 + u];
+        const float zj = s_z[j * a.r + bc.zoff + i0 + u];
 #pragma unroll
         for (int v = 0; v < 8; ++v) acc[j][v] = fmaf(zj, bf[v], acc[j][v]);
       }
@@ -333,10 +385,11 @@ __device__ __forceinline__ void expand_thread(const LoraDeltaArgs& a, const __nv
   }
 #pragma unroll
   for (int j = 0; j < RB; ++j) {
-    if (j < n) {
-      float4* d = reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f);
-      d[0] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-      d[1] = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+    const int row = j < n ? delta_row(a, r0 + j) : -1;
+    if (row >= 0) {
+      float4* d = reinterpret_cast<float4*>(a.delta + static_cast<size_t>(row) * a.NB + f);
+      d[0] = make_float4(a.scale * acc[j][0], a.scale * acc[j][1], a.scale * acc[j][2], a.scale * acc[j][3]);
+      d[1] = make_float4(a.scale * acc[j][4], a.scale * acc[j][5], a.scale * acc[j][6], a.scale * acc[j][7]);
     }
   }
 }
@@ -366,31 +419,31 @@ __device__ __forceinline__ void shrink_chunk(const LoraDeltaArgs& a, const __nv_
 
 // RBMAX = rows per chunk (the host's rb); 4 keeps the decode kernel at three CTAs per SM.
 template <int RBMAX>
-__global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(const LoraDeltaArgs a, int ks, int slice) {
+__device__ __forceinline__ void lora_fused_body(const LoraDeltaArgs& a, int item_idx, int ks, int slice, int* s_src,
+                                                float* s_z, float* s_part) {
   constexpr int rb = RBMAX;
-  __shared__ int s_src[LF_RB_MAX];
-  __shared__ float s_z[LF_RB_MAX * 128];
-  __shared__ float s_part[64 * LF_RB_MAX];  // ks * r == 64 whenever ks > 1
-  if (blockIdx.x >= *a.item_count) return;
-  const int2 item = a.items[blockIdx.x];
+  const int2 item = a.items[item_idx];
   SegInfo si = segment_info(a, item.x, false);
   si.lo = item.y;  // this CTA's chunk of the segment
   si.hi = min(si.hi, item.y + rb);
   const size_t K = a.K;
-  const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
+  const bool lora = a.delta != nullptr && a.r > 0;
   const bool do_gather = a.gather_dst != nullptr && blockIdx.y == 0;
   const bool do_quant = a.q_hi != nullptr && blockIdx.y == 0;
   if (!do_gather && !do_quant && !lora) return;
   const int f_lo = blockIdx.y * slice, f_hi = min(a.NB, f_lo + slice);
   const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
   const __nv_bfloat16* aseg = a.lora_a + slot * a.r * K;
-  const __nv_bfloat16* bseg = a.lora_b + slot * a.r * a.NB;
+  if (lora && a.split_I == 0 && si.ad >= 0 && threadIdx.x < a.r && f_hi > f_lo) {
+    // the expand's B rows head for L2 while the shrink streams A: the two loads overlap
+    prefetch_l2_bulk(a.lora_b + (slot * a.r + threadIdx.x) * a.NB + f_lo, static_cast<uint32_t>(f_hi - f_lo) * 2u);
+  }
   for (int c = blockIdx.z; si.lo + c * rb < si.hi; c += gridDim.z) {
     const int r0 = si.lo + c * rb;
     const int n = min(rb, si.hi - r0);
     __syncthreads();  // s_src / s_z of the previous chunk are no longer read
     if (threadIdx.x < LF_RB_MAX)
-      s_src[threadIdx.x] = (threadIdx.x < n) ? (a.gather ? a.gather[r0 + threadIdx.x] / a.gather_div : r0 + threadIdx.x) : 0;
+      s_src[threadIdx.x] = (threadIdx.x < n) ? gather_src(a, r0 + threadIdx.x) : 0;
     __syncthreads();
     if (do_gather) {
       const int c16 = a.K / 8;
@@ -413,7 +466,8 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
       const int w4 = (f_hi - f_lo) / 4;
       for (int idx = threadIdx.x; idx < n * w4; idx += blockDim.x) {
         const int j = idx / w4, cc = idx - j * w4;
-        reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f_lo)[cc] = z4;
+        const int row = delta_row(a, r0 + j);
+        if (row >= 0) reinterpret_cast<float4*>(a.delta + static_cast<size_t>(row) * a.NB + f_lo)[cc] = z4;
       }
       continue;
     }
@@ -423,23 +477,37 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
     else if (RBMAX == 4 || n <= 4) shrink_chunk<4, 1>(a, aseg, s_src, n, ks, s_part, s_z, 0, k8);
     else shrink_chunk<8, 1>(a, aseg, s_src, n, ks, s_part, s_z, 0, k8);
     __syncthreads();
-    if (a.z_out != nullptr) {  // shrink only: z rows (bf16) for the GEMM's expand steps
-      for (int idx = threadIdx.x; idx < n * a.r; idx += blockDim.x)
-        a.z_out[static_cast<size_t>(r0) * a.r + idx] = __float2bfloat16_rn(s_z[idx]);
-      continue;
-    }
     for (int f = f_lo + threadIdx.x * 8; f < f_hi; f += blockDim.x * 8) {
+      const BCol bc = expand_bcol(a, slot, f);
       if (n <= 1) {
-        expand_thread<1, 8>(a, bseg + f, s_z, n, r0, f);
+        expand_thread<1, 8>(a, bc, s_z, n, r0, f);
       } else if (n <= 2) {
-        expand_thread<2, 8>(a, bseg + f, s_z, n, r0, f);
+        expand_thread<2, 8>(a, bc, s_z, n, r0, f);
       } else if (RBMAX == 4 || n <= 4) {
-        expand_thread<4, 8>(a, bseg + f, s_z, n, r0, f);
+        expand_thread<4, 8>(a, bc, s_z, n, r0, f);
       } else {
-        expand_thread<8, 8>(a, bseg + f, s_z, n, r0, f);
+        expand_thread<8, 8>(a, bc, s_z, n, r0, f);
       }
     }
   }
+}
+
+// With programmatic dependent launch: the kernel behind this one (the GEMM that adds the
+// delta in its epilogue) may start at once, and a kernel launched behind another one
+// (pdl_end_wait) does not finish before that one has, so the launches after it still
+// see a completed stream.
+template <int RBMAX>
+__global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(const LoraDeltaArgs a, int ks, int slice) {
+  __shared__ int s_src[LF_RB_MAX];
+  __shared__ float s_z[LF_RB_MAX * 128];
+  __shared__ float s_part[64 * LF_RB_MAX];  // ks * r == 64 whenever ks > 1
+  if (a.pdl_trigger) pdl_trigger();
+  const int count = *a.item_count;  // a grid smaller than the work list walks it with a stride
+  for (int it = blockIdx.x; it < count; it += gridDim.x) {
+    lora_fused_body<RBMAX>(a, it, ks, slice, s_src, s_z, s_part);
+    __syncthreads();  // the next item reuses s_src / s_z
+  }
+  if (a.pdl_secondary) pdl_wait();
 }
 
 // ---- split form for adapters with long A rows (r K >= 64 Ki elements): the shrink runs
@@ -469,12 +537,16 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_shrink_part_kern
   const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
   const __nv_bfloat16* aseg = a.lora_a + slot * a.r * K;
   float* zp = a.z_part + static_cast<size_t>(blockIdx.y) * a.nrows * a.r;
+  if (a.delta != nullptr && a.split_I == 0 && si.ad >= 0 && blockIdx.y == 0 && threadIdx.x < a.r) {
+    // the expand kernel's B rows head for L2 while the shrink streams A
+    prefetch_l2_bulk(a.lora_b + (slot * a.r + threadIdx.x) * a.NB, static_cast<uint32_t>(a.NB) * 2u);
+  }
   for (int c = blockIdx.z; si.lo + c * rb < si.hi; c += gridDim.z) {
     const int r0 = si.lo + c * rb;
     const int n = min(rb, si.hi - r0);
     __syncthreads();
     if (threadIdx.x < LF_RB_MAX)
-      s_src[threadIdx.x] = (threadIdx.x < n) ? (a.gather ? a.gather[r0 + threadIdx.x] / a.gather_div : r0 + threadIdx.x) : 0;
+      s_src[threadIdx.x] = (threadIdx.x < n) ? gather_src(a, r0 + threadIdx.x) : 0;
     __syncthreads();
     if (do_gather) {
       for (int idx = threadIdx.x; idx < n * k8; idx += blockDim.x) {
@@ -511,7 +583,6 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_expand_part_kern
   si.hi = min(si.hi, item.y + rb);
   const int f_lo = blockIdx.y * slice, f_hi = min(a.NB, f_lo + slice);
   const size_t slot = static_cast<size_t>(si.ad < 0 ? 0 : si.ad) * a.E + si.e;
-  const __nv_bfloat16* bseg = a.lora_b + slot * a.r * a.NB;
   const size_t pstride = static_cast<size_t>(a.nrows) * a.r;
   for (int c = blockIdx.z; si.lo + c * rb < si.hi; c += gridDim.z) {
     const int r0 = si.lo + c * rb;
@@ -522,7 +593,8 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_expand_part_kern
       const int w4 = (f_hi - f_lo) / 4;
       for (int idx = threadIdx.x; idx < n * w4; idx += blockDim.x) {
         const int j = idx / w4, cc = idx - j * w4;
-        reinterpret_cast<float4*>(a.delta + static_cast<size_t>(r0 + j) * a.NB + f_lo)[cc] = z4;
+        const int row = delta_row(a, r0 + j);
+        if (row >= 0) reinterpret_cast<float4*>(a.delta + static_cast<size_t>(row) * a.NB + f_lo)[cc] = z4;
       }
       continue;
     }
@@ -532,15 +604,15 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_expand_part_kern
       float sum = 0.f;
       for (int ky = 0; ky < nks; ++ky) sum += __ldcg(zp + ky * pstride);
       s_z[idx] = sum;
-      if (a.z_out != nullptr && blockIdx.y == 0) a.z_out[static_cast<size_t>(r0) * a.r + idx] = __float2bfloat16_rn(sum);
     }
     __syncthreads();
     if (a.delta == nullptr) continue;
     for (int f = f_lo + threadIdx.x * 8; f < f_hi; f += blockDim.x * 8) {
-      if (n <= 1) expand_thread<1, 8>(a, bseg + f, s_z, n, r0, f);
-      else if (n <= 2) expand_thread<2, 8>(a, bseg + f, s_z, n, r0, f);
-      else if (RBMAX == 4 || n <= 4) expand_thread<4, 8>(a, bseg + f, s_z, n, r0, f);
-      else expand_thread<8, 8>(a, bseg + f, s_z, n, r0, f);
+      const BCol bc = expand_bcol(a, slot, f);
+      if (n <= 1) expand_thread<1, 8>(a, bc, s_z, n, r0, f);
+      else if (n <= 2) expand_thread<2, 8>(a, bc, s_z, n, r0, f);
+      else if (RBMAX == 4 || n <= 4) expand_thread<4, 8>(a, bc, s_z, n, r0, f);
+      else expand_thread<8, 8>(a, bc, s_z, n, r0, f);
     }
   }
 }
@@ -608,12 +680,11 @@ cudaError_t launch_lora_plan(const LoraDeltaArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_lora_plan_adapters(const LoraDeltaArgs& a, int rb, int2* items, int* count, int cap,
-                                      cudaStream_t st) {
-  if (a.nrows <= 0) return cudaSuccess;
+cudaError_t launch_lora_plan_all(const int32_t* seg_offsets, const int32_t* seg_adapter, int nseg, int L, int nrows,
+                                 int rb, int2* items, int* count, int cap, int* status, cudaStream_t st) {
+  if (nrows <= 0) return cudaSuccess;
   ProfScope ps(K_LORA, st);
-  lora_plan_kernel<<<1, 1024, 0, st>>>(a.seg_offsets, a.seg_adapter, a.nseg, a.L, a.nrows, rb, items, count, cap,
-                                       a.status, 1);
+  lora_plan_kernel<<<1, 1024, 0, st>>>(seg_offsets, seg_adapter, nseg, L, nrows, rb, items, count, cap, status, 0);
   count_launch();
   return cudaGetLastError();
 }
@@ -622,7 +693,7 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
   if (a.nrows <= 0) return cudaSuccess;
   if (a.r > 128 || a.r % 8 != 0 || a.NB % 8 != 0) return cudaErrorInvalidValue;
   if (a.items == nullptr || a.item_count == nullptr || (a.rb != 4 && a.rb != 8)) return cudaErrorInvalidValue;
-  const bool lora = (a.delta != nullptr || a.z_out != nullptr) && a.r > 0;
+  const bool lora = a.delta != nullptr && a.r > 0;
   if (!lora && a.gather_dst == nullptr && a.q_hi == nullptr) return cudaSuccess;  // nothing to do
   if (a.q_hi != nullptr && a.K % 16 != 0) return cudaErrorInvalidValue;
   const int bound = a.items_bound;
@@ -639,7 +710,8 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
   slice = (slice + 7) / 8 * 8;
   nsplit = (a.NB + slice - 1) / slice;
   const int nks = (a.K + LS_KSLICE - 1) / LS_KSLICE;
-  if (lora && a.z_part != nullptr && static_cast<long long>(a.r) * a.K >= 65536 && nks > 1 &&
+  const bool pdl = a.pdl_trigger || a.pdl_secondary;  // overlapped with a GEMM: one kernel
+  if (!pdl && lora && a.z_part != nullptr && static_cast<long long>(a.r) * a.K >= 65536 && nks > 1 &&
       static_cast<long long>(nks) * a.nrows * a.r <= a.z_part_cap) {
     ProfScope ps(K_LORA, st);
     dim3 g1(bound, nks);
@@ -652,9 +724,65 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
     return cudaGetLastError();
   }
   dim3 grid(bound, nsplit);
+  if (pdl) {
+    // running beside a GEMM (one CTA of it per SM): one persistent CTA per SM walks the
+    // work list, so that every CTA is resident at once (the GEMM behind a triggering
+    // kernel launches only when all of its CTAs have started) and fits beside the GEMM
+    grid = dim3(std::min(bound, std::max(1, a.num_sms)), 1);
+    slice = (a.NB + 7) / 8 * 8;
+  }
   ProfScope ps(K_LORA, st);
-  if (a.rb == 8) lora_fused_kernel<8><<<grid, 256, 0, st>>>(a, ks, slice);
-  else lora_fused_kernel<4><<<grid, 256, 0, st>>>(a, ks, slice);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl_secondary ? 1 : 0;
+  const cudaError_t e = a.rb == 8 ? cudaLaunchKernelEx(&cfg, lora_fused_kernel<8>, a, ks, slice)
+                                  : cudaLaunchKernelEx(&cfg, lora_fused_kernel<4>, a, ks, slice);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- row gather
+// dst[i] = src[gather[i] / div]: one warp per row, 16-byte loads and stores, four in
+// flight per lane.  A source index outside [0, nsrc) (corrupted pairs) gives a zero row.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int nsrc,
+                                                         const int32_t* __restrict__ gather, int div, int rows,
+                                                         int K, __nv_bfloat16* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * 8;
+  const int k8 = K / 8;
+  for (int row = blockIdx.x * 8 + (threadIdx.x >> 5); row < rows; row += nw) {
+    const int s = gather[row] / div;
+    const bool ok = s >= 0 && s < nsrc;
+    const uint4* sp = reinterpret_cast<const uint4*>(src + static_cast<size_t>(ok ? s : 0) * K);
+    uint4* dp = reinterpret_cast<uint4*>(dst + static_cast<size_t>(row) * K);
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    for (int c = lane; c < k8; c += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = (ok && c + 32 * u < k8) ? __ldg(sp + c + 32 * u) : z4;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c + 32 * u < k8) dp[c + 32 * u] = v[u];
+    }
+  }
+}
+
+cudaError_t launch_gather_rows(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
+                               __nv_bfloat16* dst, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (K % 8 != 0 || div <= 0) return cudaErrorInvalidValue;
+  int grid = (rows + 7) / 8;
+  if (grid > 148 * 8) grid = 148 * 8;
+  ProfScope ps(K_LORA, st);
+  gather_rows_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, dst);
   count_launch();
   return cudaGetLastError();
 }
@@ -808,6 +936,43 @@ __global__ void __launch_bounds__(256) quant_planes_kernel(const __nv_bfloat16* 
                    lo + static_cast<size_t>(row) * K, scales + 2 * static_cast<size_t>(row), lane);
 }
 
+// The e4m3 planes of gathered rows: row i of the planes is quantised from
+// src[gather[i] / div] (a zero row for an index outside [0, nsrc)).
+__global__ void __launch_bounds__(256) gather_quant_kernel(const __nv_bfloat16* __restrict__ src, int nsrc,
+                                                          const int32_t* __restrict__ gather, int div, int rows,
+                                                          int K, uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
+                                                          float* __restrict__ scales) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
+    const int sr = gather[row] / div;
+    if (sr < 0 || sr >= nsrc) {
+      for (int c = lane; c < K / 16; c += 32) {
+        reinterpret_cast<uint4*>(hi + static_cast<size_t>(row) * K)[c] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(lo + static_cast<size_t>(row) * K)[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (lane == 0) {
+        scales[2 * static_cast<size_t>(row)] = 0.f;
+        scales[2 * static_cast<size_t>(row) + 1] = 0.f;
+      }
+      continue;
+    }
+    quant_row_warp(src + static_cast<size_t>(sr) * K, K, hi + static_cast<size_t>(row) * K,
+                   lo + static_cast<size_t>(row) * K, scales + 2 * static_cast<size_t>(row), lane);
+  }
+}
+
+cudaError_t launch_gather_quant(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
+                                uint8_t* hi, uint8_t* lo, float* scales, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (K % 16 != 0 || div <= 0) return cudaErrorInvalidValue;
+  int grid = (rows + 7) / 8;
+  if (grid > 148 * 8) grid = 148 * 8;
+  ProfScope ps(K_QUANT, st);
+  gather_quant_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8_t* hi, uint8_t* lo, float* scales,
                                 cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
@@ -821,39 +986,69 @@ cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8
 }
 
 // ---------------------------------------------------------------- top-k combine
-// y[t, :] = sum_{j=0..k-1} o[t*k + j, :], summed in j order (run-to-run identical).
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o, int M, int k, int H,
+// y[t, :] = sum_{j=0..k-1} o[t*k + j, :], summed in fp32 in j order (run-to-run identical);
+// o holds the weighted per-pair outputs in bf16.  Thread = 8 features (16-byte loads).
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ o, int M, int k, int H,
+                                                     const float* __restrict__ delta,
+                                                     const __nv_bfloat16* __restrict__ delta_bf16,
+                                                     const float* __restrict__ topk_w,
                                                      __nv_bfloat16* __restrict__ y) {
   const int t = blockIdx.x;
-  const int f = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  const int f = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
   if (f >= H) return;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* base = o + static_cast<size_t>(t) * k * H + f;
+  float acc[8];
+#pragma unroll
+  for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+  const __nv_bfloat16* base = o + static_cast<size_t>(t) * k * H + f;
   for (int j0 = 0; j0 < k; j0 += 8) {  // 8 slot rows in flight, summed in slot order
-    float4 v[8];
+    uint4 v8[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u)
-      v[u] = (j0 + u < k) ? __ldg(reinterpret_cast<const float4*>(base + static_cast<size_t>(j0 + u) * H))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      v8[u] = (j0 + u < k) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(j0 + u) * H))
+                           : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (j0 + u < k) {
-        acc.x += v[u].x;
-        acc.y += v[u].y;
-        acc.z += v[u].z;
-        acc.w += v[u].w;
+        float fv[8];
+        unpack8_bf16(v8[u], fv);
+        if (delta != nullptr) {  // the down LoRA delta of the pair, weighted here
+          const size_t pr = static_cast<size_t>(t) * k + j0 + u;
+          const float w = topk_w[pr];
+          const float4* dp = reinterpret_cast<const float4*>(delta + pr * H + f);
+          const float4 d0 = __ldg(dp), d1 = __ldg(dp + 1);
+          fv[0] += w * d0.x;
+          fv[1] += w * d0.y;
+          fv[2] += w * d0.z;
+          fv[3] += w * d0.w;
+          fv[4] += w * d1.x;
+          fv[5] += w * d1.y;
+          fv[6] += w * d1.z;
+          fv[7] += w * d1.w;
+        } else if (delta_bf16 != nullptr) {
+          const size_t pr = static_cast<size_t>(t) * k + j0 + u;
+          const float w = topk_w[pr];
+          float dv[8];
+          unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(delta_bf16 + pr * H + f)), dv);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) fv[v] += w * dv[v];
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[v] += fv[v];
       }
     }
   }
-  uint2 out = make_uint2(pack2_bf16(acc.x, acc.y), pack2_bf16(acc.z, acc.w));
-  *reinterpret_cast<uint2*>(y + static_cast<size_t>(t) * H + f) = out;
+  *reinterpret_cast<uint4*>(y + static_cast<size_t>(t) * H + f) =
+      make_uint4(pack2_bf16(acc[0], acc[1]), pack2_bf16(acc[2], acc[3]), pack2_bf16(acc[4], acc[5]),
+                 pack2_bf16(acc[6], acc[7]));
 }
 
-cudaError_t launch_combine(const float* o, int M, int k, int H, __nv_bfloat16* y, cudaStream_t st) {
+cudaError_t launch_combine(const __nv_bfloat16* o, int M, int k, int H, const float* delta,
+                           const __nv_bfloat16* delta_bf16, const float* topk_w, __nv_bfloat16* y, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  dim3 grid(M, (H / 4 + 255) / 256);
+  if ((delta != nullptr || delta_bf16 != nullptr) && topk_w == nullptr) return cudaErrorInvalidValue;
+  dim3 grid(M, (H / 8 + 255) / 256);
   ProfScope ps(K_COMBINE, st);
-  combine_kernel<<<grid, 256, 0, st>>>(o, M, k, H, y);
+  combine_kernel<<<grid, 256, 0, st>>>(o, M, k, H, delta, delta_bf16, topk_w, y);
   count_launch();
   return cudaGetLastError();
 }

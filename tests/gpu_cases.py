@@ -59,7 +59,7 @@ def rel_err(y_gpu: torch.Tensor, y_ref: np.ndarray) -> float:
     return float(np.max(np.abs(yg - y_ref))) / max(denom, 1e-30) if y_ref.size else 0.0
 
 
-def run_moe_case(shape: synth.MoEShape, M: int, weights=None, tokens=None):
+def run_moe_case(shape: synth.MoEShape, M: int, weights=None, tokens=None, scale_gu=1.0, scale_d=1.0):
     """Route (from the given fp32 logits, so ids are comparable bit for bit) and
     forward on the GPU; the oracle on the same seeded inputs.
 
@@ -73,11 +73,12 @@ def run_moe_case(shape: synth.MoEShape, M: int, weights=None, tokens=None):
     lin = synth.moe_logits_in(shape, M)
     rt = ml.route(add, shape.k, shape.L, logits_in=lin.cuda())
     ids, w, sp, so = oracle_routing_from_logits(lin, ad_np, shape.E, shape.k, shape.L)
-    y = ml.forward(xd, rt, dev, k=shape.k, L=shape.L)
+    y = ml.forward(xd, rt, dev, k=shape.k, L=shape.L, scale_gu=scale_gu, scale_d=scale_d)
     torch.cuda.synchronize()
     x64 = formats.to_f64(synth.bits(x), "bf16")
     sel = np.arange(M) if tokens is None else np.asarray(tokens)
-    y_ref = ref.moe_lora_forward(x64, ids, w, ad_np, shape.I, OW.expert, OW.adapter, tokens=sel)
+    y_ref = ref.moe_lora_forward(x64, ids, w, ad_np, shape.I, OW.expert, OW.adapter, tokens=sel,
+                                 scale_gu=scale_gu, scale_d=scale_d)
     return dict(rt=rt, y=y, ids=ids, w=w, sp=sp, so=so, y_ref=y_ref, tokens=sel,
                 err=rel_err(y[torch.as_tensor(sel, dtype=torch.long, device=y.device)], y_ref),
                 x=x, ad=ad, dev=dev)

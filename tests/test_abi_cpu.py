@@ -50,12 +50,12 @@ def test_workspace_sizes():
 def _fwd(**kw):
     a = dict(x=FAKE, M=4, H=64, I=64, E=4, k=2, L=2, r=16, topk_w=FAKE, sorted_pairs=FAKE,
              seg_offsets=FAKE, w_gu=FAKE, w_d=FAKE, wdt=ml.ML_BF16, scales=None, agu=FAKE, bgu=FAKE,
-             ad=FAKE, bd=FAKE, y=FAKE, ws=FAKE, wsb=1 << 30)
+             ad=FAKE, bd=FAKE, fmt=None, y=FAKE, ws=FAKE, wsb=1 << 30)
     a.update(kw)
     return ml.lib().moe_lora_forward(a["x"], a["M"], a["H"], a["I"], a["E"], a["k"], a["L"], a["r"],
                                      a["topk_w"], a["sorted_pairs"], a["seg_offsets"], a["w_gu"], a["w_d"],
-                                     a["wdt"], a["scales"], a["agu"], a["bgu"], a["ad"], a["bd"], a["y"],
-                                     a["ws"], a["wsb"], None)
+                                     a["wdt"], a["scales"], a["agu"], a["bgu"], a["ad"], a["bd"], a["fmt"],
+                                     a["y"], a["ws"], a["wsb"], None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -73,6 +73,8 @@ def _fwd(**kw):
     (dict(wdt=7), ml.ERR_INVALID_ARG),
     (dict(agu=None), ml.ERR_INVALID_ARG),       # adapters present but A missing
     (dict(seg_offsets=MIS), ml.ERR_INVALID_ARG),
+    (dict(fmt=ctypes.pointer(ml.AdapterFormat(2, 1.0, 1.0))), ml.ERR_INVALID_ARG),   # bad layout
+    (dict(fmt=ctypes.pointer(ml.AdapterFormat(1, 1.0, 1.0)), r=128), ml.ERR_UNSUPPORTED),  # split: r <= 64
 ])
 def test_forward_host_validation(kw, code):
     assert _fwd(**kw) == code

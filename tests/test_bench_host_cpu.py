@@ -27,22 +27,27 @@ def test_routing_stats_counts_touched_experts_and_pairs():
     assert bench.routing_stats({"seg_offsets": so}, shape) == (2, 2)
 
 
-def test_expand_placement_boundary():
+def test_lora_placement_boundary(monkeypatch):
+    monkeypatch.delenv("MOE_LORA_EXPAND", raising=False)
     s = synth.MOE_DECODE_BF16  # E = 64, k = 8: more than 64 rows per expert above M = 512
-    assert not bench.expand_in_gemm(s, 512)
-    assert bench.expand_in_gemm(s, 513)
+    assert bench.lora_place(s, 512) == "delta"
+    assert bench.lora_place(s, 513) == "tc"
+    monkeypatch.setenv("MOE_LORA_EXPAND", "tc")
+    assert bench.lora_place(s, 1) == "tc"
 
 
-def test_gateup_bytes_hand_counted():
+def test_gateup_bytes_hand_counted(monkeypatch):
+    monkeypatch.delenv("MOE_LORA_EXPAND", raising=False)
     # delta form (3 rows <= 64 per expert): weights 2*2I*H*2 = 256, x 3*H*2 = 48,
     # fp32 delta 3*2I*4 = 96, act 3*I*2 = 24
     assert bench.gateup_alg_bytes(TINY, 3, experts=2, pairs=1) == 256 + 48 + 96 + 24
     # e4m3 weights: 1 byte per weight, x as two planes plus two fp32 scales per row
     f8 = TINY.with_(wdtype="e4m3")
     assert bench.gateup_alg_bytes(f8, 3, experts=2, pairs=1) == 128 + 3 * (2 * 8 + 8) + 96 + 24
-    # expand inside the GEMM (100 rows on one expert): z rows 100*r*2 and the B slice r*2I*2
+    # tensor-core LoRA kernel (100 rows on one expert): the bf16 delta 100*2I*2
     one = TINY.with_(E=1)
-    assert bench.gateup_alg_bytes(one, 100, experts=1, pairs=1) == 128 + 1600 + (400 + 32) + 800
+    assert bench.gateup_alg_bytes(one, 100, experts=1, pairs=1) == 128 + 1600 + 1600 + 800
+    assert bench.gateup_alg_flops(one, 100) == 2 * 100 * 8 * 8
 
 
 def test_layer_bytes_hand_counted():

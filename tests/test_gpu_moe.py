@@ -35,11 +35,12 @@ def test_forward_small_shapes(shape, M):
     assert res["err"] <= TOL_BF16, res["err"]
 
 
-@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("where", ["delta", "tc"])
 @pytest.mark.parametrize("bn", [16, 32, 64, 128, 256])
 def test_forward_every_n_tile(bn, where, monkeypatch):
-    """Every N tile, with the LoRA expand both as extra MMA K steps of the GEMM and as
-    the fp32 delta of the LoRA kernel added by the GEMM epilogue."""
+    """Every N tile, with the LoRA expand as extra MMA K steps of the GEMM, as the fp32
+    delta of the SIMT LoRA kernel and as the bf16 delta of the tensor-core LoRA kernel,
+    each added by the GEMM epilogue."""
     monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
     res = run_moe_case(SMALL[0], 300)
@@ -48,12 +49,12 @@ def test_forward_every_n_tile(bn, where, monkeypatch):
     assert res["err"] <= TOL_BF16, res["err"]
 
 
-@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("where", ["delta", "tc"])
 @pytest.mark.parametrize("shape,M", [(SMALL[1], 37), (SMALL[2], 300), (SMALL[3], 37), (SMALL[7], 37),
                                      (SMALL[8], 300), (SMALL[8], 1), (SMALL[9], 37), (SMALL[9], 300)],
                          ids=lambda v: getattr(v, "name", str(v)))
 def test_forward_expand_placement(shape, M, where, monkeypatch):
-    """Both placements of the LoRA expand on ragged shapes, r = 8 .. 128, E = 1."""
+    """Every placement of the LoRA work on ragged shapes, r = 8 .. 128, E = 1."""
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
     res = run_moe_case(shape, M)
     assert res["err"] <= TOL_BF16, res["err"]
@@ -70,7 +71,7 @@ def test_forward_stream_k(shape, M, monkeypatch):
     assert res["err"] <= TOL_BF16, res["err"]
 
 
-@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("where", ["delta", "tc"])
 @pytest.mark.parametrize("bn", [128, 256])
 def test_forward_cta_pairs(bn, where, monkeypatch):
     """N tiles of 128 / 256 on CTA pairs (tcgen05 cta_group::2): each CTA holds its 128
@@ -140,6 +141,53 @@ def test_forward_moe_prefill_bf16_full(prefill_weights):
     ml.check_status(res["rt"]["workspace"])
 
 
+# ---------------------------------------------------------------- adapter formats: separate
+# gate and up adapters, per-projection scales
+SPLIT = [
+    synth.MoEShape("sp_a", 230, E=8, k=2, H=384, I=192, L=3, r=16, gu_split=True, no_adapter_frac=0.2),
+    synth.MoEShape("sp_r64", 231, E=4, k=2, H=256, I=128, L=4, r=64, gu_split=True, adapter_dist="zipf"),
+    synth.MoEShape("sp_r8", 232, E=6, k=3, H=520, I=256, L=2, r=8, gu_split=True, no_adapter_frac=0.25),
+]
+
+
+@pytest.mark.parametrize("where", ["delta", "tc"])
+@pytest.mark.parametrize("shape", SPLIT, ids=lambda s: s.name)
+@pytest.mark.parametrize("M", [37, 300])
+def test_forward_split_gate_up_with_scales(shape, M, where, monkeypatch):
+    monkeypatch.setenv("MOE_LORA_EXPAND", where)
+    res = run_moe_case(shape, M, scale_gu=0.5, scale_d=2.0)
+    assert res["err"] <= TOL_BF16, res["err"]
+
+
+def test_forward_split_ragged_intermediate_decode():
+    """Separate gate and up adapters with I not a multiple of 64 (the CUDA-core LoRA path)."""
+    s = synth.MoEShape("sp_ragged", 233, E=6, k=3, H=520, I=136, L=2, r=32, gu_split=True)
+    res = run_moe_case(s, 37, scale_gu=1.5, scale_d=0.25)
+    assert res["err"] <= TOL_BF16, res["err"]
+
+
+@pytest.mark.parametrize("M", [64, 1024])
+def test_forward_split_decode_bf16_shape(M):
+    """The bf16 decode layer's shape (E=64, H=2048, I=1408) with separate gate and up
+    adapters and scales: M=64 runs the CUDA-core LoRA path, M=1024 (128 rows per expert)
+    the tensor-core one."""
+    s = synth.MOE_DECODE_BF16.with_(name="decode_split", wid=234, gu_split=True)
+    res = run_moe_case(s, M, scale_gu=0.25, scale_d=0.5)
+    assert res["err"] <= TOL_BF16, res["err"]
+
+
+def test_forward_split_prefill_shape_sampled():
+    """The prefill layer's shape (M=4096, E=128, H=4096, I=1536, r=64) with separate gate
+    and up adapters and scales, on 320 tokens the oracle computes one by one."""
+    s = synth.MOE_PREFILL_BF16.with_(name="prefill_split", wid=235, gu_split=True)
+    toks = np.unique(np.concatenate([np.arange(32), np.arange(4096 - 32, 4096),
+                                     np.random.default_rng(2).choice(4096, 256, replace=False)]))
+    cpu, dev, _ = moe_weights_both(s)
+    res = run_moe_case(s, 4096, weights=(cpu, dev, CpuWeightsOracle(s, cpu, cache=False)), tokens=toks,
+                       scale_gu=2.0, scale_d=0.5)
+    assert res["err"] <= TOL_BF16, res["err"]
+
+
 # ---------------------------------------------------------------- FP8 (e4m3) expert weights
 def check_fp8(res, label, record_property):
     """The stated FP8 gate and the tighter bound of the two-plane activation design;
@@ -164,7 +212,7 @@ def test_forward_fp8_small_shapes(shape, M, record_property):
     check_fp8(run_moe_case(shape, M), f"{shape.name} M={M}", record_property)
 
 
-@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("where", ["delta", "tc"])
 @pytest.mark.parametrize("bn", [16, 32, 64, 256])
 def test_forward_fp8_every_n_tile(bn, where, monkeypatch, record_property):
     monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))

@@ -51,11 +51,12 @@ def test_sgmv_shrink_expand(s):
     assert rel_err(y0, d_ref) <= (1e-5 if s.dtype == "f32" else 1e-2)
 
 
-@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("where", ["delta", "tc"])
 @pytest.mark.parametrize("s", CASES, ids=lambda s: s.name)
 def test_dense_lora_forward(s, where, monkeypatch):
-    """bf16: the expand both inside the GEMM (extra MMA K steps) and as the LoRA
-    kernel's delta added by the GEMM epilogue (fp32 cases take the SIMT path)."""
+    """bf16: the expand inside the GEMM (extra MMA K steps), as the SIMT LoRA kernel's
+    fp32 delta and as the tensor-core LoRA kernel's bf16 delta, each added by the GEMM
+    epilogue (fp32 cases take the SIMT path)."""
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
     d = dense_f64(s)
     y = ml.dense_lora_forward(d["x"].cuda(), d["w"]["w"].cuda(), d["w"]["a"].cuda(), d["w"]["b"].cuda(),
@@ -100,11 +101,11 @@ def test_sgmv_bad_adapter_sets_status():
     assert ei.value.status == ml.ERR_DEVICE_CHECK
 
 
-@pytest.mark.parametrize("where", ["gemm", "delta"])
+@pytest.mark.parametrize("where", ["delta", "tc"])
 def test_dense_many_segments(where, monkeypatch):
     """Tokens in arrival order (not grouped by adapter): every maximal run of one adapter
-    is a segment, ~200 of them, so a 256-token tile meets more than 64 segments (the
-    GEMM's segment scan then also walks candidates one by one)."""
+    is a segment, ~200 of them, interleaved with segments without an adapter, so the
+    LoRA work list holds ~200 short items and one GEMM tile meets many of them."""
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
     s = synth.DENSE_DECODE_BF16.with_(name="bf16_many_segs", wid=305, T=300, h_in=256, h_out=640, L=4,
                                       r=64, adapter_dist="uniform")
