@@ -46,11 +46,6 @@
  *   MOE_LORA_FORCE_BN=16|32|64|128|256  the GEMM's token tile (default: from the mean rows
  *                               per group: <= 12 -> 16, <= 24 -> 32, <= 64 -> 64, <= 96 -> 128,
  *                               else 256).
- *   MOE_LORA_STREAMK=1          stream-K split of the GEMM's (tile, K stage) iterations over
- *                               all SMs when there are fewer than two tiles per SM (off by
- *                               default: measured slower on the dense decode GEMM).
- *   MOE_LORA_PAIR=1             N tiles of 128/256 on CTA pairs (tcgen05 cta_group::2, M = 256;
- *                               off by default: measured slower at prefill).
  */
 #ifndef MOE_LORA_H
 #define MOE_LORA_H

@@ -180,16 +180,8 @@ int shrink_rows_per_cta(long long rows) {
   return static_cast<int>(rb);
 }
 
-// Stream-K scratch of the grouped GEMM (few tiles): flags right after the status word,
-// so the per-call clear of the status also re-arms them, and the partial accumulators.
-constexpr int kSkSlots = 160;                       // >= SMs of the device
-constexpr size_t kSkFlagBytes = kSkSlots * 4;
-constexpr size_t kSkPartFloats = static_cast<size_t>(kSkSlots) * 128 * 64;
-
 struct ForwardWs {
   int* status;
-  int* sk_flag;
-  float* sk_part;
   __nv_bfloat16* x_sorted;
   __nv_bfloat16* act;
   float* delta_gu;     // expand in the LoRA kernel: deltas the GEMM epilogues add
@@ -200,7 +192,7 @@ struct ForwardWs {
   long long z_part_cap;
   int2* items;         // LoRA work list and its length
   int* item_count;
-  int2* items_tc;      // expand in the GEMMs: tiles of the tensor-core shrink (adapter segments)
+  int2* items_tc;      // tensor-core LoRA kernel: chunks of <= 128 rows of each segment
   int* item_count_tc;
   __nv_bfloat16* o;   // per-pair weighted outputs [M*k][H], summed by the combine
   uint8_t* q_hi;      // e4m3 weights: activation planes [M*k][max(H, I)]
@@ -221,7 +213,6 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
     return p;
   };
   w.status = reinterpret_cast<int*>(b);
-  w.sk_flag = reinterpret_cast<int*>(take(mk > 0 ? kSkFlagBytes : 0));  // must stay first
   w.x_sorted = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
   w.act = reinterpret_cast<__nv_bfloat16*>(take(mk * I * 2));
   w.delta_gu = reinterpret_cast<float*>(take(dl ? mk * 2 * I * 4 : 0));
@@ -236,7 +227,6 @@ ForwardWs forward_layout(void* base, int M, int H, int I, int k, int r, bool fp8
   w.items_tc = reinterpret_cast<int2*>(
       take(tc ? static_cast<size_t>(lora_items_bound(static_cast<int>(mk), nkeys, kLtN)) * 8 : 0));
   w.item_count_tc = reinterpret_cast<int*>(take(tc ? 4 : 0));
-  w.sk_part = reinterpret_cast<float*>(take(mk > 0 ? kSkPartFloats * 4 : 0));
   w.o = reinterpret_cast<__nv_bfloat16*>(take(mk * H * 2));
   const size_t kmax = H > I ? H : I;
   w.q_hi = reinterpret_cast<uint8_t*>(take(fp8 ? mk * kmax : 0));
@@ -274,8 +264,6 @@ RouteWs route_layout(void* base, int M, int E, int L) {
 
 struct DenseWs {
   int* status;
-  int* sk_flag;         // bf16 path: stream-K scratch (see ForwardWs)
-  float* sk_part;
   float* z;             // fp32 path: shrink output
   int32_t* row_adapter; // fp32 path
   float* delta;         // bf16 path, expand in the LoRA kernel: delta the GEMM adds
@@ -284,7 +272,7 @@ struct DenseWs {
   long long z_part_cap;
   int2* items;          // bf16 path: LoRA work list and its length
   int* item_count;
-  int2* items_tc;       // bf16 path, expand in the GEMM: tiles of the tensor-core shrink
+  int2* items_tc;       // bf16 path, tensor-core LoRA kernel: its work list
   int* item_count_tc;
   size_t bytes;
 };
@@ -300,7 +288,6 @@ DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, Lo
     return p;
   };
   w.status = reinterpret_cast<int*>(b);
-  if (!f32) w.sk_flag = reinterpret_cast<int*>(take(T > 0 ? kSkFlagBytes : 0));  // must stay first
   if (f32) {
     w.z = reinterpret_cast<float*>(take(static_cast<size_t>(T) * r * 4));
     w.row_adapter = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * 4));
@@ -313,7 +300,6 @@ DenseWs dense_layout(void* base, int T, int h_in, int h_out, int r, bool f32, Lo
     w.item_count = reinterpret_cast<int*>(take(T > 0 ? 4 : 0));
     w.items_tc = reinterpret_cast<int2*>(take(tc ? static_cast<size_t>(lora_items_bound(T, T, kLtN)) * 8 : 0));
     w.item_count_tc = reinterpret_cast<int*>(take(tc ? 4 : 0));
-    w.sk_part = reinterpret_cast<float*>(take(T > 0 ? kSkPartFloats * 4 : 0));
   }
   w.bytes = off;
   return w;
@@ -543,8 +529,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   const bool tcl = rr && place == LORA_TC;  // tensor-core LoRA kernel, bf16 deltas
   const int mk = M * k;
   const int nkeys = E * (L + 1);
-  // status word and the stream-K flags that follow it
-  ML_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes + kSkFlagBytes, cs), "status clear");
+  ML_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes, cs), "status clear");
 
   // 1. gather x rows into (expert, adapter) order, and the gate_up LoRA:
   //    LORA_DELTA: one SIMT kernel gathers, shrinks z = x A_gu per (adapter, expert)
@@ -663,10 +648,6 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     g.b_scales = w.q_scales;
   }
   g.num_sms = num_sms();
-  g.sk_part = w.sk_part;
-  g.sk_part_cap = static_cast<long long>(kSkPartFloats);
-  g.sk_flag = w.sk_flag;
-  g.sk_slots = kSkSlots;
   // tests only: the gate_up GEMM's first stage in CTA 0 never arrives and every bounded
   // wait is shortened to MOE_LORA_TEST_STALL milliseconds (exercises the abort path)
   g.test_stall_ms = env_int("MOE_LORA_TEST_STALL", 0);
@@ -854,7 +835,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const DenseWs ws = dense_layout(workspace, T, h_in, h_out, rr, f32, place);
   const bool tcl = rr && place == LORA_TC;  // tensor-core LoRA kernel, bf16 delta
-  ML_CUDA(cudaMemsetAsync(workspace, 0, f32 ? 8 : kStatusBytes + kSkFlagBytes, cs), "status clear");
+  ML_CUDA(cudaMemsetAsync(workspace, 0, f32 ? 8 : kStatusBytes, cs), "status clear");
 
   if (f32) {
     ShrinkArgs a{};
@@ -916,6 +897,8 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     l.items_bound = lora_items_bound(T, S, l.rb);
     l.items = ws.items;
     l.item_count = ws.item_count;
+    l.r_exp = rr;
+    l.scale = 1.f;  // the dense adapters carry their scale in B
     if (tcl) {  // shrink and expand on the tensor cores, bf16 delta for the epilogue
       const int bound = lora_items_bound(T, S, kLtN);
       ML_CUDA(launch_lora_plan_all(seg_offsets, seg_adapter, S, L, T, kLtN, ws.items_tc, ws.item_count_tc, bound,
@@ -941,6 +924,8 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
       t.status = ws.status;
       t.work_counter = ws.status + 2;  // inside the status block: cleared with it by every call
       t.num_sms = num_sms();
+      t.r_exp = rr;
+      t.scale = 1.f;
       ML_CUDA(launch_lora_tc(t, cs), "dense tensor-core LoRA launch");
     } else {
       // the LoRA kernel lets the GEMM start at once: the GEMM streams W while it runs,
@@ -971,10 +956,6 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   g.pdl_secondary = rr && place == LORA_DELTA ? 1 : 0;
 
   g.num_sms = num_sms();
-  g.sk_part = ws.sk_part;
-  g.sk_part_cap = static_cast<long long>(kSkPartFloats);
-  g.sk_flag = ws.sk_flag;
-  g.sk_slots = kSkSlots;
   ML_CUDA(launch_gemm_tc(g, cs), "dense GEMM launch");
   return MOE_LORA_OK;
 }

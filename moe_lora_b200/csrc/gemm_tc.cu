@@ -52,7 +52,6 @@ constexpr int kEpiThreads = 128;
 constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMaxGroups = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-constexpr int kPfDist = 8;                         // stages of L2 prefetch lead
 
 struct TcParams {
   int epi;
@@ -78,14 +77,6 @@ struct TcParams {
   const float* b_scales;  // e4m3: [rows][2] = (s, s / 16) of the activation planes
   int m_tiles;
   int stages;
-  // stream-K (few tiles): CTA b takes the (tile, K stage) iterations
-  // [b T / G, (b + 1) T / G) of T = tiles * stages; a CTA that starts inside a tile writes
-  // its partial accumulator to sk_part[b] and raises sk_flag[b]; the CTA holding the
-  // tile's first stages adds the partials in CTA order and runs the epilogue
-  int sk;
-  float* sk_part;               // [grid][128][BN] fp32
-  int* sk_flag;                 // [grid], zero on entry, zero again on exit
-  int m_tiles2;                 // CTA pairs: pairs of 128-row tiles
   // limit of every bounded wait (ns); test_stall: CTA 0 never issues the copies of its
   // first stage, so the MMA's wait runs out and the abort path runs (tests only)
   uint64_t wait_ns;
@@ -97,56 +88,29 @@ struct TcParams {
   // streams faster than 128-byte runs
   int kpb;
   int stage_bytes;    // kpb * TileCfg::kStageBytes
-  int l2_prefetch;    // prefetch boxes kPfDist stages ahead into L2
 };
 
-// A unit of work: tile t, K stages [k0, k1).
+// A unit of work: tile t, K stages [k0, k1) (every unit is a whole tile).
 struct Unit {
   int t, k0, k1;
 };
 struct UnitIter {
-  long long pos, end;
   int t;
 };
 
-__device__ __forceinline__ long long sk_start(long long b, long long T, long long G) { return b * T / G; }
-// CTA whose stream-K range holds iteration i
-__device__ __forceinline__ int sk_owner(long long i, long long T, long long G) {
-  return static_cast<int>(((i + 1) * G + T - 1) / T - 1);
-}
-
-// CTA bb's stream-K range is non-empty (it holds at least one iteration)
-__device__ __forceinline__ bool sk_busy(long long bb, long long T, long long G) {
-  return sk_start(bb, T, G) < sk_start(bb + 1, T, G);
-}
-
-// CTA pairs: unit index space is per cluster (two CTAs walk the same units)
-__device__ __forceinline__ int unit_cta(const TcParams& p) { return p.m_tiles2 ? blockIdx.x >> 1 : blockIdx.x; }
-__device__ __forceinline__ int unit_ctas(const TcParams& p) { return p.m_tiles2 ? gridDim.x >> 1 : gridDim.x; }
-
-__device__ __forceinline__ UnitIter unit_begin(const TcParams& p, int total_tiles, int nk) {
+__device__ __forceinline__ UnitIter unit_begin() {
   UnitIter it;
-  it.t = unit_cta(p);
-  const long long T = static_cast<long long>(total_tiles) * nk;
-  it.pos = sk_start(blockIdx.x, T, gridDim.x);
-  it.end = sk_start(blockIdx.x + 1, T, gridDim.x);
+  it.t = blockIdx.x;
   return it;
 }
 
-__device__ __forceinline__ bool unit_next(const TcParams& p, int total_tiles, int nk, UnitIter& it, Unit& u) {
-  if (!p.sk) {
-    if (it.t >= total_tiles) return false;
-    u.t = it.t;
-    u.k0 = 0;
-    u.k1 = nk;
-    it.t += unit_ctas(p);
-    return true;
-  }
-  if (it.pos >= it.end) return false;
-  u.t = static_cast<int>(it.pos / nk);
-  u.k0 = static_cast<int>(it.pos - static_cast<long long>(u.t) * nk);
-  u.k1 = static_cast<int>(min(static_cast<long long>(nk), u.k0 + (it.end - it.pos)));
-  it.pos += u.k1 - u.k0;
+// persistent tile loop: CTA b takes tiles b, b + G, b + 2 G, ...
+__device__ __forceinline__ bool unit_next(int total_tiles, int nk, UnitIter& it, Unit& u) {
+  if (it.t >= total_tiles) return false;
+  u.t = it.t;
+  u.k0 = 0;
+  u.k1 = nk;
+  it.t += gridDim.x;
   return true;
 }
 
@@ -183,13 +147,10 @@ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-// TWO: the CTA pair (cta_group::2) computes 256 weight rows x BN tokens; each CTA holds
-// its 128 weight rows and half of the BN token rows.
-template <int BN, bool W8, bool TWO = false>
+template <int BN, bool W8>
 struct TileCfg {
   static constexpr int kKB = W8 ? 128 : 64;                  // K per stage (128 bytes per row)
-  static constexpr int kBRows = TWO ? BN / 2 : BN;           // token rows held by this CTA
-  static constexpr int kBTileBytes = kBRows * 128;           // one token tile (or plane)
+  static constexpr int kBTileBytes = BN * 128;               // one token tile (or plane)
   static constexpr int kStageBytes = kATileBytes + (W8 ? 2 : 1) * kBTileBytes;
   static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
   static constexpr int kAccPerBuf = W8 ? 2 : 1;              // e4m3: hi and lo side by side (N = 2 BN)
@@ -198,7 +159,6 @@ struct TileCfg {
   static constexpr int kSlotBytes = static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024);
   static constexpr int kThreads = 224;
   static_assert(!W8 || kPrefetch, "e4m3 weights use N tiles <= 64");
-  static_assert(!TWO || (!W8 && BN >= 128), "CTA pairs: bf16 weights, N tiles of 128 or 256");
 };
 
 struct TileInfo {
@@ -227,13 +187,13 @@ __device__ __forceinline__ int delta_col(int epi, int m, int f0, int I) {
   return f0 + m;
 }
 
-template <int BN, bool W8, bool TWO>
-__global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
+template <int BN, bool W8>
+__global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tml, const __grid_constant__ CUtensorMap tmd,
                    const TcParams p) {
   // tml: the lo activation plane (e4m3 weights); tmd: the fp32 LoRA delta (N tiles <= 64)
-  using Cfg = TileCfg<BN, W8, TWO>;
+  using Cfg = TileCfg<BN, W8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;                                 // stages: [A tile][token tile(s)]
@@ -242,21 +202,17 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
   volatile int* abort_flag = &sm.abort_flag;
-  // CTA pairs: rank 0 (leader) issues the MMAs for both; the barriers the MMA consumes
-  // live in the leader's shared memory
-  const uint32_t rank = TWO ? cluster_ctarank() : 0;
-  auto leader_bar = [&](uint64_t* bar) -> uint32_t { return TWO ? mapa_shared(smem_u32(bar), 0) : smem_u32(bar); };
 
   if (p.pdl_trigger) pdl_trigger();
   // ---- setup: barriers, TMEM, tile list prefix
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&sm.full[s], TWO ? 2 : 1);  // pair: the leader's and the peer's producer
+      mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
-      mbar_init(&sm.tempty[b], TWO ? 2 * kEpiThreads : kEpiThreads);
+      mbar_init(&sm.tempty[b], kEpiThreads);
       mbar_init(&sm.sfull[b], 1);
       mbar_init(&sm.sempty[b], kEpiThreads);
     }
@@ -270,10 +226,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     if (W8) tma_prefetch_desc(&tml);
     if (p.delta != nullptr) tma_prefetch_desc(&tmd);
   }
-  if (warp == 1) {
-    if constexpr (TWO) tmem_alloc_pair(&sm.tmem_base, Cfg::kTmemCols);
-    else tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
-  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
   // group offsets clamped to [0, total_rows]: offsets that are out of range or not
   // monotone (flagged by the work-list kernel) can leave rows uncomputed, never make a
   // tile reach outside the operands
@@ -312,17 +265,11 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     if (lane == 31) sm.chunk_pref[p.E] = incl;
   }
   tc_fence_before();
-  if constexpr (TWO) cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
-  else __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
-  const int total_tiles = sm.chunk_pref[p.E] * (TWO ? p.m_tiles2 : p.m_tiles);
-  // this CTA's tile of a unit (pairs: the unit is a pair of 128-row tiles, rank picks one)
-  auto tile_of = [&](int t) -> TileInfo {
-    TileInfo ti = decode_tile(sm, t, TWO ? p.m_tiles2 : p.m_tiles, p.E, BN);
-    if constexpr (TWO) ti.mt = 2 * ti.mt + static_cast<int>(rank);
-    return ti;
-  };
+  const int total_tiles = sm.chunk_pref[p.E] * p.m_tiles;
+  auto tile_of = [&](int t) -> TileInfo { return decode_tile(sm, t, p.m_tiles, p.E, BN); };
   const int nk = (p.K + Cfg::kKB * p.kpb - 1) / (Cfg::kKB * p.kpb);  // stages per tile
 
   if (warp == 0) {
@@ -334,10 +281,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     uint32_t phase = 0;
     uint32_t filled_mask = 0, last_parity = 0;
     bool ok = true;
-    UnitIter uit = unit_begin(p, total_tiles, nk);
+    UnitIter uit = unit_begin();
     Unit u;
     int itp = 0;  // unit index, the same sequence as the MMA thread's
-    while (ok && unit_next(p, total_tiles, nk, uit, u)) {
+    while (ok && unit_next(total_tiles, nk, uit, u)) {
       if (*abort_flag) break;
       const TileInfo ti = tile_of(u.t);
       int wrow0, wrow1;
@@ -355,42 +302,17 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
         const bool stall = p.test_stall && blockIdx.x == 0 && itp == 0 && kb == u.k0;  // never arrives
         if (lane == 0 && !stall) {
           uint8_t* a_s = ring + stage * p.stage_bytes;
-          uint8_t* b_s = a_s + kATileBytes;
           const int kc = kb * Cfg::kKB * p.kpb;  // first K element of the stage
-          if constexpr (TWO) {
-            // both CTAs' copies complete on the leader's barrier: the leader expects the
-            // pair's bytes, the peer adds its arrival
-            const uint32_t fb = leader_bar(&sm.full[stage]);
-            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2 * Cfg::kStageBytes);
-            tma_load_2d_pair(a_s, &tmw, fb, kc, wrow0);
-            tma_load_2d_pair(a_s + kATileBytes / 2, &tmw, fb, kc, wrow1);
-            // MMA N = the tile's rows rounded to 32; the peer holds columns [N/2, N)
-            const int n_pair = min(BN, (ti.nvalid + 31) & ~31);
-            tma_load_2d_pair(b_s, &tmb, fb, kc, ti.row0 + static_cast<int>(rank) * (n_pair / 2));
-            if (rank != 0) mbar_arrive_cluster(fb);
-          } else {
-            const int nj = min(p.kpb, (p.K - kc + Cfg::kKB - 1) / Cfg::kKB);  // sub-stages inside K
-            // the boxes of the stage kPfDist stages ahead (same tile) head for L2: with only a
-            // few large stages in the ring, their loads would otherwise wait on DRAM
-            const int kpf = kc + kPfDist * Cfg::kKB * p.kpb;
-            if (p.l2_prefetch && kpf < p.K) {
-              for (int j = 0; j < p.kpb && kpf + j * Cfg::kKB < p.K; ++j) {
-                tma_prefetch_l2_2d(&tmw, kpf + j * Cfg::kKB, wrow0);
-                tma_prefetch_l2_2d(&tmw, kpf + j * Cfg::kKB, wrow1);
-                tma_prefetch_l2_2d(&tmb, kpf + j * Cfg::kKB, ti.row0);
-                if constexpr (W8) tma_prefetch_l2_2d(&tml, kpf + j * Cfg::kKB, ti.row0);
-              }
-            }
-            mbar_arrive_expect_tx(&sm.full[stage], nj * Cfg::kStageBytes);
-            for (int j = 0; j < nj; ++j) {  // sub-stage j: K block kc + j kKB
-              uint8_t* aj = a_s + j * Cfg::kStageBytes;
-              uint8_t* bj = aj + kATileBytes;
-              const int kcj = kc + j * Cfg::kKB;
-              tma_load_2d(aj, &tmw, &sm.full[stage], kcj, wrow0);
-              tma_load_2d(aj + kATileBytes / 2, &tmw, &sm.full[stage], kcj, wrow1);
-              tma_load_2d(bj, &tmb, &sm.full[stage], kcj, ti.row0);
-              if constexpr (W8) tma_load_2d(bj + Cfg::kBTileBytes, &tml, &sm.full[stage], kcj, ti.row0);
-            }
+          const int nj = min(p.kpb, (p.K - kc + Cfg::kKB - 1) / Cfg::kKB);  // sub-stages inside K
+          mbar_arrive_expect_tx(&sm.full[stage], nj * Cfg::kStageBytes);
+          for (int j = 0; j < nj; ++j) {  // sub-stage j: K block kc + j kKB
+            uint8_t* aj = a_s + j * Cfg::kStageBytes;
+            uint8_t* bj = aj + kATileBytes;
+            const int kcj = kc + j * Cfg::kKB;
+            tma_load_2d(aj, &tmw, &sm.full[stage], kcj, wrow0);
+            tma_load_2d(aj + kATileBytes / 2, &tmw, &sm.full[stage], kcj, wrow1);
+            tma_load_2d(bj, &tmb, &sm.full[stage], kcj, ti.row0);
+            if constexpr (W8) tma_load_2d(bj + Cfg::kBTileBytes, &tml, &sm.full[stage], kcj, ti.row0);
           }
           filled_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -402,7 +324,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
       }
       ++itp;
     }
-    if (lane == 0 && *abort_flag && rank == 0) {  // pairs: the leader's barriers count both CTAs' copies
+    if (lane == 0 && *abort_flag) {
       // let our own copies land before the CTA exits
       for (int s = 0; s < S; ++s)
         if (filled_mask & (1u << s)) {
@@ -412,30 +334,21 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // pairs: the leader issues the MMAs of both CTAs (M = 256: its 128 rows and the
-    // peer's), commits reach both CTAs' barriers; the peer waits for the last commit
-    if (lane == 0 && TWO && rank != 0) {
-      volatile int dummy = 0;
-      mbar_wait(&sm.tdone, 0, &dummy, nullptr, p.wait_ns, 0);
-    } else if (lane == 0) {
-      constexpr int kMM = TWO ? 2 * kBM : kBM;  // MMA M
-      auto commit = [&](uint64_t* bar) {
-        if constexpr (TWO) umma_commit_pair(bar, 3);
-        else umma_commit(bar);
-      };
+    if (lane == 0) {
+      auto commit = [&](uint64_t* bar) { umma_commit(bar); };
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      UnitIter uit = unit_begin(p, total_tiles, nk);
+      UnitIter uit = unit_begin();
       Unit u;
-      for (; !*abort_flag && unit_next(p, total_tiles, nk, uit, u); ++it) {
+      for (; !*abort_flag && unit_next(total_tiles, nk, uit, u); ++it) {
         // the last chunk of a group is ragged: N = its rows rounded up to 16, so a
         // skewed expert load does not pay MMAs on padding rows
         const TileInfo ti = tile_of(u.t);
         // e4m3: the hi and lo planes sit back to back in the ring, so one instruction of
         // N = 2 BN covers both and each weight tile is read from shared memory once
-        const int n_mma = TWO ? min(BN, (ti.nvalid + 31) & ~31) : min(BN, (ti.nvalid + 15) & ~15);
-        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, 2 * BN) : umma_idesc_bf16(kMM, n_mma);
+        const int n_mma = min(BN, (ti.nvalid + 15) & ~15);
+        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, 2 * BN) : umma_idesc_bf16(kBM, n_mma);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(&sm.tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns, 2)) break;
@@ -458,8 +371,6 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
               const uint32_t acc = (kb != u.k0 || j != 0 || k != 0) ? 1u : 0u;
               if constexpr (W8) {
                 umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // columns [0, BN) hi, [BN, 2 BN) lo
-              } else if constexpr (TWO) {
-                umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
               } else {
                 umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
               }
@@ -485,41 +396,14 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
     const int g4 = warp & 3;           // TMEM lane quarter this warp may access
     const int m = g4 * 32 + lane;      // accumulator row = weight row within the tile
     int it = 0;
-    UnitIter uit = unit_begin(p, total_tiles, nk);
+    UnitIter uit = unit_begin();
     Unit u;
-    const long long skT = static_cast<long long>(total_tiles) * nk;
-    for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
+    for (; unit_next(total_tiles, nk, uit, u); ++it) {
       const TileInfo ti = tile_of(u.t);
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, p.wait_ns, 4);
       got = got && mbar_wait(&sm.sfull[buf], use & 1u, abort_flag, p.status, p.wait_ns, 7);
-      // stream-K roles: a later part stores its partial; the first part of a split tile
-      // waits (bounded) for the later parts' flags, then adds their partials in CTA order
-      const bool sk_store = p.sk && u.k0 != 0;
-      int sk_b1 = 0, sk_b2 = -1;  // CTAs holding the later parts of this tile
-      if (p.sk && u.k0 == 0 && u.k1 != nk) {
-        sk_b1 = static_cast<int>(blockIdx.x) + 1;
-        sk_b2 = sk_owner(static_cast<long long>(u.t) * nk + nk - 1, skT, gridDim.x);
-        if (got && et == 0) {
-          const uint64_t t0 = globaltimer_ns();
-          for (int bb = sk_b1; bb <= sk_b2 && got; ++bb) {
-            if (!sk_busy(bb, skT, gridDim.x)) continue;  // empty range: holds no part
-            while (ld_acquire_gpu(p.sk_flag + bb) == 0) {
-              if (*abort_flag) {
-                got = false;
-                break;
-              }
-              if (globaltimer_ns() - t0 > p.wait_ns) {
-                *abort_flag = 1;
-                set_status(p.status, MOE_LORA_ERR_TIMEOUT, 11);
-                got = false;
-                break;
-              }
-            }
-          }
-        }
-      }
       if (!named_bar_and(2, kEpiThreads, got)) break;  // the four warps leave together
       tc_fence_after();
 
@@ -571,26 +455,6 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
         } else {
 #pragma unroll
           for (int n = 0; n < 32; ++n) v[n] *= scale;
-        }
-        if (sk_store) {  // later part of a split tile: keep the partial, nothing else
-          float4* dst = reinterpret_cast<float4*>(p.sk_part + (static_cast<size_t>(blockIdx.x) * kBM + m) * BN + c0);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (c0 + 4 * q < BN) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          continue;
-        }
-        for (int bb = sk_b1; bb <= sk_b2; ++bb) {  // first part: add the later parts in order
-          if (!sk_busy(bb, skT, gridDim.x)) continue;
-          const float4* src = reinterpret_cast<const float4*>(p.sk_part + (static_cast<size_t>(bb) * kBM + m) * BN + c0);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (c0 + 4 * q < BN) {
-              const float4 w4 = __ldcg(src + q);
-              v[4 * q] += w4.x;
-              v[4 * q + 1] += w4.y;
-              v[4 * q + 2] += w4.z;
-              v[4 * q + 3] += w4.w;
-            }
         }
         if (p.delta != nullptr) {
           if constexpr (Cfg::kPrefetch) {
@@ -675,21 +539,8 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
           }
         }
       }
-      if (sk_store || sk_b2 >= sk_b1) {
-        __threadfence();                 // this thread's partial row is visible GPU-wide
-        named_bar_sync(1, kEpiThreads);  // every partial row stored / every partial read
-        if (et == 0) {
-          if (sk_store) {
-            __threadfence();
-            st_release_gpu(p.sk_flag + blockIdx.x, 1);
-          } else {
-            for (int bb = sk_b1; bb <= sk_b2; ++bb) p.sk_flag[bb] = 0;  // consumed: re-armed for the next launch
-          }
-        }
-      }
       tc_fence_before();
-      if constexpr (TWO) mbar_arrive_cluster(leader_bar(&sm.tempty[buf]));  // the leader's MMA reuses it
-      else mbar_arrive(&sm.tempty[buf]);
+      mbar_arrive(&sm.tempty[buf]);
       mbar_arrive(&sm.sempty[buf]);
     }
   } else if (warp == 6) {
@@ -699,9 +550,9 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
       if (p.pdl_secondary) pdl_wait();
       uint32_t issued_mask = 0, issued_parity = 0;
       int it = 0;
-      UnitIter uit = unit_begin(p, total_tiles, nk);
+      UnitIter uit = unit_begin();
       Unit u;
-      for (; unit_next(p, total_tiles, nk, uit, u); ++it) {
+      for (; unit_next(total_tiles, nk, uit, u); ++it) {
         const TileInfo ti = tile_of(u.t);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
@@ -750,13 +601,9 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, 1)
   }
 
   tc_fence_before();
-  if constexpr (TWO) cluster_sync_all();  // no CTA leaves while its peer may still signal it
-  else __syncthreads();
+  __syncthreads();
   tc_fence_after();
-  if (warp == 1) {
-    if constexpr (TWO) tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
-    else tmem_dealloc(tmem_base, Cfg::kTmemCols);
-  }
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
 }
 
 // ---------------------------------------------------------------------------- host side
@@ -788,13 +635,13 @@ CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-template <int BN, bool W8, bool TWO = false>
+template <int BN, bool W8>
 static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
-  using Cfg = TileCfg<BN, W8, TWO>;
+  using Cfg = TileCfg<BN, W8>;
   const int fixed = static_cast<int>(sizeof(SmemCore)) + 2 * Cfg::kSlotBytes;
   const int budget = 232448 - 1024 - fixed;
   // two K blocks per stage for the weight-streaming (decode) tiles: plain base stages only
-  const int kpb = (!TWO && BN <= 64 && a.K > Cfg::kKB) ? 2 : 1;
+  const int kpb = (BN <= 64 && a.K > Cfg::kKB) ? 2 : 1;
   const int stage_bytes = kpb * Cfg::kStageBytes;
   int stages = budget / stage_bytes;
   stages = stages > 8 ? 8 : stages;
@@ -806,7 +653,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   const int dev = current_device_index();
   if (dev < 0) return cudaErrorInvalidDevice;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO>,
+    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
@@ -825,7 +672,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2, kBK,
                        64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
-                       static_cast<uint64_t>(a.K) * 2, kBK, Cfg::kBRows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                       static_cast<uint64_t>(a.K) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     tml = tmb;  // unused
   }
@@ -860,39 +707,17 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.b_scales = a.b_scales;
   p.m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
   p.stages = stages;
-  p.m_tiles2 = TWO ? (p.m_tiles + 1) / 2 : 0;
   p.wait_ns = a.test_stall_ms > 0 ? static_cast<uint64_t>(a.test_stall_ms) * 1000000ull : kWaitLimitNs;
   p.test_stall = a.test_stall_ms > 0 ? 1 : 0;
   p.pdl_trigger = a.pdl_trigger;
   p.pdl_secondary = a.pdl_secondary;
   p.kpb = kpb;
   p.stage_bytes = stage_bytes;
-  // deep prefetch where the ring is shallow (wide token tiles); MOE_LORA_L2PF=0|1 overrides
-  {
-    const char* pf = std::getenv("MOE_LORA_L2PF");
-    p.l2_prefetch = pf ? (std::atoi(pf) != 0) : (stages < 6 ? 1 : 0);
-  }
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
-  const long long tiles_ub = chunks_ub * (TWO ? p.m_tiles2 : p.m_tiles);
+  const long long tiles_ub = chunks_ub * p.m_tiles;
   int grid = a.num_sms;
-  // stream-K when the tiles would leave SMs idle or unbalanced (< two waves)
-  p.sk = 0;
-  p.sk_part = a.sk_part;
-  p.sk_flag = a.sk_flag;
-  // Opt-in (MOE_LORA_STREAMK=1), for fewer than two tiles per SM.  Measured on the dense
-  // decode GEMM (86 tiles): all SMs stream but each at half the rate, 40.6 us against
-  // 36.3 us for 86 whole tiles, so whole tiles stay the default.
-  const char* skv = std::getenv("MOE_LORA_STREAMK");
-  const bool sk_want = skv != nullptr && std::atoi(skv) != 0 && tiles_ub < 2LL * grid;
-  if (!TWO && a.sk_part != nullptr && a.sk_flag != nullptr && BN <= 64 && sk_want &&
-      grid <= a.sk_slots && static_cast<long long>(grid) * kBM * BN <= a.sk_part_cap) {
-    p.sk = 1;
-  } else if (TWO) {
-    grid = (grid / 2 < tiles_ub ? grid / 2 : static_cast<int>(tiles_ub)) * 2;  // whole pairs
-  } else {
-    if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
-  }
-  if (grid < (TWO ? 2 : 1)) grid = TWO ? 2 : 1;
+  if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
+  if (grid < 1) grid = 1;
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP
                : a.epi == EPI_DOWN ? K_GEMM_DOWN
                : a.epi == EPI_LOGITS ? K_ROUTE_LOGITS
@@ -902,15 +727,8 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(Cfg::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   int na = 0;
-  if constexpr (TWO) {  // clusters of two CTAs (the MMA pair)
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = 2;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    ++na;
-  }
   if (a.pdl_secondary) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
@@ -918,19 +736,10 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO>, tmw, tmb, tml, tmd, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8>, tmw, tmb, tml, tmd, p);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
-}
-
-// N tiles of 128 and 256 on CTA pairs (cta_group::2), opt-in with MOE_LORA_PAIR=1.  On a
-// prefill-shaped case (256 rows per expert, H = 4096) the pair kernel is correct but
-// slower than one CTA per tile (gate_up 283 us against 156 us, tensor pipe active 17.5%),
-// so single-CTA tiles stay the default.
-static bool pairs_on() {
-  const char* v = std::getenv("MOE_LORA_PAIR");
-  return v != nullptr && std::atoi(v) != 0;
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
@@ -949,8 +758,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
     case 16: return launch_bn<16, false>(a, st);
     case 32: return launch_bn<32, false>(a, st);
     case 64: return launch_bn<64, false>(a, st);
-    case 128: return pairs_on() ? launch_bn<128, false, true>(a, st) : launch_bn<128, false>(a, st);
-    case 256: return pairs_on() ? launch_bn<256, false, true>(a, st) : launch_bn<256, false>(a, st);
+    case 128: return launch_bn<128, false>(a, st);
+    case 256: return launch_bn<256, false>(a, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -90,10 +90,10 @@ struct LoraDeltaArgs {
   const int32_t* scatter;
   // expand: r_exp rank rows of B per delta feature (r for fused adapters); split_I > 0:
   // separate gate and up adapters (A = the 2 r_exp rows of both, B = [2][r_exp][split_I]);
-  // every delta value is multiplied by scale
-  int r_exp;
-  int split_I;
-  float scale;
+  // every delta value is multiplied by scale; r_exp = 0 means r
+  int r_exp = 0;
+  int split_I = 0;
+  float scale = 1.f;
   // programmatic dependent launch: pdl_trigger lets the next kernel start right away;
   // pdl_secondary launches this one behind the running kernel ahead of it, and the
   // kernel then waits for that kernel before it exits.  Either forces the one-kernel form.
@@ -130,9 +130,9 @@ struct LoraTcArgs {
   int num_sms;
   // separate gate and up adapters: split_I = I (a multiple of 64), r = 2 r_exp (A holds
   // both adapters' rows), B [L][E][2][r_exp][I]; 0 = one fused adapter (B [..][r][F])
-  int split_I;
-  int r_exp;
-  float scale;                  // multiplies every delta value
+  int split_I = 0;
+  int r_exp = 0;                // 0 means r
+  float scale = 1.f;            // multiplies every delta value
 };
 cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st);
 
@@ -211,12 +211,6 @@ struct GemmArgs {
   const float* b_scales;       // [total_rows][2] = (s, s / 16)
   int bn;                      // N tile (16..256)
   int num_sms;
-  // optional stream-K scratch (used when the tiles are fewer than two per SM, N <= 64):
-  // partial accumulators [sk_slots][128][BN] fp32 and flags [sk_slots], zero on entry
-  float* sk_part;
-  long long sk_part_cap;       // floats at sk_part
-  int* sk_flag;
-  int sk_slots;
   // tests only: > 0 makes CTA 0 skip the copies of its first stage and shortens every
   // bounded wait to this many milliseconds (the MMA's wait runs out: MOE_LORA_ERR_TIMEOUT)
   int test_stall_ms;

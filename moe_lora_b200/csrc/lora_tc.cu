@@ -36,7 +36,6 @@ constexpr int kLtThreads = 192;
 constexpr int kLtEpi = 128;
 constexpr int kLtAcc = 3;                          // expand accumulators
 constexpr int kLtMaxStages = 8;
-constexpr int kLtPfDist = 6;                       // shrink stages of L2 prefetch lead
 constexpr uint64_t kLtWaitNs = 2000000000ull;      // 2 s
 
 struct LoraTcParams {
@@ -223,13 +222,6 @@ __global__ void __launch_bounds__(kLtThreads, 1)
           }
           uint8_t* s = ring + stage * p.stage_bytes;
           const int np = min(t.kpb, nk - kb);
-          // the boxes kLtPfDist stages ahead head for L2, hiding DRAM latency behind the ring
-          for (int j = 0; j < t.kpb; ++j) {
-            const int kf = kb + kLtPfDist * t.kpb + j;
-            if (kf >= nk) break;
-            tma_prefetch_l2_2d(&tma, kf * 64, arow);
-            tma_prefetch_l2_2d(xm, kf * 64, t.lo);
-          }
           mbar_arrive_expect_tx(&sm.full[stage], pair * static_cast<uint32_t>(np));
           for (int j = 0; j < np; ++j) {
             tma_load_2d(s + j * pair, &tma, &sm.full[stage], (kb + j) * 64, arow);

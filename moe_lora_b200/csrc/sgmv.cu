@@ -689,7 +689,9 @@ cudaError_t launch_lora_plan_all(const int32_t* seg_offsets, const int32_t* seg_
   return cudaGetLastError();
 }
 
-cudaError_t launch_lora_delta(const LoraDeltaArgs& a, cudaStream_t st) {
+cudaError_t launch_lora_delta(const LoraDeltaArgs& args, cudaStream_t st) {
+  LoraDeltaArgs a = args;
+  if (a.r_exp == 0) a.r_exp = a.r;
   if (a.nrows <= 0) return cudaSuccess;
   if (a.r > 128 || a.r % 8 != 0 || a.NB % 8 != 0) return cudaErrorInvalidValue;
   if (a.items == nullptr || a.item_count == nullptr || (a.rb != 4 && a.rb != 8)) return cudaErrorInvalidValue;

@@ -60,30 +60,6 @@ def test_forward_expand_placement(shape, M, where, monkeypatch):
     assert res["err"] <= TOL_BF16, res["err"]
 
 
-@pytest.mark.parametrize("shape,M", [(SMALL[0], 1), (SMALL[1], 3), (SMALL[9], 1), (SMALL[6], 37)],
-                         ids=lambda v: getattr(v, "name", str(v)))
-def test_forward_stream_k(shape, M, monkeypatch):
-    """Stream-K split of few tiles over all SMs: partial accumulators summed in CTA order
-    (tiles split into up to nine parts, some CTAs with empty ranges)."""
-    monkeypatch.setenv("MOE_LORA_STREAMK", "1")
-    monkeypatch.setenv("MOE_LORA_EXPAND", "delta")
-    res = run_moe_case(shape, M)
-    assert res["err"] <= TOL_BF16, res["err"]
-
-
-@pytest.mark.parametrize("where", ["delta", "tc"])
-@pytest.mark.parametrize("bn", [128, 256])
-def test_forward_cta_pairs(bn, where, monkeypatch):
-    """N tiles of 128 / 256 on CTA pairs (tcgen05 cta_group::2): each CTA holds its 128
-    weight rows and half of the token rows; ragged tiles, odd tile counts, LoRA units."""
-    monkeypatch.setenv("MOE_LORA_PAIR", "1")
-    monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
-    monkeypatch.setenv("MOE_LORA_EXPAND", where)
-    for shape, M in ((SMALL[0], 300), (SMALL[1], 37), (SMALL[3], 37), (SMALL[9], 300)):
-        res = run_moe_case(shape, M)
-        assert res["err"] <= TOL_BF16, (shape.name, res["err"])
-
-
 @pytest.fixture(scope="module")
 def decode_weights():
     return moe_weights_both(synth.MOE_DECODE_BF16)

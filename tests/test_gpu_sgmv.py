@@ -68,18 +68,6 @@ def test_dense_lora_forward(s, where, monkeypatch):
     assert err <= (1e-5 if s.dtype == "f32" else TOL_BF16), err
 
 
-@pytest.mark.parametrize("s", [synth.DENSE_DECODE_BF16, CASES[3]], ids=lambda s: s.name)
-def test_dense_stream_k(s, monkeypatch):
-    """The dense GEMM with its K range split over all SMs (stream-K)."""
-    monkeypatch.setenv("MOE_LORA_STREAMK", "1")
-    d = dense_f64(s)
-    y = ml.dense_lora_forward(d["x"].cuda(), d["w"]["w"].cuda(), d["w"]["a"].cuda(), d["w"]["b"].cuda(),
-                              d["offs"].cuda(), d["segs"].cuda())
-    torch.cuda.synchronize()
-    y_ref = ref.dense_lora_forward(d["x64"], d["w64"], d["a64"], d["b64"], d["offs"].numpy(), d["segs"].numpy())
-    assert rel_err(y, y_ref) <= TOL_BF16
-
-
 def test_dense_no_adapters_L0():
     s = synth.DENSE_DECODE_BF16.with_(name="L0", wid=304, T=20, h_in=256, h_out=256, L=0, r=16)
     d = dense_f64(s)
