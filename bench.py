@@ -659,7 +659,8 @@ def measure_moe(args, shape: synth.MoEShape, M: int, W: dict, world, local, *, s
     # ---- per-kernel device times: each batch's step captured as a CUDA graph with an
     #      event pair around every launch (event nodes), replayed; the last replay of
     #      every graph is read, and the instrumented replay itself is timed
-    names = ("route", "router_logits", "topk", "sort", "lora", "quant", "gemm_gateup", "gemm_down", "combine")
+    names = ("route", "router_logits", "topk", "sort", "gather", "lora", "quant", "gemm_gateup", "lora_down",
+             "gemm_down", "combine")
     nb = len(batches)
     if not args.no_graph:
         pgraphs = capture(step, nb, profile=nb * 24 + 64)

@@ -279,8 +279,9 @@ MOE_LORA_API const char* moe_lora_last_error(void);
  * stream, for up to n launches; n = 0 disables and frees the pool.  Kernel ids:
  *   0 router logits, 1 top-k, 2 sort, 3 SGMV shrink, 4 gate_up GEMM, 5 down GEMM,
  *   6 combine, 7 SGMV expand, 8 fp32 dense GEMM, 9 dense bf16 GEMM,
- *   10 e4m3 activation planes, 11 fused segmented LoRA (shrink + expand),
- *   12 one-launch routing (small batches).
+ *   10 e4m3 activation planes, 11 segmented LoRA of gate_up (or dense) and the LoRA
+ *   work lists, 12 one-launch routing (small batches), 13 segmented LoRA of down,
+ *   14 token-row gather into (expert, adapter) order.
  * Launches captured into a CUDA graph record their events as graph nodes, so every
  * replay of the graph re-records them (the last replay's times are read).
  * moe_lora_profile_read() waits for the recorded events and returns the summed

@@ -25,7 +25,8 @@ EXPORTS = ("moe_lora_route", "moe_lora_forward", "sgmv_shrink", "sgmv_expand", "
            "moe_lora_route_noalloc")
 KERNEL_IDS = {"router_logits": 0, "topk": 1, "sort": 2, "shrink": 3, "gemm_gateup": 4, "gemm_down": 5,
               "combine": 6, "expand": 7, "dense_f32": 8, "gemm_dense": 9, "quant": 10,
-              "lora": 11, "route": 12}
+              "lora": 11, "route": 12, "lora_down": 13,
+              "gather": 14}
 
 
 class AdapterFormat(ctypes.Structure):

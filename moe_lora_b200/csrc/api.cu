@@ -669,6 +669,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     t2.r_exp = rr;
     t2.split_I = 0;
     t2.scale = fmt.scale_d;
+    t2.prof_id = K_LORA_DOWN;
     t2.delta = w.dd;
     t2.scatter = sorted_pairs;  // pair order: the combine adds it
     t2.work_counter = w.status + 3;
@@ -709,6 +710,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     l2.r_exp = rr;
     l2.split_I = 0;
     l2.scale = fmt.scale_d;
+    l2.prof_id = K_LORA_DOWN;
     l2.delta = w.delta_d;
     l2.scatter = sorted_pairs;  // pair order, for the combine
     l2.pdl_trigger = 0;

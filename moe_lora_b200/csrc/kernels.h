@@ -94,6 +94,7 @@ struct LoraDeltaArgs {
   int r_exp = 0;
   int split_I = 0;
   float scale = 1.f;
+  int prof_id = 11;  // measurement hook id of the launch (K_LORA or K_LORA_DOWN)
   // programmatic dependent launch: pdl_trigger lets the next kernel start right away;
   // pdl_secondary launches this one behind the running kernel ahead of it, and the
   // kernel then waits for that kernel before it exits.  Either forces the one-kernel form.
@@ -133,6 +134,7 @@ struct LoraTcArgs {
   int split_I = 0;
   int r_exp = 0;                // 0 means r
   float scale = 1.f;            // multiplies every delta value
+  int prof_id = 11;             // measurement hook id of the launch (K_LORA or K_LORA_DOWN)
 };
 cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st);
 

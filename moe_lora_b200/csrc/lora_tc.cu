@@ -524,7 +524,7 @@ cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st) {
   int grid = a.num_sms > 0 ? a.num_sms : 148;
   if (a.items_bound < grid) grid = a.items_bound;
   if (grid < 1) grid = 1;
-  ProfScope ps(K_LORA, st);
+  ProfScope ps(a.prof_id, st);
   lora_tc_kernel<<<grid, kLtThreads, smem, st>>>(tx[0], tx[1], tx[2], tx[3], ta, tb, p);
   count_launch();
   return cudaGetLastError();

@@ -21,7 +21,9 @@ enum KernelId : int {
   K_QUANT = 10,
   K_LORA = 11,
   K_ROUTE = 12,
-  K_COUNT = 13
+  K_LORA_DOWN = 13,  // the down projection's LoRA kernel (K_LORA: gate_up's and the work lists)
+  K_GATHER = 14,     // token rows gathered into (expert, adapter) order
+  K_COUNT = 15
 };
 
 void prof_begin(int id, cudaStream_t st);

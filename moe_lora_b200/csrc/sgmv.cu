@@ -715,7 +715,7 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& args, cudaStream_t st) {
   const bool pdl = a.pdl_trigger || a.pdl_secondary;  // overlapped with a GEMM: one kernel
   if (!pdl && lora && a.z_part != nullptr && static_cast<long long>(a.r) * a.K >= 65536 && nks > 1 &&
       static_cast<long long>(nks) * a.nrows * a.r <= a.z_part_cap) {
-    ProfScope ps(K_LORA, st);
+    ProfScope ps(a.prof_id, st);
     dim3 g1(bound, nks);
     if (a.rb == 8) lora_shrink_part_kernel<8><<<g1, 256, 0, st>>>(a, ks);
     else lora_shrink_part_kernel<4><<<g1, 256, 0, st>>>(a, ks);
@@ -733,7 +733,7 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& args, cudaStream_t st) {
     grid = dim3(std::min(bound, std::max(1, a.num_sms)), 1);
     slice = (a.NB + 7) / 8 * 8;
   }
-  ProfScope ps(K_LORA, st);
+  ProfScope ps(a.prof_id, st);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(256);
@@ -783,7 +783,7 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* src, int nsrc, const int32_t
   if (K % 8 != 0 || div <= 0) return cudaErrorInvalidValue;
   int grid = (rows + 7) / 8;
   if (grid > 148 * 8) grid = 148 * 8;
-  ProfScope ps(K_LORA, st);
+  ProfScope ps(K_GATHER, st);
   gather_rows_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, dst);
   count_launch();
   return cudaGetLastError();
