@@ -15,8 +15,8 @@ Default workload: the MoE prefill layer, the largest configuration that fits one
 4096 tokens, bf16 experts, E=128, top-8, H=4096, I=1536, 16 adapters of rank 64 on
 gate_up and down (Zipf adapter ids, router bias skewing the expert load).  The same line
 carries a `sweep` of the decode layers (bf16 E=64 at M = 1, 8, 32, 64; e4m3 experts
-E=128 at M = 1, 4, 16, 64) and the dense decode projection, measured in the same
-process.  For N > 1 (torchrun) every rank runs an independent replica (weak scaling, no
+E=128 at M = 1, 4, 16, 64, and the same e4m3 layer at 4096 tokens: FP8 prefill) and the
+dense decode projection, measured in the same process.  For N > 1 (torchrun) every rank runs an independent replica (weak scaling, no
 collective on the data path); timing is the max over ranks.  Prints one JSON line on
 rank 0.
 """
@@ -46,7 +46,8 @@ DEFAULT_WORKLOAD = synth.MOE_PREFILL_BF16.name
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 # decode layers measured in the same process as the headline line
-SWEEP = ((synth.MOE_DECODE_BF16.name, (1, 8, 32, 64)), (synth.MOE_DECODE_FP8.name, (1, 4, 16, 64)),
+# (the e4m3-expert layer also at 4096 tokens: FP8 prefill on the same weights)
+SWEEP = ((synth.MOE_DECODE_BF16.name, (1, 8, 32, 64)), (synth.MOE_DECODE_FP8.name, (1, 4, 16, 64, 4096)),
          (synth.DENSE_DECODE_BF16.name, (64,)))
 
 # ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM, with the

@@ -73,6 +73,7 @@ struct LtSmem {
   int q[4];
   uint32_t tmem_base;
   int abort_flag;
+  int rowmap[kLtN];           // delta row of each row of the epilogue's current item
 };
 
 struct LtItem {
@@ -362,12 +363,16 @@ __global__ void __launch_bounds__(kLtThreads, 1)
       if (it < 0) break;
       const LtItem t = lt_item(p, it);
       if (t.n <= 0) continue;
+      // the item's delta rows, read once (the previous item's readers are past the
+      // queue barrier above)
+      for (int j = et; j < t.n; j += kLtEpi) sm.rowmap[j] = lt_delta_row(p, t.lo + j);
+      named_bar_sync(3, kLtEpi);
       if (!t.lora) {  // no adapter: delta = 0 on the segment's rows
         const int f8 = p.F / 8;
         const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
         for (int idx = et; idx < t.n * f8; idx += kLtEpi) {
           const int j = idx / f8, c = idx - j * f8;
-          const int row = lt_delta_row(p, t.lo + j);
+          const int row = sm.rowmap[j];
           if (row >= 0) reinterpret_cast<uint4*>(p.delta + static_cast<size_t>(row) * p.F)[c] = z4;
         }
         continue;
@@ -435,7 +440,7 @@ __global__ void __launch_bounds__(kLtThreads, 1)
             const int c = c0 + j;
             const int blk = c / t.n_mma, tr = c - blk * t.n_mma;
             const int f8 = (g * bpb + blk) * 128 + g4 * 32 + 8 * q;
-            const int row = (c < cols && tr < t.n && f8 + 8 <= p.F) ? lt_delta_row(p, t.lo + tr) : -1;
+            const int row = (c < cols && tr < t.n && f8 + 8 <= p.F) ? sm.rowmap[tr] : -1;
             if (row >= 0)
               *reinterpret_cast<uint4*>(p.delta + static_cast<size_t>(row) * p.F + f8) =
                   *reinterpret_cast<const uint4*>(wst + j * kLtStgPitch + 16 * q);

@@ -727,11 +727,17 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& args, cudaStream_t st) {
   }
   dim3 grid(bound, nsplit);
   if (pdl) {
-    // running beside a GEMM (one CTA of it per SM): one persistent CTA per SM walks the
-    // work list, so that every CTA is resident at once (the GEMM behind a triggering
-    // kernel launches only when all of its CTAs have started) and fits beside the GEMM
-    grid = dim3(std::min(bound, std::max(1, a.num_sms)), 1);
-    slice = (a.NB + 7) / 8 * 8;
+    // running beside a GEMM (one CTA of it per SM): at most one CTA per SM, so that every
+    // CTA is resident at once (the GEMM behind a triggering kernel launches only when all
+    // of its CTAs have started) and fits beside the GEMM.  Few work items (small batches):
+    // the features are split into slices so that the SMs share the B stream, each slice
+    // CTA redoing the item's shrink (A from L2 after the first); many items: one CTA per
+    // SM walks the list, whole rows of features per item.
+    const int sms = std::max(1, a.num_sms);
+    int ns = lora ? std::max(1, std::min(sms / std::max(1, bound), std::max(1, a.NB / 256))) : 1;
+    slice = ((a.NB + ns - 1) / ns + 7) / 8 * 8;
+    ns = (a.NB + slice - 1) / slice;
+    grid = dim3(std::max(1, std::min(bound, sms / ns)), ns);
   }
   ProfScope ps(a.prof_id, st);
   cudaLaunchConfig_t cfg{};
@@ -1002,19 +1008,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
 #pragma unroll
   for (int v = 0; v < 8; ++v) acc[v] = 0.f;
   const __nv_bfloat16* base = o + static_cast<size_t>(t) * k * H + f;
-  for (int j0 = 0; j0 < k; j0 += 8) {  // 8 slot rows in flight, summed in slot order
-    uint4 v8[8];
+  for (int j0 = 0; j0 < k; j0 += 8) {  // 8 slot rows (and their bf16 deltas) in flight
+    uint4 v8[8], d8[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u)
       v8[u] = (j0 + u < k) ? __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(j0 + u) * H))
                            : make_uint4(0u, 0u, 0u, 0u);
+    if (delta_bf16 != nullptr) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 8; ++u) {
+        const size_t pr = static_cast<size_t>(t) * k + j0 + u;
+        d8[u] = (j0 + u < k) ? __ldg(reinterpret_cast<const uint4*>(delta_bf16 + pr * H + f))
+                             : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {  // summed in slot order
       if (j0 + u < k) {
         float fv[8];
         unpack8_bf16(v8[u], fv);
+        const size_t pr = static_cast<size_t>(t) * k + j0 + u;
         if (delta != nullptr) {  // the down LoRA delta of the pair, weighted here
-          const size_t pr = static_cast<size_t>(t) * k + j0 + u;
           const float w = topk_w[pr];
           const float4* dp = reinterpret_cast<const float4*>(delta + pr * H + f);
           const float4 d0 = __ldg(dp), d1 = __ldg(dp + 1);
@@ -1027,10 +1041,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
           fv[6] += w * d1.z;
           fv[7] += w * d1.w;
         } else if (delta_bf16 != nullptr) {
-          const size_t pr = static_cast<size_t>(t) * k + j0 + u;
           const float w = topk_w[pr];
           float dv[8];
-          unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(delta_bf16 + pr * H + f)), dv);
+          unpack8_bf16(d8[u], dv);
 #pragma unroll
           for (int v = 0; v < 8; ++v) fv[v] += w * dv[v];
         }

@@ -206,3 +206,17 @@ def test_forward_moe_decode_fp8_full(fp8_weights, M, record_property):
     res = run_moe_case(synth.MOE_DECODE_FP8, M, weights=fp8_weights)
     check_fp8(res, f"{synth.MOE_DECODE_FP8.name} M={M}", record_property)
     ml.check_status(res["rt"]["workspace"])
+
+
+def test_forward_moe_prefill_fp8_sampled(fp8_weights, record_property):
+    """FP8 prefill: the e4m3 experts and rank-32 adapters of the FP8 decode layer at 4096
+    tokens (256 pairs per expert: the tensor-core LoRA kernel and N tiles of 256 on the
+    kind::f8f6f4 GEMM), on 320 tokens the oracle computes one by one (the first and last
+    32, and 256 drawn at random)."""
+    s = synth.MOE_DECODE_FP8
+    cpu, dev, _ = fp8_weights
+    toks = np.unique(np.concatenate([np.arange(32), np.arange(4096 - 32, 4096),
+                                     np.random.default_rng(3).choice(4096, 256, replace=False)]))
+    res = run_moe_case(s, 4096, weights=(cpu, dev, CpuWeightsOracle(s, cpu, cache=False)), tokens=toks)
+    check_fp8(res, f"{s.name} M=4096 ({len(toks)} tokens)", record_property)
+    ml.check_status(res["rt"]["workspace"])
