@@ -567,10 +567,13 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   l1.item_count = w.item_count;
   LoraTcArgs t1{};
   if (tcl) {
-    ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs),
-            "row gather launch");
-    if (fp8)
-      ML_CUDA(launch_quant_planes(w.x_sorted, mk, H, w.q_hi, w.q_lo, w.q_scales, cs), "activation planes launch");
+    if (fp8)  // one pass over x: the gathered bf16 rows (the LoRA kernel's operand) and their planes
+      ML_CUDA(launch_gather_quant(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.q_hi, w.q_lo,
+                                  w.q_scales, w.x_sorted, cs),
+              "gather and activation planes launch");
+    else
+      ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs),
+              "row gather launch");
     const int bound = lora_items_bound(mk, nkeys, kLtN);
     ML_CUDA(launch_lora_plan_all(seg_offsets, nullptr, nkeys, L, mk, kLtN, w.items_tc, w.item_count_tc, bound,
                                  w.status, cs),
@@ -605,7 +608,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     // LoRA kernel runs, and only its epilogue loader waits for the delta
     if (fp8)
       ML_CUDA(launch_gather_quant(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.q_hi, w.q_lo,
-                                  w.q_scales, cs),
+                                  w.q_scales, nullptr, cs),
               "activation planes launch");
     else
       ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs),
@@ -613,6 +616,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     if (rr) {
       l1.gather_dst = nullptr;
       l1.pdl_trigger = 1;
+      l1.pdl_after_plan = 1;
       ML_CUDA(launch_lora_plan(l1, cs), "LoRA plan launch");
       ML_CUDA(launch_lora_delta(l1, cs), "gate_up LoRA launch");
     }
@@ -715,6 +719,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     l2.scatter = sorted_pairs;  // pair order, for the combine
     l2.pdl_trigger = 0;
     l2.pdl_secondary = 1;
+    l2.pdl_after_plan = 0;  // behind the down GEMM, not the work-list kernel
     ML_CUDA(launch_lora_delta(l2, cs), "down LoRA launch");
   }
 
@@ -933,6 +938,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
       // the LoRA kernel lets the GEMM start at once: the GEMM streams W while it runs,
       // and only the GEMM's epilogue loader waits for the delta
       l.pdl_trigger = 1;
+      l.pdl_after_plan = 1;
       ML_CUDA(launch_lora_plan(l, cs), "LoRA plan launch");
       ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
     }

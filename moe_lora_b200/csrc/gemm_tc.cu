@@ -41,6 +41,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstddef>
 #include <cstdlib>
 #include <mutex>
 
@@ -52,6 +53,7 @@ constexpr int kEpiThreads = 128;
 constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMaxGroups = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr bool kPairDefault = false;               // CTA pairs for N tiles of 256
 
 struct TcParams {
   int epi;
@@ -88,6 +90,10 @@ struct TcParams {
   // streams faster than 128-byte runs
   int kpb;
   int stage_bytes;    // kpb * TileCfg::kStageBytes
+  // epilogue slots: two (the loader fills tile i+1's while the epilogue reads tile i's)
+  // or one (wide fp32 deltas, where shared memory is better spent on ring stages)
+  int nslots, slot_bytes;
+  int slot_delta;     // the loader TMA-prefetches the fp32 delta into the slots
 };
 
 // A unit of work: tile t, K stages [k0, k1) (every unit is a whole tile).
@@ -98,19 +104,22 @@ struct UnitIter {
   int t;
 };
 
+// persistent tile loop: CTA b takes tiles b, b + G, b + 2 G, ...; with CTA pairs both
+// CTAs of a cluster walk the same units (pair b / 2 of G / 2)
+template <bool TWO>
 __device__ __forceinline__ UnitIter unit_begin() {
   UnitIter it;
-  it.t = blockIdx.x;
+  it.t = TWO ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   return it;
 }
 
-// persistent tile loop: CTA b takes tiles b, b + G, b + 2 G, ...
+template <bool TWO>
 __device__ __forceinline__ bool unit_next(int total_tiles, int nk, UnitIter& it, Unit& u) {
   if (it.t >= total_tiles) return false;
   u.t = it.t;
   u.k0 = 0;
   u.k1 = nk;
-  it.t += gridDim.x;
+  it.t += TWO ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   return true;
 }
 
@@ -131,14 +140,15 @@ struct SmemCore {
 };
 
 // Epilogue prefetch slot, filled one tile ahead by the loader warp: the tile's pair ids,
-// routing weights and plane scales, and (N tiles <= 64) its LoRA delta [2 halves][BN][64].
+// routing weights and plane scales, and (N tiles <= 64, fp32 LoRA delta) its delta
+// [2 halves][BN][64].  Without a delta a slot ends before `delta` (TcParams::slot_bytes).
 template <int BN>
 struct EpiSlot {
-  float delta[BN <= 64 ? 2 * BN * 64 : 4];
   int col_pair[BN];
   float col_w[BN];
   float col_sh[BN];
   float col_sl[BN];
+  float delta[BN <= 64 ? 2 * BN * 64 : 4];  // 128-byte aligned: 16 BN bytes in
 };
 
 constexpr int pow2_at_least(int v) {
@@ -147,18 +157,21 @@ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int BN, bool W8>
+// TWO: a CTA pair (cta_group::2) computes 256 weight rows x BN tokens; each CTA holds its
+// 128 weight rows and half of the BN token rows of every stage.
+template <int BN, bool W8, bool TWO = false>
 struct TileCfg {
   static constexpr int kKB = W8 ? 128 : 64;                  // K per stage (128 bytes per row)
-  static constexpr int kBTileBytes = BN * 128;               // one token tile (or plane)
+  static constexpr int kBRows = TWO ? BN / 2 : BN;           // token rows held by this CTA
+  static constexpr int kBTileBytes = kBRows * 128;           // one token tile (or plane)
   static constexpr int kStageBytes = kATileBytes + (W8 ? 2 : 1) * kBTileBytes;
   static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
   static constexpr int kAccPerBuf = W8 ? 2 : 1;              // e4m3: hi and lo side by side (N = 2 BN)
   static constexpr int kTmemCols = pow2_at_least(2 * kAccPerBuf * kAccStride);
   static constexpr bool kPrefetch = BN <= 64;                // LoRA delta prefetched into the slots
-  static constexpr int kSlotBytes = static_cast<int>((sizeof(EpiSlot<BN>) + 1023) / 1024 * 1024);
   static constexpr int kThreads = 224;
   static_assert(!W8 || kPrefetch, "e4m3 weights use N tiles <= 64");
+  static_assert(!TWO || (!W8 && BN == 256), "CTA pairs: bf16 weights, N tiles of 256");
 };
 
 struct TileInfo {
@@ -187,21 +200,25 @@ __device__ __forceinline__ int delta_col(int epi, int m, int f0, int I) {
   return f0 + m;
 }
 
-template <int BN, bool W8>
-__global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
+template <int BN, bool W8, bool TWO>
+__global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tml, const __grid_constant__ CUtensorMap tmd,
                    const TcParams p) {
   // tml: the lo activation plane (e4m3 weights); tmd: the fp32 LoRA delta (N tiles <= 64)
-  using Cfg = TileCfg<BN, W8>;
+  using Cfg = TileCfg<BN, W8, TWO>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;                                 // stages: [A tile][token tile(s)]
   uint8_t* slots = ring + p.stages * p.stage_bytes;  // epilogue prefetch slots
-  SmemCore& sm = *reinterpret_cast<SmemCore*>(slots + 2 * Cfg::kSlotBytes);
+  SmemCore& sm = *reinterpret_cast<SmemCore*>(slots + p.nslots * p.slot_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages;
   volatile int* abort_flag = &sm.abort_flag;
+  // CTA pairs: rank 0 (the leader) issues the MMAs of both CTAs; the stage and TMEM
+  // barriers it consumes live in its shared memory
+  const uint32_t rank = TWO ? cluster_ctarank() : 0u;
+  auto leader_bar = [&](uint64_t* bar) -> uint32_t { return TWO ? mapa_shared(smem_u32(bar), 0) : smem_u32(bar); };
 
   if (p.pdl_trigger) pdl_trigger();
   // ---- setup: barriers, TMEM, tile list prefix
@@ -212,7 +229,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
-      mbar_init(&sm.tempty[b], kEpiThreads);
+      mbar_init(&sm.tempty[b], TWO ? 2 * kEpiThreads : kEpiThreads);  // pairs: both CTAs' epilogues
       mbar_init(&sm.sfull[b], 1);
       mbar_init(&sm.sempty[b], kEpiThreads);
     }
@@ -226,7 +243,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     if (W8) tma_prefetch_desc(&tml);
     if (p.delta != nullptr) tma_prefetch_desc(&tmd);
   }
-  if (warp == 1) tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
+  if (warp == 1) {
+    if constexpr (TWO) tmem_alloc_pair(&sm.tmem_base, Cfg::kTmemCols);
+    else tmem_alloc(&sm.tmem_base, Cfg::kTmemCols);
+  }
   // group offsets clamped to [0, total_rows]: offsets that are out of range or not
   // monotone (flagged by the work-list kernel) can leave rows uncomputed, never make a
   // tile reach outside the operands
@@ -265,11 +285,18 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     if (lane == 31) sm.chunk_pref[p.E] = incl;
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (TWO) cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
-  const int total_tiles = sm.chunk_pref[p.E] * p.m_tiles;
-  auto tile_of = [&](int t) -> TileInfo { return decode_tile(sm, t, p.m_tiles, p.E, BN); };
+  // pairs: a unit is a pair of 128-row weight tiles (an even count per group), rank picks one
+  const int unit_m = TWO ? p.m_tiles / 2 : p.m_tiles;
+  const int total_tiles = sm.chunk_pref[p.E] * unit_m;
+  auto tile_of = [&](int t) -> TileInfo {
+    TileInfo ti = decode_tile(sm, t, unit_m, p.E, BN);
+    if constexpr (TWO) ti.mt = 2 * ti.mt + static_cast<int>(rank);
+    return ti;
+  };
   const int nk = (p.K + Cfg::kKB * p.kpb - 1) / (Cfg::kKB * p.kpb);  // stages per tile
 
   if (warp == 0) {
@@ -281,10 +308,10 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     uint32_t phase = 0;
     uint32_t filled_mask = 0, last_parity = 0;
     bool ok = true;
-    UnitIter uit = unit_begin();
+    UnitIter uit = unit_begin<TWO>();
     Unit u;
     int itp = 0;  // unit index, the same sequence as the MMA thread's
-    while (ok && unit_next(total_tiles, nk, uit, u)) {
+    while (ok && unit_next<TWO>(total_tiles, nk, uit, u)) {
       if (*abort_flag) break;
       const TileInfo ti = tile_of(u.t);
       int wrow0, wrow1;
@@ -304,6 +331,16 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           uint8_t* a_s = ring + stage * p.stage_bytes;
           const int kc = kb * Cfg::kKB * p.kpb;  // first K element of the stage
           const int nj = min(p.kpb, (p.K - kc + Cfg::kKB - 1) / Cfg::kKB);  // sub-stages inside K
+          if constexpr (TWO) {
+            // both CTAs' copies complete on the leader's barrier, which expects the pair's
+            // bytes; the MMA's N is the tile's rows rounded to 32, the peer holds [N/2, N)
+            const uint32_t fb = leader_bar(&sm.full[stage]);
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2u * Cfg::kStageBytes);
+            const int n_pair = min(BN, (ti.nvalid + 31) & ~31);
+            tma_load_2d_pair(a_s, &tmw, fb, kc, wrow0);
+            tma_load_2d_pair(a_s + kATileBytes / 2, &tmw, fb, kc, wrow1);
+            tma_load_2d_pair(a_s + kATileBytes, &tmb, fb, kc, ti.row0 + static_cast<int>(rank) * (n_pair / 2));
+          } else {
           mbar_arrive_expect_tx(&sm.full[stage], nj * Cfg::kStageBytes);
           for (int j = 0; j < nj; ++j) {  // sub-stage j: K block kc + j kKB
             uint8_t* aj = a_s + j * Cfg::kStageBytes;
@@ -313,6 +350,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
             tma_load_2d(aj + kATileBytes / 2, &tmw, &sm.full[stage], kcj, wrow1);
             tma_load_2d(bj, &tmb, &sm.full[stage], kcj, ti.row0);
             if constexpr (W8) tma_load_2d(bj + Cfg::kBTileBytes, &tml, &sm.full[stage], kcj, ti.row0);
+          }
           }
           filled_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -325,30 +363,42 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       ++itp;
     }
     if (lane == 0 && *abort_flag) {
-      // let our own copies land before the CTA exits
-      for (int s = 0; s < S; ++s)
-        if (filled_mask & (1u << s)) {
-          volatile int dummy = 0;
-          mbar_wait(&sm.full[s], (last_parity >> s) & 1u, &dummy, nullptr, p.wait_ns / 4, 0);
+      // let our own copies land before the CTA exits (pairs: the peer's copies complete on
+      // the leader's barriers, so the peer gives them a fixed 50 us)
+      if (TWO && rank != 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 50000ull) {
         }
+      } else {
+        for (int s = 0; s < S; ++s)
+          if (filled_mask & (1u << s)) {
+            volatile int dummy = 0;
+            mbar_wait(&sm.full[s], (last_parity >> s) & 1u, &dummy, nullptr, p.wait_ns / 4, 0);
+          }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      auto commit = [&](uint64_t* bar) { umma_commit(bar); };
+    // pairs: the leader issues the MMAs of both CTAs (M = 256: its 128 rows and the
+    // peer's); its commits arrive on the barrier at the same offset in both CTAs
+    if (lane == 0 && (!TWO || rank == 0)) {
+      auto commit = [&](uint64_t* bar) {
+        if constexpr (TWO) umma_commit_pair(bar, 3);
+        else umma_commit(bar);
+      };
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      UnitIter uit = unit_begin();
+      UnitIter uit = unit_begin<TWO>();
       Unit u;
-      for (; !*abort_flag && unit_next(total_tiles, nk, uit, u); ++it) {
+      for (; !*abort_flag && unit_next<TWO>(total_tiles, nk, uit, u); ++it) {
         // the last chunk of a group is ragged: N = its rows rounded up to 16, so a
         // skewed expert load does not pay MMAs on padding rows
         const TileInfo ti = tile_of(u.t);
         // e4m3: the hi and lo planes sit back to back in the ring, so one instruction of
         // N = 2 BN covers both and each weight tile is read from shared memory once
-        const int n_mma = min(BN, (ti.nvalid + 15) & ~15);
-        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, 2 * BN) : umma_idesc_bf16(kBM, n_mma);
+        const int n_mma = TWO ? min(BN, (ti.nvalid + 31) & ~31) : min(BN, (ti.nvalid + 15) & ~15);
+        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, 2 * BN) : umma_idesc_bf16(TWO ? 2 * kBM : kBM, n_mma);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(&sm.tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns, 2)) break;
@@ -371,6 +421,8 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
               const uint32_t acc = (kb != u.k0 || j != 0 || k != 0) ? 1u : 0u;
               if constexpr (W8) {
                 umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // columns [0, BN) hi, [BN, 2 BN) lo
+              } else if constexpr (TWO) {
+                umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
               } else {
                 umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
               }
@@ -386,7 +438,8 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
         commit(&sm.tfull[buf]);
       }
       // all MMAs issued by this thread complete before TMEM is released
-      commit(&sm.tdone);
+      if constexpr (TWO) umma_commit_pair(&sm.tdone, 1);
+      else commit(&sm.tdone);
       volatile int dummy = 0;
       mbar_wait(&sm.tdone, 0, &dummy, nullptr, p.wait_ns, 0);
     }
@@ -396,14 +449,16 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
     const int g4 = warp & 3;           // TMEM lane quarter this warp may access
     const int m = g4 * 32 + lane;      // accumulator row = weight row within the tile
     int it = 0;
-    UnitIter uit = unit_begin();
+    UnitIter uit = unit_begin<TWO>();
     Unit u;
-    for (; unit_next(total_tiles, nk, uit, u); ++it) {
+    for (; unit_next<TWO>(total_tiles, nk, uit, u); ++it) {
       const TileInfo ti = tile_of(u.t);
       const int buf = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int sb = p.nslots == 2 ? buf : 0;  // epilogue slot and its use count
+      const uint32_t su = p.nslots == 2 ? use : static_cast<uint32_t>(it);
       bool got = mbar_wait(&sm.tfull[buf], use & 1u, abort_flag, p.status, p.wait_ns, 4);
-      got = got && mbar_wait(&sm.sfull[buf], use & 1u, abort_flag, p.status, p.wait_ns, 7);
+      got = got && mbar_wait(&sm.sfull[sb], su & 1u, abort_flag, p.status, p.wait_ns, 7);
       if (!named_bar_and(2, kEpiThreads, got)) break;  // the four warps leave together
       tc_fence_after();
 
@@ -420,7 +475,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
       const int dcol = delta_col(p.epi, m, f0, p.I);
       float scale = 1.f;
       if (p.w_scales != nullptr) scale = p.w_scales[ti.g * 2 + p.scale_idx];
-      const EpiSlot<BN>* slot = reinterpret_cast<const EpiSlot<BN>*>(slots + buf * Cfg::kSlotBytes);
+      const EpiSlot<BN>* slot = reinterpret_cast<const EpiSlot<BN>*>(slots + sb * p.slot_bytes);
 
       // bf16 delta [rows][delta_cols] (token-major): lane L of a warp loads row c0 + L's 32
       // delta columns of the warp (64 contiguous bytes, one chunk ahead), the warp passes
@@ -457,12 +512,13 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
           for (int n = 0; n < 32; ++n) v[n] *= scale;
         }
         if (p.delta != nullptr) {
-          if constexpr (Cfg::kPrefetch) {
+          if (Cfg::kPrefetch && p.slot_delta) {
             const float* dl = slot->delta + ((m >> 6) * BN + c0) * 64 + (m & 63);
 #pragma unroll
             for (int n = 0; n < 32; ++n)
               if (c0 + n < BN) v[n] += dl[n * 64];
           } else if (dcol < p.delta_cols) {
+            if (p.pdl_secondary) pdl_wait();  // the delta comes from the kernel ahead
             const float* dg = p.delta + static_cast<size_t>(ti.row0 + c0) * p.delta_cols + dcol;
 #pragma unroll
             for (int n = 0; n < 32; ++n)
@@ -540,27 +596,29 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&sm.tempty[buf]);
-      mbar_arrive(&sm.sempty[buf]);
+      if constexpr (TWO) mbar_arrive_remote(leader_bar(&sm.tempty[buf]));  // the leader's MMA reuses it
+      else mbar_arrive(&sm.tempty[buf]);
+      mbar_arrive(&sm.sempty[sb]);
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------ epilogue loader
     {
-      // the LoRA delta (and nothing else this kernel reads) comes from the kernel ahead
-      if (p.pdl_secondary) pdl_wait();
+      // the LoRA delta (and nothing else this kernel reads) comes from the kernel ahead:
+      // the loader waits for it only when it prefetches the delta
+      if (p.pdl_secondary && p.slot_delta && p.delta != nullptr) pdl_wait();
       uint32_t issued_mask = 0, issued_parity = 0;
       int it = 0;
-      UnitIter uit = unit_begin();
+      UnitIter uit = unit_begin<TWO>();
       Unit u;
-      for (; unit_next(total_tiles, nk, uit, u); ++it) {
+      for (; unit_next<TWO>(total_tiles, nk, uit, u); ++it) {
         const TileInfo ti = tile_of(u.t);
-        const int buf = it & 1;
-        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        const int buf = p.nslots == 2 ? (it & 1) : 0;
+        const uint32_t use = p.nslots == 2 ? static_cast<uint32_t>(it >> 1) : static_cast<uint32_t>(it);
         const bool got = mbar_wait(&sm.sempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns, 8);
         if (!__all_sync(0xffffffffu, got)) break;
-        EpiSlot<BN>* slot = reinterpret_cast<EpiSlot<BN>*>(slots + buf * Cfg::kSlotBytes);
+        EpiSlot<BN>* slot = reinterpret_cast<EpiSlot<BN>*>(slots + buf * p.slot_bytes);
         if constexpr (Cfg::kPrefetch) {
-          if (lane == 0 && p.delta != nullptr) {
+          if (lane == 0 && p.delta != nullptr && p.slot_delta) {
             const int f0 = (p.epi == EPI_GATEUP) ? ti.mt * 64 : ti.mt * kBM;
             const int c1 = (p.epi == EPI_GATEUP) ? p.I + f0 : f0 + 64;
             mbar_expect_tx(&sm.sfull[buf], 2 * BN * 64 * 4);
@@ -601,9 +659,13 @@ __global__ void __launch_bounds__(TileCfg<BN, W8>::kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (TWO) cluster_sync_all();  // no CTA leaves while its peer may still signal it
+  else __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  if (warp == 1) {
+    if constexpr (TWO) tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+    else tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
 }
 
 // ---------------------------------------------------------------------------- host side
@@ -635,17 +697,32 @@ CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-template <int BN, bool W8>
+template <int BN, bool W8, bool TWO = false>
 static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
-  using Cfg = TileCfg<BN, W8>;
-  const int fixed = static_cast<int>(sizeof(SmemCore)) + 2 * Cfg::kSlotBytes;
-  const int budget = 232448 - 1024 - fixed;
+  using Cfg = TileCfg<BN, W8, TWO>;
   // two K blocks per stage for the weight-streaming (decode) tiles: plain base stages only
   const int kpb = (BN <= 64 && a.K > Cfg::kKB) ? 2 : 1;
+  const int m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
+  if (TWO && (m_tiles % 2 != 0 || kpb != 1)) return cudaErrorInvalidValue;  // whole pairs of weight tiles
+  // epilogue slots: the fp32 delta part only when the loader prefetches it (whole tiles,
+  // N <= 64); one slot instead of two where that buys another ring stage
+  const bool dslot = a.delta != nullptr && Cfg::kPrefetch;
+  const int slot_bytes = static_cast<int>(((dslot ? sizeof(EpiSlot<BN>) : offsetof(EpiSlot<BN>, delta)) + 1023) /
+                                          1024 * 1024);
   const int stage_bytes = kpb * Cfg::kStageBytes;
-  int stages = budget / stage_bytes;
-  stages = stages > 8 ? 8 : stages;
+  // overlapped with a LoRA kernel (PDL: launched behind one, or letting one start) the
+  // GEMM leaves room for one of its CTAs on every SM (228 KB per SM, 1 KB reserved per
+  // CTA), so both run side by side
+  const bool coloc = a.pdl_secondary || a.pdl_trigger;
+  const int smem_cap = coloc ? 228 * 1024 - 1024 - kLoraCoresidentSmem : 232448;
+  auto stages_for = [&](int ns) {
+    const int s = (smem_cap - 1024 - static_cast<int>(sizeof(SmemCore)) - ns * slot_bytes) / stage_bytes;
+    return s > 8 ? 8 : s;
+  };
+  const int nslots = stages_for(1) > stages_for(2) ? 1 : 2;
+  const int stages = stages_for(nslots);
   if (stages < 2) return cudaErrorInvalidConfiguration;
+  const int fixed = static_cast<int>(sizeof(SmemCore)) + nslots * slot_bytes;
   const size_t smem = 1024 + static_cast<size_t>(stages) * stage_bytes + fixed;
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   // the raised shared-memory limit is a per-device function attribute
@@ -653,7 +730,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   const int dev = current_device_index();
   if (dev < 0) return cudaErrorInvalidDevice;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8>,
+    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
@@ -672,7 +749,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2, kBK,
                        64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
-                       static_cast<uint64_t>(a.K) * 2, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                       static_cast<uint64_t>(a.K) * 2, kBK, Cfg::kBRows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     tml = tmb;  // unused
   }
@@ -705,7 +782,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.scale_idx = a.scale_idx;
   p.status = a.status;
   p.b_scales = a.b_scales;
-  p.m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
+  p.m_tiles = m_tiles;
   p.stages = stages;
   p.wait_ns = a.test_stall_ms > 0 ? static_cast<uint64_t>(a.test_stall_ms) * 1000000ull : kWaitLimitNs;
   p.test_stall = a.test_stall_ms > 0 ? 1 : 0;
@@ -713,11 +790,19 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.pdl_secondary = a.pdl_secondary;
   p.kpb = kpb;
   p.stage_bytes = stage_bytes;
+  p.nslots = nslots;
+  p.slot_bytes = slot_bytes;
+  p.slot_delta = dslot ? 1 : 0;
   const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
-  const long long tiles_ub = chunks_ub * p.m_tiles;
+  const long long tiles_ub = chunks_ub * (TWO ? p.m_tiles / 2 : p.m_tiles);
   int grid = a.num_sms;
-  if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
-  if (grid < 1) grid = 1;
+  if constexpr (TWO) {  // whole clusters of two CTAs
+    grid = (grid / 2 < tiles_ub ? grid / 2 : static_cast<int>(tiles_ub)) * 2;
+    if (grid < 2) grid = 2;
+  } else {
+    if (tiles_ub < grid) grid = static_cast<int>(tiles_ub);
+    if (grid < 1) grid = 1;
+  }
   ProfScope ps(a.epi == EPI_GATEUP ? K_GEMM_GATEUP
                : a.epi == EPI_DOWN ? K_GEMM_DOWN
                : a.epi == EPI_LOGITS ? K_ROUTE_LOGITS
@@ -727,8 +812,15 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(Cfg::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   int na = 0;
+  if constexpr (TWO) {  // clusters of two CTAs: the MMA pair
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   if (a.pdl_secondary) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
@@ -736,7 +828,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8>, tmw, tmb, tml, tmd, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO>, tmw, tmb, tml, tmd, p);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -759,7 +851,16 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
     case 32: return launch_bn<32, false>(a, st);
     case 64: return launch_bn<64, false>(a, st);
     case 128: return launch_bn<128, false>(a, st);
-    case 256: return launch_bn<256, false>(a, st);
+    case 256: {
+      // N tiles of 256 on CTA pairs (tcgen05 cta_group::2, M = 256): per CTA and stage one
+      // 16 KB weight tile and half of the token tile, so the same shared memory holds more
+      // stages and each byte staged feeds twice the MMA work.  MOE_LORA_PAIR=0|1 overrides.
+      const int m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
+      const char* v = std::getenv("MOE_LORA_PAIR");
+      const bool pair = (v != nullptr ? std::atoi(v) != 0 : kPairDefault) && m_tiles % 2 == 0 && a.K > kBK &&
+                        (a.epi == EPI_GATEUP || a.epi == EPI_DOWN || a.epi == EPI_DENSE);
+      return pair ? launch_bn<256, false, true>(a, st) : launch_bn<256, false>(a, st);
+    }
     default: return cudaErrorInvalidValue;
   }
 }

@@ -57,6 +57,11 @@ cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st);
 // shrink z = src . A^T; then either write z (bf16) for a GEMM that runs the expand as
 // extra MMA K steps, or expand delta = z . B into an fp32 buffer that the GEMM epilogue
 // adds (rows without an adapter get delta = 0).  bf16 only; one kernel launch.
+// Shared memory a CTA of the SIMT LoRA kernel needs on an SM beside a GEMM CTA (its
+// static arrays and the driver's per-CTA reservation): a GEMM launched behind that kernel
+// leaves this much free.
+constexpr int kLoraCoresidentSmem = 8192;
+
 struct LoraDeltaArgs {
   const __nv_bfloat16* src;   // rows [*, K]
   const int32_t* gather;      // if set: source row of output row s = gather[s] / gather_div
@@ -97,9 +102,12 @@ struct LoraDeltaArgs {
   int prof_id = 11;  // measurement hook id of the launch (K_LORA or K_LORA_DOWN)
   // programmatic dependent launch: pdl_trigger lets the next kernel start right away;
   // pdl_secondary launches this one behind the running kernel ahead of it, and the
-  // kernel then waits for that kernel before it exits.  Either forces the one-kernel form.
+  // kernel then waits for that kernel before it exits; pdl_after_plan launches it behind
+  // the work-list kernel, whose list it waits for before reading it.  Any of them forces
+  // the one-kernel form.
   int pdl_trigger;
   int pdl_secondary;
+  int pdl_after_plan = 0;
 };
 int lora_rows_per_chunk(int nrows, int nseg);
 int lora_items_bound(int nrows, int nseg, int rb);
@@ -235,9 +243,9 @@ cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8
 cudaError_t launch_combine(const __nv_bfloat16* o, int M, int k, int H, const float* delta,
                            const __nv_bfloat16* delta_bf16, const float* topk_w, __nv_bfloat16* y, cudaStream_t st);
 // The e4m3 activation planes of gathered rows (see launch_quant_planes): plane row i from
-// src[gather[i] / div].
+// src[gather[i] / div]; copy (if set) also receives the gathered bf16 rows.
 cudaError_t launch_gather_quant(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
-                                uint8_t* hi, uint8_t* lo, float* scales, cudaStream_t st);
+                                uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy, cudaStream_t st);
 
 // Host state that CUDA keeps per device (function attributes, SM counts, capability)
 // is cached per device index, for processes that drive several GPUs.

@@ -167,8 +167,9 @@ cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st) {
 // relative 2^-8; the FP8-weight GEMM multiplies both planes on the kind::f8f6f4 tensor
 // core.  |x / s| <= 448 and |(x - hi s) / (s / 16)| <= 448 by construction.
 // One warp quantises one bf16 row of K elements into the two e4m3 planes (see below).
+// copy_row (if set) also receives the bf16 row itself.
 __device__ __forceinline__ void quant_row_warp(const __nv_bfloat16* src_row, int K, uint8_t* hi_row, uint8_t* lo_row,
-                                               float* scale2, int lane) {
+                                               float* scale2, int lane, __nv_bfloat16* copy_row = nullptr) {
   const uint4* xr = reinterpret_cast<const uint4*>(src_row);
   const int k8 = K / 8;
   float amax = 0.f;
@@ -184,7 +185,9 @@ __device__ __forceinline__ void quant_row_warp(const __nv_bfloat16* src_row, int
   const float inv = 1.f / s, inv_lo = 16.f / s;
   for (int c = lane; c < k8; c += 32) {
     float f[8];
-    unpack8_bf16(__ldg(xr + c), f);
+    const uint4 raw = __ldg(xr + c);
+    if (copy_row != nullptr) reinterpret_cast<uint4*>(copy_row)[c] = raw;
+    unpack8_bf16(raw, f);
     uint32_t hq[2], lq[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -501,7 +504,10 @@ __global__ void __launch_bounds__(256, RBMAX == 4 ? 3 : 2) lora_fused_kernel(con
   __shared__ int s_src[LF_RB_MAX];
   __shared__ float s_z[LF_RB_MAX * 128];
   __shared__ float s_part[64 * LF_RB_MAX];  // ks * r == 64 whenever ks > 1
+  static_assert(sizeof(s_src) + sizeof(s_z) + sizeof(s_part) + 1024 <= kLoraCoresidentSmem,
+                "the LoRA CTA must fit beside a GEMM CTA");
   if (a.pdl_trigger) pdl_trigger();
+  if (a.pdl_after_plan) pdl_wait();  // the work list comes from the kernel ahead
   const int count = *a.item_count;  // a grid smaller than the work list walks it with a stride
   for (int it = blockIdx.x; it < count; it += gridDim.x) {
     lora_fused_body<RBMAX>(a, it, ks, slice, s_src, s_z, s_part);
@@ -633,6 +639,7 @@ __global__ void __launch_bounds__(1024) lora_plan_kernel(const int32_t* __restri
                                                          int* __restrict__ count, int cap, int* status,
                                                          int adapters_only) {
   __shared__ int s_scan[32];
+  pdl_trigger();  // a LoRA kernel launched behind this one may start (it waits for the list)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = (nseg + blockDim.x - 1) / blockDim.x;
   const int q0 = threadIdx.x * per, q1 = min(nseg, q0 + per);
@@ -712,7 +719,7 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& args, cudaStream_t st) {
   slice = (slice + 7) / 8 * 8;
   nsplit = (a.NB + slice - 1) / slice;
   const int nks = (a.K + LS_KSLICE - 1) / LS_KSLICE;
-  const bool pdl = a.pdl_trigger || a.pdl_secondary;  // overlapped with a GEMM: one kernel
+  const bool pdl = a.pdl_trigger || a.pdl_secondary || a.pdl_after_plan;  // overlapped: one kernel
   if (!pdl && lora && a.z_part != nullptr && static_cast<long long>(a.r) * a.K >= 65536 && nks > 1 &&
       static_cast<long long>(nks) * a.nrows * a.r <= a.z_part_cap) {
     ProfScope ps(a.prof_id, st);
@@ -749,7 +756,7 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& args, cudaStream_t st) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = a.pdl_secondary ? 1 : 0;
+  cfg.numAttrs = (a.pdl_secondary || a.pdl_after_plan) ? 1 : 0;
   const cudaError_t e = a.rb == 8 ? cudaLaunchKernelEx(&cfg, lora_fused_kernel<8>, a, ks, slice)
                                   : cudaLaunchKernelEx(&cfg, lora_fused_kernel<4>, a, ks, slice);
   count_launch();
@@ -949,7 +956,8 @@ __global__ void __launch_bounds__(256) quant_planes_kernel(const __nv_bfloat16* 
 __global__ void __launch_bounds__(256) gather_quant_kernel(const __nv_bfloat16* __restrict__ src, int nsrc,
                                                           const int32_t* __restrict__ gather, int div, int rows,
                                                           int K, uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
-                                                          float* __restrict__ scales) {
+                                                          float* __restrict__ scales,
+                                                          __nv_bfloat16* __restrict__ copy) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
     const int sr = gather[row] / div;
@@ -958,6 +966,9 @@ __global__ void __launch_bounds__(256) gather_quant_kernel(const __nv_bfloat16* 
         reinterpret_cast<uint4*>(hi + static_cast<size_t>(row) * K)[c] = make_uint4(0u, 0u, 0u, 0u);
         reinterpret_cast<uint4*>(lo + static_cast<size_t>(row) * K)[c] = make_uint4(0u, 0u, 0u, 0u);
       }
+      if (copy != nullptr)
+        for (int c = lane; c < K / 8; c += 32)
+          reinterpret_cast<uint4*>(copy + static_cast<size_t>(row) * K)[c] = make_uint4(0u, 0u, 0u, 0u);
       if (lane == 0) {
         scales[2 * static_cast<size_t>(row)] = 0.f;
         scales[2 * static_cast<size_t>(row) + 1] = 0.f;
@@ -965,18 +976,19 @@ __global__ void __launch_bounds__(256) gather_quant_kernel(const __nv_bfloat16* 
       continue;
     }
     quant_row_warp(src + static_cast<size_t>(sr) * K, K, hi + static_cast<size_t>(row) * K,
-                   lo + static_cast<size_t>(row) * K, scales + 2 * static_cast<size_t>(row), lane);
+                   lo + static_cast<size_t>(row) * K, scales + 2 * static_cast<size_t>(row), lane,
+                   copy != nullptr ? copy + static_cast<size_t>(row) * K : nullptr);
   }
 }
 
 cudaError_t launch_gather_quant(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
-                                uint8_t* hi, uint8_t* lo, float* scales, cudaStream_t st) {
+                                uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   if (K % 16 != 0 || div <= 0) return cudaErrorInvalidValue;
   int grid = (rows + 7) / 8;
   if (grid > 148 * 8) grid = 148 * 8;
   ProfScope ps(K_QUANT, st);
-  gather_quant_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales);
+  gather_quant_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales, copy);
   count_launch();
   return cudaGetLastError();
 }
