@@ -646,7 +646,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.b = w.x_sorted;
   g.bn = choose_bn(mk, E);
   if (fp8) {
-    if (g.bn > 64) g.bn = 64;  // e4m3 tiles use the prefetching epilogue (N <= 64)
+    if (g.bn > 128) g.bn = 128;  // e4m3: the hi and lo planes make the MMA's N = 2 BN <= 256
     g.b_hi = w.q_hi;
     g.b_lo = w.q_lo;
     g.b_scales = w.q_scales;

@@ -32,6 +32,12 @@
 //   warp 6      epilogue loader: one tile ahead of the epilogue, the per-column data
 //               (pair ids, routing weights, activation plane scales) and, for N tiles
 //               <= 64, a TMA of the tile's fp32 LoRA delta into a two-slot ring
+// N tiles of 256 (prefill) run on CTA pairs (a cluster of two, tcgen05 cta_group::2):
+// the pair computes 256 weight rows x 256 tokens, each CTA staging its own 128 weight
+// rows and half of the token rows (the MMA reads both halves), so every staged byte
+// feeds twice the MMA work; the leader CTA's thread issues the MMAs of both and alone
+// expects the pair's bytes on its stage barriers, its commits reach both CTAs, and both
+// CTAs' epilogues release the accumulator on the leader's barrier.
 // Every mbarrier wait is bounded; on expiry the CTA records MOE_LORA_ERR_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include "common.cuh"
@@ -40,6 +46,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstddef>
 #include <cstdlib>
@@ -53,7 +60,7 @@ constexpr int kEpiThreads = 128;
 constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kMaxGroups = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-constexpr bool kPairDefault = false;               // CTA pairs for N tiles of 256
+constexpr bool kPairDefault = true;                // CTA pairs for N tiles of 256
 
 struct TcParams {
   int epi;
@@ -170,7 +177,7 @@ struct TileCfg {
   static constexpr int kTmemCols = pow2_at_least(2 * kAccPerBuf * kAccStride);
   static constexpr bool kPrefetch = BN <= 64;                // LoRA delta prefetched into the slots
   static constexpr int kThreads = 224;
-  static_assert(!W8 || kPrefetch, "e4m3 weights use N tiles <= 64");
+  static_assert(!W8 || BN <= 128, "e4m3 weights use N tiles <= 128 (hi and lo planes: N = 2 BN)");
   static_assert(!TWO || (!W8 && BN == 256), "CTA pairs: bf16 weights, N tiles of 256");
 };
 
@@ -335,11 +342,15 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 :
             // both CTAs' copies complete on the leader's barrier, which expects the pair's
             // bytes; the MMA's N is the tile's rows rounded to 32, the peer holds [N/2, N)
             const uint32_t fb = leader_bar(&sm.full[stage]);
-            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2u * Cfg::kStageBytes);
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2u * nj * Cfg::kStageBytes);
             const int n_pair = min(BN, (ti.nvalid + 31) & ~31);
-            tma_load_2d_pair(a_s, &tmw, fb, kc, wrow0);
-            tma_load_2d_pair(a_s + kATileBytes / 2, &tmw, fb, kc, wrow1);
-            tma_load_2d_pair(a_s + kATileBytes, &tmb, fb, kc, ti.row0 + static_cast<int>(rank) * (n_pair / 2));
+            for (int j = 0; j < nj; ++j) {
+              uint8_t* aj = a_s + j * Cfg::kStageBytes;
+              const int kcj = kc + j * Cfg::kKB;
+              tma_load_2d_pair(aj, &tmw, fb, kcj, wrow0);
+              tma_load_2d_pair(aj + kATileBytes / 2, &tmw, fb, kcj, wrow1);
+              tma_load_2d_pair(aj + kATileBytes, &tmb, fb, kcj, ti.row0 + static_cast<int>(rank) * (n_pair / 2));
+            }
           } else {
           mbar_arrive_expect_tx(&sm.full[stage], nj * Cfg::kStageBytes);
           for (int j = 0; j < nj; ++j) {  // sub-stage j: K block kc + j kKB
@@ -700,10 +711,11 @@ CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
 template <int BN, bool W8, bool TWO = false>
 static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   using Cfg = TileCfg<BN, W8, TWO>;
-  // two K blocks per stage for the weight-streaming (decode) tiles: plain base stages only
-  const int kpb = (BN <= 64 && a.K > Cfg::kKB) ? 2 : 1;
+  // two K blocks per stage for the weight-streaming (decode) tiles, and for CTA pairs
+  // (64 KB stages: eight MMAs of M = 256 between the commits that free a stage)
+  const int kpb = ((BN <= 64 || TWO) && a.K > Cfg::kKB) ? 2 : 1;
   const int m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
-  if (TWO && (m_tiles % 2 != 0 || kpb != 1)) return cudaErrorInvalidValue;  // whole pairs of weight tiles
+  if (TWO && m_tiles % 2 != 0) return cudaErrorInvalidValue;  // whole pairs of weight tiles
   // epilogue slots: the fp32 delta part only when the loader prefetches it (whole tiles,
   // N <= 64); one slot instead of two where that buys another ring stage
   const bool dslot = a.delta != nullptr && Cfg::kPrefetch;
@@ -843,7 +855,8 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
     switch (a.bn) {
       case 16: return launch_bn<16, true>(a, st);
       case 32: return launch_bn<32, true>(a, st);
-      default: return launch_bn<64, true>(a, st);
+      case 64: return launch_bn<64, true>(a, st);
+      default: return launch_bn<128, true>(a, st);
     }
   }
   switch (a.bn) {

@@ -47,6 +47,10 @@ struct LoraTcParams {
   int L, E;                   // slot of (adapter a, group e) = a E + e (dense: E = 1, e = 0)
   int K, r, rbox, F, nrows;
   int stages, stage_bytes;
+  // expand stages hold bps feature blocks of expand_bytes each (several per stage, so the
+  // MMA thread commits a stage after more MMAs: a commit costs about as much as several
+  // small MMAs)
+  int bps, expand_bytes;
   __nv_bfloat16* delta;       // [nrows][F]
   const int32_t* scatter;     // delta row of row s: scatter[s] (pair order); null = s
   int* status;
@@ -230,25 +234,29 @@ __global__ void __launch_bounds__(kLtThreads, 1)
           }
           advance();
         }
-        for (int fb = 0; fb < nf && ok; ++fb) {
+        for (int fb0 = 0; fb0 < nf && ok; fb0 += p.bps) {
           ok = acquire();
           if (!ok) break;
-          uint8_t* s = ring + stage * p.stage_bytes;
-          mbar_arrive_expect_tx(&sm.full[stage], 2u * static_cast<uint32_t>(p.rbox) * 128u);
-          if (p.split_I == 0) {
-            tma_load_2d(s, &tmb, &sm.full[stage], fb * 128, arow);
-            tma_load_2d(s + p.rbox * 128, &tmb, &sm.full[stage], fb * 128 + 64, arow);
-          } else {
-            // each 64-feature box: K rows [0, r_exp) then [r_exp, 2 r_exp), one of them the
-            // adapter's B rows and the other zeros (a box past the tensor's last row)
-            const int zrow = p.L * p.E * p.r;  // first row past B
-            for (int h = 0; h < 2; ++h) {
-              const int f = fb * 128 + 64 * h;
-              const bool up = f >= p.split_I;
-              const int fc = up ? f - p.split_I : f;
-              uint8_t* bx = s + h * (p.rbox * 128);
-              tma_load_2d(bx, &tmb, &sm.full[stage], fc, up ? zrow : arow);
-              tma_load_2d(bx + p.r_exp * 128, &tmb, &sm.full[stage], fc, up ? arow + p.r_exp : zrow);
+          const int nb = min(p.bps, nf - fb0);
+          mbar_arrive_expect_tx(&sm.full[stage], static_cast<uint32_t>(nb) * 2u * static_cast<uint32_t>(p.rbox) * 128u);
+          for (int jb = 0; jb < nb; ++jb) {
+            const int fb = fb0 + jb;
+            uint8_t* s = ring + stage * p.stage_bytes + jb * p.expand_bytes;
+            if (p.split_I == 0) {
+              tma_load_2d(s, &tmb, &sm.full[stage], fb * 128, arow);
+              tma_load_2d(s + p.rbox * 128, &tmb, &sm.full[stage], fb * 128 + 64, arow);
+            } else {
+              // each 64-feature box: K rows [0, r_exp) then [r_exp, 2 r_exp), one of them the
+              // adapter's B rows and the other zeros (a box past the tensor's last row)
+              const int zrow = p.L * p.E * p.r;  // first row past B
+              for (int h = 0; h < 2; ++h) {
+                const int f = fb * 128 + 64 * h;
+                const bool up = f >= p.split_I;
+                const int fc = up ? f - p.split_I : f;
+                uint8_t* bx = s + h * (p.rbox * 128);
+                tma_load_2d(bx, &tmb, &sm.full[stage], fc, up ? zrow : arow);
+                tma_load_2d(bx + p.r_exp * 128, &tmb, &sm.full[stage], fc, up ? arow + p.r_exp : zrow);
+              }
             }
           }
           advance();
@@ -313,6 +321,7 @@ __global__ void __launch_bounds__(kLtThreads, 1)
         // segment's whole expand fits in the three accumulators, so the MMAs of the next
         // item's shrink need not wait for this item's epilogue
         const int bpb = 128 / t.n_mma, ng = (nf + bpb - 1) / bpb;
+        int bsub = 0;  // block within the current expand stage
         for (int g = 0; g < ng && ok; ++g, ++acc_i) {
           const int buf = acc_i % kLtAcc;
           const uint32_t use = static_cast<uint32_t>(acc_i / kLtAcc);
@@ -321,19 +330,25 @@ __global__ void __launch_bounds__(kLtThreads, 1)
             break;
           }
           for (int j = 0; j < bpb && g * bpb + j < nf; ++j) {
-            if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kLtWaitNs, 25)) {
-              ok = false;
-              break;
+            if (bsub == 0) {
+              if (!mbar_wait(&sm.full[stage], phase, abort_flag, p.status, kLtWaitNs, 25)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
-            tc_fence_after();
-            const uint64_t adesc = umma_desc_mn_sw128(smem_u32(ring + stage * p.stage_bytes), zdesc_lbo);
+            const uint64_t adesc =
+                umma_desc_mn_sw128(smem_u32(ring + stage * p.stage_bytes + bsub * p.expand_bytes), zdesc_lbo);
             const uint32_t td = tz + 128 + buf * 128 + j * t.n_mma;
             for (int kk = 0; kk < p.rbox / 16; ++kk)  // 16 rank rows (2048 B) per instruction
               umma_bf16(td, adesc + 128 * kk, zdesc + 128 * kk, lidesc, kk > 0 ? 1u : 0u);
-            umma_commit(&sm.empty[stage]);
-            if (++stage == S) {
-              stage = 0;
-              phase ^= 1u;
+            if (++bsub == p.bps || g * bpb + j == nf - 1) {  // the stage's last block: release it
+              bsub = 0;
+              umma_commit(&sm.empty[stage]);
+              if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+              }
             }
           }
           if (!ok) break;
@@ -473,7 +488,9 @@ cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st) {
   if (a.split_I != 0 && (a.split_I % 64 != 0 || a.r != 2 * a.r_exp || a.r % 16 != 0)) return cudaErrorInvalidValue;
   const int shrink_bytes = a.r * 128 + kLtN * 128;
   const int expand_bytes = 2 * rbox * 128;
-  const int stage_bytes = (std::max(shrink_bytes, expand_bytes) + 1023) / 1024 * 1024;
+  // 48 KB stages: several shrink K blocks or expand feature blocks per stage
+  const int stage_bytes = (std::max(std::max(shrink_bytes, expand_bytes), 49152) + 1023) / 1024 * 1024;
+  const int bps = std::min(4, stage_bytes / expand_bytes);
   // after the ring: z tile, epilogue staging, barriers; the shrink MMA reads 128 A rows
   // (16 KB) from each box pair's start, which may reach past the ring into these
   const int tail = 2 * rbox * 128 + 4 * kLtStgWarp + static_cast<int>(sizeof(LtSmem));
@@ -518,6 +535,8 @@ cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st) {
   p.nrows = a.nrows;
   p.stages = stages;
   p.stage_bytes = stage_bytes;
+  p.bps = bps;
+  p.expand_bytes = expand_bytes;
   p.delta = a.delta;
   p.scatter = a.scatter;
   p.status = a.status;

@@ -38,9 +38,8 @@ def test_forward_small_shapes(shape, M):
 @pytest.mark.parametrize("where", ["delta", "tc"])
 @pytest.mark.parametrize("bn", [16, 32, 64, 128, 256])
 def test_forward_every_n_tile(bn, where, monkeypatch):
-    """Every N tile, with the LoRA expand as extra MMA K steps of the GEMM, as the fp32
-    delta of the SIMT LoRA kernel and as the bf16 delta of the tensor-core LoRA kernel,
-    each added by the GEMM epilogue."""
+    """Every N tile, with the LoRA delta from the SIMT LoRA kernel (fp32) and from the
+    tensor-core LoRA kernel (bf16), each added by the GEMM epilogue."""
     monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
     res = run_moe_case(SMALL[0], 300)
@@ -58,6 +57,19 @@ def test_forward_expand_placement(shape, M, where, monkeypatch):
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
     res = run_moe_case(shape, M)
     assert res["err"] <= TOL_BF16, res["err"]
+
+
+@pytest.mark.parametrize("pair", ["0", "1"])
+@pytest.mark.parametrize("shape,M", [(SMALL[0], 300), (SMALL[2], 700), (SMALL[3], 300), (SMALL[7], 600),
+                                     (SMALL[8], 400), (SMALL[9], 300)], ids=lambda v: getattr(v, "name", str(v)))
+def test_forward_n256_single_and_pair(shape, M, pair, monkeypatch):
+    """N tiles of 256 on one CTA and on CTA pairs (cta_group::2): ragged last chunks (the
+    pair's N rounded to 32, split between the CTAs), odd chunk counts, r = 64 and 128,
+    E = 1, K with a ragged last K block."""
+    monkeypatch.setenv("MOE_LORA_FORCE_BN", "256")
+    monkeypatch.setenv("MOE_LORA_PAIR", pair)
+    res = run_moe_case(shape, M)
+    assert res["err"] <= TOL_BF16, (shape.name, res["err"])
 
 
 @pytest.fixture(scope="module")
@@ -189,8 +201,10 @@ def test_forward_fp8_small_shapes(shape, M, record_property):
 
 
 @pytest.mark.parametrize("where", ["delta", "tc"])
-@pytest.mark.parametrize("bn", [16, 32, 64, 256])
+@pytest.mark.parametrize("bn", [16, 32, 64, 128, 256])
 def test_forward_fp8_every_n_tile(bn, where, monkeypatch, record_property):
+    """Every N tile of the e4m3 GEMM (256 is clamped to 128: the two activation planes
+    make the MMA's N twice the tile's)."""
     monkeypatch.setenv("MOE_LORA_FORCE_BN", str(bn))
     monkeypatch.setenv("MOE_LORA_EXPAND", where)
     check_fp8(run_moe_case(SMALL_FP8[1], 150), f"{SMALL_FP8[1].name} bn={bn} {where}", record_property)
