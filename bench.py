@@ -16,9 +16,9 @@ Default workload: the MoE prefill layer, the largest configuration that fits one
 gate_up and down (Zipf adapter ids, router bias skewing the expert load).  The same line
 carries a `sweep` of the decode layers (bf16 E=64 at M = 1, 8, 32, 64; e4m3 experts
 E=128 at M = 1, 4, 16, 64, and the same e4m3 layer at 4096 tokens: FP8 prefill) and the
-dense decode projection, measured in the same process.  For N > 1 (torchrun) every rank runs an independent replica (weak scaling, no
-collective on the data path); timing is the max over ranks.  Prints one JSON line on
-rank 0.
+dense decode projection, measured in the same process.  For N > 1 (torchrun) every rank
+runs an independent replica (weak scaling, no collective on the data path); timing is
+the max over ranks.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
@@ -53,7 +53,8 @@ SWEEP = ((synth.MOE_DECODE_BF16.name, (1, 8, 32, 64)), (synth.MOE_DECODE_FP8.nam
 # ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM, with the
 # hash of the kernel source it was taken on and the case it was taken on; reported as
 # null when the source has changed since or the case differs.  Filled from profiles/.
-NCU_TRAFFIC = {"gemm_tc.cu": "", "bytes_per_launch": 0.0, "workload": "", "M": 0}
+NCU_TRAFFIC = {"gemm_tc.cu": "6769753932579f83", "bytes_per_launch": 4952061184.0 + 108819968.0,
+               "workload": "moe_prefill_bf16_e128_h4096_i1536", "M": 4096}
 
 
 def parse(argv=None):
@@ -860,10 +861,17 @@ def run_sweep(args, world, local, skip: str) -> list:
             est = measure_moe(args, shape, M, W, world, local, steps=10, warmup=3, full=False)
             n = sweep_steps(est["ms_per_step"], args.sweep_seconds)
             m = measure_moe(args, shape, M, W, world, local, steps=n, warmup=10, full=False)
-            res.append({"workload": name, "M": M, "tokens_per_s": m["value"], "ms_per_step": m["ms_per_step"],
-                        "steps": n, "layer_frac_of_hbm_peak": m["layer"]["frac_of_hbm_peak"],
-                        "gate_up": {kk: m["roofline"][kk] for kk in ("bound", "achieved", "unit", "frac")},
-                        "kernel_ms_per_step": m["layer"]["kernel_ms_per_step"], "gpu_launches": m["gpu_launches"]})
+            ent = {"workload": name, "M": M, "tokens_per_s": m["value"], "ms_per_step": m["ms_per_step"],
+                   "steps": n, "layer_frac_of_hbm_peak": m["layer"]["frac_of_hbm_peak"],
+                   "gate_up": {kk: m["roofline"][kk] for kk in ("bound", "achieved", "unit", "frac")},
+                   "kernel_ms_per_step": m["layer"]["kernel_ms_per_step"], "gpu_launches": m["gpu_launches"],
+                   "launches_per_step": m["gpu_launches"] / max(1, n)}
+            frac, ms = m["layer"]["frac_of_hbm_peak"], m["ms_per_step"]
+            if frac < 0.70:  # what holds the step below the layer's copy-peak time
+                ent["bound_by"] = (f"launch latency: {ent['launches_per_step']:.0f} dependent kernel launches per "
+                                   f"step; the layer's bytes at the copy peak take {frac * ms * 1e3:.1f} us of "
+                                   f"{ms * 1e3:.1f} us")
+            res.append(ent)
         del W
         torch.cuda.empty_cache()
     return res

@@ -64,6 +64,12 @@ struct LoraTcParams {
   float scale;                // multiplies every delta value
 };
 
+struct LtItem {
+  int lo, hi, n, n_mma, box, slot;
+  int kpb;                    // K blocks of 64 per shrink stage (short segments: several)
+  bool lora;                  // the segment has an adapter (else delta = 0 rows)
+};
+
 struct LtSmem {
   uint64_t full[kLtMaxStages];
   uint64_t empty[kLtMaxStages];
@@ -75,16 +81,12 @@ struct LtSmem {
   uint64_t qfull[4];          // work-item queue: the producer claims items ...
   uint64_t qempty[4];         // ... and the MMA thread and the epilogue release the slot
   int q[4];
+  LtItem qi[4];               // the claimed items, decoded once by the producer
   uint32_t tmem_base;
   int abort_flag;
   int rowmap[kLtN];           // delta row of each row of the epilogue's current item
 };
 
-struct LtItem {
-  int lo, hi, n, n_mma, box, slot;
-  int kpb;                    // K blocks of 64 per shrink stage (short segments: several)
-  bool lora;                  // the segment has an adapter (else delta = 0 rows)
-};
 
 constexpr int kLtStgPitch = 80;               // bytes per staged row of 32 bf16 (16-byte aligned)
 constexpr int kLtStgWarp = 32 * kLtStgPitch;  // one epilogue warp's staging block
@@ -201,10 +203,11 @@ __global__ void __launch_bounds__(kLtThreads, 1)
         if (!mbar_wait(&sm.qempty[qs], ((qi >> 2) & 1) ^ 1u, abort_flag, p.status, kLtWaitNs, 20)) break;
         int it = atomicAdd(p.work_counter, 1);
         if (it >= count) it = -1;
+        const LtItem t = it >= 0 ? lt_item(p, it) : LtItem{};
         sm.q[qs] = it;
+        sm.qi[qs] = t;
         mbar_arrive(&sm.qfull[qs]);
         if (it < 0) break;
-        const LtItem t = lt_item(p, it);
         if (!t.lora) continue;
         const int arow = t.slot * p.r;
         const CUtensorMap* xm = t.box == 0 ? &tmx16 : t.box == 1 ? &tmx32 : t.box == 2 ? &tmx64 : &tmx128;
@@ -282,9 +285,9 @@ __global__ void __launch_bounds__(kLtThreads, 1)
         const int qs = qi & 3;
         if (!mbar_wait(&sm.qfull[qs], (qi >> 2) & 1, abort_flag, p.status, kLtWaitNs, 28)) break;
         const int it = static_cast<volatile int*>(sm.q)[qs];
+        const LtItem t = sm.qi[qs];
         mbar_arrive(&sm.qempty[qs]);
         if (it < 0) break;
-        const LtItem t = lt_item(p, it);
         if (!t.lora) continue;
         // shrink: z[i][j] = sum_k A[i][k] x[j][k]; rows i >= r of the accumulator are unused
         const uint32_t idesc = umma_idesc_bf16(128, t.n_mma);
@@ -373,10 +376,10 @@ __global__ void __launch_bounds__(kLtThreads, 1)
       const int qs = qi & 3;
       const bool gq = mbar_wait(&sm.qfull[qs], (qi >> 2) & 1, abort_flag, p.status, kLtWaitNs, 29);
       const int it = gq ? static_cast<volatile int*>(sm.q)[qs] : -1;
+      const LtItem t = sm.qi[qs];
       if (!named_bar_and(3, kLtEpi, gq)) break;  // every thread has read the slot
       if (et == 0) mbar_arrive(&sm.qempty[qs]);
       if (it < 0) break;
-      const LtItem t = lt_item(p, it);
       if (t.n <= 0) continue;
       // the item's delta rows, read once (the previous item's readers are past the
       // queue barrier above)

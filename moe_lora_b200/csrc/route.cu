@@ -171,18 +171,42 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 }
 
 // ---------------------------------------------------------------- stable scatter
+// Slot j of token t routed to expert e, or -1: the token's k ids read as 16-byte
+// vectors when k is a multiple of 4 (one load chain per token instead of k).
+__device__ __forceinline__ int slot_of(const int32_t* __restrict__ topk_ids, int t, int k, int e) {
+  const int32_t* row = topk_ids + static_cast<size_t>(t) * k;
+  if ((k & 3) == 0 && k <= 16) {
+    int4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (4 * q < k) v[q] = __ldg(reinterpret_cast<const int4*>(row) + q);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (4 * q < k) {
+        if (v[q].x == e) return 4 * q;
+        if (v[q].y == e) return 4 * q + 1;
+        if (v[q].z == e) return 4 * q + 2;
+        if (v[q].w == e) return 4 * q + 3;
+      }
+    return -1;
+  }
+  for (int j = 0; j < k; ++j)
+    if (row[j] == e) return j;
+  return -1;
+}
+
 // One block per expert e.  (1) Exclusive prefix of the key counts gives the CSR
-// offsets of e's L+1 keys.  (2) The 8 warps split the tokens into 8 contiguous
+// offsets of e's L+1 keys.  (2) The 16 warps split the tokens into 16 contiguous
 // ranges; each warp counts its pairs per adapter key, the counts are prefixed over
 // warps, then each warp walks its range in token order and places its pairs with a
 // warp match on the key: positions are stable (ascending token within a key).
-__global__ void __launch_bounds__(256) sort_scatter_kernel(const int32_t* __restrict__ topk_ids,
+__global__ void __launch_bounds__(512) sort_scatter_kernel(const int32_t* __restrict__ topk_ids,
                                                           const int32_t* __restrict__ a_key,
                                                           const int32_t* __restrict__ key_count,
                                                           int M, int k, int E, int L,
                                                           int32_t* __restrict__ sorted_pairs,
                                                           int32_t* __restrict__ seg_offsets) {
-  constexpr int NW = 8;
+  constexpr int NW = 16;
   __shared__ int s_red[NW];
   __shared__ int s_off[65];
   __shared__ int s_wcnt[NW][65];
@@ -216,14 +240,8 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(const int32_t* __rest
   // (2a) per-warp counts
   const int chunk = (M + NW - 1) / NW;
   const int tb = warp * chunk, te = min(M, tb + chunk);
-  for (int t = tb + lane; t < te; t += 32) {
-    for (int j = 0; j < k; ++j) {
-      if (topk_ids[static_cast<size_t>(t) * k + j] == e) {
-        atomicAdd(&s_wcnt[warp][a_key[t]], 1);
-        break;
-      }
-    }
-  }
+  for (int t = tb + lane; t < te; t += 32)
+    if (slot_of(topk_ids, t, k, e) >= 0) atomicAdd(&s_wcnt[warp][a_key[t]], 1);
   __syncthreads();
   if (threadIdx.x < LA) {
     int acc = 0;
@@ -240,11 +258,7 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(const int32_t* __rest
     const int t = tb32 + lane;
     int jf = -1, ap = 0;
     if (t < te) {
-      for (int j = 0; j < k; ++j)
-        if (topk_ids[static_cast<size_t>(t) * k + j] == e) {
-          jf = j;
-          break;
-        }
+      jf = slot_of(topk_ids, t, k, e);
       ap = a_key[t];
     }
     const int keyv = (jf >= 0) ? ap : (LA + lane);
@@ -552,7 +566,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   }
   {
     ProfScope ps(K_SORT, st);
-    sort_scatter_kernel<<<a.E, 256, 0, st>>>(a.topk_ids, a.a_key, a.key_count, a.M, a.k, a.E, a.L,
+    sort_scatter_kernel<<<a.E, 512, 0, st>>>(a.topk_ids, a.a_key, a.key_count, a.M, a.k, a.E, a.L,
                                              a.sorted_pairs, a.seg_offsets);
     count_launch();
   }

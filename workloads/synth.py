@@ -92,8 +92,13 @@ MOE_DECODE_FP8 = MoEShape("moe_decode_fp8_e128_h7168_i2048", 4, E=128, k=8, H=71
                           L=32, r=32, wdtype="e4m3", bias=True, adapter_dist="zipf",
                           M_list=(1, 4, 16, 64))
 
+# A profiling-size cut of the prefill layer: a quarter of the experts and tokens, so 256
+# pairs per expert (the full layer's tile shapes) with about 2 GB of weights on the device.
+MOE_PREFILL_BF16_SMALL = MOE_PREFILL_BF16.with_(name="moe_prefill_bf16_e32_h4096_i1536", wid=5, E=32,
+                                                M_list=(1024,))
+
 WORKLOADS = {w.name: w for w in (SGMV_F32, DENSE_DECODE_BF16, MOE_DECODE_BF16,
-                                 MOE_PREFILL_BF16, MOE_DECODE_FP8)}
+                                 MOE_PREFILL_BF16, MOE_DECODE_FP8, MOE_PREFILL_BF16_SMALL)}
 
 
 def rng(*key: int) -> np.random.Generator:
