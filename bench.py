@@ -793,8 +793,32 @@ def measure_moe(args, shape: synth.MoEShape, M: int, W: dict, world, local, *, s
             "lora_overhead_ms_per_step": step_ms - t_none, "base_only_ms_per_step": t_none,
             "same_adapter_ms_per_step": t_same, "distinct_adapters_ms_per_step": step_ms,
             "adapters": f"{shape.adapter_dist} over L={L}",
-            "swap_ab": "not measured: only the swapped (weights in the 128-row MMA M slot) tile exists",
         }
+        if M * k >= 256 * shape.E and shape.wdtype == "bf16":
+            # the operand swap at prefill tiles: weights in M (one CTA per 128 x 256 tile, and
+            # CTA pairs, the default) against tokens in M (128 tokens x 256 weight rows)
+            def with_env(env, fn):
+                old = {kk: os.environ.get(kk) for kk in env}
+                os.environ.update(env)
+                try:
+                    return fn()
+                finally:
+                    for kk, vv in old.items():
+                        if vv is None:
+                            os.environ.pop(kk, None)
+                        else:
+                            os.environ[kk] = vv
+            same = lambda ab: ab  # noqa: E731
+            t_single = with_env({"MOE_LORA_PAIR": "0"}, lambda: timed_variant(same))
+            t_unswapped = with_env({"MOE_LORA_SWAP": "0"}, lambda: timed_variant(same))
+            out["secondary"]["swap_ab"] = {
+                "weights_in_m_cta_pairs_ms_per_step": step_ms, "weights_in_m_one_cta_ms_per_step": t_single,
+                "tokens_in_m_ms_per_step": t_unswapped,
+                "tiles": "weights in M: 128 (one CTA) or 256 (pair) weight rows x 256 tokens; tokens in M: 128 "
+                         "tokens x 256 weight rows; both GEMMs of the layer"}
+        else:
+            out["secondary"]["swap_ab"] = ("decode: only the swapped tile (weights in M) is built; a tile with "
+                                           "tokens in M would leave most of the MMA's 128 rows empty")
 
     # ---- e2e: pinned host inputs -> device, route + forward, y -> pinned host, every step
     e2e_steps = args.e2e_steps or steps

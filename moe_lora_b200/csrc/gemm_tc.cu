@@ -166,7 +166,11 @@ constexpr int pow2_at_least(int v) {
 
 // TWO: a CTA pair (cta_group::2) computes 256 weight rows x BN tokens; each CTA holds its
 // 128 weight rows and half of the BN token rows of every stage.
-template <int BN, bool W8, bool TWO = false>
+// NS (not swapped, for the operand-swap comparison): tokens in the MMA's M slot (chunks of
+// kNsTok = 128 token rows), weight rows in N (BN = 256: for gate_up 128 gate rows and the
+// matching 128 up rows, for down 256 output rows).
+constexpr int kNsTok = 128;
+template <int BN, bool W8, bool TWO = false, bool NS = false>
 struct TileCfg {
   static constexpr int kKB = W8 ? 128 : 64;                  // K per stage (128 bytes per row)
   static constexpr int kBRows = TWO ? BN / 2 : BN;           // token rows held by this CTA
@@ -179,6 +183,8 @@ struct TileCfg {
   static constexpr int kThreads = 224;
   static_assert(!W8 || BN <= 128, "e4m3 weights use N tiles <= 128 (hi and lo planes: N = 2 BN)");
   static_assert(!TWO || (!W8 && BN == 256), "CTA pairs: bf16 weights, N tiles of 256");
+  static_assert(!NS || (!W8 && !TWO && BN == 256), "tokens in M: bf16 weights, 256 weight rows in N");
+  static constexpr int kTokRows = NS ? kNsTok : BN;          // token rows per tile
 };
 
 struct TileInfo {
@@ -207,13 +213,13 @@ __device__ __forceinline__ int delta_col(int epi, int m, int f0, int I) {
   return f0 + m;
 }
 
-template <int BN, bool W8, bool TWO>
-__global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 : 1)
+template <int BN, bool W8, bool TWO, bool NS>
+__global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ? 2 : 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tml, const __grid_constant__ CUtensorMap tmd,
                    const TcParams p) {
   // tml: the lo activation plane (e4m3 weights); tmd: the fp32 LoRA delta (N tiles <= 64)
-  using Cfg = TileCfg<BN, W8, TWO>;
+  using Cfg = TileCfg<BN, W8, TWO, NS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;                                 // stages: [A tile][token tile(s)]
@@ -271,7 +277,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 :
       int c = 0;
       if (g < p.E) {
         const int n = sm.grp_off[g + 1] - sm.grp_off[g];
-        c = n > 0 ? (n + BN - 1) / BN : 0;
+        c = n > 0 ? (n + Cfg::kTokRows - 1) / Cfg::kTokRows : 0;
       }
       cnt[i] = c;
       tot += c;
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 :
   const int unit_m = TWO ? p.m_tiles / 2 : p.m_tiles;
   const int total_tiles = sm.chunk_pref[p.E] * unit_m;
   auto tile_of = [&](int t) -> TileInfo {
-    TileInfo ti = decode_tile(sm, t, unit_m, p.E, BN);
+    TileInfo ti = decode_tile(sm, t, unit_m, p.E, Cfg::kTokRows);
     if constexpr (TWO) ti.mt = 2 * ti.mt + static_cast<int>(rank);
     return ti;
   };
@@ -322,7 +328,15 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 :
       if (*abort_flag) break;
       const TileInfo ti = tile_of(u.t);
       int wrow0, wrow1;
-      if (p.epi == EPI_GATEUP) {
+      if constexpr (NS) {  // 128-row weight boxes: gate and up halves, or two halves of 256 rows
+        if (p.epi == EPI_GATEUP) {
+          wrow0 = ti.g * p.rows_per_group + ti.mt * 128;
+          wrow1 = ti.g * p.rows_per_group + p.I + ti.mt * 128;
+        } else {
+          wrow0 = ti.g * p.rows_per_group + ti.mt * 256;
+          wrow1 = wrow0 + 128;
+        }
+      } else if (p.epi == EPI_GATEUP) {
         wrow0 = ti.g * p.rows_per_group + ti.mt * 64;
         wrow1 = ti.g * p.rows_per_group + p.I + ti.mt * 64;
       } else {
@@ -350,6 +364,16 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 :
               tma_load_2d_pair(aj, &tmw, fb, kcj, wrow0);
               tma_load_2d_pair(aj + kATileBytes / 2, &tmw, fb, kcj, wrow1);
               tma_load_2d_pair(aj + kATileBytes, &tmb, fb, kcj, ti.row0 + static_cast<int>(rank) * (n_pair / 2));
+            }
+          } else if constexpr (NS) {
+            // A = the chunk's 128 token rows, B = the two 128-row weight boxes
+            mbar_arrive_expect_tx(&sm.full[stage], nj * Cfg::kStageBytes);
+            for (int j = 0; j < nj; ++j) {
+              uint8_t* aj = a_s + j * Cfg::kStageBytes;
+              const int kcj = kc + j * Cfg::kKB;
+              tma_load_2d(aj, &tmb, &sm.full[stage], kcj, ti.row0);
+              tma_load_2d(aj + kATileBytes, &tmw, &sm.full[stage], kcj, wrow0);
+              tma_load_2d(aj + kATileBytes + Cfg::kBTileBytes / 2, &tmw, &sm.full[stage], kcj, wrow1);
             }
           } else {
           mbar_arrive_expect_tx(&sm.full[stage], nj * Cfg::kStageBytes);
@@ -408,7 +432,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 :
         const TileInfo ti = tile_of(u.t);
         // e4m3: the hi and lo planes sit back to back in the ring, so one instruction of
         // N = 2 BN covers both and each weight tile is read from shared memory once
-        const int n_mma = TWO ? min(BN, (ti.nvalid + 31) & ~31) : min(BN, (ti.nvalid + 15) & ~15);
+        const int n_mma = NS ? BN : TWO ? min(BN, (ti.nvalid + 31) & ~31) : min(BN, (ti.nvalid + 15) & ~15);
         const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, 2 * BN) : umma_idesc_bf16(TWO ? 2 * kBM : kBM, n_mma);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
@@ -487,6 +511,94 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO>::kThreads, BN <= 64 ? 2 :
       float scale = 1.f;
       if (p.w_scales != nullptr) scale = p.w_scales[ti.g * 2 + p.scale_idx];
       const EpiSlot<BN>* slot = reinterpret_cast<const EpiSlot<BN>*>(slots + sb * p.slot_bytes);
+
+      if constexpr (NS) {
+        // tokens in the TMEM lanes: thread m holds token row row0 + m, the columns are
+        // weight rows (gate_up: 128 gate columns, then the matching 128 up columns)
+        const int row = ti.row0 + m;
+        const bool tok_ok = m < ti.nvalid;
+        const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(g4 * 32) << 16) + buf * Cfg::kAccPerBuf * Cfg::kAccStride;
+        if (p.epi == EPI_GATEUP) {
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            float gv[32], uv[32];
+            tmem_ld_32x32b_x32(t_acc + c0, gv);
+            tmem_ld_32x32b_x32(t_acc + 128 + c0, uv);
+            const int f = ti.mt * 128 + c0;
+            if (!tok_ok || f >= p.I) continue;
+#pragma unroll
+            for (int n = 0; n < 32; ++n) {
+              gv[n] *= scale;
+              uv[n] *= scale;
+            }
+            if (p.delta_bf16 != nullptr) {  // this row's 32 gate and 32 up delta values
+              const __nv_bfloat16* dr = p.delta_bf16 + static_cast<size_t>(row) * p.delta_cols;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                if (f + 8 * q + 8 > p.I) break;
+                float dg[8], du[8];
+                unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(dr + f + 8 * q)), dg);
+                unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(dr + p.I + f + 8 * q)), du);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  gv[8 * q + e] += dg[e];
+                  uv[8 * q + e] += du[e];
+                }
+              }
+            }
+            uint32_t packed[16];
+#pragma unroll
+            for (int n = 0; n < 16; ++n)
+              packed[n] = pack2_bf16(silu(gv[2 * n]) * uv[2 * n], silu(gv[2 * n + 1]) * uv[2 * n + 1]);
+            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(row) * p.I + f;
+            if (f + 32 <= p.I) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                reinterpret_cast<uint4*>(dst)[q] =
+                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            } else {
+              for (int n = 0; n < 32 && f + n < p.I; ++n)
+                reinterpret_cast<uint16_t*>(dst)[n] =
+                    static_cast<uint16_t>((n & 1) ? (packed[n >> 1] >> 16) : (packed[n >> 1] & 0xFFFFu));
+            }
+          }
+        } else {  // EPI_DOWN: the routing pair of this row, weighted
+          int pr = 0;
+          float w = 0.f;
+          if (tok_ok) {
+            pr = p.sorted_pairs[row];
+            if (pr < 0 || pr >= p.total_rows) {  // a corrupted pair index is not followed
+              set_status(p.status, MOE_LORA_ERR_DEVICE_CHECK, row);
+              pr = -1;
+            } else {
+              w = p.topk_w[pr];
+            }
+          }
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            float v[32];
+            tmem_ld_32x32b_x32(t_acc + c0, v);
+            const int f = ti.mt * 256 + c0;
+            if (!tok_ok || pr < 0 || f >= p.n_out) continue;
+            uint32_t packed[16];
+#pragma unroll
+            for (int n = 0; n < 16; ++n) packed[n] = pack2_bf16(w * scale * v[2 * n], w * scale * v[2 * n + 1]);
+            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(pr) * p.n_out + f;
+            if (f + 32 <= p.n_out) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                reinterpret_cast<uint4*>(dst)[q] =
+                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            } else {
+              for (int n = 0; n < 32 && f + n < p.n_out; ++n)
+                reinterpret_cast<uint16_t*>(dst)[n] =
+                    static_cast<uint16_t>((n & 1) ? (packed[n >> 1] >> 16) : (packed[n >> 1] & 0xFFFFu));
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.tempty[buf]);
+        mbar_arrive(&sm.sempty[sb]);
+        continue;
+      }
 
       // bf16 delta [rows][delta_cols] (token-major): lane L of a warp loads row c0 + L's 32
       // delta columns of the warp (64 contiguous bytes, one chunk ahead), the warp passes
@@ -708,14 +820,16 @@ CUresult encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-template <int BN, bool W8, bool TWO = false>
+template <int BN, bool W8, bool TWO = false, bool NS = false>
 static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
-  using Cfg = TileCfg<BN, W8, TWO>;
+  using Cfg = TileCfg<BN, W8, TWO, NS>;
   // two K blocks per stage for the weight-streaming (decode) tiles, and for CTA pairs
   // (64 KB stages: eight MMAs of M = 256 between the commits that free a stage)
   const int kpb = ((BN <= 64 || TWO) && a.K > Cfg::kKB) ? 2 : 1;
-  const int m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
+  const int m_tiles = NS ? ((a.epi == EPI_GATEUP) ? (a.I + 127) / 128 : (a.n_out + 255) / 256)
+                         : (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
   if (TWO && m_tiles % 2 != 0) return cudaErrorInvalidValue;  // whole pairs of weight tiles
+  if (NS && (a.delta != nullptr || (a.epi != EPI_GATEUP && a.epi != EPI_DOWN))) return cudaErrorInvalidValue;
   // epilogue slots: the fp32 delta part only when the loader prefetches it (whole tiles,
   // N <= 64); one slot instead of two where that buys another ring stage
   const bool dslot = a.delta != nullptr && Cfg::kPrefetch;
@@ -742,7 +856,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   const int dev = current_device_index();
   if (dev < 0) return cudaErrorInvalidDevice;
   if (!attr_set[dev].load(std::memory_order_acquire)) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO>,
+    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, W8, TWO, NS>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
@@ -759,9 +873,10 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
       return cudaErrorInvalidValue;
   } else {
     if (encode_tmap_2d(&tmw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.w, a.K, wrows, static_cast<uint64_t>(a.K) * 2, kBK,
-                       64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+                       NS ? 128 : 64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         encode_tmap_2d(&tmb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
-                       static_cast<uint64_t>(a.K) * 2, kBK, Cfg::kBRows, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                       static_cast<uint64_t>(a.K) * 2, kBK, NS ? kNsTok : Cfg::kBRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     tml = tmb;  // unused
   }
@@ -805,7 +920,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.nslots = nslots;
   p.slot_bytes = slot_bytes;
   p.slot_delta = dslot ? 1 : 0;
-  const long long chunks_ub = (a.total_rows + BN - 1) / BN + a.E;
+  const long long chunks_ub = (a.total_rows + Cfg::kTokRows - 1) / Cfg::kTokRows + a.E;
   const long long tiles_ub = chunks_ub * (TWO ? p.m_tiles / 2 : p.m_tiles);
   int grid = a.num_sms;
   if constexpr (TWO) {  // whole clusters of two CTAs
@@ -840,7 +955,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO>, tmw, tmb, tml, tmd, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, W8, TWO, NS>, tmw, tmb, tml, tmd, p);
   count_launch();
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -869,6 +984,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
       // 16 KB weight tile and half of the token tile, so the same shared memory holds more
       // stages and each byte staged feeds twice the MMA work.  MOE_LORA_PAIR=0|1 overrides.
       const int m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
+      // MOE_LORA_SWAP=0: tokens in M and weights in N (the operand-swap comparison)
+      const char* sw = std::getenv("MOE_LORA_SWAP");
+      if (sw != nullptr && std::atoi(sw) == 0 && a.delta == nullptr && (a.epi == EPI_GATEUP || a.epi == EPI_DOWN))
+        return launch_bn<256, false, false, true>(a, st);
       const char* v = std::getenv("MOE_LORA_PAIR");
       const bool pair = (v != nullptr ? std::atoi(v) != 0 : kPairDefault) && m_tiles % 2 == 0 && a.K > kBK &&
                         (a.epi == EPI_GATEUP || a.epi == EPI_DOWN || a.epi == EPI_DENSE);

@@ -59,15 +59,19 @@ def test_forward_expand_placement(shape, M, where, monkeypatch):
     assert res["err"] <= TOL_BF16, res["err"]
 
 
-@pytest.mark.parametrize("pair", ["0", "1"])
+@pytest.mark.parametrize("variant", ["single", "pair", "tokens_in_m"])
 @pytest.mark.parametrize("shape,M", [(SMALL[0], 300), (SMALL[2], 700), (SMALL[3], 300), (SMALL[7], 600),
                                      (SMALL[8], 400), (SMALL[9], 300)], ids=lambda v: getattr(v, "name", str(v)))
-def test_forward_n256_single_and_pair(shape, M, pair, monkeypatch):
-    """N tiles of 256 on one CTA and on CTA pairs (cta_group::2): ragged last chunks (the
-    pair's N rounded to 32, split between the CTAs), odd chunk counts, r = 64 and 128,
-    E = 1, K with a ragged last K block."""
+def test_forward_n256_single_pair_and_unswapped(shape, M, variant, monkeypatch):
+    """Tiles of 256 tokens on one CTA and on CTA pairs (cta_group::2: ragged last chunks,
+    the pair's N rounded to 32 and split between the CTAs, odd chunk counts), and the
+    unswapped tile (128 tokens in M, 256 weight rows in N); r = 64 and 128, E = 1, K with
+    a ragged last K block, I and H not multiples of the weight tile."""
     monkeypatch.setenv("MOE_LORA_FORCE_BN", "256")
-    monkeypatch.setenv("MOE_LORA_PAIR", pair)
+    monkeypatch.setenv("MOE_LORA_EXPAND", "tc")
+    monkeypatch.setenv("MOE_LORA_PAIR", "1" if variant == "pair" else "0")
+    if variant == "tokens_in_m":
+        monkeypatch.setenv("MOE_LORA_SWAP", "0")
     res = run_moe_case(shape, M)
     assert res["err"] <= TOL_BF16, (shape.name, res["err"])
 
