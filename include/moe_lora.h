@@ -45,6 +45,9 @@
  *                               Default: "tc" above 64 rows per expert, "delta" below.
  *   MOE_LORA_PAIR=0|1           N tiles of 256 on CTA pairs (tcgen05 cta_group::2, M = 256);
  *                               default 1.
+ *   MOE_LORA_SWAP=0             tiles of 256 with tokens in the MMA's M (128 tokens x 256 weight
+ *                               rows per CTA) instead of weights in M; bf16 weights and the
+ *                               tensor-core LoRA placement only (default: weights in M).
  *   MOE_LORA_FORCE_BN=16|32|64|128|256  the GEMM's token tile (default: from the mean rows
  *                               per group: <= 12 -> 16, <= 24 -> 32, <= 64 -> 64, <= 96 -> 128,
  *                               else 256).

@@ -695,12 +695,31 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
             }
           }
         } else if (p.epi == EPI_DOWN) {
-          if (row_ok) {
-            const int* cp = slot->col_pair + c0;
-            const float* cw = slot->col_w + c0;
+          // through ebuf (thread m's 32 columns into row m), then lane n of warp g4 writes
+          // the 32 features [32 g4, 32 g4 + 32) of token column n as four 16-byte runs, so
+          // a routing pair's row leaves as whole 64-byte pieces
 #pragma unroll
-            for (int n = 0; n < 32; ++n)
-              if (n < ncol) p.out_bf16[static_cast<size_t>(cp[n]) * p.n_out + feat] = __float2bfloat16_rn(v[n] * cw[n]);
+          for (int n = 0; n < 32; ++n) sm.ebuf[m][n] = v[n];
+          named_bar_sync(1, kEpiThreads);
+          const int n = lane;
+          const int fbase = f0 + g4 * 32;
+          if (n < ncol && fbase < p.n_out) {
+            const float w = slot->col_w[c0 + n];
+            __nv_bfloat16* dst = p.out_bf16 + static_cast<size_t>(slot->col_pair[c0 + n]) * p.n_out + fbase;
+            uint32_t packed[16];
+#pragma unroll
+            for (int f = 0; f < 16; ++f)
+              packed[f] = pack2_bf16(w * sm.ebuf[g4 * 32 + 2 * f][n], w * sm.ebuf[g4 * 32 + 2 * f + 1][n]);
+            if (fbase + 32 <= p.n_out) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                reinterpret_cast<uint4*>(dst)[q] =
+                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            } else {
+              for (int f = 0; f < 32 && fbase + f < p.n_out; ++f)
+                reinterpret_cast<uint16_t*>(dst)[f] =
+                    static_cast<uint16_t>((f & 1) ? (packed[f >> 1] >> 16) : (packed[f >> 1] & 0xFFFFu));
+            }
           }
         } else if (p.epi == EPI_LOGITS) {
           if (row_ok) {

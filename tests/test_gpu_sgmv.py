@@ -24,6 +24,12 @@ CASES = [
     # r h_in >= 65536: split LoRA shrink with a ragged last K slice
     synth.DENSE_DECODE_BF16.with_(name="bf16_split", wid=304, T=45, h_in=2056, h_out=264, L=5, r=32,
                                   no_adapter_frac=0.2),
+    # 8 weight tiles, the last one 104 rows, K = 4096
+    synth.DENSE_DECODE_BF16.with_(name="bf16_k4096_ragged_m", wid=306, T=50, h_in=4096, h_out=1000, L=6, r=16,
+                                  no_adapter_frac=0.2),
+    # two token chunks (256 + a ragged 44) of 5 weight tiles each
+    synth.DENSE_DECODE_BF16.with_(name="bf16_two_chunks", wid=307, T=300, h_in=2048, h_out=640, L=4,
+                                  r=32),
 ]
 
 
@@ -109,3 +115,4 @@ def test_dense_many_segments(where, monkeypatch):
     y_ref = ref.dense_lora_forward(d["x64"], d["w64"], d["a64"], d["b64"], offs, segs)
     err = rel_err(y, y_ref)
     assert err <= TOL_BF16, err
+
