@@ -253,8 +253,8 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmw);
     tma_prefetch_desc(&tmb);
-    if (W8) tma_prefetch_desc(&tml);
-    if (p.delta != nullptr) tma_prefetch_desc(&tmd);
+    if (W8 || TWO) tma_prefetch_desc(&tml);
+    if (p.delta != nullptr || TWO) tma_prefetch_desc(&tmd);
   }
   if (warp == 1) {
     if constexpr (TWO) tmem_alloc_pair(&sm.tmem_base, Cfg::kTmemCols);
@@ -356,14 +356,19 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
             // both CTAs' copies complete on the leader's barrier, which expects the pair's
             // bytes; the MMA's N is the tile's rows rounded to 32, the peer holds [N/2, N)
             const uint32_t fb = leader_bar(&sm.full[stage]);
-            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2u * nj * Cfg::kStageBytes);
             const int n_pair = min(BN, (ti.nvalid + 31) & ~31);
+            // each CTA's half of the token rows from the smallest box that holds it (32, 64
+            // or 128 rows), so a ragged chunk does not stream the next group's rows
+            const int half = n_pair / 2;
+            const CUtensorMap* bm = half <= 32 ? &tml : half <= 64 ? &tmd : &tmb;
+            const uint32_t bbytes = (half <= 32 ? 32u : half <= 64 ? 64u : 128u) * 128u;
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2u * nj * (kATileBytes + bbytes));
             for (int j = 0; j < nj; ++j) {
               uint8_t* aj = a_s + j * Cfg::kStageBytes;
               const int kcj = kc + j * Cfg::kKB;
               tma_load_2d_pair(aj, &tmw, fb, kcj, wrow0);
               tma_load_2d_pair(aj + kATileBytes / 2, &tmw, fb, kcj, wrow1);
-              tma_load_2d_pair(aj + kATileBytes, &tmb, fb, kcj, ti.row0 + static_cast<int>(rank) * (n_pair / 2));
+              tma_load_2d_pair(aj + kATileBytes, bm, fb, kcj, ti.row0 + static_cast<int>(rank) * half);
             }
           } else if constexpr (NS) {
             // A = the chunk's 128 token rows, B = the two 128-row weight boxes
@@ -898,8 +903,17 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
                        CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     tml = tmb;  // unused
+    if constexpr (TWO) {  // token boxes of 32 and 64 rows for ragged chunks (tml, tmd)
+      if (encode_tmap_2d(&tml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
+                         static_cast<uint64_t>(a.K) * 2, kBK, 32, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+          encode_tmap_2d(&tmd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.b, a.K, a.total_rows,
+                         static_cast<uint64_t>(a.K) * 2, kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    }
   }
-  if (a.delta != nullptr && Cfg::kPrefetch) {
+  if (TWO) {
+    // tmd holds the 64-row token box (pairs take no fp32 delta)
+  } else if (a.delta != nullptr && Cfg::kPrefetch) {
     if (encode_tmap_2d(&tmd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.delta, a.delta_cols, a.total_rows,
                        static_cast<uint64_t>(a.delta_cols) * 4, 64, BN, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
