@@ -53,7 +53,7 @@ SWEEP = ((synth.MOE_DECODE_BF16.name, (1, 8, 32, 64)), (synth.MOE_DECODE_FP8.nam
 # ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM, with the
 # hash of the kernel source it was taken on and the case it was taken on; reported as
 # null when the source has changed since or the case differs.  Filled from profiles/.
-NCU_TRAFFIC = {"gemm_tc.cu": "6769753932579f83", "bytes_per_launch": 4952061184.0 + 108819968.0,
+NCU_TRAFFIC = {"gemm_tc.cu": "19dc9a8ae004c27c", "bytes_per_launch": 4617012992.0 + 111399936.0,
                "workload": "moe_prefill_bf16_e128_h4096_i1536", "M": 4096}
 
 
@@ -859,6 +859,21 @@ def sweep_steps(est_ms: float, seconds: float) -> int:
     return int(min(4000, max(20, seconds * 1e3 / max(est_ms, 1e-3))))
 
 
+def bound_by(ent: dict, gemm: dict) -> str:
+    """What holds a sweep step below the layer's copy-peak time: the GEMMs' share against
+    the rest of the step, kernel by kernel (event-timed), and the launches per step."""
+    ms = ent["ms_per_step"]
+    kt = {k: v for k, v in ent["kernel_ms_per_step"].items() if v > 0}
+    g = sum(v for k, v in kt.items() if k.startswith("gemm"))
+    rest = sorted(((k, v) for k, v in kt.items() if not k.startswith("gemm")), key=lambda kv: -kv[1])
+    lead = (f"the GEMMs take {g * 1e3:.1f} of {ms * 1e3:.1f} us (gate_up at {gemm['frac']:.2f} of the "
+            f"{'tensor' if gemm['bound'] == 'tensor' else 'HBM copy'} peak)")
+    tail = ", ".join(f"{k} {v * 1e3:.1f} us" for k, v in rest[:4])
+    return (f"{lead}; the other kernels: {tail}; the layer's bytes at the copy peak take "
+            f"{ent['layer_frac_of_hbm_peak'] * ms * 1e3:.1f} us; {ent['launches_per_step']:.0f} dependent launches "
+            f"per step")
+
+
 def run_sweep(args, world, local, skip: str) -> list:
     """The decode layers (and the dense decode projection) measured in the same process:
     tokens/s, the layer's fraction of the HBM copy peak and the gate_up GEMM's roofline,
@@ -873,10 +888,14 @@ def run_sweep(args, world, local, skip: str) -> list:
             est = measure_dense(args, shape, world, local, steps=20, warmup=3, full=False)
             n = sweep_steps(est["ms_per_step"], args.sweep_seconds)
             m = measure_dense(args, shape, world, local, steps=n, warmup=10, full=False)
-            res.append({"workload": name, "M": shape.T, "tokens_per_s": m["value"], "ms_per_step": m["ms_per_step"],
-                        "steps": n, "layer_frac_of_hbm_peak": m["layer"]["frac_of_hbm_peak"],
-                        "gemm": {kk: m["roofline"][kk] for kk in ("bound", "achieved", "unit", "frac")},
-                        "kernel_ms_per_step": m["layer"]["kernel_ms_per_step"], "gpu_launches": m["gpu_launches"]})
+            ent = {"workload": name, "M": shape.T, "tokens_per_s": m["value"], "ms_per_step": m["ms_per_step"],
+                   "steps": n, "layer_frac_of_hbm_peak": m["layer"]["frac_of_hbm_peak"],
+                   "gemm": {kk: m["roofline"][kk] for kk in ("bound", "achieved", "unit", "frac")},
+                   "kernel_ms_per_step": m["layer"]["kernel_ms_per_step"], "gpu_launches": m["gpu_launches"],
+                   "launches_per_step": m["gpu_launches"] / max(1, n)}
+            if ent["layer_frac_of_hbm_peak"] < 0.70:
+                ent["bound_by"] = bound_by(ent, ent["gemm"])
+            res.append(ent)
             continue
         W = synth.moe_weights_device(shape, dev)
         for M in Ms:
@@ -890,11 +909,8 @@ def run_sweep(args, world, local, skip: str) -> list:
                    "gate_up": {kk: m["roofline"][kk] for kk in ("bound", "achieved", "unit", "frac")},
                    "kernel_ms_per_step": m["layer"]["kernel_ms_per_step"], "gpu_launches": m["gpu_launches"],
                    "launches_per_step": m["gpu_launches"] / max(1, n)}
-            frac, ms = m["layer"]["frac_of_hbm_peak"], m["ms_per_step"]
-            if frac < 0.70:  # what holds the step below the layer's copy-peak time
-                ent["bound_by"] = (f"launch latency: {ent['launches_per_step']:.0f} dependent kernel launches per "
-                                   f"step; the layer's bytes at the copy peak take {frac * ms * 1e3:.1f} us of "
-                                   f"{ms * 1e3:.1f} us")
+            if ent["layer_frac_of_hbm_peak"] < 0.70:
+                ent["bound_by"] = bound_by(ent, ent["gate_up"])
             res.append(ent)
         del W
         torch.cuda.empty_cache()
