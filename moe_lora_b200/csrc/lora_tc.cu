@@ -21,7 +21,7 @@
 //
 // Structure (one CTA per SM, persistent over the device-side work list, 12 warps):
 //   warp 0      claims items (a queue of kLtQ slots) and loads the shrink stages: A_a box +
-//               the rows' box (one of four heights, so a short segment does not load 128
+//               the rows' box (one of six heights, so a short segment does not load 128
 //               rows), several K blocks per stage
 //   warp 1      shrink MMAs into the z accumulator (TMEM columns [0, 128))
 //   warp 2      loads the expand stages: B_a^T boxes of 64 features
@@ -106,7 +106,13 @@ struct LtSmem {
 constexpr int kLtStgPitch = 80;               // bytes per staged row of 32 bf16 (16-byte aligned)
 constexpr int kLtStgWarp = 32 * kLtStgPitch;  // one epilogue warp's staging block
 
-__device__ __forceinline__ int lt_box_rows(int box) { return 16 << box; }
+// heights of the rows' box (a short segment loads no more rows than it needs, to the next
+// multiple of 8 or 16; the shrink MMA's N rounds up to 16 and reads past a 24-row box into
+// rows whose z columns are never used)
+constexpr int kLtBoxes = 6;
+__device__ __forceinline__ int lt_box_rows(int box) {
+  return box == 0 ? 16 : box == 1 ? 24 : box == 2 ? 32 : box == 3 ? 48 : box == 4 ? 64 : 128;
+}
 
 // Work item `it`: rows [lo, hi) of segment q with hi - lo <= kLtN.
 __device__ __forceinline__ LtItem lt_item(const LoraTcParams& p, int it) {
@@ -117,7 +123,7 @@ __device__ __forceinline__ LtItem lt_item(const LoraTcParams& p, int it) {
   t.hi = (q >= 0 && q < p.nseg) ? min(min(p.seg_off[q + 1], t.lo + kLtN), p.nrows) : t.lo;
   t.n = max(0, t.hi - t.lo);
   t.n_mma = (t.n + 15) & ~15;
-  t.box = t.n <= 16 ? 0 : t.n <= 32 ? 1 : t.n <= 64 ? 2 : 3;
+  t.box = t.n <= 16 ? 0 : t.n <= 24 ? 1 : t.n <= 32 ? 2 : t.n <= 48 ? 3 : t.n <= 64 ? 4 : 5;
   int ad, e = 0;
   if (p.seg_adapter != nullptr) {
     ad = (q >= 0 && q < p.nseg) ? p.seg_adapter[q] : -1;
@@ -130,7 +136,7 @@ __device__ __forceinline__ LtItem lt_item(const LoraTcParams& p, int it) {
   t.slot = t.lora ? ad * p.E + e : 0;
   // a shrink stage holds as many (A box, rows box) pairs as fit, up to 4: short segments
   // then keep as many bytes in flight as long ones
-  t.kpb = min(4, max(1, p.s_stage_bytes / (p.r * 128 + (16 << t.box) * 128)));
+  t.kpb = min(4, max(1, p.s_stage_bytes / (p.r * 128 + lt_box_rows(t.box) * 128)));
   return t;
 }
 
@@ -157,7 +163,8 @@ __device__ __forceinline__ bool lt_take(LtSmem& sm, int qi, int& it, LtItem& t, 
 }
 
 __global__ void __launch_bounds__(kLtThreads, 1)
-    lora_tc_kernel(const __grid_constant__ CUtensorMap tmx16, const __grid_constant__ CUtensorMap tmx32,
+    lora_tc_kernel(const __grid_constant__ CUtensorMap tmx16, const __grid_constant__ CUtensorMap tmx24,
+                   const __grid_constant__ CUtensorMap tmx32, const __grid_constant__ CUtensorMap tmx48,
                    const __grid_constant__ CUtensorMap tmx64, const __grid_constant__ CUtensorMap tmx128,
                    const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                    const LoraTcParams p) {
@@ -201,7 +208,9 @@ __global__ void __launch_bounds__(kLtThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmx16);
+    tma_prefetch_desc(&tmx24);
     tma_prefetch_desc(&tmx32);
+    tma_prefetch_desc(&tmx48);
     tma_prefetch_desc(&tmx64);
     tma_prefetch_desc(&tmx128);
     tma_prefetch_desc(&tma);
@@ -239,7 +248,8 @@ __global__ void __launch_bounds__(kLtThreads, 1)
         if (it < 0) break;
         if (!t.lora) continue;
         const int arow = t.slot * p.r;
-        const CUtensorMap* xm = t.box == 0 ? &tmx16 : t.box == 1 ? &tmx32 : t.box == 2 ? &tmx64 : &tmx128;
+        const CUtensorMap* xm = t.box == 0 ? &tmx16 : t.box == 1 ? &tmx24 : t.box == 2 ? &tmx32
+                              : t.box == 3 ? &tmx48 : t.box == 4 ? &tmx64 : &tmx128;
         const uint32_t xbytes = static_cast<uint32_t>(lt_box_rows(t.box)) * 128u;
         const uint32_t pair = static_cast<uint32_t>(p.r) * 128u + xbytes;  // one (A, rows) box pair
         // the item's B_a rows head for L2 in pieces, one per shrink stage, so the expand
@@ -638,10 +648,11 @@ cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  CUtensorMap tx[4], ta, tb;
-  for (int b = 0; b < 4; ++b)
+  CUtensorMap tx[kLtBoxes], ta, tb;
+  const uint32_t box_rows[kLtBoxes] = {16, 24, 32, 48, 64, 128};
+  for (int b = 0; b < kLtBoxes; ++b)
     if (encode_tmap_2d(&tx[b], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.src, a.K, a.nrows,
-                       static_cast<uint64_t>(a.K) * 2, 64, 16u << b, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                       static_cast<uint64_t>(a.K) * 2, 64, box_rows[b], CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   const uint64_t slot_rows = static_cast<uint64_t>(a.L) * a.E * a.r;
   if (encode_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.lora_a, a.K, slot_rows, static_cast<uint64_t>(a.K) * 2,
@@ -682,7 +693,7 @@ cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st) {
   if (a.items_bound < grid) grid = a.items_bound;
   if (grid < 1) grid = 1;
   ProfScope ps(a.prof_id, st);
-  lora_tc_kernel<<<grid, kLtThreads, smem, st>>>(tx[0], tx[1], tx[2], tx[3], ta, tb, p);
+  lora_tc_kernel<<<grid, kLtThreads, smem, st>>>(tx[0], tx[1], tx[2], tx[3], tx[4], tx[5], ta, tb, p);
   count_launch();
   return cudaGetLastError();
 }
