@@ -600,6 +600,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     t1.delta = w.dgu;
     t1.status = w.status;
     t1.work_counter = w.status + 2;  // inside the status block: cleared with it by every call
+    t1.pdl_trigger = 1;  // the gate_up GEMM takes each SM this kernel leaves
     t1.num_sms = num_sms();
     ML_CUDA(launch_lora_tc(t1, cs), "gate_up tensor-core LoRA launch");
   } else {
@@ -637,7 +638,10 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.delta_cols = 2 * I;
   g.delta = rr && place == LORA_DELTA ? w.delta_gu : nullptr;
   g.delta_bf16 = tcl ? w.dgu : nullptr;
-  g.pdl_secondary = rr && place == LORA_DELTA ? 1 : 0;
+  // behind the LoRA kernel (PDL): the GEMM streams its weights while that kernel ends, and
+  // only what reads the delta waits for it
+  g.pdl_secondary = (rr && place == LORA_DELTA) || tcl ? 1 : 0;
+  g.pdl_full_smem = tcl ? 1 : 0;
   g.out_bf16 = w.act;
   g.w_scales = w_dtype == ML_E4M3 ? w_scales : nullptr;
   g.scale_idx = 0;
@@ -659,6 +663,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   g.test_stall_ms = 0;
 
   g.pdl_secondary = 0;
+  g.pdl_full_smem = 0;
 
   // 3. down LoRA shrink + expand on act: delta_d = (act A_d) B_d (LORA_DELTA: after the
   //    down GEMM's launch, overlapped with it, into a pair-order delta the combine adds)
@@ -677,6 +682,7 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     t2.delta = w.dd;
     t2.scatter = sorted_pairs;  // pair order: the combine adds it
     t2.work_counter = w.status + 3;
+    t2.pdl_trigger = 1;  // the down GEMM (which does not read this delta) starts as SMs free up
     ML_CUDA(launch_lora_tc(t2, cs), "down tensor-core LoRA launch");
   }
 
@@ -691,6 +697,8 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   d.delta = nullptr;
   d.delta_bf16 = nullptr;  // the down LoRA delta (delta and tc placements) goes to the combine
   d.pdl_trigger = rr && place == LORA_DELTA ? 1 : 0;
+  d.pdl_end_wait = tcl ? 1 : 0;  // behind the tensor-core down LoRA: waits for it only to finish
+  d.pdl_full_smem = tcl ? 1 : 0;
   d.out_bf16 = w.o;
   d.out_f32 = nullptr;
   d.sorted_pairs = sorted_pairs;

@@ -91,7 +91,9 @@ struct TcParams {
   uint64_t wait_ns;
   int test_stall;
   int pdl_trigger;    // let the next kernel launch at once
-  int pdl_secondary;  // launched behind the LoRA kernel: the loader waits for it
+  int pdl_secondary;  // launched behind the LoRA kernel: whatever reads its delta waits for it
+  int pdl_end_wait;   // launched behind a kernel whose output it does not read: it waits for
+                      // that kernel only before it exits, so the launches after it see both done
   // base stages hold kpb consecutive K blocks (sub-stages of TileCfg::kStageBytes): two
   // give 256-byte runs of every weight row per stage at decode, which the memory system
   // streams faster than 128-byte runs
@@ -536,6 +538,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
               uv[n] *= scale;
             }
             if (p.delta_bf16 != nullptr) {  // this row's 32 gate and 32 up delta values
+              if (p.pdl_secondary) pdl_wait();  // the delta comes from the kernel ahead
               const __nv_bfloat16* dr = p.delta_bf16 + static_cast<size_t>(row) * p.delta_cols;
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
@@ -621,6 +624,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
                        : make_uint4(0u, 0u, 0u, 0u);
         }
       };
+      if (dbf && p.pdl_secondary) pdl_wait();  // the delta comes from the kernel ahead
       if (dbf) dload(0);
       for (int c0 = 0; c0 < ti.nvalid; c0 += 32) {
         named_bar_sync(1, kEpiThreads);  // the previous chunk is done with smem
@@ -805,6 +809,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
     }
   }
 
+  if (p.pdl_end_wait) pdl_wait();
   tc_fence_before();
   if constexpr (TWO) cluster_sync_all();  // no CTA leaves while its peer may still signal it
   else __syncthreads();
@@ -860,10 +865,11 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   const int slot_bytes = static_cast<int>(((dslot ? sizeof(EpiSlot<BN>) : offsetof(EpiSlot<BN>, delta)) + 1023) /
                                           1024 * 1024);
   const int stage_bytes = kpb * Cfg::kStageBytes;
-  // overlapped with a LoRA kernel (PDL: launched behind one, or letting one start) the
-  // GEMM leaves room for one of its CTAs on every SM (228 KB per SM, 1 KB reserved per
-  // CTA), so both run side by side
-  const bool coloc = a.pdl_secondary || a.pdl_trigger;
+  // overlapped with the SIMT LoRA kernel (PDL: launched behind one, or letting one start)
+  // the GEMM leaves room for one of its CTAs on every SM (228 KB per SM, 1 KB reserved per
+  // CTA), so both run side by side; behind the tensor-core LoRA kernel (pdl_full_smem)
+  // nothing shares an SM, and a GEMM CTA starts on each SM that kernel has left
+  const bool coloc = (a.pdl_secondary || a.pdl_trigger) && !a.pdl_full_smem;
   const int smem_cap = coloc ? 228 * 1024 - 1024 - kLoraCoresidentSmem : 232448;
   auto stages_for = [&](int ns) {
     const int s = (smem_cap - 1024 - static_cast<int>(sizeof(SmemCore)) - ns * slot_bytes) / stage_bytes;
@@ -948,6 +954,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
   p.test_stall = a.test_stall_ms > 0 ? 1 : 0;
   p.pdl_trigger = a.pdl_trigger;
   p.pdl_secondary = a.pdl_secondary;
+  p.pdl_end_wait = a.pdl_end_wait;
   p.kpb = kpb;
   p.stage_bytes = stage_bytes;
   p.nslots = nslots;
@@ -981,7 +988,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     attr[na].val.clusterDim.z = 1;
     ++na;
   }
-  if (a.pdl_secondary) {
+  if (a.pdl_secondary || a.pdl_end_wait) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;

@@ -143,6 +143,7 @@ struct LoraTcArgs {
   int r_exp = 0;                // 0 means r
   float scale = 1.f;            // multiplies every delta value
   int prof_id = 11;             // measurement hook id of the launch (K_LORA or K_LORA_DOWN)
+  int pdl_trigger = 0;          // the kernel behind this one (PDL) may launch at once
 };
 cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st);
 
@@ -230,6 +231,12 @@ struct GemmArgs {
   // so the weight stream and the MMAs start at once
   int pdl_trigger;
   int pdl_secondary;
+  // launched behind a kernel whose output it does not read (PDL): it waits for that
+  // kernel only before it exits
+  int pdl_end_wait = 0;
+  // the kernel ahead holds its SMs' shared memory (the tensor-core LoRA kernel): keep the
+  // full shared memory, nothing runs beside this kernel's CTAs
+  int pdl_full_smem = 0;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st);
 

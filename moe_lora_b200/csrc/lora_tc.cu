@@ -74,6 +74,7 @@ struct LoraTcParams {
   int split_I;
   int r_exp;
   float scale;                // multiplies every delta value
+  int pdl_trigger;            // the kernel behind this one (PDL) may launch at once
 };
 
 struct LtItem {
@@ -177,6 +178,9 @@ __global__ void __launch_bounds__(kLtThreads, 1)
   LtSmem& sm = *reinterpret_cast<LtSmem*>(stg + 4 * kLtStgWarp);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sm.abort_flag;
+  // the GEMM behind this kernel takes each SM this kernel leaves; only what reads the delta
+  // waits for this kernel to finish
+  if (p.pdl_trigger) pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.s_stages; ++s) {
@@ -689,6 +693,7 @@ cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st) {
   p.split_I = a.split_I;
   p.r_exp = a.split_I ? a.r_exp : a.r;
   p.scale = a.scale;
+  p.pdl_trigger = a.pdl_trigger;
   int grid = a.num_sms > 0 ? a.num_sms : 148;
   if (a.items_bound < grid) grid = a.items_bound;
   if (grid < 1) grid = 1;
