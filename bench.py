@@ -53,7 +53,7 @@ SWEEP = ((synth.MOE_DECODE_BF16.name, (1, 8, 32, 64)), (synth.MOE_DECODE_FP8.nam
 # ncu-measured DRAM traffic (read + write bytes per launch) of the gate_up GEMM, with the
 # hash of the kernel source it was taken on and the case it was taken on; reported as
 # null when the source has changed since or the case differs.  Filled from profiles/.
-NCU_TRAFFIC = {"gemm_tc.cu": "19dc9a8ae004c27c", "bytes_per_launch": 4617012992.0 + 111399936.0,
+NCU_TRAFFIC = {"gemm_tc.cu": "f1929774665d1ca1", "bytes_per_launch": 4554427136.0 + 110045184.0,
                "workload": "moe_prefill_bf16_e128_h4096_i1536", "M": 4096}
 
 
@@ -820,38 +820,91 @@ def measure_moe(args, shape: synth.MoEShape, M: int, W: dict, world, local, *, s
             out["secondary"]["swap_ab"] = ("decode: only the swapped tile (weights in M) is built; a tile with "
                                            "tokens in M would leave most of the MMA's 128 rows empty")
 
-    # ---- e2e: pinned host inputs -> device, route + forward, y -> pinned host, every step
+    # ---- e2e: pinned host inputs -> device, route + forward, y -> pinned host, every step.
+    #      Serving pipeline: the compute of step i on this stream, the input copy of step
+    #      i + 1 and the output copy of step i - 1 on two copy streams (double-buffered
+    #      device inputs and outputs), the first input copy and the last output copy inside
+    #      the timed region; the same steps one after another are reported beside it
     e2e_steps = args.e2e_steps or steps
     hx = [b[0].cpu().pin_memory() for b in batches]
     ha = [b[1].cpu().pin_memory() for b in batches]
     hy = torch.empty((M, shape.H), dtype=torch.bfloat16).pin_memory()
-    dx = torch.empty_like(batches[0][0])
-    da = torch.empty_like(batches[0][1])
+    dxs = [torch.empty_like(batches[0][0]) for _ in range(2)]
+    das = [torch.empty_like(batches[0][1]) for _ in range(2)]
+    ys = [y, torch.empty_like(y)]
+    for b in range(2):  # real inputs before the graphs' warm-up calls
+        dxs[b].copy_(batches[b % nb][0])
+        das[b].copy_(batches[b % nb][1])
 
-    def e2e_step(j):
-        dx.copy_(hx[j], non_blocking=True)
-        da.copy_(ha[j], non_blocking=True)
-        call(dx, da)
-        hy.copy_(y, non_blocking=True)
+    def e2e_compute(b):
+        rt = ml.route(das[b], k, L, x=dxs[b], w_router=W["w_router"], bias=W["bias"], out=rbufs, workspace=rws)
+        ml.forward(dxs[b], rt, W, k=k, L=L, y=ys[b], workspace=fws)
 
-    e2e_graphs = capture(e2e_step, nb) if not args.no_graph else []
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(e2e_steps):
-        e2e_graphs[i % nb].replay() if e2e_graphs else e2e_step(i % nb)
-    e1.record()
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    del graphs, e2e_graphs
+    def e2e_serial(j):
+        dxs[0].copy_(hx[j], non_blocking=True)
+        das[0].copy_(ha[j], non_blocking=True)
+        e2e_compute(0)
+        hy.copy_(ys[0], non_blocking=True)
+
+    cgraphs = capture(lambda b: e2e_compute(b % 2), 2) if not args.no_graph else []
+    sgraphs = capture(e2e_serial, nb) if not args.no_graph else []
+    cs = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def h2d(i, b):
+        with torch.cuda.stream(s_in):
+            dxs[b].copy_(hx[i % nb], non_blocking=True)
+            das[b].copy_(ha[i % nb], non_blocking=True)
+            in_done[b].record(s_in)
+
+    def pipelined(n):
+        s_in.wait_stream(cs)
+        s_out.wait_stream(cs)
+        h2d(0, 0)
+        for i in range(n):
+            b = i % 2
+            cs.wait_event(in_done[b])
+            if i >= 2:
+                cs.wait_event(out_done[b])  # ys[b] of step i - 2 has been copied out
+            cgraphs[b].replay() if cgraphs else e2e_compute(b)
+            comp_done[b].record(cs)
+            if i + 1 < n:
+                if i >= 1:
+                    s_in.wait_event(comp_done[1 - b])  # step i - 1 is done with its inputs
+                h2d(i + 1, 1 - b)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                hy.copy_(ys[b], non_blocking=True)
+                out_done[b].record(s_out)
+        cs.wait_stream(s_out)
+        cs.wait_stream(s_in)
+
+    def timed(fn):
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(e0.elapsed_time(e1), world)
+
+    pipelined(min(4, e2e_steps))  # warm the copy streams
+    e2e_ms = timed(lambda: pipelined(e2e_steps))
+    serial_ms = timed(lambda: [sgraphs[i % nb].replay() if sgraphs else e2e_serial(i % nb) for i in range(e2e_steps)])
+    del graphs, cgraphs, sgraphs
     ml.check_status(fws)
     ml.check_status(rws)
     out["e2e"] = {"value": world * M * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                   "h2d_bytes_per_step": M * shape.H * 2 + M * 4, "d2h_bytes_per_step": M * shape.H * 2,
-                  "how": "graph replay of H2D copy, route, forward, D2H copy" if not args.no_graph
-                  else "plain API calls"}
+                  "how": ("serving pipeline: route + forward of step i (graph replay) while step i + 1's "
+                          "inputs go in and step i - 1's y comes out on two copy streams; pinned host "
+                          "buffers, every step's copies inside the timed region"),
+                  "serial_value": world * M * e2e_steps / (serial_ms / 1e3),
+                  "serial_how": "H2D copy, route, forward, D2H copy one after another (graph replay)"}
     return out
 
 
