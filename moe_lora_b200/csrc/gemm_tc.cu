@@ -145,6 +145,7 @@ struct SmemCore {
   int abort_flag;
   int chunk_pref[kMaxGroups + 1];
   int grp_off[kMaxGroups + 1];
+  short chunk_rows[kMaxGroups];  // token rows per chunk of group g (<= the tile's)
   float ebuf[kBM][33];
 };
 
@@ -204,8 +205,9 @@ __device__ __forceinline__ TileInfo decode_tile(const SmemCore& sm, int t, int m
     else hi = mid;
   }
   ti.g = lo;
-  ti.row0 = sm.grp_off[lo] + (c - sm.chunk_pref[lo]) * BN;
-  ti.nvalid = min(BN, sm.grp_off[lo + 1] - ti.row0);
+  const int cr = sm.chunk_rows[lo];
+  ti.row0 = sm.grp_off[lo] + (c - sm.chunk_pref[lo]) * cr;
+  ti.nvalid = min(cr, sm.grp_off[lo + 1] - ti.row0);
   return ti;
 }
 
@@ -280,6 +282,15 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
       if (g < p.E) {
         const int n = sm.grp_off[g + 1] - sm.grp_off[g];
         c = n > 0 ? (n + Cfg::kTokRows - 1) / Cfg::kTokRows : 0;
+        // a group whose last chunk would hold less than half a tile splits its rows evenly
+        // over its chunks instead (rounded up to 16): the small last chunk would cost
+        // about as many MMA issue slots as a full one
+        int cr = Cfg::kTokRows;
+        if (c >= 2 && n - (c - 1) * Cfg::kTokRows < Cfg::kTokRows / 2) {
+          cr = min(Cfg::kTokRows, ((n + c - 1) / c + 15) & ~15);
+          c = (n + cr - 1) / cr;  // every chunk keeps at least one row
+        }
+        sm.chunk_rows[g] = static_cast<short>(cr);
       }
       cnt[i] = c;
       tot += c;

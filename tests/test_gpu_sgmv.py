@@ -116,3 +116,22 @@ def test_dense_many_segments(where, monkeypatch):
     err = rel_err(y, y_ref)
     assert err <= TOL_BF16, err
 
+
+
+def test_dense_tc_lora_every_row_box(monkeypatch):
+    """Segments whose lengths sit on both sides of every rows'-box height of the tensor-core
+    LoRA kernel (16, 24, 32, 48, 64, 128 rows), and one longer than an item (two items)."""
+    monkeypatch.setenv("MOE_LORA_EXPAND", "tc")
+    lens = [1, 16, 17, 24, 25, 32, 33, 48, 49, 64, 65, 127, 128, 200]
+    T = sum(lens)
+    s = synth.DENSE_DECODE_BF16.with_(name="bf16_boxes", wid=308, T=T, h_in=256, h_out=384, L=4, r=32,
+                                      adapter_dist="uniform")
+    d = dense_f64(s)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    segs = (np.arange(len(lens)) % s.L).astype(np.int32)
+    y = ml.dense_lora_forward(d["x"].cuda(), d["w"]["w"].cuda(), d["w"]["a"].cuda(), d["w"]["b"].cuda(),
+                              torch.from_numpy(offs).cuda(), torch.from_numpy(segs).cuda())
+    torch.cuda.synchronize()
+    y_ref = ref.dense_lora_forward(d["x64"], d["w64"], d["a64"], d["b64"], offs, segs)
+    err = rel_err(y, y_ref)
+    assert err <= TOL_BF16, err
