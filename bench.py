@@ -16,9 +16,12 @@ Default workload: the MoE prefill layer, the largest configuration that fits one
 gate_up and down (Zipf adapter ids, router bias skewing the expert load).  The same line
 carries a `sweep` of the decode layers (bf16 E=64 at M = 1, 8, 32, 64; e4m3 experts
 E=128 at M = 1, 4, 16, 64, and the same e4m3 layer at 4096 tokens: FP8 prefill) and the
-dense decode projection, measured in the same process.  For N > 1 (torchrun) every rank
-runs an independent replica (weak scaling, no collective on the data path); timing is
-the max over ranks.  Prints one JSON line on rank 0.
+dense decode projection, measured in the same process.  `e2e` is the same step through the
+public API with pinned host buffers, run as a serving pipeline (each step's inputs copied in
+and its y copied out on two copy streams while the neighbouring step computes, every copy
+inside the timed region); `e2e.serial_value` is the same with copies and compute one after
+another.  For N > 1 (torchrun) every rank runs an independent replica (weak scaling, no
+collective on the data path); timing is the max over ranks.  Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
