@@ -176,16 +176,18 @@ constexpr int kNsTok = 128;
 template <int BN, bool W8, bool TWO = false, bool NS = false>
 struct TileCfg {
   static constexpr int kKB = W8 ? 128 : 64;                  // K per stage (128 bytes per row)
-  static constexpr int kBRows = TWO ? BN / 2 : BN;           // token rows held by this CTA
+  // token rows held by this CTA: pairs of bf16 tiles split the tokens, pairs of e4m3 tiles
+  // split the planes (the leader stages the hi plane, its peer the lo plane, all BN rows)
+  static constexpr int kBRows = (TWO && !W8) ? BN / 2 : BN;
   static constexpr int kBTileBytes = kBRows * 128;           // one token tile (or plane)
-  static constexpr int kStageBytes = kATileBytes + (W8 ? 2 : 1) * kBTileBytes;
+  static constexpr int kStageBytes = kATileBytes + ((W8 && !TWO) ? 2 : 1) * kBTileBytes;
   static constexpr int kAccStride = BN < 32 ? 32 : BN;       // TMEM columns per accumulator
   static constexpr int kAccPerBuf = W8 ? 2 : 1;              // e4m3: hi and lo side by side (N = 2 BN)
   static constexpr int kTmemCols = pow2_at_least(2 * kAccPerBuf * kAccStride);
   static constexpr bool kPrefetch = BN <= 64;                // LoRA delta prefetched into the slots
   static constexpr int kThreads = 224;
   static_assert(!W8 || BN <= 128, "e4m3 weights use N tiles <= 128 (hi and lo planes: N = 2 BN)");
-  static_assert(!TWO || (!W8 && BN == 256), "CTA pairs: bf16 weights, N tiles of 256");
+  static_assert(!TWO || (!W8 && BN == 256) || (W8 && BN == 128), "CTA pairs: bf16 N tiles of 256, e4m3 of 128");
   static_assert(!NS || (!W8 && !TWO && BN == 256), "tokens in M: bf16 weights, 256 weight rows in N");
   static constexpr int kTokRows = NS ? kNsTok : BN;          // token rows per tile
 };
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
     tma_prefetch_desc(&tmw);
     tma_prefetch_desc(&tmb);
     if (W8 || TWO) tma_prefetch_desc(&tml);
-    if (p.delta != nullptr || TWO) tma_prefetch_desc(&tmd);
+    if (p.delta != nullptr || (TWO && !W8)) tma_prefetch_desc(&tmd);
   }
   if (warp == 1) {
     if constexpr (TWO) tmem_alloc_pair(&sm.tmem_base, Cfg::kTmemCols);
@@ -365,7 +367,19 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
           uint8_t* a_s = ring + stage * p.stage_bytes;
           const int kc = kb * Cfg::kKB * p.kpb;  // first K element of the stage
           const int nj = min(p.kpb, (p.K - kc + Cfg::kKB - 1) / Cfg::kKB);  // sub-stages inside K
-          if constexpr (TWO) {
+          if constexpr (TWO && W8) {
+            // e4m3 pairs: the MMA's N is both planes (2 BN rows); the leader stages the hi
+            // plane of the chunk's BN token rows, its peer the lo plane
+            const uint32_t fb = leader_bar(&sm.full[stage]);
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2u * nj * Cfg::kStageBytes);
+            for (int j = 0; j < nj; ++j) {
+              uint8_t* aj = a_s + j * Cfg::kStageBytes;
+              const int kcj = kc + j * Cfg::kKB;
+              tma_load_2d_pair(aj, &tmw, fb, kcj, wrow0);
+              tma_load_2d_pair(aj + kATileBytes / 2, &tmw, fb, kcj, wrow1);
+              tma_load_2d_pair(aj + kATileBytes, rank == 0 ? &tmb : &tml, fb, kcj, ti.row0);
+            }
+          } else if constexpr (TWO) {
             // both CTAs' copies complete on the leader's barrier, which expects the pair's
             // bytes; the MMA's N is the tile's rows rounded to 32, the peer holds [N/2, N)
             const uint32_t fb = leader_bar(&sm.full[stage]);
@@ -451,7 +465,7 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
         // e4m3: the hi and lo planes sit back to back in the ring, so one instruction of
         // N = 2 BN covers both and each weight tile is read from shared memory once
         const int n_mma = NS ? BN : TWO ? min(BN, (ti.nvalid + 31) & ~31) : min(BN, (ti.nvalid + 15) & ~15);
-        const uint32_t idesc = W8 ? umma_idesc_e4m3(kBM, 2 * BN) : umma_idesc_bf16(TWO ? 2 * kBM : kBM, n_mma);
+        const uint32_t idesc = W8 ? umma_idesc_e4m3(TWO ? 2 * kBM : kBM, 2 * BN) : umma_idesc_bf16(TWO ? 2 * kBM : kBM, n_mma);
         const int buf = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         if (!mbar_wait(&sm.tempty[buf], (use & 1u) ^ 1u, abort_flag, p.status, p.wait_ns, 2)) break;
@@ -472,7 +486,9 @@ __global__ void __launch_bounds__(TileCfg<BN, W8, TWO, NS>::kThreads, BN <= 64 ?
 #pragma unroll
             for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
               const uint32_t acc = (kb != u.k0 || j != 0 || k != 0) ? 1u : 0u;
-              if constexpr (W8) {
+              if constexpr (W8 && TWO) {
+                umma_e4m3_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // hi from the leader, lo from the peer
+              } else if constexpr (W8) {
                 umma_e4m3(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);  // columns [0, BN) hi, [BN, 2 BN) lo
               } else if constexpr (TWO) {
                 umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, acc);
@@ -928,7 +944,7 @@ static cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     }
   }
-  if (TWO) {
+  if (TWO && !W8) {
     // tmd holds the 64-row token box (pairs take no fp32 delta)
   } else if (a.delta != nullptr && Cfg::kPrefetch) {
     if (encode_tmap_2d(&tmd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.delta, a.delta_cols, a.total_rows,
@@ -1022,7 +1038,15 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t st) {
       case 16: return launch_bn<16, true>(a, st);
       case 32: return launch_bn<32, true>(a, st);
       case 64: return launch_bn<64, true>(a, st);
-      default: return launch_bn<128, true>(a, st);
+      default: {
+        // CTA pairs (M = 256): each CTA stages one plane, so a stage holds one weight tile
+        // and one plane and every staged byte feeds twice the MMA work
+        const int m_tiles = (a.epi == EPI_GATEUP) ? (a.I + 63) / 64 : (a.n_out + kBM - 1) / kBM;
+        const char* v = std::getenv("MOE_LORA_PAIR");
+        const bool pair = (v != nullptr ? std::atoi(v) != 0 : kPairDefault) && m_tiles % 2 == 0 && a.K > 128 &&
+                          (a.epi == EPI_GATEUP || a.epi == EPI_DOWN);
+        return pair ? launch_bn<128, true, true>(a, st) : launch_bn<128, true>(a, st);
+      }
     }
   }
   switch (a.bn) {

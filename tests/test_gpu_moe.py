@@ -214,6 +214,21 @@ def test_forward_fp8_every_n_tile(bn, where, monkeypatch, record_property):
     check_fp8(run_moe_case(SMALL_FP8[1], 150), f"{SMALL_FP8[1].name} bn={bn} {where}", record_property)
 
 
+F8_PAIR = synth.MoEShape("f8_pair", 223, E=6, k=3, H=512, I=256, L=2, r=32, wdtype="e4m3", bias=True,
+                         adapter_dist="zipf", no_adapter_frac=0.25)
+
+
+@pytest.mark.parametrize("variant", ["single", "pair"])
+@pytest.mark.parametrize("M", [37, 300])
+def test_forward_fp8_single_and_pair(M, variant, monkeypatch, record_property):
+    """e4m3 tiles of 128 tokens on one CTA and on CTA pairs (cta_group::2, M = 256: the
+    leader stages the hi activation plane, its peer the lo plane), over even weight-tile
+    counts with a router bias that skews the groups, so chunks are ragged and uneven."""
+    monkeypatch.setenv("MOE_LORA_FORCE_BN", "128")
+    monkeypatch.setenv("MOE_LORA_PAIR", "1" if variant == "pair" else "0")
+    check_fp8(run_moe_case(F8_PAIR, M), f"{F8_PAIR.name} M={M} {variant}", record_property)
+
+
 @pytest.fixture(scope="module")
 def fp8_weights():
     return moe_weights_both(synth.MOE_DECODE_FP8)
