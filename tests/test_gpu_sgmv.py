@@ -57,6 +57,25 @@ def test_sgmv_shrink_expand(s):
     assert rel_err(y0, d_ref) <= (1e-5 if s.dtype == "f32" else 1e-2)
 
 
+@pytest.mark.parametrize("T", [5, 33, 64])
+def test_dense_n64_tile(T, monkeypatch):
+    """The dense projection's N tile of 64 with the SIMT LoRA kernel's fp32 delta added in
+    the epilogue: tiny, ragged and full token counts, a ragged last weight tile and a K
+    that ends inside a block."""
+    monkeypatch.setenv("MOE_LORA_FORCE_BN", "64")
+    monkeypatch.setenv("MOE_LORA_EXPAND", "delta")
+    s = synth.DENSE_DECODE_BF16.with_(name="bf16_n64", wid=309, T=T, h_in=1000, h_out=1000, L=5, r=16,
+                                      no_adapter_frac=0.2)
+    d = dense_f64(s)
+    y = ml.dense_lora_forward(d["x"].cuda(), d["w"]["w"].cuda(), d["w"]["a"].cuda(), d["w"]["b"].cuda(),
+                              d["offs"].cuda(), d["segs"].cuda())
+    torch.cuda.synchronize()
+    y_ref = ref.dense_lora_forward(d["x64"], d["w64"], d["a64"], d["b64"], d["offs"].numpy(),
+                                   d["segs"].numpy())
+    err = rel_err(y, y_ref)
+    assert err <= TOL_BF16, err
+
+
 @pytest.mark.parametrize("where", ["delta", "tc"])
 @pytest.mark.parametrize("s", CASES, ids=lambda s: s.name)
 def test_dense_lora_forward(s, where, monkeypatch):
