@@ -254,9 +254,10 @@ RouteWs route_layout(void* base, int M, int E, int L) {
     return p;
   };
   w.status = reinterpret_cast<int*>(b);
-  w.key_count = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * (L + 1) * 4));
-  // adapter key per token; tickets of the one-launch routing (ceil(M / 8) + 1)
+  // adapter key per token; tickets of the one-launch routing (ceil(M / 8) + 1), right
+  // behind the status block so that one memset clears both
   w.a_key = reinterpret_cast<int32_t*>(take(static_cast<size_t>(M > (M + 7) / 8 + 1 ? M : (M + 7) / 8 + 1) * 4));
+  w.key_count = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * (L + 1) * 4));
   w.logits = reinterpret_cast<float*>(take(static_cast<size_t>(M) * E * 4));
   w.bytes = off;
   return w;
@@ -445,7 +446,10 @@ moe_lora_status moe_lora_route(const void* x, const void* w_router, const float*
   if (st != MOE_LORA_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const RouteWs w = route_layout(workspace, M, E, L);
-  ML_CUDA(cudaMemsetAsync(workspace, 0, 8, cs), "status clear");
+  // one memset for the status word and, for the one-launch routing, its tickets
+  const int tickets = route_fused_tickets(M, k);
+  ML_CUDA(cudaMemsetAsync(workspace, 0, tickets > 0 ? kStatusBytes + 4 * static_cast<size_t>(tickets) : 8, cs),
+          "status clear");
   RouteArgs a{};
   a.x = static_cast<const __nv_bfloat16*>(x);
   a.w_router = static_cast<const __nv_bfloat16*>(w_router);
@@ -467,6 +471,7 @@ moe_lora_status moe_lora_route(const void* x, const void* w_router, const float*
   a.a_key = w.a_key;
   a.status = w.status;
   a.num_sms = num_sms();
+  a.tickets_zeroed = tickets > 0 ? 1 : 0;
   ML_CUDA(launch_route(a, cs), "moe_lora_route launch");
   return MOE_LORA_OK;
 }
@@ -529,7 +534,9 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   const bool tcl = rr && place == LORA_TC;  // tensor-core LoRA kernel, bf16 deltas
   const int mk = M * k;
   const int nkeys = E * (L + 1);
-  ML_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes, cs), "status clear");
+  // the status block (status word, work counters) is zeroed by the call's first kernel,
+  // the row gather below, which writes no status itself; every later kernel of the call
+  // starts after it has finished
 
   // 1. gather x rows into (expert, adapter) order, and the gate_up LoRA:
   //    LORA_DELTA: one SIMT kernel gathers, shrinks z = x A_gu per (adapter, expert)
@@ -569,10 +576,11 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
   if (tcl) {
     if (fp8)  // one pass over x: the gathered bf16 rows (the LoRA kernel's operand) and their planes
       ML_CUDA(launch_gather_quant(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.q_hi, w.q_lo,
-                                  w.q_scales, w.x_sorted, cs),
+                                  w.q_scales, w.x_sorted, cs, w.status),
               "gather and activation planes launch");
     else
-      ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs),
+      ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs,
+                                 w.status),
               "row gather launch");
     const int bound = lora_items_bound(mk, nkeys, kLtN);
     ML_CUDA(launch_lora_plan_all(seg_offsets, nullptr, nkeys, L, mk, kLtN, w.items_tc, w.item_count_tc, bound,
@@ -609,10 +617,11 @@ moe_lora_status moe_lora_forward(const void* x, int M, int H, int I, int E, int 
     // LoRA kernel runs, and only its epilogue loader waits for the delta
     if (fp8)
       ML_CUDA(launch_gather_quant(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.q_hi, w.q_lo,
-                                  w.q_scales, nullptr, cs),
+                                  w.q_scales, nullptr, cs, w.status),
               "activation planes launch");
     else
-      ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs),
+      ML_CUDA(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), M, sorted_pairs, k, mk, H, w.x_sorted, cs,
+                                 w.status),
               "row gather launch");
     if (rr) {
       l1.gather_dst = nullptr;
@@ -850,7 +859,10 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const DenseWs ws = dense_layout(workspace, T, h_in, h_out, rr, f32, place);
   const bool tcl = rr && place == LORA_TC;  // tensor-core LoRA kernel, bf16 delta
-  ML_CUDA(cudaMemsetAsync(workspace, 0, f32 ? 8 : kStatusBytes, cs), "status clear");
+  // with adapters (bf16) the LoRA work-list kernel comes first and zeroes the status block
+  // itself; the kernels behind it write status only after they have waited for it
+  const bool plan_clears = !f32 && rr > 0;
+  if (!plan_clears) ML_CUDA(cudaMemsetAsync(workspace, 0, f32 ? 8 : kStatusBytes, cs), "status clear");
 
   if (f32) {
     ShrinkArgs a{};
@@ -917,7 +929,7 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
     if (tcl) {  // shrink and expand on the tensor cores, bf16 delta for the epilogue
       const int bound = lora_items_bound(T, S, kLtN);
       ML_CUDA(launch_lora_plan_all(seg_offsets, seg_adapter, S, L, T, kLtN, ws.items_tc, ws.item_count_tc, bound,
-                                   ws.status, cs),
+                                   ws.status, cs, true),
               "LoRA work list launch");
       LoraTcArgs t{};
       t.src = static_cast<const __nv_bfloat16*>(x);
@@ -947,7 +959,9 @@ moe_lora_status dense_lora_forward(const void* x, const void* w, const void* lor
       // and only the GEMM's epilogue loader waits for the delta
       l.pdl_trigger = 1;
       l.pdl_after_plan = 1;
+      l.clear_status = 1;
       ML_CUDA(launch_lora_plan(l, cs), "LoRA plan launch");
+      l.clear_status = 0;
       ML_CUDA(launch_lora_delta(l, cs), "dense LoRA launch");
     }
   }

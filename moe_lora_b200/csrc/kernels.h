@@ -28,8 +28,12 @@ struct RouteArgs {
                           // tickets of the one-launch routing
   int* status;
   int num_sms;
+  int tickets_zeroed = 0;  // the caller's status clear already zeroed the tickets
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+// Tickets (ints at a_key) of the one-launch routing for M tokens of k pairs, or 0 when the
+// routing takes the multi-kernel path.
+int route_fused_tickets(int M, int k);
 
 // Segmented shrink z[s] = src_row(s) . A_seg(s)^T (SIMT: 128-bit loads, warp-shuffle
 // split-K reduction).  Segments come either from a dense (offsets, adapter) table or
@@ -108,6 +112,7 @@ struct LoraDeltaArgs {
   int pdl_trigger;
   int pdl_secondary;
   int pdl_after_plan = 0;
+  int clear_status = 0;  // launch_lora_plan: zero the status block first (the call's first kernel)
 };
 int lora_rows_per_chunk(int nrows, int nseg);
 int lora_items_bound(int nrows, int nseg, int rb);
@@ -149,11 +154,15 @@ cudaError_t launch_lora_tc(const LoraTcArgs& a, cudaStream_t st);
 
 // dst[i] = src[gather[i] / div] for i < rows (bf16 rows of K elements; a source index
 // outside [0, nsrc) gives a zero row).
+// clear_status (if set): the call's status block, zeroed by the kernel's first CTA before
+// any later kernel of the call runs (so the first kernel of a call replaces a memset).
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
-                               __nv_bfloat16* dst, cudaStream_t st);
+                               __nv_bfloat16* dst, cudaStream_t st, int* clear_status = nullptr);
 // Work list of every non-empty segment (with or without an adapter), chunks of rb rows.
+// clear_status: zero the status block first (the plan kernel is then the call's first).
 cudaError_t launch_lora_plan_all(const int32_t* seg_offsets, const int32_t* seg_adapter, int nseg, int L, int nrows,
-                                 int rb, int2* items, int* count, int cap, int* status, cudaStream_t st);
+                                 int rb, int2* items, int* count, int cap, int* status, cudaStream_t st,
+                                 bool clear_status = false);
 
 // y[t] += z[t] . B_a(t) for dense segments (f32 or bf16 y and B).
 struct ExpandArgs {
@@ -252,7 +261,8 @@ cudaError_t launch_combine(const __nv_bfloat16* o, int M, int k, int H, const fl
 // The e4m3 activation planes of gathered rows (see launch_quant_planes): plane row i from
 // src[gather[i] / div]; copy (if set) also receives the gathered bf16 rows.
 cudaError_t launch_gather_quant(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
-                                uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy, cudaStream_t st);
+                                uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy, cudaStream_t st,
+                                int* clear_status = nullptr);
 
 // Host state that CUDA keeps per device (function attributes, SM counts, capability)
 // is cached per device index, for processes that drive several GPUs.

@@ -488,13 +488,18 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteArgs a, con
   }
 }
 
+int route_fused_tickets(int M, int k) {
+  return (M > 0 && static_cast<long long>(M) * k <= RF_MAX_PAIRS) ? (M + RF_TB - 1) / RF_TB + 1 : 0;
+}
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   const int nk = a.E * (a.L + 1);
   if (a.M == 0) return cudaMemsetAsync(a.seg_offsets, 0, sizeof(int32_t) * (nk + 1), st);
   if (static_cast<long long>(a.M) * a.k <= RF_MAX_PAIRS) {
-    // one launch; a_key[0, n_tb] holds the tickets
+    // one launch; a_key[0, n_tb] holds the tickets (zeroed here unless the caller's
+    // status clear covered them)
     const int n_tb = (a.M + RF_TB - 1) / RF_TB;
-    cudaError_t err = cudaMemsetAsync(a.a_key, 0, sizeof(int32_t) * (n_tb + 1), st);
+    cudaError_t err = a.tickets_zeroed ? cudaSuccess : cudaMemsetAsync(a.a_key, 0, sizeof(int32_t) * (n_tb + 1), st);
     if (err != cudaSuccess) return err;
     const size_t smem = route_fused_smem(a.E, a.L, a.M, a.k);
     // the raised shared-memory limit is a per-device function attribute

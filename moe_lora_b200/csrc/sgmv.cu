@@ -637,9 +637,13 @@ __global__ void __launch_bounds__(1024) lora_plan_kernel(const int32_t* __restri
                                                          const int32_t* __restrict__ seg_adapter, int nseg, int L,
                                                          int nrows, int rb, int2* __restrict__ items,
                                                          int* __restrict__ count, int cap, int* status,
-                                                         int adapters_only) {
+                                                         int adapters_only, int clear_status) {
   __shared__ int s_scan[32];
   pdl_trigger();  // a LoRA kernel launched behind this one may start (it waits for the list)
+  if (clear_status) {  // the call's first kernel: its status block starts at zero
+    for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) status[i] = 0;
+    __syncthreads();
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = (nseg + blockDim.x - 1) / blockDim.x;
   const int q0 = threadIdx.x * per, q1 = min(nseg, q0 + per);
@@ -682,16 +686,18 @@ cudaError_t launch_lora_plan(const LoraDeltaArgs& a, cudaStream_t st) {
   if (a.nrows <= 0) return cudaSuccess;
   ProfScope ps(K_LORA, st);
   lora_plan_kernel<<<1, 1024, 0, st>>>(a.seg_offsets, a.seg_adapter, a.nseg, a.L, a.nrows, a.rb, a.items,
-                                       a.item_count, a.items_bound, a.status, 0);
+                                       a.item_count, a.items_bound, a.status, 0, a.clear_status);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_lora_plan_all(const int32_t* seg_offsets, const int32_t* seg_adapter, int nseg, int L, int nrows,
-                                 int rb, int2* items, int* count, int cap, int* status, cudaStream_t st) {
+                                 int rb, int2* items, int* count, int cap, int* status, cudaStream_t st,
+                                 bool clear_status) {
   if (nrows <= 0) return cudaSuccess;
   ProfScope ps(K_LORA, st);
-  lora_plan_kernel<<<1, 1024, 0, st>>>(seg_offsets, seg_adapter, nseg, L, nrows, rb, items, count, cap, status, 0);
+  lora_plan_kernel<<<1, 1024, 0, st>>>(seg_offsets, seg_adapter, nseg, L, nrows, rb, items, count, cap, status, 0,
+                                       clear_status ? 1 : 0);
   count_launch();
   return cudaGetLastError();
 }
@@ -769,7 +775,10 @@ cudaError_t launch_lora_delta(const LoraDeltaArgs& args, cudaStream_t st) {
 // flight per lane.  A source index outside [0, nsrc) (corrupted pairs) gives a zero row.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ src, int nsrc,
                                                          const int32_t* __restrict__ gather, int div, int rows,
-                                                         int K, __nv_bfloat16* __restrict__ dst) {
+                                                         int K, __nv_bfloat16* __restrict__ dst,
+                                                         int* __restrict__ clear_status) {
+  if (clear_status != nullptr && blockIdx.x == 0)  // the call's first kernel: its status block
+    for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) clear_status[i] = 0;
   const int lane = threadIdx.x & 31;
   const int nw = gridDim.x * 8;
   const int k8 = K / 8;
@@ -791,13 +800,13 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
 }
 
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
-                               __nv_bfloat16* dst, cudaStream_t st) {
+                               __nv_bfloat16* dst, cudaStream_t st, int* clear_status) {
   if (rows <= 0) return cudaSuccess;
   if (K % 8 != 0 || div <= 0) return cudaErrorInvalidValue;
   int grid = (rows + 7) / 8;
   if (grid > 148 * 8) grid = 148 * 8;
   ProfScope ps(K_GATHER, st);
-  gather_rows_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, dst);
+  gather_rows_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, dst, clear_status);
   count_launch();
   return cudaGetLastError();
 }
@@ -957,7 +966,10 @@ __global__ void __launch_bounds__(256) gather_quant_kernel(const __nv_bfloat16* 
                                                           const int32_t* __restrict__ gather, int div, int rows,
                                                           int K, uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
                                                           float* __restrict__ scales,
-                                                          __nv_bfloat16* __restrict__ copy) {
+                                                          __nv_bfloat16* __restrict__ copy,
+                                                          int* __restrict__ clear_status) {
+  if (clear_status != nullptr && blockIdx.x == 0)  // the call's first kernel: its status block
+    for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) clear_status[i] = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
     const int sr = gather[row] / div;
@@ -982,13 +994,14 @@ __global__ void __launch_bounds__(256) gather_quant_kernel(const __nv_bfloat16* 
 }
 
 cudaError_t launch_gather_quant(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
-                                uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy, cudaStream_t st) {
+                                uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy, cudaStream_t st,
+                                int* clear_status) {
   if (rows <= 0) return cudaSuccess;
   if (K % 16 != 0 || div <= 0) return cudaErrorInvalidValue;
   int grid = (rows + 7) / 8;
   if (grid > 148 * 8) grid = 148 * 8;
   ProfScope ps(K_QUANT, st);
-  gather_quant_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales, copy);
+  gather_quant_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales, copy, clear_status);
   count_launch();
   return cudaGetLastError();
 }
