@@ -291,9 +291,23 @@ constexpr int RF_EB = 4;
 constexpr int RF_TB = 8;
 constexpr int RF_MAX_PAIRS = 1024;
 
-// key counts [E (L+1)], pair keys [M k], unnormalised weights [RF_TB][k]
+// key counts [E (L+1)], pair keys [M k], unnormalised weights [RF_TB][k], pair ranks [M k]
 size_t route_fused_smem(int E, int L, int M, int k) {
-  return (static_cast<size_t>(E) * (L + 1) + static_cast<size_t>(M) * k + static_cast<size_t>(RF_TB) * k) * 4;
+  return (static_cast<size_t>(E) * (L + 1) + 2 * static_cast<size_t>(M) * k + static_cast<size_t>(RF_TB) * k) * 4;
+}
+
+// Order-preserving unsigned key of a logit for the arg-max: larger logit, larger key;
+// +0 and -0 share a key (they compare equal); NaN gets 0, the key of "not a candidate",
+// since a NaN logit never wins a comparison.  -inf stays a candidate (key >= 1).
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  uint32_t b = __float_as_uint(v);
+  if (v != v) return 0u;
+  if ((b & 0x7fffffffu) == 0u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 // true in exactly one CTA: the one whose arrival completes `ticket` to `count`
@@ -375,16 +389,16 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteArgs a, con
     tb = blockIdx.x;
   }
 
-  // ---- phase 2: top-k of the token block, one warp per token
+  // ---- phase 2: top-k of the token block, one warp per token.  Each step takes the
+  // largest logit left (the smallest expert id among equal ones) with two warp
+  // reductions: the largest order-preserving key, then the smallest id holding it.
   const int t = tb * RF_TB + warp;
   if (t < a.M) {
-    float v[8];
-    bool used[8];
+    uint32_t kv[8];  // candidate keys; 0 once taken, for NaN and for ids >= E
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane + 32 * i;
-      v[i] = (e < a.E) ? __ldcg(lg + static_cast<size_t>(t) * a.E + e) : -INFINITY;
-      used[i] = (e >= a.E);
+      kv[i] = (e < a.E) ? logit_key(__ldcg(lg + static_cast<size_t>(t) * a.E + e)) : 0u;
     }
     int ad = a.adapter_ids[t];
     if (ad < -1 || ad >= a.L) {
@@ -394,33 +408,25 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteArgs a, con
     float top_v0 = 0.f, denom = 0.f;
     float* wrow = s_w + warp * a.k;
     for (int j = 0; j < a.k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+      uint32_t lk = 0u, le = 0xffffffffu;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        if (!used[i] && (v[i] > bv || (v[i] == bv && e < be))) {
-          bv = v[i];
-          be = e;
+      for (int i = 0; i < 8; ++i)
+        if (kv[i] > lk) {  // ascending i: the lane's smallest id among its largest keys
+          lk = kv[i];
+          le = static_cast<uint32_t>(lane + 32 * i);
         }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if ((be & 31) == lane) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (be == lane + 32 * i) used[i] = true;
-      }
-      if (be >= a.E) {  // only NaN logits remain: flag the token, keep the indices in range
+      const uint32_t bk = __reduce_max_sync(0xffffffffu, lk);
+      int be = static_cast<int>(__reduce_min_sync(0xffffffffu, (bk != 0u && lk == bk) ? le : 0xffffffffu));
+      float bv;
+      if (bk == 0u) {  // only NaN logits remain: flag the token, keep the indices in range
         if (lane == 0) set_status(a.status, MOE_LORA_ERR_DEVICE_CHECK, t);
         be = j % a.E;
+        bv = -INFINITY;
+      } else {
+        bv = key_logit(bk);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (be == lane + 32 * i) kv[i] = 0u;
       }
       if (j == 0) top_v0 = bv;
       const float ex = expf(bv - top_v0);
@@ -469,20 +475,27 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteArgs a, con
     base += c;
   }
   if (threadIdx.x == 0) a.seg_offsets[nk] = mk;
+  // rank of each pair among the earlier pairs of its 32-pair chunk with the same key, and
+  // for the first of them the chunk's count of that key (all warps, one chunk each)
+  int* s_rank = reinterpret_cast<int*>(s_w + RF_TB * a.k);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int p0 = warp * 32; p0 < mk; p0 += 8 * 32) {
+    const int p = p0 + lane;
+    const int key = (p < mk) ? s_key[p] : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (p < mk) s_rank[p] = __popc(peers & lt) | (((peers & lt) == 0u) ? __popc(peers) << 16 : 0);
+  }
   __syncthreads();
+  // stable placement, chunk after chunk: a pair goes to its key's next free slot plus its
+  // rank; the chunk's first pair of each key then moves that key's slot on
   if (warp == 0) {
-    const unsigned lt = (1u << lane) - 1u;
     for (int p0 = 0; p0 < mk; p0 += 32) {
       const int p = p0 + lane;
-      const int key = (p < mk) ? s_key[p] : -1 - lane;
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
-      int pos = 0;
-      if (p < mk) pos = s_cnt[key] + __popc(peers & lt);
+      const int key = (p < mk) ? s_key[p] : 0;
+      const int rk = (p < mk) ? s_rank[p] : 0;
+      if (p < mk) a.sorted_pairs[s_cnt[key] + (rk & 0xffff)] = p;
       __syncwarp();
-      if (p < mk) {
-        a.sorted_pairs[pos] = p;
-        if ((peers & lt) == 0) s_cnt[key] += __popc(peers);
-      }
+      if (p < mk && (rk >> 16) != 0) s_cnt[key] += rk >> 16;
       __syncwarp();
     }
   }
