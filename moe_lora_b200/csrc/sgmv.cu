@@ -168,6 +168,34 @@ cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t st) {
 // core.  |x / s| <= 448 and |(x - hi s) / (s / 16)| <= 448 by construction.
 // One warp quantises one bf16 row of K elements into the two e4m3 planes (see below).
 // copy_row (if set) also receives the bf16 row itself.
+// The two e4m3 planes of 8 bf16 values (one 16-byte chunk) at scale s: hi = e4m3(v / s)
+// and lo = e4m3((v - hi s) 16 / s), 8 bytes each.
+__device__ __forceinline__ void quant8(const uint4 raw, float s, float inv, float inv_lo, uint2& hq8, uint2& lq8) {
+  float f[8];
+  unpack8_bf16(raw, f);
+  uint32_t hq[2], lq[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t hw = 0, lw = 0;
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const int v = 4 * h + 2 * pr;
+      const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(make_float2(f[v] * inv, f[v + 1] * inv),
+                                                              __NV_SATFINITE, __NV_E4M3);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
+      const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      const __nv_fp8x2_storage_t ql = __nv_cvt_float2_to_fp8x2(
+          make_float2((f[v] - d.x * s) * inv_lo, (f[v + 1] - d.y * s) * inv_lo), __NV_SATFINITE, __NV_E4M3);
+      hw |= static_cast<uint32_t>(q) << (16 * pr);
+      lw |= static_cast<uint32_t>(ql) << (16 * pr);
+    }
+    hq[h] = hw;
+    lq[h] = lw;
+  }
+  hq8 = make_uint2(hq[0], hq[1]);
+  lq8 = make_uint2(lq[0], lq[1]);
+}
+
 __device__ __forceinline__ void quant_row_warp(const __nv_bfloat16* src_row, int K, uint8_t* hi_row, uint8_t* lo_row,
                                                float* scale2, int lane, __nv_bfloat16* copy_row = nullptr) {
   const uint4* xr = reinterpret_cast<const uint4*>(src_row);
@@ -184,31 +212,12 @@ __device__ __forceinline__ void quant_row_warp(const __nv_bfloat16* src_row, int
   const float s = amax > 0.f ? amax / 448.f : 1.f;
   const float inv = 1.f / s, inv_lo = 16.f / s;
   for (int c = lane; c < k8; c += 32) {
-    float f[8];
     const uint4 raw = __ldg(xr + c);
     if (copy_row != nullptr) reinterpret_cast<uint4*>(copy_row)[c] = raw;
-    unpack8_bf16(raw, f);
-    uint32_t hq[2], lq[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t hw = 0, lw = 0;
-#pragma unroll
-      for (int pr = 0; pr < 2; ++pr) {
-        const int v = 4 * h + 2 * pr;
-        const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(make_float2(f[v] * inv, f[v + 1] * inv),
-                                                                __NV_SATFINITE, __NV_E4M3);
-        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
-        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-        const __nv_fp8x2_storage_t ql = __nv_cvt_float2_to_fp8x2(
-            make_float2((f[v] - d.x * s) * inv_lo, (f[v + 1] - d.y * s) * inv_lo), __NV_SATFINITE, __NV_E4M3);
-        hw |= static_cast<uint32_t>(q) << (16 * pr);
-        lw |= static_cast<uint32_t>(ql) << (16 * pr);
-      }
-      hq[h] = hw;
-      lq[h] = lw;
-    }
-    reinterpret_cast<uint2*>(hi_row)[c] = make_uint2(hq[0], hq[1]);
-    reinterpret_cast<uint2*>(lo_row)[c] = make_uint2(lq[0], lq[1]);
+    uint2 hq, lq;
+    quant8(raw, s, inv, inv_lo, hq, lq);
+    reinterpret_cast<uint2*>(hi_row)[c] = hq;
+    reinterpret_cast<uint2*>(lo_row)[c] = lq;
   }
   if (lane == 0) {
     scale2[0] = s;
@@ -993,14 +1002,85 @@ __global__ void __launch_bounds__(256) gather_quant_kernel(const __nv_bfloat16* 
   }
 }
 
+// Rows of up to 8192 elements: one CTA per row, the row's 16-byte chunks held in
+// registers (U per thread), so each row is read once; the same arithmetic as
+// quant_row_warp (the row maximum does not depend on the order it is taken in).  gather
+// null: row i of src; an index outside [0, nsrc) gives zero planes and zero scales.
+template <int U>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __restrict__ src, int nsrc,
+                                                        const int32_t* __restrict__ gather, int div, int rows, int K,
+                                                        uint8_t* __restrict__ hi, uint8_t* __restrict__ lo,
+                                                        float* __restrict__ scales, __nv_bfloat16* __restrict__ copy,
+                                                        int* __restrict__ clear_status) {
+  __shared__ float s_amax[8];
+  if (clear_status != nullptr && blockIdx.x == 0)  // the call's first kernel: its status block
+    for (int i = threadIdx.x; i < static_cast<int>(kStatusBytes / 4); i += blockDim.x) clear_status[i] = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k8 = K / 8;
+  for (int row = blockIdx.x; row < rows; row += gridDim.x) {
+    const int sr = gather != nullptr ? gather[row] / div : row;
+    const bool ok = sr >= 0 && sr < nsrc;
+    const uint4* xr = reinterpret_cast<const uint4*>(src + static_cast<size_t>(ok ? sr : 0) * K);
+    uint4 raw[U];
+    float amax = 0.f;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = threadIdx.x + 256 * u;
+      raw[u] = (ok && c < k8) ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+      float f[8];
+      unpack8_bf16(raw[u], f);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) amax = fmaxf(amax, fabsf(f[v]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) s_amax[warp] = amax;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = fmaxf(amax, s_amax[w]);
+    const float s = amax > 0.f ? amax / 448.f : 1.f;
+    const float inv = 1.f / s, inv_lo = 16.f / s;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = threadIdx.x + 256 * u;
+      if (c < k8) {
+        if (copy != nullptr) reinterpret_cast<uint4*>(copy + static_cast<size_t>(row) * K)[c] = raw[u];
+        uint2 hq, lq;
+        quant8(raw[u], s, inv, inv_lo, hq, lq);  // zero chunks give zero bytes
+        reinterpret_cast<uint2*>(hi + static_cast<size_t>(row) * K)[c] = hq;
+        reinterpret_cast<uint2*>(lo + static_cast<size_t>(row) * K)[c] = lq;
+      }
+    }
+    if (threadIdx.x == 0) {
+      scales[2 * static_cast<size_t>(row)] = ok ? s : 0.f;
+      scales[2 * static_cast<size_t>(row) + 1] = ok ? s / 16.f : 0.f;
+    }
+    __syncthreads();  // s_amax is rewritten for the next row
+  }
+}
+
+// quant_rows_kernel for K <= 8192 (one row per CTA), else the warp-per-row kernels
+static cudaError_t launch_quant_rows(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows,
+                                     int K, uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy,
+                                     int* clear_status, cudaStream_t st) {
+  const int k8 = K / 8;
+  const int grid = rows < 148 * 8 ? rows : 148 * 8;
+  if (k8 <= 256) quant_rows_kernel<1><<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales, copy, clear_status);
+  else if (k8 <= 512) quant_rows_kernel<2><<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales, copy, clear_status);
+  else quant_rows_kernel<4><<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales, copy, clear_status);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gather_quant(const __nv_bfloat16* src, int nsrc, const int32_t* gather, int div, int rows, int K,
                                 uint8_t* hi, uint8_t* lo, float* scales, __nv_bfloat16* copy, cudaStream_t st,
                                 int* clear_status) {
   if (rows <= 0) return cudaSuccess;
   if (K % 16 != 0 || div <= 0) return cudaErrorInvalidValue;
+  ProfScope ps(K_QUANT, st);
+  if (K / 8 <= 1024) return launch_quant_rows(src, nsrc, gather, div, rows, K, hi, lo, scales, copy, clear_status, st);
   int grid = (rows + 7) / 8;
   if (grid > 148 * 8) grid = 148 * 8;
-  ProfScope ps(K_QUANT, st);
   gather_quant_kernel<<<grid, 256, 0, st>>>(src, nsrc, gather, div, rows, K, hi, lo, scales, copy, clear_status);
   count_launch();
   return cudaGetLastError();
@@ -1010,9 +1090,10 @@ cudaError_t launch_quant_planes(const __nv_bfloat16* src, int rows, int K, uint8
                                 cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   if (K % 16 != 0) return cudaErrorInvalidValue;
+  ProfScope ps(K_QUANT, st);
+  if (K / 8 <= 1024) return launch_quant_rows(src, rows, nullptr, 1, rows, K, hi, lo, scales, nullptr, nullptr, st);
   int grid = (rows + 7) / 8;
   if (grid > 148 * 8) grid = 148 * 8;
-  ProfScope ps(K_QUANT, st);
   quant_planes_kernel<<<grid, 256, 0, st>>>(src, rows, K, hi, lo, scales);
   count_launch();
   return cudaGetLastError();
