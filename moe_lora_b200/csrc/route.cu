@@ -440,7 +440,10 @@ __global__ void __launch_bounds__(256) route_fused_kernel(const RouteArgs a, con
     const float inv = 1.0f / denom;
     for (int j = lane; j < a.k; j += 32) a.topk_w[t * a.k + j] = wrow[j] * inv;
   }
-  if (!arrive_last(tickets + n_tb, n_tb, &s_flag)) return;
+  // one token block (M <= 8): this CTA is the only one past phase 2, and a block barrier
+  // makes its top-k visible to its phase 3
+  if (n_tb == 1) __syncthreads();
+  else if (!arrive_last(tickets + n_tb, n_tb, &s_flag)) return;
 
   // ---- phase 3: key counts, CSR offsets, stable placement (one CTA)
   for (int i = threadIdx.x; i < nk; i += blockDim.x) s_cnt[i] = 0;
